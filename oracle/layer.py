@@ -1,0 +1,345 @@
+"""fp64 oracle: the plain definition of one pre-LayerNorm GPT layer with Megatron-style
+tensor-parallel partitioning, forward and hand-written reverse-mode backward.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring). Float64 numpy throughout; the only
+library primitives are matmul, exp, log, tanh and scipy's erf.
+
+Sources (web pages about Megatron-LM; they print no formulas, so each reading is stated):
+  [TP]   "Megatron-LM 3D并行原理与万亿参数训练实战指南" (trdm.cn), section 2.1 (tensor
+         parallelism): W_q/W_k/W_v column-split, x broadcast to every shard, each shard
+         computes its own heads without communication; W_o row-split, each shard's partial
+         output summed by AllReduce; the softmax needs whole heads, hence column-then-row.
+  [API]  "Megatron-LM：NVIDIA大模型训练框架" (second-brain-czx), section "张量并行":
+         ColumnParallelLinear(h, 3h, gather_output=False) then RowParallelLinear(h, h,
+         input_is_parallel=True) around the attention.
+  [MD]   the trdm.cn page, section 3.2 (model definition): LayerNorm statistics global over the
+         hidden dimension; hidden and head counts divisible by tp_size; softmax in fp32
+         (attention_softmax_in_fp32); apply_query_key_layer_scaling flag.
+  [ACT]  the trdm.cn page, section 3.3 (launch flags): GeLU is the default MLP activation.
+  [RC]   the trdm.cn page, section 4.1 (checkpointing / recompute): only the layer input is
+         kept and intermediates are recomputed in backward -- mathematically the identity.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * LayerNorm: biased variance (divide by h), eps inside the square root, affine gamma/beta.
+  * Pre-LN block with two LayerNorms and two residuals: y = h1 + MLP(LN2(h1)),
+    h1 = x + Attn(LN1(x)).
+  * Softmax scale 1/sqrt(d); query-key layer scaling is an identity under an fp32 softmax.
+  * Causal mask: key j visible to query i iff j <= i; masked probabilities are exactly 0.
+  * Row-parallel biases (b_o, b2) are added once, after the shard sum.
+  * GeLU exact: u * Phi(u); the tanh form is selected by gelu_tanh=1.
+  * QKV packing: shard-major, then [Q|K|V], then head, then head_dim.
+  * No dropout.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf
+
+f64 = np.float64
+
+
+# ----------------------------------------------------------------------------- LayerNorm
+def layer_norm(x, gamma, beta, eps):
+    """LN over the last axis of x [rows, h]: mean, biased variance, xhat=(x-mean)*rstd,
+    y = gamma*xhat + beta. Statistics are over the full hidden dimension on every shard
+    ([MD]: the normalisation statistics must agree across the TP group; under the column/row
+    split the LN input is replicated, so each shard sees the whole row).
+    Returns (y, mean, rstd, xhat)."""
+    x = np.asarray(x, f64)
+    mean = x.mean(axis=-1)
+    var = ((x - mean[:, None]) ** 2).mean(axis=-1)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xhat = (x - mean[:, None]) * rstd[:, None]
+    return xhat * gamma + beta, mean, rstd, xhat
+
+
+def layer_norm_grad(dy, xhat, rstd, gamma):
+    """Reverse of layer_norm given the upstream grad dy [rows, h].
+    With g = dy*gamma: dx = rstd * (g - mean(g) - xhat * mean(g*xhat)),
+    dgamma = sum_rows dy*xhat, dbeta = sum_rows dy."""
+    g = dy * gamma
+    dx = rstd[:, None] * (g - g.mean(axis=-1, keepdims=True)
+                          - xhat * (g * xhat).mean(axis=-1, keepdims=True))
+    return dx, (dy * xhat).sum(axis=0), dy.sum(axis=0)
+
+
+# ----------------------------------------------------------------------------- GeLU ([ACT])
+_SQRT_2_OVER_PI = math.sqrt(2.0 / math.pi)
+_TANH_C = 0.044715
+
+
+def gelu(u, tanh_approx=0):
+    """Exact GeLU u*Phi(u) = u/2 * (1 + erf(u/sqrt 2)); tanh form if tanh_approx."""
+    if tanh_approx:
+        return 0.5 * u * (1.0 + np.tanh(_SQRT_2_OVER_PI * (u + _TANH_C * u ** 3)))
+    return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))
+
+
+def gelu_grad(u, tanh_approx=0):
+    """d GeLU / du: exact form Phi(u) + u*phi(u)."""
+    if tanh_approx:
+        z = _SQRT_2_OVER_PI * (u + _TANH_C * u ** 3)
+        t = np.tanh(z)
+        return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * _SQRT_2_OVER_PI * (
+            1.0 + 3.0 * _TANH_C * u * u)
+    cdf = 0.5 * (1.0 + erf(u / math.sqrt(2.0)))
+    pdf = np.exp(-0.5 * u * u) / math.sqrt(2.0 * math.pi)
+    return cdf + u * pdf
+
+
+# ----------------------------------------------------------------------------- attention
+def causal_softmax(S):
+    """Row-wise softmax of S [s, s] over the visible keys j <= i; masked entries are 0.
+    Returns (P, lse) with lse_i = log sum_{j<=i} exp(S_ij)."""
+    s = S.shape[0]
+    mask = np.tril(np.ones((s, s), dtype=bool))
+    Sm = np.where(mask, S, -np.inf)
+    m = Sm.max(axis=1)
+    e = np.where(mask, np.exp(Sm - m[:, None]), 0.0)
+    z = e.sum(axis=1)
+    return e / z[:, None], m + np.log(z)
+
+
+def attention_head_fwd(q, k, v):
+    """One head of causal attention on q, k, v [s, d]: S = q k^T / sqrt(d) (scale reading),
+    P = causal softmax (kept in full precision, [MD]), o = P v. Returns (o, lse, P)."""
+    d = q.shape[1]
+    P, lse = causal_softmax((q @ k.T) / math.sqrt(d))
+    return P @ v, lse, P
+
+
+def attention_head_bwd(q, k, v, P, do):
+    """Reverse of attention_head_fwd: dv = P^T do; dP = do v^T; dS = P*(dP - rowsum(P*dP));
+    dq = dS k / sqrt(d); dk = dS^T q / sqrt(d)."""
+    d = q.shape[1]
+    dv = P.T @ do
+    dP = do @ v.T
+    D = (P * dP).sum(axis=1)
+    dS = P * (dP - D[:, None])
+    return dS @ k / math.sqrt(d), dS.T @ q / math.sqrt(d), dv
+
+
+def attention_fwd(qkv, b, s, heads, tp):
+    """Causal attention over a packed qkv [b*s, p, 3, H/p, d]: each shard owns whole heads
+    ([TP]: column-split Q/K/V let each shard run its heads' softmax locally).
+    Returns O [b*s, p, H/p, d] and lse [b, H, s]."""
+    T = b * s
+    hp = heads // tp
+    d = qkv.shape[-1]
+    O = np.empty((T, tp, hp, d))
+    lse = np.empty((b, heads, s))
+    for bi in range(b):
+        rows = slice(bi * s, (bi + 1) * s)
+        for t in range(tp):
+            for j in range(hp):
+                o, l, _ = attention_head_fwd(qkv[rows, t, 0, j], qkv[rows, t, 1, j],
+                                             qkv[rows, t, 2, j])
+                O[rows, t, j] = o
+                lse[bi, t * hp + j] = l
+    return O, lse
+
+
+def attention_bwd(qkv, dO, b, s, heads, tp):
+    """Backward of attention_fwd; P is recomputed from q and k ([RC]). Returns dqkv in the
+    packed layout of qkv."""
+    hp = heads // tp
+    dqkv = np.empty_like(qkv)
+    for bi in range(b):
+        rows = slice(bi * s, (bi + 1) * s)
+        for t in range(tp):
+            for j in range(hp):
+                q, k, v = qkv[rows, t, 0, j], qkv[rows, t, 1, j], qkv[rows, t, 2, j]
+                _, _, P = attention_head_fwd(q, k, v)
+                dq, dk, dv = attention_head_bwd(q, k, v, P, dO[rows, t, j])
+                dqkv[rows, t, 0, j] = dq
+                dqkv[rows, t, 1, j] = dk
+                dqkv[rows, t, 2, j] = dv
+    return dqkv
+
+
+# ----------------------------------------------------------------------------- the layer
+def _np(a):
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().to(dtype=__import__("torch").float64).numpy()
+    return np.asarray(a, f64)
+
+
+def layer_fwd(cfg, params, x):
+    """Forward of the layer on packed per-shard parameters (the TP path).
+
+    cfg: object with hidden, heads, ffn, seq, micro_batch, tp_size, ln_eps, gelu_tanh.
+    params: dict of packed arrays (layouts in the mgt_inputs docstring). x: [b, s, h].
+    Returns (y [b, s, h], saved dict of every intermediate)."""
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    b, s = cfg.micro_batch, cfg.seq
+    T, d, hp = b * s, h // H, H // p
+    P = {k: _np(v) for k, v in params.items()}
+    x2 = _np(x).reshape(T, h)
+
+    ln1, mu1, rstd1, xhat1 = layer_norm(x2, P["ln1_g"], P["ln1_b"], cfg.ln_eps)
+    # Column-parallel QKV ([TP], [API]): every shard multiplies the replicated ln1 by its own
+    # row block of W_qkv; no reduction.
+    qkv = np.empty((T, p, 3, hp, d))
+    for t in range(p):
+        w_t = P["w_qkv"][t].reshape(3 * hp * d, h)
+        qkv[:, t] = (ln1 @ w_t.T + P["b_qkv"][t].reshape(-1)).reshape(T, 3, hp, d)
+    O, lse = attention_fwd(qkv, b, s, H, p)
+    # Row-parallel out-proj ([TP]): shard t multiplies its slice of the attention output by
+    # its input-column block of W_o; the partials are summed (the AllReduce), then b_o is
+    # added once and the residual x.
+    acc = np.zeros((T, h))
+    for t in range(p):
+        acc += O[:, t].reshape(T, h // p) @ P["w_o"][t].T
+    h1 = x2 + P["b_o"] + acc
+    ln2, mu2, rstd2, xhat2 = layer_norm(h1, P["ln2_g"], P["ln2_b"], cfg.ln_eps)
+    # Column-parallel fc1 + GeLU, row-parallel fc2 with shard sum, bias once, residual.
+    u = np.empty((T, p, f // p))
+    for t in range(p):
+        u[:, t] = ln2 @ P["w1"][t].T + P["b1"][t]
+    a = gelu(u, cfg.gelu_tanh)
+    acc2 = np.zeros((T, h))
+    for t in range(p):
+        acc2 += a[:, t] @ P["w2"][t].T
+    y = h1 + P["b2"] + acc2
+    saved = dict(x=x2, ln1=ln1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, qkv=qkv, O=O, lse=lse,
+                 h1=h1, ln2=ln2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, u=u, a=a)
+    return y.reshape(b, s, h), saved
+
+
+def layer_bwd(cfg, params, saved, dy):
+    """Hand-written reverse of layer_fwd (packed TP path). Returns (dx [b,s,h], grads in the
+    packed parameter layout, intermediate grads)."""
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    b, s = cfg.micro_batch, cfg.seq
+    T, d, hp = b * s, h // H, H // p
+    P = {k: _np(v) for k, v in params.items()}
+    dy2 = _np(dy).reshape(T, h)
+    g = {}
+    # fc2 (row-parallel): y = h1 + b2 + sum_t a_t W2_t^T
+    g["b2"] = dy2.sum(axis=0)
+    g["w2"] = np.empty((p, h, f // p))
+    da = np.empty((T, p, f // p))
+    for t in range(p):
+        g["w2"][t] = dy2.T @ saved["a"][:, t]
+        da[:, t] = dy2 @ P["w2"][t]
+    du = da * gelu_grad(saved["u"], cfg.gelu_tanh)
+    # fc1 (column-parallel): the input ln2 was broadcast to every shard, so its gradient is
+    # the sum of the shards' contributions.
+    g["b1"] = du.sum(axis=0)
+    g["w1"] = np.empty((p, f // p, h))
+    dln2 = np.zeros((T, h))
+    for t in range(p):
+        g["w1"][t] = du[:, t].T @ saved["ln2"]
+        dln2 += du[:, t] @ P["w1"][t]
+    d_ln, g["ln2_g"], g["ln2_b"] = layer_norm_grad(dln2, saved["xhat2"], saved["rstd2"],
+                                                   P["ln2_g"])
+    dh1 = dy2 + d_ln
+    # out-proj (row-parallel)
+    g["b_o"] = dh1.sum(axis=0)
+    g["w_o"] = np.empty((p, h, h // p))
+    dO = np.empty((T, p, hp, d))
+    for t in range(p):
+        g["w_o"][t] = dh1.T @ saved["O"][:, t].reshape(T, h // p)
+        dO[:, t] = (dh1 @ P["w_o"][t]).reshape(T, hp, d)
+    dqkv = attention_bwd(saved["qkv"], dO, b, s, H, p)
+    # QKV (column-parallel)
+    g["b_qkv"] = np.empty((p, 3, hp, d))
+    g["w_qkv"] = np.empty((p, 3, hp, d, h))
+    dln1 = np.zeros((T, h))
+    for t in range(p):
+        dq_t = dqkv[:, t].reshape(T, 3 * hp * d)
+        g["b_qkv"][t] = dq_t.sum(axis=0).reshape(3, hp, d)
+        g["w_qkv"][t] = (dq_t.T @ saved["ln1"]).reshape(3, hp, d, h)
+        dln1 += dq_t @ P["w_qkv"][t].reshape(3 * hp * d, h)
+    d_ln1, g["ln1_g"], g["ln1_b"] = layer_norm_grad(dln1, saved["xhat1"], saved["rstd1"],
+                                                    P["ln1_g"])
+    dx = dh1 + d_ln1
+    inter = dict(du=du, dln2=dln2, dh1=dh1, dO=dO, dqkv=dqkv, dln1=dln1)
+    return dx.reshape(b, s, h), g, inter
+
+
+def layer_fwd_full(cfg, params, x):
+    """The same layer on full, unsharded matrices (no tensor parallelism): w_qkv [3h, h] with
+    rows [Q | K | V], head n of each at rows n*d..(n+1)*d-1; w_o [h, h]; w1 [f, h]; w2 [h, f].
+    Used to check that the sharded computation equals the unsharded one."""
+    h, H = cfg.hidden, cfg.heads
+    b, s = cfg.micro_batch, cfg.seq
+    T, d = b * s, h // H
+    P = {k: _np(v) for k, v in params.items()}
+    x2 = _np(x).reshape(T, h)
+    ln1, mu1, rstd1, xhat1 = layer_norm(x2, P["ln1_g"], P["ln1_b"], cfg.ln_eps)
+    qkv = ln1 @ P["w_qkv"].T + P["b_qkv"]
+    O = np.empty((T, h))
+    for bi in range(b):
+        rows = slice(bi * s, (bi + 1) * s)
+        for n in range(H):
+            c = slice(n * d, (n + 1) * d)
+            o, _, _ = attention_head_fwd(qkv[rows, c], qkv[rows, h:][:, c],
+                                         qkv[rows, 2 * h:][:, c])
+            O[rows, c] = o
+    h1 = x2 + O @ P["w_o"].T + P["b_o"]
+    ln2, mu2, rstd2, xhat2 = layer_norm(h1, P["ln2_g"], P["ln2_b"], cfg.ln_eps)
+    u = ln2 @ P["w1"].T + P["b1"]
+    a = gelu(u, cfg.gelu_tanh)
+    y = h1 + a @ P["w2"].T + P["b2"]
+    saved = dict(x=x2, ln1=ln1, xhat1=xhat1, rstd1=rstd1, qkv=qkv, O=O, h1=h1, ln2=ln2,
+                 xhat2=xhat2, rstd2=rstd2, u=u, a=a)
+    return y.reshape(b, s, h), saved
+
+
+def layer_bwd_full(cfg, params, saved, dy):
+    """Reverse of layer_fwd_full. Returns (dx, grads in the full layout)."""
+    h, H = cfg.hidden, cfg.heads
+    b, s = cfg.micro_batch, cfg.seq
+    T, d = b * s, h // H
+    P = {k: _np(v) for k, v in params.items()}
+    dy2 = _np(dy).reshape(T, h)
+    g = {}
+    g["b2"] = dy2.sum(axis=0)
+    g["w2"] = dy2.T @ saved["a"]
+    du = (dy2 @ P["w2"]) * gelu_grad(saved["u"], cfg.gelu_tanh)
+    g["b1"] = du.sum(axis=0)
+    g["w1"] = du.T @ saved["ln2"]
+    d_ln, g["ln2_g"], g["ln2_b"] = layer_norm_grad(du @ P["w1"], saved["xhat2"],
+                                                   saved["rstd2"], P["ln2_g"])
+    dh1 = dy2 + d_ln
+    g["b_o"] = dh1.sum(axis=0)
+    g["w_o"] = dh1.T @ saved["O"]
+    dO = dh1 @ P["w_o"]
+    qkv = saved["qkv"]
+    dqkv = np.empty_like(qkv)
+    for bi in range(b):
+        rows = slice(bi * s, (bi + 1) * s)
+        for n in range(H):
+            c = slice(n * d, (n + 1) * d)
+            q, k, v = qkv[rows, c], qkv[rows, h:][:, c], qkv[rows, 2 * h:][:, c]
+            _, _, Pm = attention_head_fwd(q, k, v)
+            dq, dk, dv = attention_head_bwd(q, k, v, Pm, dO[rows, c])
+            dqkv[rows, n * d:(n + 1) * d] = dq
+            dqkv[rows, h + n * d:h + (n + 1) * d] = dk
+            dqkv[rows, 2 * h + n * d:2 * h + (n + 1) * d] = dv
+    g["b_qkv"] = dqkv.sum(axis=0)
+    g["w_qkv"] = dqkv.T @ saved["ln1"]
+    d_ln1, g["ln1_g"], g["ln1_b"] = layer_norm_grad(dqkv @ P["w_qkv"], saved["xhat1"],
+                                                    saved["rstd1"], P["ln1_g"])
+    dx = dh1 + d_ln1
+    return dx.reshape(b, s, h), g
+
+
+def gather_grads(cfg, g):
+    """Packed per-shard gradients -> full layout (index permutation, the inverse of the
+    packing), so sharded results can be compared with layer_bwd_full."""
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    d, hp = h // H, H // p
+    out = dict(g)
+    out["w_qkv"] = np.asarray(g["w_qkv"]).reshape(p, 3, hp, d, h).transpose(1, 0, 2, 3, 4) \
+        .reshape(3 * h, h)
+    out["b_qkv"] = np.asarray(g["b_qkv"]).reshape(p, 3, hp, d).transpose(1, 0, 2, 3) \
+        .reshape(3 * h)
+    out["w_o"] = np.asarray(g["w_o"]).reshape(p, h, h // p).transpose(1, 0, 2).reshape(h, h)
+    out["w1"] = np.asarray(g["w1"]).reshape(f, h)
+    out["b1"] = np.asarray(g["b1"]).reshape(f)
+    out["w2"] = np.asarray(g["w2"]).reshape(p, h, f // p).transpose(1, 0, 2).reshape(h, f)
+    return out
