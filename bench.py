@@ -1,0 +1,326 @@
+"""Benchmark: forward + backward of the Megatron-style tensor-parallel GPT layer on B200.
+
+Default workload: the h=4096 layer (32 heads of 128, ffn 11008, seq 2048, micro-batch 1,
+logical tp_size 2, bf16 with fp32 accumulation), synthetic seeded inputs. One "step" = one
+mgt_layer_fwd + one mgt_layer_bwd over one batch. With --gpus N (launched by torchrun) every
+rank runs its own replica on its own batch (data parallel, no collective on the data path):
+weak scaling, value = tokens of all ranks / max-over-ranks time.
+
+Prints ONE JSON line (rank 0). --impl reference times the fp64 CPU oracle instead, on a bounded
+sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "layer fwd+bwd tokens/s and TFLOP/s (fraction of B200 bf16 peak) at h=4096"
+DEFAULT_WORKLOAD = "gpt-h4096-tp2-bf16"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels per launch of each profiled family (the C ABI times families, some launch several)
+KERNELS_PER_LAUNCH = {"gemm_tc": 1, "gemm_simt": 1, "attn_fwd": 1, "attn_bwd": 3, "ln_fwd": 1,
+                      "ln_bwd": 2, "colsum": 1}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: d[k] for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def run_mgt(args):
+    import torch
+
+    import tensor_transformer_layer_megatron_b200 as mgt
+    from mgt_inputs import config_by_name, make_inputs, pack_params
+    from tensor_transformer_layer_megatron_b200.runner import LayerRun
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = config_by_name(args.config)
+    t = make_inputs(cfg)
+    packed = pack_params(cfg, t)
+    layer = mgt.Layer.from_config(cfg)
+    run = LayerRun(layer, packed, t["x"], t["dy"], device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        run.step()
+    run.check()
+    torch.cuda.synchronize()
+
+    # ---- timed region: device events, per-kernel events inside the C ABI
+    layer.profile(True)
+    layer.profile_read()  # reset totals
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    prof = layer.profile_read()
+    layer.profile(False)
+    run.check()
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / args.steps
+    tokens = cfg.tokens * world
+    value = tokens / (ms_step / 1e3)
+    flops_step = cfg.model_flops() * world
+    tflops = flops_step / (ms_step / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    x_h = run.x.cpu().pin_memory()
+    dy_h = run.dy.cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    dx_h = torch.empty_like(x_h).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        run.x.copy_(x_h, non_blocking=True)
+        run.dy.copy_(dy_h, non_blocking=True)
+        run.step()
+        y_h.copy_(run.y, non_blocking=True)
+        dx_h.copy_(run.dx, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = tokens / (e2e_ms / args.steps / 1e3)
+    h2d = (x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size())
+    d2h = (y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size())
+
+    # ---- roofline of the dominant kernel family (the tcgen05 GEMM)
+    peaks, peak_src = load_peaks()
+    fam = max(prof.items(), key=lambda kv: kv[1]["ms"]) if prof else (None, None)
+    roof = None
+    if fam[0] is not None:
+        name, st = fam
+        if st["flops"] > 0:
+            achieved = st["flops"] / (st["ms"] / 1e3) / 1e12
+            roof = {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                    "peak_source": peak_src + " bf16_tflops_sustained (kernel timed inside "
+                                   "the step)",
+                    "traffic": None,
+                    "launches": st["launches"], "avg_launch_ms": round(st["ms"] / st["launches"], 4),
+                    "share_of_step": round(st["ms"] / ms, 4)}
+        else:
+            achieved = st["bytes"] / (st["ms"] / 1e3) / 1e9
+            roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+    kernels = {k: {"launches": v["launches"], "ms_per_step": round(v["ms"] / args.steps, 4),
+                   **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)}
+                      if v["flops"] else {}),
+                   **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)}
+                      if v["bytes"] else {})}
+               for k, v in prof.items()}
+    launches = sum(v["launches"] * KERNELS_PER_LAUNCH.get(k, 1) for k, v in prof.items())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, args.cpu_tokens)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs and N(0,0.02) random-init weights)",
+            "tflops": round(tflops, 1),
+            "frac_of_nominal_2250": round(tflops / NOMINAL_BF16_TFLOPS, 4),
+            "frac_of_measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+            "frac_of_measured_burst": round(tflops / peaks["bf16_tflops"], 4),
+            "config": {"workload": cfg.name, "hidden": cfg.hidden, "heads": cfg.heads,
+                       "ffn": cfg.ffn, "seq_len": cfg.seq, "micro_batch": cfg.micro_batch,
+                       "tp_size": cfg.tp_size, "tokens_per_gpu": cfg.tokens,
+                       "global_batch": cfg.micro_batch * world,
+                       "parallelism": "dp%d (independent replicas), logical tp%d per replica"
+                                      % (world, cfg.tp_size),
+                       "l2": "no flush: per-step working set (weights 315 MB bf16 + fp32 grads "
+                             "630 MB + activations) exceeds the 126 MB L2"},
+            "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "x, dy pinned host -> device; fwd+bwd via the C ABI; y, dx -> host"},
+            "roofline": roof,
+            "kernels": kernels,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def cpu_baseline(cfg, tokens):
+    """The fp64 oracle, as it stands, on a bounded sample: one sequence of `tokens` tokens of
+    the same layer (weights of the full shape), forward + backward, on this host's cores."""
+    import torch
+
+    import oracle
+    from mgt_inputs import make_inputs, pack_params
+    sub = cfg.replace(seq=tokens, micro_batch=1)
+    t = make_inputs(sub)
+    packed = pack_params(sub, t)
+    t0 = time.time()
+    _, saved = oracle.layer_fwd(sub, packed, t["x"])
+    oracle.layer_bwd(sub, packed, saved, t["dy"])
+    dt = time.time() - t0
+    return {"value": round(tokens / dt, 3), "unit": "tokens/s",
+            "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": "fp64 numpy oracle fwd+bwd of one %d-token sequence of the %s layer "
+                      "(full weight shapes), %.1f s" % (tokens, cfg.name, dt)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from mgt_inputs import config_by_name
+    cfg = config_by_name(args.config)
+    import torch
+    samples = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(cfg, args.cpu_tokens)
+        if i >= args.warmup:
+            samples.append(r)
+    v = sum(s["value"] for s in samples) / len(samples)
+    ms_step = cfg.tokens / v * 1e3
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(ms_step, 1), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": cfg.name, "tokens_per_step_sampled": args.cpu_tokens},
+           "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s",
+                            "cores": torch.get_num_threads(), "kind": "oracle",
+                            "sample": samples[0]["sample"]},
+           "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mgt", choices=["mgt", "reference"])
+    ap.add_argument("--config", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mgt(args)
+
+
+if __name__ == "__main__":
+    main()

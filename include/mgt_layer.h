@@ -1,0 +1,189 @@
+/*
+ * mgt_layer.h -- C ABI of a B200-native (sm_100a) Megatron-style tensor-parallel GPT layer.
+ *
+ * One pre-LayerNorm GPT block, forward and backward, on one GPU with a *logical* tp_size:
+ *
+ *   ln1 = LN(x; g1, b1)
+ *   qkv = ln1 W_qkv^T + b_qkv        column-parallel: each shard owns whole heads
+ *   o   = causal softmax attention per head (scale 1/sqrt(d), softmax in fp32)
+ *   h1  = x + b_o + sum_t o_t W_o,t^T     row-parallel: shard partials summed on-device
+ *   ln2 = LN(h1; g2, b2)
+ *   a   = GeLU(ln2 W1^T + b1)         column-parallel
+ *   y   = h1 + b2 + sum_t a_t W2,t^T      row-parallel
+ *
+ * Sources: the page "Megatron-LM 3D并行原理与万亿参数训练实战指南" (trdm.cn), section 2.1
+ * (tensor parallelism: W_q/W_k/W_v split by output columns with x broadcast and no
+ * communication; W_o split by input rows with partial outputs summed by AllReduce), section 3.2
+ * (LayerNorm statistics global over hidden; hidden and heads divisible by tp_size; softmax in
+ * fp32), section 3.3 (GeLU is the default activation); and the page "Megatron-LM：NVIDIA大模型
+ * 训练框架" (second-brain-czx), section "张量并行" (ColumnParallelLinear with
+ * gather_output=False feeding RowParallelLinear with input_is_parallel=True). The pages give no
+ * formulas; the readings taken (LN eps 1e-5 inside the square root with biased variance, exact
+ * erf GeLU, biases of row-parallel layers added once after the shard sum, two LNs and two
+ * residuals) are documented with the oracle.
+ *
+ * Conventions
+ *   - Row-major everywhere. Weights are nn.Linear style [out, in]; y = x W^T + b.
+ *   - Packed per-shard weights (column split = block of output rows, row split = block of
+ *     input columns):
+ *         w_qkv [p][3][H/p][d][h]   b_qkv [p][3][H/p][d]
+ *         w_o   [p][h][h/p]         b_o   [h]
+ *         w1    [p][f/p][h]         b1    [p][f/p]
+ *         w2    [p][h][f/p]         b2    [h]
+ *         ln1_g, ln1_b, ln2_g, ln2_b [h]
+ *   - x, y, dx, dy: [b, s, h], tokens flattened as T = b*s with s fastest.
+ *   - dtype MGT_BF16: activations, weights and biases are bf16; LN gamma/beta are fp32.
+ *     dtype MGT_F32: everything fp32. All gradients of parameters are written in fp32 and
+ *     OVERWRITTEN (not accumulated); dx is in the activation dtype.
+ *   - All device pointers are owned by the caller. The handle owns host state only (config,
+ *     derived sizes, optional profiling events). Calls are asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - The library never allocates device memory. `saved` (written by fwd, read by bwd) and
+ *     `workspace` are caller buffers of the sizes mgt_layer_sizes reports, 256-byte aligned.
+ *     The first 256 bytes of `workspace` hold the device status word: zero the workspace once
+ *     after allocating it; device errors accumulate there until mgt_layer_get_error reads and
+ *     clears them.
+ *
+ * Errors: synchronous validation returns MGT_EINVAL / MGT_EUNSUPPORTED without touching the
+ * GPU; a failed launch returns MGT_ECUDA; a device-side bounded wait that runs out records
+ * MGT_ETIMEOUT in the status word (read by mgt_layer_get_error). Nothing aborts or traps.
+ */
+#ifndef MGT_LAYER_H
+#define MGT_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mgt_status {
+  MGT_OK = 0,
+  MGT_EINVAL = 1,        /* bad sizes, null pointers, divisibility (h%p, H%p, h%H, f%p) */
+  MGT_EUNSUPPORTED = 2,  /* dtype, head_dim, alignment outside what the kernels implement */
+  MGT_ECUDA = 3,         /* a CUDA runtime/driver call or kernel launch failed */
+  MGT_ETIMEOUT = 4,      /* a device-side bounded wait gave up (see mgt_layer_get_error) */
+  MGT_ENOMEM = 5         /* a caller buffer is smaller than required */
+} mgt_status;
+
+typedef enum mgt_dtype { MGT_F32 = 0, MGT_BF16 = 1 } mgt_dtype;
+
+/* Layer shape and numerics. Mirrors TransformerConfig(hidden_size, num_attention_heads,
+ * ffn_hidden_size, seq_length) plus micro-batch and the logical tensor-parallel size.
+ * Valid: all sizes > 0; hidden % heads == 0; hidden % tp_size == 0; heads % tp_size == 0;
+ * ffn % tp_size == 0; head_dim in {64, 128} for bf16, <= 64 for f32; for bf16 also
+ * hidden/tp_size and ffn/tp_size multiples of 64. causal must be 1 (the GPT mask);
+ * recompute_attn is accepted for either value -- attention probabilities are never stored,
+ * the backward always recomputes them from the saved log-sum-exp. */
+typedef struct mgt_layer_config {
+  int32_t hidden;
+  int32_t heads;
+  int32_t ffn;
+  int32_t seq;
+  int32_t micro_batch;
+  int32_t tp_size;
+  int32_t dtype;          /* mgt_dtype */
+  int32_t causal;         /* must be 1 */
+  float ln_eps;           /* LayerNorm epsilon, added to the biased variance */
+  int32_t recompute_attn; /* informational; see above */
+  int32_t gelu_tanh;      /* 0: exact erf GeLU; 1: tanh approximation */
+} mgt_layer_config;
+
+/* Parameters (device pointers, packed layouts above). */
+typedef struct mgt_layer_params {
+  const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o;
+  const void *ln2_g, *ln2_b, *w1, *b1, *w2, *b2;
+} mgt_layer_params;
+
+/* Parameter gradients (device pointers, fp32, same packed layouts). */
+typedef struct mgt_layer_grads {
+  void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o;
+  void *ln2_g, *ln2_b, *w1, *b1, *w2, *b2;
+} mgt_layer_grads;
+
+typedef struct mgt_layer mgt_layer; /* opaque handle, host memory only */
+
+/* Validate `cfg` and create a handle. Host only: makes no CUDA call. On error *out = NULL. */
+mgt_status mgt_layer_init(const mgt_layer_config* cfg, mgt_layer** out);
+
+/* Bytes the caller must provide for `saved` (fwd -> bwd activations) and `workspace`. */
+mgt_status mgt_layer_sizes(const mgt_layer* layer, size_t* saved_bytes, size_t* workspace_bytes);
+
+/* Where each intermediate lives, for inspection and tests. `region` is an mgt_region value;
+ * regions below 64 are offsets into `saved`, regions from 64 up are offsets into `workspace`.
+ * Element types: ACT = activation dtype, F32 = float. Shapes use T = b*s. */
+typedef enum mgt_region {
+  MGT_SAVED_LN1 = 0,        /* ACT [T, h]          LN1 output                          */
+  MGT_SAVED_LN1_MEAN = 1,   /* F32 [T]                                                 */
+  MGT_SAVED_LN1_RSTD = 2,   /* F32 [T]             1/sqrt(var + eps)                   */
+  MGT_SAVED_QKV = 3,        /* ACT [T][p][3][H/p][d]                                   */
+  MGT_SAVED_ATTN_O = 4,     /* ACT [T][p][H/p][d]  attention output (= [T, h])         */
+  MGT_SAVED_ATTN_LSE = 5,   /* F32 [b][H][s]       natural-log sum of exp of scores    */
+  MGT_SAVED_H1 = 6,         /* ACT [T, h]          first residual stream               */
+  MGT_SAVED_LN2 = 7,        /* ACT [T, h]                                              */
+  MGT_SAVED_LN2_MEAN = 8,   /* F32 [T]                                                 */
+  MGT_SAVED_LN2_RSTD = 9,   /* F32 [T]                                                 */
+  MGT_SAVED_FC1_U = 10,     /* ACT [T][p][f/p]     fc1 pre-activation                  */
+  MGT_SAVED_FC1_A = 11,     /* ACT [T][p][f/p]     GeLU(u)                             */
+  MGT_SAVED_COUNT = 12,
+  MGT_WS_STATUS = 64,       /* int32 device status word (first 256 bytes)              */
+  MGT_WS_DU = 65,           /* ACT [T, f]   dL/du                                      */
+  MGT_WS_DLN2 = 66,         /* ACT [T, h]   dL/d ln2 (shard contributions summed)      */
+  MGT_WS_DH1 = 67,          /* ACT [T, h]   dL/d h1                                    */
+  MGT_WS_DO = 68,           /* ACT [T, h]   dL/d attention output                      */
+  MGT_WS_DQKV = 69,         /* ACT [T, 3h]  dL/d qkv (packed like qkv)                 */
+  MGT_WS_DLN1 = 70,         /* ACT [T, h]   dL/d ln1                                   */
+  MGT_WS_ATTN_D = 71,       /* F32 [b][H][s] rowsum(dO * O)                            */
+  MGT_WS_DQ_ACC = 72,       /* F32 [T, h]   dQ accumulator of the attention backward   */
+  MGT_WS_LN_PARTIAL = 73,   /* F32 [blocks][2][h] per-block LayerNorm dgamma/dbeta     */
+  MGT_WS_COUNT = 74
+} mgt_region;
+mgt_status mgt_layer_region(const mgt_layer* layer, int region, size_t* offset, size_t* bytes);
+
+/* Forward. Reads x [b,s,h]; writes y [b,s,h] and every region of `saved`.
+ * Launch order on `stream`: LN1, QKV GEMM(+bias), attention, out-proj GEMM (+shard sum,
+ * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores u and a), fc2 GEMM (+shard sum, +b2, +h1). */
+mgt_status mgt_layer_fwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
+                         void* y, void* saved, void* workspace, void* stream);
+
+/* Backward. Reads x, saved (from the matching fwd) and dy; writes dx and every gradient in
+ * `grads` (fp32, overwritten). Uses `workspace` for intermediate gradients. */
+mgt_status mgt_layer_bwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
+                         const void* saved, const void* dy, void* dx, const mgt_layer_grads* grads,
+                         void* workspace, void* stream);
+
+/* Synchronise `stream`, read and clear the device status word in `workspace`.
+ * Returns MGT_OK, MGT_ETIMEOUT (a bounded wait gave up) or MGT_ECUDA. */
+mgt_status mgt_layer_get_error(mgt_layer* layer, void* workspace, void* stream);
+
+/* Per-kernel timing with CUDA events recorded around every launch of this handle
+ * (enable = 1 creates the events and needs a GPU; 0 stops recording). */
+typedef struct mgt_kernel_stat {
+  char name[32];     /* kernel family, e.g. "gemm_tc", "attn_fwd", "ln_fwd"         */
+  int64_t launches;  /* launches recorded                                          */
+  double ms;         /* summed device time of those launches                       */
+  double flops;      /* summed algorithmic FLOPs (dense contractions)              */
+  double bytes;      /* summed algorithmic HBM bytes (memory-bound kernels)        */
+} mgt_kernel_stat;
+mgt_status mgt_layer_profile(mgt_layer* layer, int enable);
+/* Synchronises the recorded events, folds them into per-family totals, copies up to `cap`
+ * entries to `out`, sets *n, and resets the totals. */
+mgt_status mgt_layer_profile_read(mgt_layer* layer, mgt_kernel_stat* out, int cap, int* n);
+
+void mgt_layer_destroy(mgt_layer* layer);
+const char* mgt_status_string(mgt_status s);
+
+/* Plain bf16 GEMM on the tensor-core path used inside the layer, exported for unit tests:
+ *   C[m, n] = sum_k A(m, k) * B(n, k),  C fp32 row-major with leading dimension ldc.
+ * A(m, k) = A[m*lda + k] if a_mn_major == 0, else A[k*lda + m]; likewise B(n, k) with
+ * b_mn_major. lda/ldb in elements, multiples of 8; pointers 16-byte aligned; M, N, K >= 1.
+ * `status` is an int32 device word (zeroed by the caller) that receives timeout codes. */
+mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major,
+                         int32_t b_mn_major, const void* A, int64_t lda, const void* B,
+                         int64_t ldb, float* C, int64_t ldc, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MGT_LAYER_H */

@@ -1,0 +1,203 @@
+"""Python binding of libmgt.so, the B200 (sm_100a) tensor-parallel GPT layer.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels behind the C ABI
+declared in include/mgt_layer.h. PyTorch is used for device memory and streams. There is no
+fallback: if the shared library is missing or fails to load, importing the binding's Layer raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+__all__ = ["Layer", "MgtError", "load_library", "gemm_bf16", "REGIONS", "PARAM_ORDER",
+           "lib_path"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG, "libmgt.so")
+
+PARAM_ORDER = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
+               "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
+
+REGIONS = {
+    "ln1": 0, "ln1_mean": 1, "ln1_rstd": 2, "qkv": 3, "attn_o": 4, "attn_lse": 5, "h1": 6,
+    "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_u": 10, "fc1_a": 11,
+    "status": 64, "du": 65, "dln2": 66, "dh1": 67, "dO": 68, "dqkv": 69, "dln1": 70,
+    "attn_D": 71, "dq_acc": 72, "ln_partial": 73,
+}
+
+STATUS = {0: "MGT_OK", 1: "MGT_EINVAL", 2: "MGT_EUNSUPPORTED", 3: "MGT_ECUDA",
+          4: "MGT_ETIMEOUT", 5: "MGT_ENOMEM"}
+
+
+class MgtError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("heads", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("seq", ctypes.c_int32), ("micro_batch", ctypes.c_int32),
+                ("tp_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("ln_eps", ctypes.c_float),
+                ("recompute_attn", ctypes.c_int32), ("gelu_tanh", ctypes.c_int32)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in PARAM_ORDER]
+
+
+class _KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("ms", ctypes.c_double), ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
+_LIB = None
+
+
+def load_library():
+    """Load libmgt.so (raises OSError if it is missing: there is no fallback)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(lib_path):
+        raise OSError("libmgt.so is not built (%s); run python -m "
+                      "tensor_transformer_layer_megatron_b200.build" % lib_path)
+    lib = ctypes.CDLL(lib_path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.mgt_layer_init.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(vp)]
+    lib.mgt_layer_sizes.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.mgt_layer_region.argtypes = [vp, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.mgt_layer_fwd.argtypes = [vp, ctypes.POINTER(_Params), vp, vp, vp, vp, vp]
+    lib.mgt_layer_bwd.argtypes = [vp, ctypes.POINTER(_Params), vp, vp, vp, vp,
+                                  ctypes.POINTER(_Params), vp, vp]
+    lib.mgt_layer_get_error.argtypes = [vp, vp, vp]
+    lib.mgt_layer_profile.argtypes = [vp, ctypes.c_int]
+    lib.mgt_layer_profile_read.argtypes = [vp, ctypes.POINTER(_KernelStat), ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int)]
+    lib.mgt_layer_destroy.argtypes = [vp]
+    lib.mgt_layer_destroy.restype = None
+    lib.mgt_status_string.argtypes = [ctypes.c_int]
+    lib.mgt_status_string.restype = ctypes.c_char_p
+    lib.mgt_gemm_bf16.argtypes = [i32, i32, i32, i32, i32, vp, ctypes.c_int64, vp,
+                                  ctypes.c_int64, vp, ctypes.c_int64, vp, vp]
+    for name in ("mgt_layer_init", "mgt_layer_sizes", "mgt_layer_region", "mgt_layer_fwd",
+                 "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
+                 "mgt_layer_profile_read", "mgt_gemm_bf16"):
+        getattr(lib, name).restype = ctypes.c_int
+    _LIB = lib
+    return lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise MgtError(code, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+class Layer:
+    """One tensor-parallel GPT layer (logical tp_size shards on one GPU).
+
+    dtype: "bf16" or "f32". Parameters are passed as a dict of device tensors in the packed
+    per-shard layouts of include/mgt_layer.h (see PARAM_ORDER)."""
+
+    def __init__(self, hidden, heads, ffn, seq, micro_batch, tp_size=1, dtype="bf16",
+                 ln_eps=1e-5, gelu_tanh=0, causal=1):
+        self.lib = load_library()
+        self.cfg = _Config(hidden, heads, ffn, seq, micro_batch, tp_size,
+                           1 if dtype == "bf16" else 0, causal, ln_eps, 1, gelu_tanh)
+        self.dtype = dtype
+        h = ctypes.c_void_p()
+        _check(self.lib.mgt_layer_init(ctypes.byref(self.cfg), ctypes.byref(h)), "mgt_layer_init")
+        self.handle = h
+
+    @classmethod
+    def from_config(cls, cfg):
+        """Build from any object with hidden, heads, ffn, seq, micro_batch, tp_size, dtype,
+        ln_eps, gelu_tanh attributes."""
+        return cls(cfg.hidden, cfg.heads, cfg.ffn, cfg.seq, cfg.micro_batch, cfg.tp_size,
+                   cfg.dtype, cfg.ln_eps, cfg.gelu_tanh)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            self.lib.mgt_layer_destroy(h)
+            self.handle = None
+
+    # ------------------------------------------------------------------ sizes / regions
+    def sizes(self):
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(self.lib.mgt_layer_sizes(self.handle, ctypes.byref(a), ctypes.byref(b)),
+               "mgt_layer_sizes")
+        return a.value, b.value
+
+    def region(self, name):
+        o, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(self.lib.mgt_layer_region(self.handle, REGIONS[name], ctypes.byref(o),
+                                         ctypes.byref(n)), "mgt_layer_region")
+        return o.value, n.value
+
+    def alloc_buffers(self, device="cuda"):
+        """Caller-owned `saved` and (zeroed) `workspace` byte buffers."""
+        import torch
+        s, w = self.sizes()
+        return (torch.empty(max(s, 256), dtype=torch.uint8, device=device),
+                torch.zeros(max(w, 256), dtype=torch.uint8, device=device))
+
+    def view(self, buf, name, dtype, shape):
+        """Typed view of one region of a saved/workspace buffer (for inspection and tests)."""
+        import math
+        o, n = self.region(name)
+        esz = buf.new_empty(0, dtype=dtype).element_size()
+        cnt = math.prod(shape)
+        assert cnt * esz == n, (name, cnt * esz, n)
+        return buf[o:o + n].view(dtype).view(*shape)
+
+    # ------------------------------------------------------------------ compute
+    @staticmethod
+    def _params(p: Dict) -> _Params:
+        return _Params(*[_ptr(p[n]) for n in PARAM_ORDER])
+
+    def fwd(self, params, x, y, saved, workspace, stream=None):
+        _check(self.lib.mgt_layer_fwd(self.handle, ctypes.byref(self._params(params)),
+                                      _ptr(x), _ptr(y), _ptr(saved), _ptr(workspace),
+                                      _stream_handle(stream)), "mgt_layer_fwd")
+
+    def bwd(self, params, x, saved, dy, dx, grads, workspace, stream=None):
+        _check(self.lib.mgt_layer_bwd(self.handle, ctypes.byref(self._params(params)),
+                                      _ptr(x), _ptr(saved), _ptr(dy), _ptr(dx),
+                                      ctypes.byref(self._params(grads)), _ptr(workspace),
+                                      _stream_handle(stream)), "mgt_layer_bwd")
+
+    def get_error(self, workspace, stream=None) -> int:
+        return self.lib.mgt_layer_get_error(self.handle, _ptr(workspace), _stream_handle(stream))
+
+    def profile(self, enable=True):
+        _check(self.lib.mgt_layer_profile(self.handle, 1 if enable else 0), "mgt_layer_profile")
+
+    def profile_read(self):
+        arr = (_KernelStat * 64)()
+        n = ctypes.c_int()
+        _check(self.lib.mgt_layer_profile_read(self.handle, arr, 64, ctypes.byref(n)),
+               "mgt_layer_profile_read")
+        return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms,
+                                           flops=arr[i].flops, bytes=arr[i].bytes)
+                for i in range(n.value)}
+
+
+def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):
+    """C[m, n] = sum_k A(m, k) B(n, k) on the tcgen05 path (see mgt_gemm_bf16)."""
+    lib = load_library()
+    _check(lib.mgt_gemm_bf16(M, N, K, a_mn, b_mn, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
+                             _ptr(status), _stream_handle(stream)), "mgt_gemm_bf16")

@@ -1,0 +1,491 @@
+// Tensor-core GEMM for sm_100a: TMA -> shared-memory ring -> tcgen05.mma (one issuing thread)
+// -> fp32 accumulators in tensor memory -> epilogue warps (tcgen05.ld) -> global memory.
+//
+// This one kernel serves every contraction of the layer:
+//   forward  QKV / fc1 (column-parallel): A = activations (K-major), B = packed weight rows
+//            (K-major); out-proj / fc2 (row-parallel): the K loop runs over the tp shards
+//            (K groups), so the shard partials are summed in the tensor-memory accumulator
+//            -- the on-device equivalent of the AllReduce after RowParallelLinear described
+//            on the trdm.cn page, section 2.1.
+//   backward dgrad: B = weight read N-major (no transpose copy); for row-parallel layers the
+//            N dimension is grouped by shard. wgrad: A = dY^T and B = X, both read MN-major
+//            along the token dimension; fp32 output written straight into the packed layout.
+//
+// CTA: 192 threads. warp 0 = TMA producer (one lane), warp 1 = TMEM owner + MMA issuer (one
+// lane), warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31). Persistent: grid =
+// min(#tiles, #SMs); tiles are taken round-robin. Accumulators are double-buffered in TMEM so
+// the epilogue of tile i overlaps the main loop of tile i+1.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "mgt_device.cuh"
+
+namespace mgt {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes = one 128B-swizzle row
+constexpr int kThreads = 192;
+constexpr int kChunkBytes = 64 * BK * 2;  // one [64 x 64] bf16 box = 8 KB
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+};
+
+struct TileCoord {
+  int ng, mb, nb;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n) {
+  TileCoord t;
+  const int per_group = num_m * num_n;
+  t.ng = tile / per_group;
+  const int r = tile - t.ng * per_group;
+  t.nb = r / num_m;  // m fastest: consecutive CTAs share the same weight (B) tile
+  t.mb = r - t.nb * num_m;
+  return t;
+}
+
+// ---------------------------------------------------------------------------- epilogue
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int col,
+                                               int count, float (&v)[32]) {
+  const long long off = (long long)(col / a.out_ng) * a.out_gs + (long long)row * a.ldc +
+                        (col % a.out_ng);
+  if constexpr (EPI == kEpiStoreF32) {
+    float* o = reinterpret_cast<float*>(a.out) + off;
+    if (count == 32) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+      for (int i = 0; i < count; ++i) o[i] = v[i];
+    }
+    return;
+  } else {
+    // bias / residual / aux come in the activation dtype (bf16)
+    const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+    if (EPI == kEpiBf16 || EPI == kEpiGelu) {
+      if (bias) {
+        if (count == 32) {
+          const uint4* bp = reinterpret_cast<const uint4*>(bias + col);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w = __ldg(bp + q);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              v[q * 8 + 2 * j] += bf16_lo(ww[j]);
+              v[q * 8 + 2 * j + 1] += bf16_hi(ww[j]);
+            }
+          }
+        } else {
+          for (int i = 0; i < count; ++i) v[i] += __bfloat162float(bias[col + i]);
+        }
+      }
+    }
+    if (EPI == kEpiBf16 && a.res) {
+      const __nv_bfloat16* r =
+          reinterpret_cast<const __nv_bfloat16*>(a.res) + (long long)row * a.ldr + col;
+      if (count == 32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4*>(r + q * 8);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[q * 8 + 2 * j] += bf16_lo(ww[j]);
+            v[q * 8 + 2 * j + 1] += bf16_hi(ww[j]);
+          }
+        }
+      } else {
+        for (int i = 0; i < count; ++i) v[i] += __bfloat162float(r[i]);
+      }
+    }
+    if (EPI == kEpiDGelu) {
+      const __nv_bfloat16* u =
+          reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col;
+      if (count == 32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4*>(u + q * 8);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[q * 8 + 2 * j] *= gelu_grad_f(bf16_lo(ww[j]), a.gelu_tanh);
+            v[q * 8 + 2 * j + 1] *= gelu_grad_f(bf16_hi(ww[j]), a.gelu_tanh);
+          }
+        }
+      } else {
+        for (int i = 0; i < count; ++i) v[i] *= gelu_grad_f(__bfloat162float(u[i]), a.gelu_tanh);
+      }
+    }
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + off;
+    if (EPI == kEpiGelu) {
+      __nv_bfloat16* o2 = reinterpret_cast<__nv_bfloat16*>(a.out2) + off;
+      if (count == 32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 wu, wa;
+          wu.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+          wu.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+          wu.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+          wu.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+          *reinterpret_cast<uint4*>(o2 + q * 8) = wu;
+          wa.x = pack_bf16x2(gelu_f(v[q * 8 + 0], a.gelu_tanh), gelu_f(v[q * 8 + 1], a.gelu_tanh));
+          wa.y = pack_bf16x2(gelu_f(v[q * 8 + 2], a.gelu_tanh), gelu_f(v[q * 8 + 3], a.gelu_tanh));
+          wa.z = pack_bf16x2(gelu_f(v[q * 8 + 4], a.gelu_tanh), gelu_f(v[q * 8 + 5], a.gelu_tanh));
+          wa.w = pack_bf16x2(gelu_f(v[q * 8 + 6], a.gelu_tanh), gelu_f(v[q * 8 + 7], a.gelu_tanh));
+          *reinterpret_cast<uint4*>(o + q * 8) = wa;
+        }
+      } else {
+        for (int i = 0; i < count; ++i) {
+          o2[i] = __float2bfloat16_rn(v[i]);
+          o[i] = __float2bfloat16_rn(gelu_f(v[i], a.gelu_tanh));
+        }
+      }
+      return;
+    }
+    if (count == 32) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+        *reinterpret_cast<uint4*>(o + q * 8) = w;
+      }
+    } else {
+      for (int i = 0; i < count; ++i) o[i] = __float2bfloat16_rn(v[i]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- kernel
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB, const GemmArgs args, int num_m,
+                   int num_n) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  // 128B-swizzled tiles need 1024-byte alignment in the shared window itself.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kt_per_group = (args.Kg + BK - 1) / BK;
+  const int k_iters = args.KG * kt_per_group;
+  const int num_tiles = args.NG * num_m * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (k_iters > 0 && warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileCoord tc = tile_coord(tile, num_m, num_n);
+      for (int kg = 0; kg < args.KG && ok; ++kg) {
+        for (int kt = 0; kt < kt_per_group; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, args.err, kErrTimeoutProducer, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          if constexpr (!A_MN) {
+            tma_load_3d(&tmA, &full[stage], a_dst, kt * BK, kg, tc.mb * BM);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_3d(&tmA, &full[stage], a_dst + c * kChunkBytes, tc.mb * BM + c * 64,
+                          kt * BK, 0);
+          }
+          if constexpr (!B_MN) {
+            tma_load_3d(&tmB, &full[stage], b_dst, kt * BK, tc.nb * BN, kg);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_3d(&tmB, &full[stage], b_dst + c * kChunkBytes, tc.nb * BN + c * 64,
+                          kt * BK, tc.ng);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+    {
+      // Let every load this thread issued land before the CTA can exit (after a timeout too).
+      // The slots issued most recently are the STAGES before the cursor; wait (bounded) for
+      // their phase. Slots never issued report their previous phase as complete.
+      for (int i = 1; i <= C::STAGES; ++i) {
+        int s = stage - i;
+        uint32_t ph = phase;
+        if (s < 0) {
+          s += C::STAGES;
+          ph ^= 1;
+        }
+        mbar_wait(&full[s], ph, args.err, kErrTimeoutDrain, nullptr);
+      }
+    }
+  } else if (k_iters > 0 && warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1, args.err, kErrTimeoutMma, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int it = 0; it < k_iters; ++it) {
+        if (!mbar_wait(&full[stage], phase, args.err, kErrTimeoutMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+        const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          // K-major: advance 16 elements (32 bytes) inside the 128-byte swizzle row.
+          // MN-major: advance 16 rows of 128 bytes; 64-wide MN chunks are kChunkBytes apart.
+          const uint64_t ad = A_MN ? smem_desc_sw128(a_addr + k * 2048, kChunkBytes, 1024)
+                                   : smem_desc_sw128(a_addr + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * 2048, kChunkBytes, 1024)
+                                   : smem_desc_sw128(b_addr + k * 32, 16, 1024);
+          tc_mma_f16(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[stage]);  // frees the slot once these MMAs have read it
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      tc_commit(&tfull[acc]);  // accumulator ready once all MMAs above complete
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    // Make sure no MMA is still writing tensor memory when the CTA frees it.
+    tc_commit(drain);
+    mbar_wait(drain, 0, args.err, kErrTimeoutDrain, nullptr);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const TileCoord tc = tile_coord(tile, num_m, num_n);
+      const int row = tc.mb * BM + ew * 32 + lane;
+      if (k_iters > 0) {
+        if (!mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue, abort_flag))
+          break;
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        if (k_iters > 0) {
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN + c * 32,
+                             v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        const int n0 = tc.nb * BN + c * 32;
+        if (row < args.M && n0 < args.Ng) {
+          const int count = min(32, args.Ng - n0);
+          epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, count, v);
+        }
+      }
+      if (k_iters > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map with 128-byte swizzle. dims/strides as in GemmArgs' comment;
+// stride values in elements (converted to bytes here).
+bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+              const uint32_t box[3]) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t gs[2] = {strides[0] * 2, strides[1] * 2};
+  cuuint32_t bd[3] = {box[0], box[1], box[2]};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gd, gs, bd,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+cudaError_t launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                        int num_sms, cudaStream_t stream) {
+  using C = Cfg<BN>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int num_m = (a.M + BM - 1) / BM;
+  const int num_n = (a.Ng + BN - 1) / BN;
+  const int tiles = a.NG * num_m * num_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, num_m, num_n);
+  return cudaGetLastError();
+}
+
+template <int BN, bool A_MN, bool B_MN>
+cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                       int num_sms, cudaStream_t s) {
+  switch (a.epi) {
+    case kEpiStoreF32: return launch_inst<BN, A_MN, B_MN, kEpiStoreF32>(ta, tb, a, num_sms, s);
+    case kEpiBf16: return launch_inst<BN, A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, s);
+    case kEpiGelu: return launch_inst<BN, A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, s);
+    case kEpiDGelu: return launch_inst<BN, A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                      int num_sms, cudaStream_t s) {
+  if (!a.a_mn && !a.b_mn) return launch_epi<BN, false, false>(ta, tb, a, num_sms, s);
+  if (!a.a_mn && a.b_mn) return launch_epi<BN, false, true>(ta, tb, a, num_sms, s);
+  if (a.a_mn && !a.b_mn) return launch_epi<BN, true, false>(ta, tb, a, num_sms, s);
+  return launch_epi<BN, true, true>(ta, tb, a, num_sms, s);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  // Shape rules of the tensor maps (checked by the callers too).
+  if (a.M <= 0 || a.Ng <= 0 || a.NG <= 0 || a.Kg <= 0 || a.KG <= 0) return cudaErrorInvalidValue;
+  if ((a.a_mn && a.KG != 1) || (a.b_mn && a.KG != 1) || (!a.b_mn && a.NG != 1))
+    return cudaErrorInvalidValue;
+  const int BN = (a.Ng <= 128) ? 128 : 256;
+  CUtensorMap ta, tb;
+  {
+    uint64_t dims[3], str[2];
+    uint32_t box[3];
+    if (!a.a_mn) {
+      dims[0] = a.Kg; dims[1] = a.KG; dims[2] = a.M;
+      str[0] = a.KG > 1 ? (uint64_t)a.Kg : (uint64_t)a.lda;
+      str[1] = a.lda;
+      box[0] = BK; box[1] = 1; box[2] = BM;
+    } else {
+      dims[0] = a.M; dims[1] = a.Kg; dims[2] = 1;
+      str[0] = a.lda; str[1] = a.lda;
+      box[0] = 64; box[1] = BK; box[2] = 1;
+    }
+    if (!make_map(&ta, a.A, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[3], str[2];
+    uint32_t box[3];
+    if (!a.b_mn) {
+      dims[0] = a.Kg; dims[1] = a.Ng; dims[2] = a.KG;
+      str[0] = a.ldb;
+      str[1] = a.KG > 1 ? (uint64_t)a.b_kgs : (uint64_t)a.ldb;
+      box[0] = BK; box[1] = BN; box[2] = 1;
+    } else {
+      dims[0] = a.Ng; dims[1] = a.Kg; dims[2] = a.NG;
+      str[0] = a.ldb;
+      str[1] = a.NG > 1 ? (uint64_t)a.b_ngs : (uint64_t)a.ldb;
+      box[0] = 64; box[1] = BK; box[2] = 1;
+    }
+    if (!make_map(&tb, a.B, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  if (BN == 128) return launch_bn<128>(ta, tb, a, num_sms, stream);
+  return launch_bn<256>(ta, tb, a, num_sms, stream);
+}
+
+}  // namespace mgt

@@ -1,0 +1,86 @@
+// Internal declarations shared by the kernel translation units and the C-ABI host code.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mgt {
+
+// Device status codes written into the caller's status word (first failure wins).
+enum DeviceError : int {
+  kErrNone = 0,
+  kErrTimeoutProducer = 0x100,  // TMA producer waited too long for a free stage
+  kErrTimeoutMma = 0x101,       // MMA issuer waited too long for data or a free accumulator
+  kErrTimeoutEpilogue = 0x102,  // epilogue waited too long for an accumulator
+  kErrTimeoutDrain = 0x103,     // unwinding after a timeout waited too long
+  kErrTimeoutAttn = 0x110,
+};
+
+// Epilogue applied to each fp32 accumulator tile of the GEMM.
+enum Epilogue : int {
+  kEpiStoreF32 = 0,  // out (fp32) = acc                     (weight gradients)
+  kEpiBf16 = 1,      // out (act) = acc [+ bias] [+ residual] (QKV, out-proj, fc2, dgrads)
+  kEpiGelu = 2,      // u = acc + bias -> out2; out = GeLU(u) (fc1)
+  kEpiDGelu = 3,     // out = acc * GeLU'(aux)                (fc2 dgrad -> du)
+};
+
+// One GEMM  C[m, col] = sum_{kg < KG} sum_{kk < Kg} A(m, kg, kk) * B(ng, n, kg, kk)
+// over tiles (ng < NG, m < M, n < Ng), col = ng*Ng + n. Operands are described by 3-D TMA
+// tensor maps built on the host (bf16 path) or by strides (fp32 SIMT path):
+//   A K-major : A[m*lda + kg*Kg + kk]              tensor map dims {Kg, KG, M}
+//   A M-major : A[(kg*Kg + kk)*lda + m]            tensor map dims {M, Kg*KG, 1}
+//   B K-major : B[kg*b_kgs + n*ldb + kk]           tensor map dims {Kg, Ng, KG}
+//   B N-major : B[ng*b_ngs + (kg*Kg + kk)*ldb + n] tensor map dims {Ng, Kg*KG, NG}
+// Output element (m, col) lives at out[(col / out_ng) * out_gs + m * ldc + col % out_ng].
+struct GemmArgs {
+  int M, Ng, NG, Kg, KG;
+  int a_mn, b_mn;                       // operand majorness (0 = K-major)
+  // SIMT path only (fp32): raw operand pointers and strides in elements.
+  const void* A; long long lda;
+  const void* B; long long ldb, b_kgs, b_ngs;
+  // Epilogue.
+  int epi;
+  void* out; long long ldc; int out_ng; long long out_gs;
+  void* out2;                           // kEpiGelu: pre-activation u (same addressing as out)
+  const void* bias;                     // indexed by col; nullable
+  const void* res; long long ldr;       // residual, res[m*ldr + col]; nullable
+  const void* aux; long long ld_aux;    // kEpiDGelu: u[m*ld_aux + col]
+  int gelu_tanh;
+  int* err;                             // device status word
+};
+
+// tcgen05 / TMA GEMM for bf16 operands (fp32 accumulate in tensor memory).
+// Builds the tensor maps from the pointers in `args` (A, B, strides) and launches a persistent
+// kernel with one CTA per SM. Returns a CUDA error code.
+cudaError_t launch_gemm_tc(const GemmArgs& args, int num_sms, cudaStream_t stream);
+// Plain FFMA GEMM with the same semantics for fp32 operands.
+cudaError_t launch_gemm_simt_f32(const GemmArgs& args, cudaStream_t stream);
+
+// LayerNorm over the last dimension. dtype: 0 fp32, 1 bf16 (x, y); stats and params fp32.
+cudaError_t launch_ln_fwd(int dtype, long long rows, int h, float eps, const void* x,
+                          const float* gamma, const float* beta, void* y, float* mean,
+                          float* rstd, cudaStream_t stream);
+// dx = dres + LN'^T(dy); per-block partial dgamma/dbeta into `partial` [nblk][2][h], then a
+// second kernel reduces them into dgamma/dbeta. Returns the number of blocks used in *nblk.
+int ln_bwd_blocks(long long rows, int num_sms);
+cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, const void* dres,
+                          const void* x, const float* gamma, const float* mean,
+                          const float* rstd, void* dx, float* partial, int nblk,
+                          float* dgamma, float* dbeta, cudaStream_t stream);
+
+// Column sums of a [rows, cols] activation matrix into fp32 (bias gradients).
+cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
+                          cudaStream_t stream);
+
+// Causal attention over packed qkv [T][p][3][H/p][d]; O [T][p][H/p][d]; lse [b][H][s].
+struct AttnArgs {
+  int b, s, H, d, p;
+  const void* qkv; void* o; float* lse;
+  const void* dO; float* Dsum; float* dq_acc; void* dqkv;
+  int* err;
+};
+cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t stream);
+int attn_bwd_kernel_count(int dtype);
+
+}  // namespace mgt

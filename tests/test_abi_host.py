@@ -1,0 +1,104 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every function that
+include/mgt_layer.h declares, validates configurations synchronously, and lays out its buffers
+consistently."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tensor_transformer_layer_megatron_b200 as mgt
+from mgt_inputs import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mgt_layer.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mgt_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = mgt.load_library()
+    names = declared_functions()
+    assert "mgt_layer_fwd" in names and "mgt_layer_bwd" in names and "mgt_layer_init" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _init(**kw):
+    base = dict(hidden=64, heads=4, ffn=256, seq=32, micro_batch=2, tp_size=2, dtype=0,
+                causal=1, ln_eps=1e-5, recompute_attn=1, gelu_tanh=0)
+    base.update(kw)
+    lib = mgt.load_library()
+    cfg = mgt._Config(*[base[f] for f, _ in mgt._Config._fields_])
+    h = ctypes.c_void_p()
+    st = lib.mgt_layer_init(ctypes.byref(cfg), ctypes.byref(h))
+    if st == 0:
+        lib.mgt_layer_destroy(h)
+    else:
+        assert not h.value
+    return st
+
+
+def test_golden_tp_divisibility():
+    path = os.path.join(ROOT, "tests", "golden", "tp_divisibility.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert rows
+    for hidden, heads, tp, expect, per_shard in rows:
+        st = _init(hidden=int(hidden), heads=int(heads), ffn=4 * int(hidden), seq=16,
+                   micro_batch=1, tp_size=int(tp), dtype=1)
+        assert mgt.STATUS[st] == "MGT_" + expect, (hidden, tp)
+        if expect == "OK":
+            assert int(hidden) // int(tp) == int(per_shard)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hidden=0), 1), (dict(seq=-1), 1), (dict(heads=3), 1),       # h % H
+    (dict(tp_size=3), 1),                                              # h % p
+    (dict(heads=8, tp_size=16, hidden=128), 1),                        # H % p
+    (dict(ffn=255), 1),                                                # f % p
+    (dict(causal=0), 2), (dict(dtype=7), 2),
+    (dict(dtype=1), 2),                   # bf16 needs head_dim 64/128 (here 16)
+    (dict(dtype=1, hidden=128, heads=2, tp_size=2, ffn=200), 2),      # f/p = 100, not a multiple of 64
+    (dict(hidden=512, heads=4), 2),       # fp32 head_dim 128 > 64
+])
+def test_init_rejects(kw, code):
+    assert _init(**kw) == code
+
+
+def test_init_accepts_every_workload():
+    for c in CONFIGS:
+        assert _init(hidden=c.hidden, heads=c.heads, ffn=c.ffn, seq=c.seq,
+                     micro_batch=c.micro_batch, tp_size=c.tp_size,
+                     dtype=1 if c.dtype == "bf16" else 0) == 0, c.name
+
+
+def test_null_handle_and_status_strings():
+    lib = mgt.load_library()
+    assert lib.mgt_layer_sizes(None, None, None) == 1
+    assert lib.mgt_layer_fwd(None, None, None, None, None, None, None) == 1
+    assert lib.mgt_status_string(4) == b"device wait timed out"
+
+
+@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: c.name)
+def test_region_layout(cfg):
+    L = mgt.Layer.from_config(cfg)
+    saved, ws = L.sizes()
+    T, h, f, e = cfg.tokens, cfg.hidden, cfg.ffn, 2 if cfg.dtype == "bf16" else 4
+    expect = {"ln1": T * h * e, "qkv": 3 * T * h * e, "attn_o": T * h * e,
+              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_u": T * f * e,
+              "fc1_a": T * f * e, "du": T * f * e, "dqkv": 3 * T * h * e}
+    spans = []
+    for name, rid in mgt.REGIONS.items():
+        o, n = L.region(name)
+        assert o % 256 == 0
+        if name in expect:
+            assert n == expect[name], name
+        spans.append((rid >= 64, o, o + n))
+        assert o + n <= (ws if rid >= 64 else saved)
+    for buf in (False, True):
+        s = sorted((a, b) for k, a, b in spans if k == buf)
+        for (a0, b0), (a1, b1) in zip(s, s[1:]):
+            assert b0 <= a1  # regions never overlap

@@ -1,0 +1,43 @@
+"""Layer parity of the CUDA path against the fp64 oracle, through the C ABI, on seeded inputs:
+small layers spanning several tiles with ragged tails (tokens, sequence, ffn per shard),
+tp_size 1/2/4, head_dim 64/128, both GeLU forms, and the fp32 correctness layer."""
+import pytest
+
+from mgt_inputs import LayerConfig, config_by_name
+from parity import full_parity, tol
+
+pytestmark = pytest.mark.gpu
+
+
+def small(name, **kw):
+    base = dict(name=name, dtype="bf16", seed=hash(name) % 10000)
+    base.update(kw)
+    return LayerConfig(**base)
+
+
+SMALL = [
+    small("h128-d64-p2-s80-b2", hidden=128, heads=2, ffn=256, seq=80, micro_batch=2, tp_size=2),
+    small("h256-d128-p2-s200", hidden=256, heads=2, ffn=512, seq=200, micro_batch=1, tp_size=2),
+    small("h512-d128-p4-s130-b3", hidden=512, heads=4, ffn=1536, seq=130, micro_batch=3,
+          tp_size=4),
+    small("h256-d64-p1-s64", hidden=256, heads=4, ffn=768, seq=64, micro_batch=1, tp_size=1),
+    small("h256-d128-p2-f640", hidden=256, heads=2, ffn=640, seq=96, micro_batch=2, tp_size=2),
+    small("h256-d64-p2-tanh", hidden=256, heads=4, ffn=512, seq=33, micro_batch=2, tp_size=2,
+          gelu_tanh=1),
+    small("h128-d64-p1-s1", hidden=128, heads=2, ffn=256, seq=1, micro_batch=4, tp_size=1),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_layer_bf16_small(cfg):
+    errs = full_parity(cfg)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("affine", [False, True])
+def test_layer_f32_tiny(affine):
+    cfg = config_by_name("tiny-h64-tp2-f32")
+    errs = full_parity(cfg, nonzero_affine=affine)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
