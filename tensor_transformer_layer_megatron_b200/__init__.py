@@ -169,12 +169,27 @@ class Layer:
     def _params(p: Dict) -> _Params:
         return _Params(*[_ptr(p[n]) for n in PARAM_ORDER])
 
+    def _check_types(self, params, acts, grads=None):
+        import torch
+        act = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        for n in PARAM_ORDER:
+            want = torch.float32 if n.startswith("ln") else act
+            if params[n].dtype != want:
+                raise TypeError("parameter %s must be %s" % (n, want))
+            if grads is not None and grads[n].dtype != torch.float32:
+                raise TypeError("gradient %s must be float32" % n)
+        for t in acts:
+            if t.dtype != act:
+                raise TypeError("activations must be %s" % act)
+
     def fwd(self, params, x, y, saved, workspace, stream=None):
+        self._check_types(params, (x, y))
         _check(self.lib.mgt_layer_fwd(self.handle, ctypes.byref(self._params(params)),
                                       _ptr(x), _ptr(y), _ptr(saved), _ptr(workspace),
                                       _stream_handle(stream)), "mgt_layer_fwd")
 
     def bwd(self, params, x, saved, dy, dx, grads, workspace, stream=None):
+        self._check_types(params, (x, dy, dx), grads)
         _check(self.lib.mgt_layer_bwd(self.handle, ctypes.byref(self._params(params)),
                                       _ptr(x), _ptr(saved), _ptr(dy), _ptr(dx),
                                       ctypes.byref(self._params(grads)), _ptr(workspace),
@@ -198,6 +213,10 @@ class Layer:
 
 def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):
     """C[m, n] = sum_k A(m, k) B(n, k) on the tcgen05 path (see mgt_gemm_bf16)."""
+    import torch
+    if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16 or C.dtype != torch.float32:
+        raise TypeError("gemm_bf16 takes bf16 A, B and an fp32 C")
     lib = load_library()
     _check(lib.mgt_gemm_bf16(M, N, K, a_mn, b_mn, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
                              _ptr(status), _stream_handle(stream)), "mgt_gemm_bf16")
+

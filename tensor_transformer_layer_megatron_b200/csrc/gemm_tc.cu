@@ -332,8 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileCoord tc = tile_coord(tile, num_m, num_n);
       const int row = tc.mb * BM + ew * 32 + lane;
       if (k_iters > 0) {
-        if (!mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue, abort_flag))
-          break;
+        const bool ok = mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue,
+                                  abort_flag);
+        // Lanes leave the polling loop independently; tcgen05.ld is .sync.aligned and needs
+        // the whole warp converged, and the exit decision must be warp-uniform.
+        if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
       }
 #pragma unroll 1

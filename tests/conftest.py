@@ -16,3 +16,14 @@ def pytest_configure(config):
 def has_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+@pytest.fixture(autouse=True)
+def _default_dtype_guard():
+    """Tests must not leak a changed torch default dtype into later tests (buffers handed to
+    the C ABI are typed explicitly, but a float64 default once turned an fp32 output buffer
+    into a float64 one)."""
+    import torch
+    before = torch.get_default_dtype()
+    yield
+    torch.set_default_dtype(before)

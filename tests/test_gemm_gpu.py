@@ -38,7 +38,7 @@ def test_gemm_bf16(M, N, K, a_mn, b_mn):
         Bs = torch.zeros(N, ldb, dtype=torch.bfloat16); Bs[:, :K] = B
     ldc = (N + 3) // 4 * 4
     dA, dB = As.cuda(), Bs.cuda()
-    C = torch.full((M, ldc), float("nan"), device="cuda")
+    C = torch.full((M, ldc), float("nan"), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     mgt.gemm_bf16(dA, dB, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status)
     torch.cuda.synchronize()

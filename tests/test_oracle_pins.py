@@ -12,7 +12,6 @@ import torch.nn.functional as F
 import oracle
 from mgt_inputs import LayerConfig, make_inputs, pack_params, unpack_params
 
-torch.set_default_dtype(torch.float64)
 
 
 def tiny(p=2, **kw):
