@@ -183,6 +183,25 @@ mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major,
                          int32_t b_mn_major, const void* A, int64_t lda, const void* B,
                          int64_t ldb, float* C, int64_t ldc, int32_t* status, void* stream);
 
+/* LayerNorm backward that allocates nothing -- the pages have no counterpart; it exists for
+ * callers that cannot call cudaMalloc where they run the backward (frameworks that own all
+ * device memory through their own pool allocator, hot loops where an allocation would
+ * synchronise the device). Computes, for `rows` rows of width h,
+ *   dx = dres + rstd * (g - mean(g) - xhat * mean(g * xhat)),  g = dy * gamma,
+ *   dgamma = sum_rows dy * xhat,  dbeta = sum_rows dy,  xhat = (x - mean) * rstd,
+ * i.e. the LayerNorm backward of mgt_layer_bwd. dtype: MGT_BF16 (dy, dres, x, dx bf16) or
+ * MGT_F32; gamma, mean, rstd, dgamma, dbeta fp32. dres may be NULL. h must be a multiple of 8
+ * (bf16) or 4 (f32) and at most 16384 (bf16) / 8192 (f32), else MGT_EUNSUPPORTED.
+ * Its per-block partial sums live in a fixed 4 MiB array of the library's own device memory,
+ * held on every GPU that loads the library until the process exits. The first call on each
+ * device looks up that array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture. All calls share the array: calls that overlap on the GPU (other
+ * streams, other threads) race on it, so serialise them. Allocates no memory. */
+mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int32_t h, const void* dy,
+                                     const void* dres, const void* x, const float* gamma,
+                                     const float* mean, const float* rstd, void* dx,
+                                     float* dgamma, float* dbeta, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

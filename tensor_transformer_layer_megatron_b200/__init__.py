@@ -10,8 +10,8 @@ import ctypes
 import os
 from typing import Dict, Optional
 
-__all__ = ["Layer", "MgtError", "load_library", "gemm_bf16", "REGIONS", "PARAM_ORDER",
-           "lib_path"]
+__all__ = ["Layer", "MgtError", "load_library", "gemm_bf16", "layernorm_bwd_noalloc", "REGIONS",
+           "PARAM_ORDER", "lib_path"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_PKG, "libmgt.so")
@@ -82,9 +82,11 @@ def load_library():
     lib.mgt_status_string.restype = ctypes.c_char_p
     lib.mgt_gemm_bf16.argtypes = [i32, i32, i32, i32, i32, vp, ctypes.c_int64, vp,
                                   ctypes.c_int64, vp, ctypes.c_int64, vp, vp]
+    lib.mgt_layernorm_bwd_noalloc.argtypes = [i32, ctypes.c_int64, i32, vp, vp, vp, vp, vp, vp,
+                                              vp, vp, vp, vp]
     for name in ("mgt_layer_init", "mgt_layer_sizes", "mgt_layer_region", "mgt_layer_fwd",
                  "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
-                 "mgt_layer_profile_read", "mgt_gemm_bf16"):
+                 "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -220,3 +222,21 @@ def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):
     _check(lib.mgt_gemm_bf16(M, N, K, a_mn, b_mn, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
                              _ptr(status), _stream_handle(stream)), "mgt_gemm_bf16")
 
+
+def layernorm_bwd_noalloc(dtype, rows, h, dy, dres, x, gamma, mean, rstd, dx, dgamma, dbeta,
+                          stream=None):
+    """LayerNorm backward with library-owned scratch (see mgt_layernorm_bwd_noalloc): for
+    callers that cannot allocate device memory. dtype: "bf16" or "f32"."""
+    import torch
+    act = torch.bfloat16 if dtype == "bf16" else torch.float32
+    for t in (dy, dres, x, dx):
+        if t is not None and t.dtype != act:
+            raise TypeError("dy, dres, x, dx must be %s" % act)
+    for t in (gamma, mean, rstd, dgamma, dbeta):
+        if t.dtype != torch.float32:
+            raise TypeError("gamma, mean, rstd, dgamma, dbeta must be float32")
+    lib = load_library()
+    _check(lib.mgt_layernorm_bwd_noalloc(1 if dtype == "bf16" else 0, rows, h, _ptr(dy),
+                                         _ptr(dres), _ptr(x), _ptr(gamma), _ptr(mean),
+                                         _ptr(rstd), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
+                                         _stream_handle(stream)), "mgt_layernorm_bwd_noalloc")
