@@ -375,6 +375,219 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------- CTA-pair kernel
+// Same contract as gemm_tc_kernel, but a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256): CTA r of the pair loads rows
+// [m0 + 128 r, +128) of A and the half [n0 + 128 r, +128) of B into its own shared memory, and
+// the pair's leader issues one MMA that reads both CTAs' halves and writes each CTA's 128
+// accumulator rows into that CTA's tensor memory. Each CTA moves 32 KB per 64-deep k-step
+// instead of 48 KB for the same MMA work per SM, which is what keeps the shared-memory port
+// below its limit at full tensor throughput.
+//
+// Synchronisation: both CTAs' TMA loads complete on the leader's `full` barrier (the leader
+// posts the expected bytes of both); the leader's tcgen05.commit multicasts to `empty` and
+// `tfull` in both CTAs; both CTAs' epilogue warps arrive on the leader's `tempty` (count 8).
+// A cluster barrier after initialisation and another before exit bracket all cross-CTA
+// traffic; every wait in between is bounded.
+constexpr int kPairStages = 6;
+constexpr int kPairAB = BM * BK * 2;            // 16 KB: this CTA's A rows or B half
+constexpr int kPairStageBytes = 2 * kPairAB;    // 32 KB per CTA per stage
+constexpr int kPairSmem = kPairStages * kPairStageBytes + 256 + 1024;
+
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args, int num_m2,
+                    int num_n) {
+  constexpr int BN = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairAB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kPairStages;
+  uint64_t* tfull = bars + 2 * kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int kt_per_group = (args.Kg + BK - 1) / BK;
+  const int k_iters = args.KG * kt_per_group;
+  const int num_tiles = args.NG * num_m2 * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrive or load
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      const TileCoord tc = tile_coord(tile, num_m2, num_n);
+      const int m0 = tc.mb * 256 + rank * 128;
+      const int n0 = tc.nb * BN + rank * 128;
+      for (int kg = 0; kg < args.KG && ok; ++kg) {
+        for (int kt = 0; kt < kt_per_group; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, args.err, kErrTimeoutProducer, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          uint8_t* a_dst = sA + stage * kPairAB;
+          uint8_t* b_dst = sB + stage * kPairAB;
+          if constexpr (!A_MN) {
+            tma_load_3d_pair(&tmA, fb, a_dst, kt * BK, kg, m0);
+          } else {
+            tma_load_3d_pair(&tmA, fb, a_dst, m0, kt * BK, 0);
+            tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, kt * BK, 0);
+          }
+          if constexpr (!B_MN) {
+            tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, n0, kg);
+          } else {
+            tma_load_3d_pair(&tmB, fb, b_dst, n0, kt * BK, tc.ng);
+            tma_load_3d_pair(&tmB, fb, b_dst + kChunkBytes, n0 + 64, kt * BK, tc.ng);
+          }
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+    // Loads of this CTA complete on the leader's barrier, so only the leader can see them
+    // land; the peer relies on the end-of-kernel cluster barrier, which the leader reaches
+    // only after its MMA issuer consumed (or gave up on) every stage.
+    if (leader) {
+      for (int i = 1; i <= kPairStages; ++i) {
+        int s = stage - i;
+        uint32_t ph = phase;
+        if (s < 0) {
+          s += kPairStages;
+          ph ^= 1;
+        }
+        mbar_wait(&full[s], ph, args.err, kErrTimeoutDrain, nullptr);
+      }
+    }
+  } else if (leader && warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    constexpr uint32_t idesc = idesc_bf16_f32(256, BN, A_MN, B_MN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1, args.err, kErrTimeoutMma, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int it = 0; it < k_iters; ++it) {
+        if (!mbar_wait(&full[stage], phase, args.err, kErrTimeoutMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sA + stage * kPairAB);
+        const uint32_t b_addr = smem_u32(sB + stage * kPairAB);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(a_addr + k * 2048, kChunkBytes, 1024)
+                                   : smem_desc_sw128(a_addr + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * 2048, kChunkBytes, 1024)
+                                   : smem_desc_sw128(b_addr + k * 32, 16, 1024);
+          tc_mma_f16_pair(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit_pair_mc(&empty[stage], 0x3);  // frees the slot in both CTAs
+        if (++stage == kPairStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      tc_commit_pair_mc(&tfull[acc], 0x3);  // both CTAs' accumulator rows are ready
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    tc_commit_pair(drain);
+    mbar_wait(drain, 0, args.err, kErrTimeoutDrain, nullptr);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const TileCoord tc = tile_coord(tile, num_m2, num_n);
+      const int row = tc.mb * 256 + rank * 128 + ew * 32 + lane;
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue,
+                                abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN + c * 32,
+                           v);
+        const int n0 = tc.nb * BN + c * 32;
+        if (row < args.M && n0 < args.Ng) {
+          const int count = min(32, args.Ng - n0);
+          epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, count, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its barriers or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 // ---------------------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -438,6 +651,45 @@ cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
   return cudaErrorInvalidValue;
 }
 
+template <bool A_MN, bool B_MN, int EPI>
+cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                             int num_sms, cudaStream_t stream) {
+  auto kern = gemm_tc2_kernel<A_MN, B_MN, EPI>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int num_m2 = (a.M + 255) / 256;
+  const int num_n = (a.Ng + 255) / 256;
+  const int tiles = a.NG * num_m2 * num_n;
+  const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  kern<<<2 * pairs, kThreads, kPairSmem, stream>>>(ta, tb, a, num_m2, num_n);
+  return cudaGetLastError();
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t launch_pair_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                            int num_sms, cudaStream_t s) {
+  switch (a.epi) {
+    case kEpiStoreF32: return launch_pair_inst<A_MN, B_MN, kEpiStoreF32>(ta, tb, a, num_sms, s);
+    case kEpiBf16: return launch_pair_inst<A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, s);
+    case kEpiGelu: return launch_pair_inst<A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, s);
+    case kEpiDGelu: return launch_pair_inst<A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                        int num_sms, cudaStream_t s) {
+  if (!a.a_mn && !a.b_mn) return launch_pair_epi<false, false>(ta, tb, a, num_sms, s);
+  if (!a.a_mn && a.b_mn) return launch_pair_epi<false, true>(ta, tb, a, num_sms, s);
+  if (a.a_mn && !a.b_mn) return launch_pair_epi<true, false>(ta, tb, a, num_sms, s);
+  return launch_pair_epi<true, true>(ta, tb, a, num_sms, s);
+}
+
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                       int num_sms, cudaStream_t s) {
@@ -454,7 +706,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
   if (a.M <= 0 || a.Ng <= 0 || a.NG <= 0 || a.Kg <= 0 || a.KG <= 0) return cudaErrorInvalidValue;
   if ((a.a_mn && a.KG != 1) || (a.b_mn && a.KG != 1) || (!a.b_mn && a.NG != 1))
     return cudaErrorInvalidValue;
+  // Wide tiles run on CTA pairs (cta_group::2, 256 x 256 per pair); narrow N on one CTA.
+  const bool pair = a.Ng > 128 && num_sms >= 2;
   const int BN = (a.Ng <= 128) ? 128 : 256;
+  const int b_rows = pair ? 128 : BN;  // B rows per CTA per k-step
   CUtensorMap ta, tb;
   {
     uint64_t dims[3], str[2];
@@ -478,7 +733,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
       dims[0] = a.Kg; dims[1] = a.Ng; dims[2] = a.KG;
       str[0] = a.ldb;
       str[1] = a.KG > 1 ? (uint64_t)a.b_kgs : (uint64_t)a.ldb;
-      box[0] = BK; box[1] = BN; box[2] = 1;
+      box[0] = BK; box[1] = b_rows; box[2] = 1;
     } else {
       dims[0] = a.Ng; dims[1] = a.Kg; dims[2] = a.NG;
       str[0] = a.ldb;
@@ -487,6 +742,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
     }
     if (!make_map(&tb, a.B, dims, str, box)) return cudaErrorInvalidValue;
   }
+  if (pair) return launch_pair(ta, tb, a, num_sms, stream);
   if (BN == 128) return launch_bn<128>(ta, tb, a, num_sms, stream);
   return launch_bn<256>(ta, tb, a, num_sms, stream);
 }
