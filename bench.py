@@ -194,8 +194,16 @@ def run_mgt(args):
     h2d = (x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size())
     d2h = (y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size())
 
-    # ---- roofline of the dominant kernel family (the tcgen05 GEMM)
+    # ---- roofline of the dominant kernel family (the tcgen05 GEMM, all call sites together)
     peaks, peak_src = load_peaks()
+    sites = {k: v for k, v in prof.items() if "/" in k}
+    families = {}
+    for k, v in prof.items():
+        f = families.setdefault(k.split("/")[0], {"launches": 0, "ms": 0.0, "flops": 0.0,
+                                                   "bytes": 0.0})
+        for q in f:
+            f[q] += v[q]
+    prof = families
     fam = max(prof.items(), key=lambda kv: kv[1]["ms"]) if prof else (None, None)
     roof = None
     if fam[0] is not None:
@@ -221,6 +229,9 @@ def run_mgt(args):
                    **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)}
                       if v["bytes"] else {})}
                for k, v in prof.items()}
+    gemm_sites = {k.split("/")[1]: {"ms_per_step": round(v["ms"] / args.steps, 4),
+                                    "tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)}
+                  for k, v in sites.items()}
     launches = sum(v["launches"] * KERNELS_PER_LAUNCH.get(k, 1) for k, v in prof.items())
 
     cpu = None
@@ -250,6 +261,7 @@ def run_mgt(args):
                     "what": "x, dy pinned host -> device; fwd+bwd via the C ABI; y, dx -> host"},
             "roofline": roof,
             "kernels": kernels,
+            "gemm_sites": gemm_sites,
             "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,

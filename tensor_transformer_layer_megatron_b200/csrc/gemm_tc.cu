@@ -11,8 +11,9 @@
 //            N dimension is grouped by shard. wgrad: A = dY^T and B = X, both read MN-major
 //            along the token dimension; fp32 output written straight into the packed layout.
 //
-// CTA: 192 threads. warp 0 = TMA producer (one lane), warp 1 = TMEM owner + MMA issuer (one
-// lane), warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31). Persistent: grid =
+// CTA: 320 threads. warp 0 = TMA producer (one lane), warp 1 = TMEM owner + MMA issuer (one
+// lane), warps 2..9 = epilogue: warp w reads TMEM lanes 32*(w%4)..+31, and the two warps of
+// each lane quarter split the tile's columns, so the epilogue keeps pace with the MMAs. Persistent: grid =
 // min(#tiles, #SMs); tiles are taken round-robin. Accumulators are double-buffered in TMEM so
 // the epilogue of tile i overlaps the main loop of tile i+1.
 #include <cudaTypedefs.h>
@@ -26,7 +27,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one 128B-swizzle row
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 2 producer/MMA warps + 8 epilogue warps
+constexpr int kEpiWarps = 8;
 constexpr int kChunkBytes = 64 * BK * 2;  // one [64 x 64] bf16 box = 8 KB
 
 template <int BN>
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -326,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp & 3;  // TMEM lane quarter this warp may access
+    const int c_begin = ((warp - 2) >> 2) * (BN / 64);  // this warp's half of the columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = c_begin; c < c_begin + BN / 64; ++c) {
         float v[32];
         if (k_iters > 0) {
           tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN + c * 32,
@@ -429,7 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&tempty[b], 2 * kEpiWarps);  // epilogue warps of both CTAs of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -548,6 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp & 3;
+    const int c_begin = ((warp - 2) >> 2) * (BN / 64);
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -559,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = c_begin; c < c_begin + BN / 64; ++c) {
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN + c * 32,
                            v);

@@ -152,10 +152,11 @@ GemmArgs gemm_base(int M, int Ng, int NG, int Kg, int KG) {
   return a;
 }
 
-cudaError_t gemm(mgt_layer* L, const GemmArgs& a, cudaStream_t s) {
+// `site` names the call ("gemm_tc/fc1_fwd", ...): profiling groups launches by this name.
+cudaError_t gemm(mgt_layer* L, const char* site, const GemmArgs& a, cudaStream_t s) {
   const double flops = 2.0 * a.M * (double)a.Ng * a.NG * (double)a.Kg * a.KG;
   if (L->cfg.dtype == MGT_BF16)
-    return run(L, "gemm_tc", flops, 0, s, [&] { return launch_gemm_tc(a, L->num_sms, s); });
+    return run(L, site, flops, 0, s, [&] { return launch_gemm_tc(a, L->num_sms, s); });
   return run(L, "gemm_simt", flops, 0, s, [&] { return launch_gemm_simt_f32(a, s); });
 }
 
@@ -284,7 +285,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, 3 * h, 1, h, 1);
     a.A = ln1; a.lda = h; a.B = P->w_qkv; a.ldb = h;
     a.epi = kEpiBf16; a.out = qkv; a.ldc = 3 * h; a.bias = P->b_qkv; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/qkv_fwd", a, s));
   }
   // 3. causal attention per head (each shard's heads are local)
   {
@@ -299,7 +300,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, h / p, p);
     a.A = O; a.lda = h; a.B = P->w_o; a.ldb = h / p; a.b_kgs = (long long)h * (h / p);
     a.epi = kEpiBf16; a.out = h1; a.ldc = h; a.bias = P->b_o; a.res = x; a.ldr = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/outproj_fwd", a, s));
   }
   // 5. LN2
   MGT_TRY(run(L, "ln_fwd", 0, ln_bytes, s, [&] {
@@ -312,14 +313,14 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
     a.epi = kEpiGelu; a.out = act; a.out2 = u; a.ldc = f; a.bias = P->b1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   }
   // 7. fc2, row-parallel with shard sum, + b2, + residual h1
   {
     GemmArgs a = gemm_base(T, h, 1, f / p, p);
     a.A = act; a.lda = f; a.B = P->w2; a.ldb = f / p; a.b_kgs = (long long)h * (f / p);
     a.epi = kEpiBf16; a.out = y; a.ldc = h; a.bias = P->b2; a.res = h1; a.ldr = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc2_fwd", a, s));
   }
   return MGT_OK;
 }
@@ -379,14 +380,14 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.b_ngs = (long long)h * (f / p);
     a.epi = kEpiDGelu; a.out = du; a.ldc = f; a.aux = u; a.ld_aux = f;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc2_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(h, f, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dy; a.lda = h; a.B = act; a.ldb = f;
     a.epi = kEpiStoreF32; a.out = G->w2; a.ldc = f / p; a.out_ng = f / p;
     a.out_gs = (long long)h * (f / p); a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, s));
   }
   // B3. fc1: db1, dgrad (sum over shards = K loop over f), wgrad
   MGT_TRY(colsum(du, f, G->b1));
@@ -394,13 +395,13 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, f, 1);
     a.b_mn = 1; a.A = du; a.lda = f; a.B = P->w1; a.ldb = h;
     a.epi = kEpiBf16; a.out = dln2; a.ldc = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc1_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(f, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f; a.B = ln2; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, s));
   }
   // B4. LN2 backward + residual gradient dy -> dh1
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
@@ -414,14 +415,14 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.b_mn = 1; a.A = dh1; a.lda = h; a.B = P->w_o; a.ldb = h / p;
     a.b_ngs = (long long)h * (h / p);
     a.epi = kEpiBf16; a.out = dO; a.ldc = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/outproj_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dh1; a.lda = h; a.B = O; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w_o; a.ldc = h / p; a.out_ng = h / p;
     a.out_gs = (long long)h * (h / p); a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/outproj_wgrad", a, s));
   }
   // B6. attention backward (probabilities recomputed from the saved log-sum-exp)
   {
@@ -436,13 +437,13 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, 3 * h, 1);
     a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = P->w_qkv; a.ldb = h;
     a.epi = kEpiBf16; a.out = dln1; a.ldc = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/qkv_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(3 * h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = ln1; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err;
-    MGT_TRY(gemm(L, a, s));
+    MGT_TRY(gemm(L, "gemm_tc/qkv_wgrad", a, s));
   }
   // B8. LN1 backward + residual gradient dh1 -> dx
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {

@@ -48,53 +48,64 @@ struct Vec<float> {
   }
 };
 
-template <int NT>
-__device__ __forceinline__ float block_sum(float v, float* red) {
+// ---------------------------------------------------------------------------- row groups
+// A row is owned by a group of W warps (W*32 threads); a 256-thread CTA holds 8/W groups. Sums
+// over the row are warp shuffles, then (W > 1) a named barrier private to the group, so groups
+// that process different numbers of rows never wait on each other.
+template <int W>
+__device__ __forceinline__ float group_sum(float v, float* red, int grp, int wg) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();  // protect `red` from the previous use
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  float s = 0.f;
+  if constexpr (W == 1) {
+    return v;
+  } else {
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) red[grp * W + wg] = v;
+    asm volatile("bar.sync %0, %1;" ::"r"(grp + 1), "r"(W * 32) : "memory");
+    float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < NT / 32; ++i) s += red[i];
-  return s;
+    for (int i = 0; i < W; ++i) s += red[grp * W + i];
+    asm volatile("bar.sync %0, %1;" ::"r"(grp + 1), "r"(W * 32) : "memory");  // red reusable
+    return s;
+  }
 }
 
 // ---------------------------------------------------------------------------- LN forward
-// One CTA of NT threads per row; each thread keeps up to MAXV 16-byte vectors of the row in
-// registers, so the row is read once: mean, then the centred second moment (two passes over
-// registers, no cancellation), then the normalised, affine output.
-template <typename T, int NT, int MAXV>
-__global__ void __launch_bounds__(NT) ln_fwd_kernel(long long rows, int h, float eps,
-                                                    const T* __restrict__ x,
-                                                    const float* __restrict__ gamma,
-                                                    const float* __restrict__ beta,
-                                                    T* __restrict__ y, float* __restrict__ mean,
-                                                    float* __restrict__ rstd) {
-  constexpr int V = Vec<T>::N;
-  __shared__ float red[NT / 32];
-  const long long row = blockIdx.x;
-  const T* xr = x + row * h;
+// Each group reads its row once into registers (up to VPL 16-byte vectors per thread), takes
+// the mean, then the centred second moment (two passes over registers, no cancellation), and
+// writes the normalised, affine output.
+template <typename T, int W, int VPL>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(long long rows, int h, float eps,
+                                                     const T* __restrict__ x,
+                                                     const float* __restrict__ gamma,
+                                                     const float* __restrict__ beta,
+                                                     T* __restrict__ y, float* __restrict__ mean,
+                                                     float* __restrict__ rstd) {
+  constexpr int V = Vec<T>::N, G = 8 / W, GT = 32 * W;
+  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, grp = warp / W, wg = warp % W;
+  const int t = wg * 32 + (threadIdx.x & 31);
+  const long long row = (long long)blockIdx.x * G + grp;
+  const bool valid = row < rows;
   const int nvec = h / V;
-  float v[MAXV][V];
+  const T* xr = x + (valid ? row : 0) * h;
+  float v[VPL][V];
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int vi = threadIdx.x + i * NT;
-    if (vi < nvec) {
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * GT;
+    if (valid && vi < nvec) {
       Vec<T>::load(xr + vi * V, v[i]);
 #pragma unroll
       for (int j = 0; j < V; ++j) s += v[i][j];
     }
   }
-  const float mu = block_sum<NT>(s, red) / h;
+  const float mu = group_sum<W>(s, red, grp, wg) / h;
   float q = 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int vi = threadIdx.x + i * NT;
-    if (vi < nvec) {
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * GT;
+    if (valid && vi < nvec) {
 #pragma unroll
       for (int j = 0; j < V; ++j) {
         const float c = v[i][j] - mu;
@@ -102,12 +113,13 @@ __global__ void __launch_bounds__(NT) ln_fwd_kernel(long long rows, int h, float
       }
     }
   }
-  const float var = block_sum<NT>(q, red) / h;
+  const float var = group_sum<W>(q, red, grp, wg) / h;
   const float rs = rsqrtf(var + eps);
+  if (!valid) return;
   T* yr = y + row * h;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int vi = threadIdx.x + i * NT;
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * GT;
     if (vi < nvec) {
       float o[V];
 #pragma unroll
@@ -118,105 +130,161 @@ __global__ void __launch_bounds__(NT) ln_fwd_kernel(long long rows, int h, float
       Vec<T>::store(yr + vi * V, o);
     }
   }
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     mean[row] = mu;
     rstd[row] = rs;
   }
 }
 
 // ---------------------------------------------------------------------------- LN backward
-// CTA b handles rows b, b+grid, ...; thread columns are fixed, so each thread accumulates its
-// columns' dgamma = sum dy*xhat and dbeta = sum dy across its rows in registers and writes one
-// partial row per CTA. dx = rstd*(g - mean(g) - xhat*mean(g*xhat)) + dres with g = dy*gamma.
-// The second pass re-reads x and dy (an L1/L2 hit) instead of holding them in registers.
-template <typename T, int NT, int MAXV>
-__global__ void __launch_bounds__(NT) ln_bwd_kernel(long long rows, int h,
-                                                    const T* __restrict__ dy,
-                                                    const T* __restrict__ dres,
-                                                    const T* __restrict__ x,
-                                                    const float* __restrict__ gamma,
-                                                    const float* __restrict__ mean,
-                                                    const float* __restrict__ rstd,
-                                                    T* __restrict__ dx,
-                                                    float* __restrict__ partial) {
-  constexpr int V = Vec<T>::N;
-  __shared__ float red[NT / 32];
+// dx for one row per group, every row in flight at once (no accumulators across rows):
+//   g = dy*gamma, dx = rstd*(g - mean(g) - xhat*mean(g*xhat)) + dres.
+template <typename T, int W, int VPL>
+__global__ void __launch_bounds__(256) ln_bwd_dx_kernel(long long rows, int h,
+                                                        const T* __restrict__ dy,
+                                                        const T* __restrict__ dres,
+                                                        const T* __restrict__ x,
+                                                        const float* __restrict__ gamma,
+                                                        const float* __restrict__ mean,
+                                                        const float* __restrict__ rstd,
+                                                        T* __restrict__ dx) {
+  constexpr int V = Vec<T>::N, G = 8 / W, GT = 32 * W;
+  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, grp = warp / W, wg = warp % W;
+  const int t = wg * 32 + (threadIdx.x & 31);
+  const long long row = (long long)blockIdx.x * G + grp;
+  const bool valid = row < rows;
+  const long long r = valid ? row : 0;
   const int nvec = h / V;
-  float dg[MAXV][V], db[MAXV][V];
+  const float mu = mean[r], rs = rstd[r];
+  float xh[VPL][V], g[VPL][V];
+  float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i)
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * GT;
+    if (valid && vi < nvec) {
+      float xv[V], dv[V];
+      Vec<T>::load(x + r * h + vi * V, xv);
+      Vec<T>::load(dy + r * h + vi * V, dv);
 #pragma unroll
-    for (int j = 0; j < V; ++j) dg[i][j] = db[i][j] = 0.f;
-
-  for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
-    const float mu = mean[row], rs = rstd[row];
-    float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int vi = threadIdx.x + i * NT;
-      if (vi < nvec) {
-        float xv[V], dv[V];
-        Vec<T>::load(x + row * h + vi * V, xv);
-        Vec<T>::load(dy + row * h + vi * V, dv);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          const float xh = (xv[j] - mu) * rs;
-          const float g = dv[j] * __ldg(gamma + vi * V + j);
-          s1 += g;
-          s2 += g * xh;
-          dg[i][j] += dv[j] * xh;
-          db[i][j] += dv[j];
-        }
-      }
-    }
-    const float m1 = block_sum<NT>(s1, red) / h;
-    const float m2 = block_sum<NT>(s2, red) / h;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int vi = threadIdx.x + i * NT;
-      if (vi < nvec) {
-        float xv[V], dv[V], r[V], o[V];
-        Vec<T>::load(x + row * h + vi * V, xv);
-        Vec<T>::load(dy + row * h + vi * V, dv);
-        if (dres) {
-          Vec<T>::load(dres + row * h + vi * V, r);
-        } else {
-#pragma unroll
-          for (int j = 0; j < V; ++j) r[j] = 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          const float xh = (xv[j] - mu) * rs;
-          const float g = dv[j] * __ldg(gamma + vi * V + j);
-          o[j] = rs * (g - m1 - xh * m2) + r[j];
-        }
-        Vec<T>::store(dx + row * h + vi * V, o);
+      for (int j = 0; j < V; ++j) {
+        xh[i][j] = (xv[j] - mu) * rs;
+        g[i][j] = dv[j] * __ldg(gamma + vi * V + j);
+        s1 += g[i][j];
+        s2 += g[i][j] * xh[i][j];
       }
     }
   }
-  float* pg = partial + (long long)blockIdx.x * 2 * h;
+  const float m1 = group_sum<W>(s1, red, grp, wg) / h;
+  const float m2 = group_sum<W>(s2, red, grp, wg) / h;
+  if (!valid) return;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int vi = threadIdx.x + i * NT;
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * GT;
     if (vi < nvec) {
+      float rv[V], o[V];
+      if (dres) {
+        Vec<T>::load(dres + r * h + vi * V, rv);
+      } else {
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        pg[vi * V + j] = dg[i][j];
-        pg[h + vi * V + j] = db[i][j];
+        for (int j = 0; j < V; ++j) rv[j] = 0.f;
       }
+#pragma unroll
+      for (int j = 0; j < V; ++j) o[j] = rs * (g[i][j] - m1 - xh[i][j] * m2) + rv[j];
+      Vec<T>::store(dx + r * h + vi * V, o);
     }
   }
 }
 
-// dgamma[c] = sum_b partial[b][0][c]; dbeta[c] = sum_b partial[b][1][c] (fixed order).
-__global__ void ln_param_reduce_kernel(int h, int nblk, const float* __restrict__ partial,
-                                       float* __restrict__ dgamma, float* __restrict__ dbeta) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= 2 * h) return;
-  const int which = c / h, col = c % h;
+// Partial dgamma = sum dy*xhat and dbeta = sum dy over one slice of rows. Block = 32 x 8
+// threads covering 32*VEC columns; blockIdx.y is the slice; the 8 row lanes are combined in
+// shared memory and written to partial[slice][2][h] (no atomics: deterministic).
+template <typename T>
+__global__ void __launch_bounds__(256) ln_bwd_param_kernel(long long rows, int h,
+                                                           const T* __restrict__ dy,
+                                                           const T* __restrict__ x,
+                                                           const float* __restrict__ mean,
+                                                           const float* __restrict__ rstd,
+                                                           float* __restrict__ partial,
+                                                           long long rows_per) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[2][8][32 * V + 1];
+  const int c0 = (blockIdx.x * 32 + threadIdx.x) * V;
+  const long long r0 = blockIdx.y * rows_per;
+  const long long r1 = min(rows, r0 + rows_per);
+  float ag[V], ab[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) ag[j] = ab[j] = 0.f;
+  if (c0 < h) {
+    long long r = r0 + threadIdx.y;
+    for (; r + 8 < r1; r += 16) {  // two independent rows in flight per thread
+      float x0[V], d0[V], x1[V], d1[V];
+      Vec<T>::load(x + r * h + c0, x0);
+      Vec<T>::load(dy + r * h + c0, d0);
+      Vec<T>::load(x + (r + 8) * h + c0, x1);
+      Vec<T>::load(dy + (r + 8) * h + c0, d1);
+      const float mu0 = mean[r], rs0 = rstd[r], mu1 = mean[r + 8], rs1 = rstd[r + 8];
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        ag[j] += d0[j] * ((x0[j] - mu0) * rs0) + d1[j] * ((x1[j] - mu1) * rs1);
+        ab[j] += d0[j] + d1[j];
+      }
+    }
+    for (; r < r1; r += 8) {
+      float x0[V], d0[V];
+      Vec<T>::load(x + r * h + c0, x0);
+      Vec<T>::load(dy + r * h + c0, d0);
+      const float mu0 = mean[r], rs0 = rstd[r];
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        ag[j] += d0[j] * ((x0[j] - mu0) * rs0);
+        ab[j] += d0[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    red[0][threadIdx.y][threadIdx.x * V + j] = ag[j];
+    red[1][threadIdx.y][threadIdx.x * V + j] = ab[j];
+  }
+  __syncthreads();
+  float* pg = partial + (long long)blockIdx.y * 2 * h;
+  const int t = threadIdx.y * 32 + threadIdx.x;
+  for (int cc = t; cc < 2 * 32 * V; cc += 256) {
+    const int which = cc / (32 * V), cl = cc % (32 * V);
+    const int col = blockIdx.x * 32 * V + cl;
+    if (col < h) {
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum += red[which][k][cl];
+      pg[which * h + col] = sum;
+    }
+  }
+}
+
+// dgamma[c] = sum_b partial[b][0][c]; dbeta[c] = sum_b partial[b][1][c]. Block = 32 columns x
+// 8 slices of the partial rows; fixed summation order.
+__global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk,
+                                                              const float* __restrict__ partial,
+                                                              float* __restrict__ dgamma,
+                                                              float* __restrict__ dbeta) {
+  __shared__ float red[8][33];
+  const int c = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int sl = threadIdx.x >> 5;
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += partial[(long long)b * 2 * h + which * h + col];
-  (which ? dbeta : dgamma)[col] = s;
+  if (c < 2 * h)
+    for (int b = sl; b < nblk; b += 8) s += partial[(long long)b * 2 * h + c];
+  red[sl][threadIdx.x & 31] = s;
+  __syncthreads();
+  if (sl == 0 && c < 2 * h) {
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) tot += red[k][threadIdx.x & 31];
+    if (c < h)
+      dgamma[c] = tot;
+    else
+      dbeta[c - h] = tot;
+  }
 }
 
 // ---------------------------------------------------------------------------- column sums
@@ -235,7 +303,17 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
 #pragma unroll
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
   if (c0 < cols) {
-    for (long long r = r0 + threadIdx.y; r < r1; r += 8) {
+    long long r = r0 + threadIdx.y;
+    for (; r + 24 < r1; r += 32) {  // four independent rows in flight per thread
+      float v0[V], v1[V], v2[V], v3[V];
+      Vec<T>::load(x + r * cols + c0, v0);
+      Vec<T>::load(x + (r + 8) * cols + c0, v1);
+      Vec<T>::load(x + (r + 16) * cols + c0, v2);
+      Vec<T>::load(x + (r + 24) * cols + c0, v3);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] += (v0[j] + v1[j]) + (v2[j] + v3[j]);
+    }
+    for (; r < r1; r += 8) {
       float v[V];
       Vec<T>::load(x + r * cols + c0, v);
 #pragma unroll
@@ -306,42 +384,85 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
   }
 }
 
-template <typename T, int NT, int MAXV>
+template <typename T, int W, int VPL>
 cudaError_t ln_fwd_inst(long long rows, int h, float eps, const void* x, const float* g,
                         const float* b, void* y, float* mean, float* rstd, cudaStream_t s) {
-  ln_fwd_kernel<T, NT, MAXV><<<(unsigned)rows, NT, 0, s>>>(
+  const long long grid = (rows + (8 / W) - 1) / (8 / W);
+  ln_fwd_kernel<T, W, VPL><<<(unsigned)grid, 256, 0, s>>>(
       rows, h, eps, reinterpret_cast<const T*>(x), g, b, reinterpret_cast<T*>(y), mean, rstd);
   return cudaGetLastError();
 }
 
-template <typename T, int NT, int MAXV>
-cudaError_t ln_bwd_inst(long long rows, int h, const void* dy, const void* dres, const void* x,
-                        const float* g, const float* mean, const float* rstd, void* dx,
-                        float* partial, int nblk, cudaStream_t s) {
-  ln_bwd_kernel<T, NT, MAXV><<<nblk, NT, 0, s>>>(
+template <typename T, int W, int VPL>
+cudaError_t ln_bwd_dx_inst(long long rows, int h, const void* dy, const void* dres,
+                           const void* x, const float* g, const float* mean, const float* rstd,
+                           void* dx, cudaStream_t s) {
+  const long long grid = (rows + (8 / W) - 1) / (8 / W);
+  ln_bwd_dx_kernel<T, W, VPL><<<(unsigned)grid, 256, 0, s>>>(
       rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(dres),
-      reinterpret_cast<const T*>(x), g, mean, rstd, reinterpret_cast<T*>(dx), partial);
+      reinterpret_cast<const T*>(x), g, mean, rstd, reinterpret_cast<T*>(dx));
+  return cudaGetLastError();
+}
+
+// Row-group shapes: a row is spread over W warps with at most VPL 16-byte vectors per thread,
+// so registers stay small and many rows are in flight. bf16: h <= 16384; fp32: h <= 8192.
+template <typename T>
+cudaError_t ln_fwd_dispatch(long long rows, int h, float eps, const void* x, const float* g,
+                            const float* b, void* y, float* mean, float* rstd, cudaStream_t s) {
+  const int nvec = h / Vec<T>::N;
+  if (nvec <= 64) return ln_fwd_inst<T, 1, 2>(rows, h, eps, x, g, b, y, mean, rstd, s);
+  if (nvec <= 128) return ln_fwd_inst<T, 1, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
+  if (nvec <= 256) return ln_fwd_inst<T, 2, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
+  if (nvec <= 512) return ln_fwd_inst<T, 4, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
+  if (nvec <= 1024) return ln_fwd_inst<T, 8, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
+  return ln_fwd_inst<T, 8, 8>(rows, h, eps, x, g, b, y, mean, rstd, s);
+}
+
+template <typename T>
+cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* dres,
+                            const void* x, const float* g, const float* mean, const float* rstd,
+                            void* dx, float* partial, int nblk, float* dgamma, float* dbeta,
+                            cudaStream_t s) {
+  const int nvec = h / Vec<T>::N;
+  cudaError_t e;
+  if (nvec <= 64)
+    e = ln_bwd_dx_inst<T, 1, 2>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  else if (nvec <= 128)
+    e = ln_bwd_dx_inst<T, 1, 4>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  else if (nvec <= 256)
+    e = ln_bwd_dx_inst<T, 2, 4>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  else if (nvec <= 512)
+    e = ln_bwd_dx_inst<T, 4, 4>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  else if (nvec <= 1024)
+    e = ln_bwd_dx_inst<T, 8, 4>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  else
+    e = ln_bwd_dx_inst<T, 8, 8>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
+  if (e != cudaSuccess) return e;
+  // dgamma/dbeta partials: one partial row pair per slice of rows, at most nblk slices.
+  const int cb = (h + 32 * Vec<T>::N - 1) / (32 * Vec<T>::N);
+  long long slices = (4LL * 148 + cb - 1) / cb;
+  if (slices > nblk) slices = nblk;
+  if (slices > (rows + 15) / 16) slices = (rows + 15) / 16;
+  if (slices < 1) slices = 1;
+  const long long rows_per = (rows + slices - 1) / slices;
+  slices = (rows + rows_per - 1) / rows_per;
+  ln_bwd_param_kernel<T><<<dim3(cb, (unsigned)slices), dim3(32, 8), 0, s>>>(
+      rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x), mean, rstd,
+      partial, rows_per);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ln_param_reduce_kernel<<<(2 * h + 31) / 32, 256, 0, s>>>(h, (int)slices, partial, dgamma,
+                                                          dbeta);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// Threads per row: enough 16-byte vectors per thread to cover h (forward: up to 256 threads
-// x 8 vectors; backward: up to 512 threads x 4 vectors). bf16: h <= 16384; fp32: h <= 8192.
 cudaError_t launch_ln_fwd(int dtype, long long rows, int h, float eps, const void* x,
                           const float* gamma, const float* beta, void* y, float* mean,
                           float* rstd, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  const int V = dtype ? 8 : 4;
-  const int nvec = h / V;
-  if (nvec <= 32 * 2)
-    return dtype ? ln_fwd_inst<__nv_bfloat16, 32, 2>(rows, h, eps, x, gamma, beta, y, mean, rstd, s)
-                 : ln_fwd_inst<float, 32, 2>(rows, h, eps, x, gamma, beta, y, mean, rstd, s);
-  if (nvec <= 128 * 4)
-    return dtype ? ln_fwd_inst<__nv_bfloat16, 128, 4>(rows, h, eps, x, gamma, beta, y, mean, rstd, s)
-                 : ln_fwd_inst<float, 128, 4>(rows, h, eps, x, gamma, beta, y, mean, rstd, s);
-  return dtype ? ln_fwd_inst<__nv_bfloat16, 256, 8>(rows, h, eps, x, gamma, beta, y, mean, rstd, s)
-               : ln_fwd_inst<float, 256, 8>(rows, h, eps, x, gamma, beta, y, mean, rstd, s);
+  return dtype ? ln_fwd_dispatch<__nv_bfloat16>(rows, h, eps, x, gamma, beta, y, mean, rstd, s)
+               : ln_fwd_dispatch<float>(rows, h, eps, x, gamma, beta, y, mean, rstd, s);
 }
 
 int ln_bwd_blocks(long long rows, int num_sms) {
@@ -355,21 +476,10 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
                           const float* rstd, void* dx, float* partial, int nblk, float* dgamma,
                           float* dbeta, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  const int V = dtype ? 8 : 4;
-  const int nvec = h / V;
-  cudaError_t e;
-  if (nvec <= 32 * 2)
-    e = dtype ? ln_bwd_inst<__nv_bfloat16, 32, 2>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s)
-              : ln_bwd_inst<float, 32, 2>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s);
-  else if (nvec <= 128 * 4)
-    e = dtype ? ln_bwd_inst<__nv_bfloat16, 128, 4>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s)
-              : ln_bwd_inst<float, 128, 4>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s);
-  else
-    e = dtype ? ln_bwd_inst<__nv_bfloat16, 512, 4>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s)
-              : ln_bwd_inst<float, 512, 4>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial, nblk, s);
-  if (e != cudaSuccess) return e;
-  ln_param_reduce_kernel<<<(2 * h + 255) / 256, 256, 0, s>>>(h, nblk, partial, dgamma, dbeta);
-  return cudaGetLastError();
+  return dtype ? ln_bwd_dispatch<__nv_bfloat16>(rows, h, dy, dres, x, gamma, mean, rstd, dx,
+                                                partial, nblk, dgamma, dbeta, s)
+               : ln_bwd_dispatch<float>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial,
+                                        nblk, dgamma, dbeta, s);
 }
 
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
