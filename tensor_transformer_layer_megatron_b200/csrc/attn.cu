@@ -4,11 +4,11 @@
 // heads without communication). Softmax arithmetic is fp32 (section 3.2,
 // attention_softmax_in_fp32). Scale 1/sqrt(d); key j visible to query i iff j <= i.
 //
-// bf16 path: FlashAttention-style tiling (online softmax, O(s) memory) on mma.sync m16n8k16
-// tensor-core instructions with ldmatrix from swizzled shared memory and cp.async double
-// buffering. The backward recomputes the probabilities from the saved log-sum-exp (the
-// page's section 4.1 recompute), keeps dK/dV in registers per key block, and accumulates dQ
-// with fp32 atomics into a workspace buffer that a last pass scales and converts.
+// bf16 path: the forward runs on tcgen05 (attn_tc.cu). The backward here is FlashAttention-
+// style tiling on mma.sync m16n8k16 with ldmatrix from swizzled shared memory and cp.async
+// double buffering; it recomputes the probabilities from the saved log-sum-exp (the page's
+// section 4.1 recompute), keeps dK/dV in registers per key block, and accumulates dQ with
+// fp32 atomics into a workspace buffer that a last pass scales and converts.
 // fp32 path: plain per-row kernels (tiny shapes only).
 #include "mgt_device.cuh"
 
@@ -16,7 +16,6 @@ namespace mgt {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 // ============================================================================ fp32 kernels
 // One thread per (batch, head, query): online softmax over keys 0..i.
@@ -145,159 +144,6 @@ __device__ __forceinline__ void load_tile(uint32_t sbase, const __nv_bfloat16* g
     const bool ok = gr < nvalid;
     const __nv_bfloat16* src = g + (long long)(ok ? gr : 0) * ld + c * 8;
     cp_async16(tile_addr<D>(sbase, r, c), src, ok);
-  }
-}
-
-// ============================================================================ bf16 forward
-// CTA = 4 warps, 64 queries (16 per warp); key blocks of 64, double-buffered.
-template <int D>
-__global__ void __launch_bounds__(128) attn_fwd_bf16_kernel(AttnArgs a, float scale_log2) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK0 = sQ + 64 * D * 2;
-  const uint32_t sV0 = sK0 + 2 * 64 * D * 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = a.s, H = a.H, hp = H / a.p;
-  const int nqb = (S + 63) / 64;
-  const int qb = nqb - 1 - blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, j = n % hp;
-  const long long ld = 3LL * H * D;
-  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.qkv) +
-                            (long long)b * S * ld + (long long)t * 3 * hp * D + (long long)j * D;
-  const __nv_bfloat16* kg = qg + (long long)hp * D;
-  const __nv_bfloat16* vg = qg + 2LL * hp * D;
-
-  load_tile<D, 128>(sQ, qg, ld, qb * 64, 64, S);
-  cp_async_commit();
-  load_tile<D, 128>(sK0, kg, ld, 0, 64, S);
-  load_tile<D, 128>(sV0, vg, ld, 0, 64, S);
-  cp_async_commit();
-  cp_async_wait<1>();
-  __syncthreads();
-
-  uint32_t qf[D / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks) {
-    const int mi = lane >> 3, r = lane & 7;
-    ldsm_x4(tile_addr<D>(sQ, warp * 16 + (mi & 1) * 8 + r, ks * 2 + (mi >> 1)), qf[ks][0],
-            qf[ks][1], qf[ks][2], qf[ks][3]);
-  }
-
-  float acc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  const int g = lane >> 2, q4 = lane & 3;
-  const int nkb = qb + 1;
-
-  for (int kb = 0; kb < nkb; ++kb) {
-    const int buf = kb & 1;
-    if (kb + 1 < nkb) {
-      load_tile<D, 128>(sK0 + (buf ^ 1) * 64 * D * 2, kg, ld, (kb + 1) * 64, 64, S);
-      load_tile<D, 128>(sV0 + (buf ^ 1) * 64 * D * 2, vg, ld, (kb + 1) * 64, 64, S);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t sK = sK0 + buf * 64 * D * 2, sV = sV0 + buf * 64 * D * 2;
-
-    float sacc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        const int mi = lane >> 3, r = lane & 7;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(tile_addr<D>(sK, np * 16 + (mi >> 1) * 8 + r, ks * 2 + (mi & 1)), b0, b1, b2, b3);
-        mma16816(sacc[2 * np], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
-        mma16816(sacc[2 * np + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
-      }
-    }
-    // scale into log2 units, causal mask on the diagonal block, online softmax
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = sacc[nt][e] * scale_log2;
-        if (kb == qb) {
-          const int qr = warp * 16 + g + (e >= 2 ? 8 : 0);
-          const int kc = nt * 8 + 2 * q4 + (e & 1);
-          if (kc > qr) v = -INFINITY;
-        }
-        sacc[nt][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-    float alpha[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-      const float mn = fmaxf(mrow[r], mx[r]);
-      alpha[r] = exp2f(mrow[r] - mn);  // exp2(-inf) = 0 on the first block
-      mrow[r] = mn;
-    }
-    float rs[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p = exp2f(sacc[nt][e] - mrow[e >> 1]);
-        sacc[nt][e] = p;
-        rs[e >> 1] += p;
-      }
-    }
-    lrow[0] = lrow[0] * alpha[0] + rs[0];
-    lrow[1] = lrow[1] * alpha[1] + rs[1];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      acc[i][0] *= alpha[0];
-      acc[i][1] *= alpha[0];
-      acc[i][2] *= alpha[1];
-      acc[i][3] *= alpha[1];
-    }
-    // O += P V
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t a0 = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
-      const uint32_t a1 = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
-      const uint32_t a2 = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
-      const uint32_t a3 = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
-#pragma unroll
-      for (int dp = 0; dp < D / 16; ++dp) {
-        const int mi = lane >> 3, r = lane & 7;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(tile_addr<D>(sV, kk * 16 + (mi & 1) * 8 + r, dp * 2 + (mi >> 1)), b0, b1, b2, b3);
-        mma16816(acc[2 * dp], a0, a1, a2, a3, b0, b1);
-        mma16816(acc[2 * dp + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    __syncthreads();  // everyone is done with this buffer before it is refilled
-  }
-
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
-    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
-  }
-  __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(a.o);
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int qrow = qb * 64 + warp * 16 + g + r * 8;
-    if (qrow < S) {
-      const float inv = 1.f / lrow[r];
-      __nv_bfloat16* orow = og + ((long long)b * S + qrow) * H * D + (long long)n * D;
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i)
-        *reinterpret_cast<uint32_t*>(orow + i * 8 + 2 * q4) =
-            pack_bf16x2(acc[i][2 * r] * inv, acc[i][2 * r + 1] * inv);
-      if (q4 == 0) a.lse[((long long)b * H + n) * S + qrow] = (mrow[r] + log2f(lrow[r])) * kLn2;
-    }
   }
 }
 
@@ -545,23 +391,7 @@ __global__ void attn_dq_convert_kernel(AttnArgs a, float scale) {
 }
 
 template <int D>
-constexpr int fwd_smem() { return (64 + 4 * 64) * D * 2; }
-template <int D>
 constexpr int bwd_smem() { return 4 * 64 * D * 2 + 64 * 32 * 2 + 4 * 32 * 4; }
-
-template <int D>
-cudaError_t fwd_bf16(const AttnArgs& a, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem<D>());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid((a.s + 63) / 64, a.b * a.H);
-  attn_fwd_bf16_kernel<D><<<grid, 128, fwd_smem<D>(), s>>>(a, kLog2e / sqrtf((float)D));
-  return cudaGetLastError();
-}
 
 template <int D>
 cudaError_t bwd_bf16(const AttnArgs& a, cudaStream_t s) {
@@ -595,9 +425,7 @@ cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t s) {
     attn_fwd_f32_kernel<64><<<(total + 127) / 128, 128, 0, s>>>(a);
     return cudaGetLastError();
   }
-  if (a.d == 64) return fwd_bf16<64>(a, s);
-  if (a.d == 128) return fwd_bf16<128>(a, s);
-  return cudaErrorInvalidValue;
+  return launch_attn_fwd_tc(a, s);  // tcgen05 kernel (attn_tc.cu)
 }
 
 cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t s) {

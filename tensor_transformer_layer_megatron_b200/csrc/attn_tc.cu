@@ -1,0 +1,322 @@
+// Causal attention forward on the fifth-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA owns one 128-query tile of one head. The heads are local to their tensor-parallel
+// shard (the column split of W_q/W_k/W_v on the trdm.cn page, section 2.1, keeps whole heads
+// on a shard), so the softmax never needs another shard's data. Softmax arithmetic is fp32
+// (section 3.2, attention_softmax_in_fp32); scale 1/sqrt(d); key j visible to query i iff
+// j <= i.
+//
+// Per key block of 128 (double-buffered K/V tiles from TMA):
+//   S = Q K^T            tcgen05.mma M=128 N=128, fp32 in TMEM (two S buffers, so the next
+//                        block's S is computed while the softmax works on this one)
+//   softmax warps        one thread per query row reads its 128 scores with tcgen05.ld, so
+//                        the row max and sum need no shuffles; P = exp2(S*scale*log2e - m)
+//                        goes to shared memory as bf16 in the 128B-swizzled K-major layout
+//   O += P V             tcgen05.mma M=128 N=d, V read N-major straight from its TMA tile
+// The running max is updated lazily: O and the row sum are rescaled only when a row's max grows
+// by more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16), and the
+// rescale of O in TMEM is done by whole warps (tcgen05.ld/st are warp-collective).
+// Finally O / l is written in bf16 and lse = (m + log2 l) * ln 2.
+//
+// Warps 0-3: softmax + output (warp w owns TMEM lanes 32w..32w+31, i.e. query rows);
+// warp 4: TMA producer; warp 5: TMEM owner and MMA issuer. Every wait is bounded.
+#include "mgt_device.cuh"
+
+namespace mgt {
+namespace {
+
+constexpr int kAttnThreads = 192;
+constexpr float kLog2eF = 1.4426950408889634f;
+constexpr float kLn2F = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdLayout {
+  static constexpr int CH = D / 64;              // 64-wide (128-byte) swizzle chunks per row
+  static constexpr int TILE = 128 * D * 2;       // one 128-row Q, K or V tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = TILE;             // 2 stages
+  static constexpr int V_OFF = K_OFF + 2 * TILE; // 2 stages
+  static constexpr int P_OFF = V_OFF + 2 * TILE; // [128 q][128 keys] bf16, 2 chunks
+  static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
+  static constexpr int BYTES = BAR_OFF + 256 + 1024;
+  static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a,
+                       float scale_log2) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.s, H = a.H, hp = H / a.p;
+  const int nqb = (S + 127) / 128;
+  const int qb = nqb - 1 - blockIdx.x;  // longest rows first
+  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
+  const int nkv = qb + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(q_full, L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c)
+        tma_load_3d(&tm, q_full, smem + L::Q_OFF + c * 16384, col_q + c * 64, qb * 128, b);
+      int issued = 0;
+      for (int kb = 0; kb < nkv; ++kb) {
+        const int st = kb & 1;
+        if (!mbar_wait(&kv_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&k_full[st], L::TILE);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c)
+          tma_load_3d(&tm, &k_full[st], smem + L::K_OFF + st * L::TILE + c * 16384,
+                      col_k + c * 64, kb * 128, b);
+        mbar_arrive_expect_tx(&v_full[st], L::TILE);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c)
+          tma_load_3d(&tm, &v_full[st], smem + L::V_OFF + st * L::TILE + c * 16384,
+                      col_v + c * 64, kb * 128, b);
+        issued = kb + 1;
+      }
+      // every issued load lands before the CTA can exit
+      mbar_wait(q_full, 0, a.err, kErrTimeoutDrain, nullptr);
+      for (int kb = issued - 2 < 0 ? 0 : issued - 2; kb < issued; ++kb) {
+        mbar_wait(&k_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+        mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
+      const uint32_t p_addr = smem_u32(smem + L::P_OFF);
+      bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag);
+      auto issue_s = [&](int kb) -> bool {
+        const int st = kb & 1;
+        if (!mbar_wait(&k_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::K_OFF + st * L::TILE);
+        const uint32_t d = tmem + (st ? L::TMEM_S1 : L::TMEM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(d, smem_desc_sw128(q_addr + off, 16, 1024),
+                     smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[st]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int kb = 0; kb < nkv && ok; ++kb) {
+        if (kb + 1 < nkv && !issue_s(kb + 1)) break;
+        if (!mbar_wait(p_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        if (!mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + L::V_OFF + (kb & 1) * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
+          const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + L::TMEM_O, smem_desc_sw128(p_addr + a_off, 16, 1024),
+                     smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(pv_done);
+        tc_commit(&kv_empty[kb & 1]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + output
+    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t p_addr = smem_u32(smem + L::P_OFF);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < nkv; ++kb) {
+      const int st = kb & 1;
+      ok = mbar_wait(&s_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float tmp[32];
+        tmem_ld_32x32b_x32(lane_base + (st ? L::TMEM_S1 : L::TMEM_S0) + c * 32, tmp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = tmp[i];
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float v = sv[i] * scale_log2;
+        if (kb == qb && i > r) v = -INFINITY;  // causal mask on the diagonal block
+        sv[i] = v;
+        mx = fmaxf(mx, v);
+      }
+      const bool need = mx > m_run + kRescaleThreshold;
+      const float alpha = need ? exp2f(m_run - mx) : 1.f;
+      if (need) m_run = mx;
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        const float p = exp2f(sv[i] - m_run);
+        sv[i] = p;
+        rs += p;
+      }
+      l_run = l_run * alpha + rs;
+      if (kb > 0) {
+        // PV of the previous block must be done before O is rescaled or P overwritten.
+        ok = mbar_wait(pv_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+          }
+        }
+      }
+      // P (bf16) -> shared memory, K-major 128B-swizzled: row r, 16-byte chunk c16
+#pragma unroll
+      for (int c16 = 0; c16 < 16; ++c16) {
+        const uint32_t addr = p_addr + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+        st_shared_v4(addr, pack_bf16x2(sv[c16 * 8 + 0], sv[c16 * 8 + 1]),
+                     pack_bf16x2(sv[c16 * 8 + 2], sv[c16 * 8 + 3]),
+                     pack_bf16x2(sv[c16 * 8 + 4], sv[c16 * 8 + 5]),
+                     pack_bf16x2(sv[c16 * 8 + 6], sv[c16 * 8 + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) {
+      ok = mbar_wait(pv_done, (nkv - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const int qrow = qb * 128 + r;
+        const float inv = 1.f / l_run;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
+                              ((long long)b * S + qrow) * H * D + (long long)n * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+          if (qrow < S) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 w;
+              w.x = pack_bf16x2(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
+              w.y = pack_bf16x2(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
+              w.z = pack_bf16x2(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
+              w.w = pack_bf16x2(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = w;
+            }
+          }
+        }
+        if (qrow < S) a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
+  using L = FwdLayout<D>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  // qkv viewed as [b][s][3h]; rows past s read as zeros, so tiles never cross sequences.
+  CUtensorMap tm;
+  const uint64_t three_h = 3ull * a.H * D;
+  const uint64_t dims[3] = {three_h, (uint64_t)a.s, (uint64_t)a.b};
+  const uint64_t strides[2] = {three_h, three_h * a.s};
+  const uint32_t box[3] = {64, 128, 1};
+  if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
+  dim3 grid((a.s + 127) / 128, a.b * a.H);
+  attn_fwd_tc_kernel<D><<<grid, kAttnThreads, L::BYTES, s>>>(tm, a, kLog2eF / sqrtf((float)D));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t s) {
+  if (a.d == 64) return fwd_tc<64>(a, s);
+  if (a.d == 128) return fwd_tc<128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace mgt

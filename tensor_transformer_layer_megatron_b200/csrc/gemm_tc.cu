@@ -607,10 +607,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor map with 128-byte swizzle. dims/strides as in GemmArgs' comment;
-// stride values in elements (converted to bytes here).
-bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
-              const uint32_t box[3]) {
+}  // namespace
+
+// 3-D bf16 tensor map with 128-byte swizzle; strides in elements (converted to bytes here).
+bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
+                             const uint64_t strides[2], const uint32_t box[3]) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t gd[3] = {dims[0], dims[1], dims[2]};
@@ -621,6 +622,13 @@ bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[3], const ui
                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+              const uint32_t box[3]) {
+  return make_tensor_map_bf16_3d(m, base, dims, strides, box);
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI>

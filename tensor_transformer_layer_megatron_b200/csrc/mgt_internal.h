@@ -49,6 +49,10 @@ struct GemmArgs {
   int* err;                             // device status word
 };
 
+// 3-D bf16 tensor map (128-byte swizzle, zero fill out of bounds); strides in elements.
+bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
+                             const uint64_t strides[2], const uint32_t box[3]);
+
 // tcgen05 / TMA GEMM for bf16 operands (fp32 accumulate in tensor memory).
 // Builds the tensor maps from the pointers in `args` (A, B, strides) and launches a persistent
 // kernel with one CTA per SM. Returns a CUDA error code.
@@ -80,6 +84,7 @@ struct AttnArgs {
   int* err;
 };
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t stream);  // bf16, d in {64, 128}
 cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 int attn_bwd_kernel_count(int dtype);
 
