@@ -135,7 +135,7 @@ typedef enum mgt_region {
   MGT_WS_DQKV = 69,         /* ACT [T, 3h]  dL/d qkv (packed like qkv)                 */
   MGT_WS_DLN1 = 70,         /* ACT [T, h]   dL/d ln1                                   */
   MGT_WS_ATTN_D = 71,       /* F32 [b][H][s] rowsum(dO * O)                            */
-  MGT_WS_DQ_ACC = 72,       /* F32 [T, h]   dQ accumulator of the attention backward   */
+  MGT_WS_DQ_ACC = 72,       /* unused (0 bytes): dQ is accumulated in tensor memory     */
   MGT_WS_LN_PARTIAL = 73,   /* F32 [blocks][2][h] per-block LayerNorm dgamma/dbeta     */
   MGT_WS_COUNT = 74
 } mgt_region;

@@ -289,6 +289,482 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
+// ============================================================================ backward
+// Two kernels, both on tcgen05 with the probabilities recomputed from the saved log-sum-exp:
+//   dK/dV kernel, one CTA per 128-key block (key-stationary), looping over query blocks:
+//     S^T = K Q^T and dP^T = V dO^T in TMEM; one thread per key row forms
+//     P^T = exp2(S^T*scale*log2e - lse*log2e) and dS^T = P^T * (dP^T - D) (D = rowsum(dO*O))
+//     and writes both back into TMEM as packed bf16; then dV += P^T dO and dK += dS^T Q run with
+//     the A operand read from TMEM and dO, Q read N-major from their TMA tiles.
+//   dQ kernel, one CTA per 128-query block (query-stationary), looping over key blocks:
+//     S = Q K^T, dP = dO V^T, dS = P * (dP - D) per query row, dQ += dS K.
+// dQ therefore needs no atomics and is written once, in bf16, scaled by 1/sqrt(d); the cost is
+// recomputing S and dP in the second kernel. TMEM: S 0-127, dP 128-255, accumulators above.
+template <int D>
+struct BwdLayout {
+  static constexpr int CH = D / 64;
+  static constexpr int TILE = 128 * D * 2;
+  // dK/dV kernel: K, V resident; Q and dO double-buffered; per-query stats double-buffered.
+  static constexpr int A_K = 0, A_V = TILE, A_Q = 2 * TILE, A_DO = 4 * TILE;
+  static constexpr int A_STAT = 6 * TILE;  // float lse2[2][128], dsum[2][128]
+  static constexpr int A_BAR = A_STAT + 4 * 128 * 4;
+  static constexpr int A_BYTES = A_BAR + 256 + 1024;
+  // dQ kernel: Q, dO resident; K and V double-buffered.
+  static constexpr int B_Q = 0, B_DO = TILE, B_K = 2 * TILE, B_V = 4 * TILE;
+  static constexpr int B_BAR = 6 * TILE;
+  static constexpr int B_BYTES = B_BAR + 256 + 1024;
+  static constexpr int T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+                            const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
+                            float scale_log2, float scale) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::A_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;   // [2]: Q and dO of one query block
+  uint64_t* q_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* mm_done = bars + 7;
+  uint64_t* drain = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lse_s = reinterpret_cast<float*>(smem + L::A_STAT);  // [2][128], log2 units
+  float* dsum_s = lse_s + 256;                                 // [2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.s, H = a.H, hp = H / a.p;
+  const int kb = blockIdx.x;  // key block; kb = 0 has the most query blocks: launched first
+  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
+  const int nq = (S + 127) / 128;
+  const int niter = nq - kb;  // query blocks qi = kb .. nq-1 see keys of this block
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(mm_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_3d(&tm_qkv, kv_full, smem + L::A_K + c * 16384, col_k + c * 64, kb * 128, b);
+        tma_load_3d(&tm_qkv, kv_full, smem + L::A_V + c * 16384, col_v + c * 64, kb * 128, b);
+      }
+      int issued = 0;
+      for (int it = 0; it < niter; ++it) {
+        const int st = it & 1, qi = kb + it;
+        if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_3d(&tm_qkv, &q_full[st], smem + L::A_Q + st * L::TILE + c * 16384,
+                      col_q + c * 64, qi * 128, b);
+          tma_load_3d(&tm_do, &q_full[st], smem + L::A_DO + st * L::TILE + c * 16384,
+                      n * D + c * 64, qi * 128, b);
+        }
+        issued = it + 1;
+      }
+      mbar_wait(kv_full, 0, a.err, kErrTimeoutDrain, nullptr);
+      for (int it = issued - 2 < 0 ? 0 : issued - 2; it < issued; ++it)
+        mbar_wait(&q_full[it & 1], (it >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      const uint32_t k_addr = smem_u32(smem + L::A_K), v_addr = smem_u32(smem + L::A_V);
+      bool ok = mbar_wait(kv_full, 0, a.err, kErrTimeoutAttn, abort_flag);
+      for (int it = 0; it < niter && ok; ++it) {
+        const int st = it & 1;
+        // the previous block's dV/dK MMAs read P and dS from the S/dP columns: wait for them
+        if (it > 0 && !mbar_wait(mm_done, (it - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        if (!mbar_wait(&q_full[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + L::A_Q + st * L::TILE);
+        const uint32_t do_addr = smem_u32(smem + L::A_DO + st * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + L::T_S, smem_desc_sw128(k_addr + off, 16, 1024),
+                     smem_desc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + L::T_DP, smem_desc_sw128(v_addr + off, 16, 1024),
+                     smem_desc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        if (!mbar_wait(p_full, it & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 128 queries, 16 per MMA
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_f16_tmem_a(tmem + L::T_ACC0, tmem + L::T_S + kk * 8,
+                            smem_desc_sw128(do_addr + kk * 2048, 16384, 1024), idesc_acc, acc);
+          tc_mma_f16_tmem_a(tmem + L::T_ACC1, tmem + L::T_DP + kk * 8,
+                            smem_desc_sw128(q_addr + kk * 2048, 16384, 1024), idesc_acc, acc);
+        }
+        tc_commit(mm_done);
+        tc_commit(&q_empty[st]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ P^T, dS^T and the output
+    const int r = warp * 32 + lane;  // key row within the block = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float* lse_g = a.lse + ((long long)b * H + n) * S;
+    const float* dsum_g = a.Dsum + ((long long)b * H + n) * S;
+    bool ok = true;
+    for (int it = 0; it < niter; ++it) {
+      const int st = it & 1, qi = kb + it;
+      {
+        const int q = qi * 128 + r;  // padded queries get lse = +inf, hence P = 0
+        lse_s[st * 128 + r] = q < S ? lse_g[q] * kLog2eF : INFINITY;
+        dsum_s[st * 128 + r] = q < S ? dsum_g[q] : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      ok = mbar_wait(s_full, it & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* ls = lse_s + st * 128;
+      const float* ds_ = dsum_s + st * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32], dp[32];
+        tmem_ld_32x32b_x32(lane_base + L::T_S + c * 32, sv);
+        tmem_ld_32x32b_x32(lane_base + L::T_DP + c * 32, dp);
+        uint32_t pw[16], dw[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = c * 32 + i + e;
+            float p = exp2f(sv[i + e] * scale_log2 - ls[col]);
+            if (qi == kb && col < r) p = 0.f;  // key > query
+            p2[e] = p;
+            d2[e] = p * (dp[i + e] - ds_[col]);
+          }
+          pw[i >> 1] = pack_bf16x2(p2[0], p2[1]);
+          dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+        }
+        tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, pw);
+        tmem_st_32x32b_x16(lane_base + L::T_DP + c * 16, dw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && niter > 0) {
+      ok = mbar_wait(mm_done, (niter - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const int key = kb * 128 + r;
+        const long long ld = 3LL * H * D;
+        __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + ((long long)b * S + key) * ld +
+                            (long long)t * 3 * hp * D + (long long)jh * D + (long long)hp * D;
+        __nv_bfloat16* dv = dk + (long long)hp * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32], k[32];
+          tmem_ld_32x32b_x32(lane_base + L::T_ACC0 + c * 32, v);
+          tmem_ld_32x32b_x32(lane_base + L::T_ACC1 + c * 32, k);
+          if (key < S) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 wv, wk;
+              wv.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              wv.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              wv.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              wv.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              wk.x = pack_bf16x2(k[q * 8 + 0] * scale, k[q * 8 + 1] * scale);
+              wk.y = pack_bf16x2(k[q * 8 + 2] * scale, k[q * 8 + 3] * scale);
+              wk.z = pack_bf16x2(k[q * 8 + 4] * scale, k[q * 8 + 5] * scale);
+              wk.w = pack_bf16x2(k[q * 8 + 6] * scale, k[q * 8 + 7] * scale);
+              *reinterpret_cast<uint4*>(dv + c * 32 + q * 8) = wv;
+              *reinterpret_cast<uint4*>(dk + c * 32 + q * 8) = wk;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+                          const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
+                          float scale_log2, float scale) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::B_BAR);
+  uint64_t* q_full = bars + 0;    // Q and dO of this query block
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* mm_done = bars + 7;
+  uint64_t* drain = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.s, H = a.H, hp = H / a.p;
+  const int nqb = (S + 127) / 128;
+  const int qb = nqb - 1 - blockIdx.x;
+  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
+  const int nkv = qb + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(mm_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_3d(&tm_qkv, q_full, smem + L::B_Q + c * 16384, col_q + c * 64, qb * 128, b);
+        tma_load_3d(&tm_do, q_full, smem + L::B_DO + c * 16384, n * D + c * 64, qb * 128, b);
+      }
+      int issued = 0;
+      for (int kb = 0; kb < nkv; ++kb) {
+        const int st = kb & 1;
+        if (!mbar_wait(&kv_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * L::TILE);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_3d(&tm_qkv, &kv_full[st], smem + L::B_K + st * L::TILE + c * 16384,
+                      col_k + c * 64, kb * 128, b);
+          tma_load_3d(&tm_qkv, &kv_full[st], smem + L::B_V + st * L::TILE + c * 16384,
+                      col_v + c * 64, kb * 128, b);
+        }
+        issued = kb + 1;
+      }
+      mbar_wait(q_full, 0, a.err, kErrTimeoutDrain, nullptr);
+      for (int kb = issued - 2 < 0 ? 0 : issued - 2; kb < issued; ++kb)
+        mbar_wait(&kv_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::B_Q), do_addr = smem_u32(smem + L::B_DO);
+      bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag);
+      for (int kb = 0; kb < nkv && ok; ++kb) {
+        const int st = kb & 1;
+        if (kb > 0 && !mbar_wait(mm_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        if (!mbar_wait(&kv_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::B_K + st * L::TILE);
+        const uint32_t v_addr = smem_u32(smem + L::B_V + st * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + L::T_S, smem_desc_sw128(q_addr + off, 16, 1024),
+                     smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + L::T_DP, smem_desc_sw128(do_addr + off, 16, 1024),
+                     smem_desc_sw128(v_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        if (!mbar_wait(p_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA; dS sits in the S columns
+          tc_mma_f16_tmem_a(tmem + L::T_ACC0, tmem + L::T_S + kk * 8,
+                            smem_desc_sw128(k_addr + kk * 2048, 16384, 1024), idesc_acc,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(mm_done);
+        tc_commit(&kv_empty[st]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else {
+    const int r = warp * 32 + lane;  // query row within the block = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int q = qb * 128 + r;
+    const float lse2 = q < S ? a.lse[((long long)b * H + n) * S + q] * kLog2eF : INFINITY;
+    const float dq_sum = q < S ? a.Dsum[((long long)b * H + n) * S + q] : 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < nkv; ++kb) {
+      ok = mbar_wait(s_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32], dp[32];
+        tmem_ld_32x32b_x32(lane_base + L::T_S + c * 32, sv);
+        tmem_ld_32x32b_x32(lane_base + L::T_DP + c * 32, dp);
+        uint32_t dw[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = c * 32 + i + e;
+            float p = exp2f(sv[i + e] * scale_log2 - lse2);
+            if (kb == qb && col > r) p = 0.f;  // key > query
+            d2[e] = p * (dp[i + e] - dq_sum);
+          }
+          dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+        }
+        tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, dw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) {
+      ok = mbar_wait(mm_done, (nkv - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const long long ld = 3LL * H * D;
+        __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + ((long long)b * S + q) * ld +
+                            (long long)t * 3 * hp * D + (long long)jh * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld_32x32b_x32(lane_base + L::T_ACC0 + c * 32, v);
+          if (q < S) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              uint4 w;
+              w.x = pack_bf16x2(v[qq * 8 + 0] * scale, v[qq * 8 + 1] * scale);
+              w.y = pack_bf16x2(v[qq * 8 + 2] * scale, v[qq * 8 + 3] * scale);
+              w.z = pack_bf16x2(v[qq * 8 + 4] * scale, v[qq * 8 + 5] * scale);
+              w.w = pack_bf16x2(v[qq * 8 + 6] * scale, v[qq * 8 + 7] * scale);
+              *reinterpret_cast<uint4*>(dq + c * 32 + qq * 8) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
+  using L = BwdLayout<D>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::A_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::B_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap tm_qkv, tm_do;
+  const uint64_t three_h = 3ull * a.H * D, hd = (uint64_t)a.H * D;
+  const uint32_t box[3] = {64, 128, 1};
+  {
+    const uint64_t dims[3] = {three_h, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {three_h, three_h * a.s};
+    if (!make_tensor_map_bf16_3d(&tm_qkv, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {hd, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {hd, hd * a.s};
+    if (!make_tensor_map_bf16_3d(&tm_do, a.dO, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const float scale = 1.f / sqrtf((float)D);
+  dim3 grid((a.s + 127) / 128, a.b * a.H);
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kAttnThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
+                                                                    kLog2eF * scale, scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_bwd_dq_tc_kernel<D><<<grid, kAttnThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
+                                                                  kLog2eF * scale, scale);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   using L = FwdLayout<D>;
@@ -312,6 +788,12 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t s) {
+  if (a.d == 64) return bwd_tc<64>(a, s);
+  if (a.d == 128) return bwd_tc<128>(a, s);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t s) {
   if (a.d == 64) return fwd_tc<64>(a, s);

@@ -113,7 +113,7 @@ void layout(mgt_layer* L) {
                                    T * 3 * h * e,
                                    T * h * e,
                                    bHs * 4,
-                                   L->cfg.dtype == MGT_BF16 ? T * h * 4 : 0,
+                                   0,
                                    nblk * 2 * h * 4};
   off = 0;
   for (int i = 0; i < MGT_WS_COUNT - 64; ++i) {
@@ -290,7 +290,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   // 3. causal attention per head (each shard's heads are local)
   {
     AttnArgs a{L->cfg.micro_batch, L->cfg.seq, L->H, L->d, p, qkv, O, lse,
-               nullptr, nullptr, nullptr, nullptr, err};
+               nullptr, nullptr, nullptr, err};
     const double fl = 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;
     MGT_TRY(run(L, "attn_fwd", fl, 0, s, [&] { return launch_attn_fwd(dt, a, s); }));
   }
@@ -363,7 +363,6 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   char* dqkv = sp(workspace, L->ws[MGT_WS_DQKV - 64]);
   char* dln1 = sp(workspace, L->ws[MGT_WS_DLN1 - 64]);
   float* Dsum = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_ATTN_D - 64]));
-  float* dq_acc = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_DQ_ACC - 64]));
   float* part = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_LN_PARTIAL - 64]));
   const int nblk = T < kMaxLnBlocks ? T : kMaxLnBlocks;
   auto colsum = [&](const void* src, int cols, void* out) {
@@ -427,8 +426,8 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   // B6. attention backward (probabilities recomputed from the saved log-sum-exp)
   {
     AttnArgs a{L->cfg.micro_batch, L->cfg.seq, L->H, L->d, p, qkv, (void*)O, (float*)lse,
-               dO, Dsum, dq_acc, dqkv, err};
-    const double fl = 2.5 * 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;
+               dO, Dsum, dqkv, err};
+    const double fl = 2.5 * 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;  // model FLOPs incl. one recompute of S
     MGT_TRY(run(L, "attn_bwd", fl, 0, s, [&] { return launch_attn_bwd(dt, a, s); }));
   }
   // B7. QKV: db_qkv, dgrad (sum over shards = K loop over 3h), wgrad

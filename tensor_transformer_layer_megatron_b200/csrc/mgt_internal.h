@@ -80,12 +80,13 @@ cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, fl
 struct AttnArgs {
   int b, s, H, d, p;
   const void* qkv; void* o; float* lse;
-  const void* dO; float* Dsum; float* dq_acc; void* dqkv;
+  const void* dO; float* Dsum; void* dqkv;
   int* err;
 };
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t stream);  // bf16, d in {64, 128}
+// bf16 backward: dK/dV kernel then dQ kernel, both tcgen05; needs a.Dsum = rowsum(dO * O).
+cudaError_t launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t stream);
-int attn_bwd_kernel_count(int dtype);
 
 }  // namespace mgt
