@@ -124,7 +124,7 @@ typedef enum mgt_region {
   MGT_SAVED_LN2 = 7,        /* ACT [T, h]                                              */
   MGT_SAVED_LN2_MEAN = 8,   /* F32 [T]                                                 */
   MGT_SAVED_LN2_RSTD = 9,   /* F32 [T]                                                 */
-  MGT_SAVED_FC1_U = 10,     /* ACT [T][p][f/p]     fc1 pre-activation                  */
+  MGT_SAVED_FC1_DGELU = 10, /* ACT [T][p][f/p]     GeLU'(u), u = fc1 pre-activation    */
   MGT_SAVED_FC1_A = 11,     /* ACT [T][p][f/p]     GeLU(u)                             */
   MGT_SAVED_COUNT = 12,
   MGT_WS_STATUS = 64,       /* int32 device status word (first 256 bytes)              */
@@ -136,14 +136,15 @@ typedef enum mgt_region {
   MGT_WS_DLN1 = 70,         /* ACT [T, h]   dL/d ln1                                   */
   MGT_WS_ATTN_D = 71,       /* F32 [b][H][s] rowsum(dO * O)                            */
   MGT_WS_DQ_ACC = 72,       /* unused (0 bytes): dQ is accumulated in tensor memory     */
-  MGT_WS_LN_PARTIAL = 73,   /* F32 [blocks][2][h] per-block LayerNorm dgamma/dbeta     */
+  MGT_WS_LN_PARTIAL = 73,   /* F32 [slices][3][h] LayerNorm dgamma/dbeta/residual-grad partial sums */
   MGT_WS_COUNT = 74
 } mgt_region;
 mgt_status mgt_layer_region(const mgt_layer* layer, int region, size_t* offset, size_t* bytes);
 
 /* Forward. Reads x [b,s,h]; writes y [b,s,h] and every region of `saved`.
  * Launch order on `stream`: LN1, QKV GEMM(+bias), attention, out-proj GEMM (+shard sum,
- * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores u and a), fc2 GEMM (+shard sum, +b2, +h1). */
+ * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores a and GeLU'(u)), fc2 GEMM (+shard sum, +b2,
+ * +h1). */
 mgt_status mgt_layer_fwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
                          void* y, void* saved, void* workspace, void* stream);
 

@@ -21,7 +21,7 @@ PARAM_ORDER = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
 
 REGIONS = {
     "ln1": 0, "ln1_mean": 1, "ln1_rstd": 2, "qkv": 3, "attn_o": 4, "attn_lse": 5, "h1": 6,
-    "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_u": 10, "fc1_a": 11,
+    "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_dgelu": 10, "fc1_a": 11,
     "status": 64, "du": 65, "dln2": 66, "dh1": 67, "dO": 68, "dqkv": 69, "dln1": 70,
     "attn_D": 71, "dq_acc": 72, "ln_partial": 73,
 }

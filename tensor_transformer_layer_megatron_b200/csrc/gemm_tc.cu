@@ -112,46 +112,51 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
         for (int i = 0; i < count; ++i) v[i] += __bfloat162float(r[i]);
       }
     }
-    if (EPI == kEpiDGelu) {
-      const __nv_bfloat16* u =
+    if (EPI == kEpiDGelu) {  // aux holds GeLU'(u), stored by the forward epilogue
+      const __nv_bfloat16* g =
           reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col;
       if (count == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 w = *reinterpret_cast<const uint4*>(u + q * 8);
+          const uint4 w = *reinterpret_cast<const uint4*>(g + q * 8);
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            v[q * 8 + 2 * j] *= gelu_grad_f(bf16_lo(ww[j]), a.gelu_tanh);
-            v[q * 8 + 2 * j + 1] *= gelu_grad_f(bf16_hi(ww[j]), a.gelu_tanh);
+            v[q * 8 + 2 * j] *= bf16_lo(ww[j]);
+            v[q * 8 + 2 * j + 1] *= bf16_hi(ww[j]);
           }
         }
       } else {
-        for (int i = 0; i < count; ++i) v[i] *= gelu_grad_f(__bfloat162float(u[i]), a.gelu_tanh);
+        for (int i = 0; i < count; ++i) v[i] *= __bfloat162float(g[i]);
       }
     }
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + off;
-    if (EPI == kEpiGelu) {
+    if (EPI == kEpiGelu) {  // out = GeLU(u), out2 = GeLU'(u) for the backward
       __nv_bfloat16* o2 = reinterpret_cast<__nv_bfloat16*>(a.out2) + off;
       if (count == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint4 wu, wa;
-          wu.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-          wu.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-          wu.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-          wu.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-          *reinterpret_cast<uint4*>(o2 + q * 8) = wu;
-          wa.x = pack_bf16x2(gelu_f(v[q * 8 + 0], a.gelu_tanh), gelu_f(v[q * 8 + 1], a.gelu_tanh));
-          wa.y = pack_bf16x2(gelu_f(v[q * 8 + 2], a.gelu_tanh), gelu_f(v[q * 8 + 3], a.gelu_tanh));
-          wa.z = pack_bf16x2(gelu_f(v[q * 8 + 4], a.gelu_tanh), gelu_f(v[q * 8 + 5], a.gelu_tanh));
-          wa.w = pack_bf16x2(gelu_f(v[q * 8 + 6], a.gelu_tanh), gelu_f(v[q * 8 + 7], a.gelu_tanh));
+          float ga[8], gd[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) gelu_and_grad_f(v[q * 8 + j], a.gelu_tanh, ga[j], gd[j]);
+          uint4 wd, wa;
+          wd.x = pack_bf16x2(gd[0], gd[1]);
+          wd.y = pack_bf16x2(gd[2], gd[3]);
+          wd.z = pack_bf16x2(gd[4], gd[5]);
+          wd.w = pack_bf16x2(gd[6], gd[7]);
+          *reinterpret_cast<uint4*>(o2 + q * 8) = wd;
+          wa.x = pack_bf16x2(ga[0], ga[1]);
+          wa.y = pack_bf16x2(ga[2], ga[3]);
+          wa.z = pack_bf16x2(ga[4], ga[5]);
+          wa.w = pack_bf16x2(ga[6], ga[7]);
           *reinterpret_cast<uint4*>(o + q * 8) = wa;
         }
       } else {
         for (int i = 0; i < count; ++i) {
-          o2[i] = __float2bfloat16_rn(v[i]);
-          o[i] = __float2bfloat16_rn(gelu_f(v[i], a.gelu_tanh));
+          float ga, gd;
+          gelu_and_grad_f(v[i], a.gelu_tanh, ga, gd);
+          o2[i] = __float2bfloat16_rn(gd);
+          o[i] = __float2bfloat16_rn(ga);
         }
       }
       return;
@@ -401,8 +406,10 @@ template <bool A_MN, bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const GemmArgs args, int num_m2,
-                    int num_n) {
-  constexpr int BN = 256;
+                    int num_n, int BN) {
+  // BN: the pair's N tile, a multiple of 32 up to 256 (256 when B is MN-major); each CTA
+  // loads BN/2 rows of B. Accumulator buffers stay 256 columns apart in TMEM.
+  const uint32_t b_bytes = (uint32_t)(BN / 2) * BK * 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
@@ -458,14 +465,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
       const TileCoord tc = tile_coord(tile, num_m2, num_n);
       const int m0 = tc.mb * 256 + rank * 128;
-      const int n0 = tc.nb * BN + rank * 128;
+      const int n0 = tc.nb * BN + rank * (BN / 2);
       for (int kg = 0; kg < args.KG && ok; ++kg) {
         for (int kt = 0; kt < kt_per_group; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.err, kErrTimeoutProducer, abort_flag)) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairAB + b_bytes));
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kPairAB;
           uint8_t* b_dst = sB + stage * kPairAB;
@@ -504,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (leader && warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer (leader only)
-    constexpr uint32_t idesc = idesc_bf16_f32(256, BN, A_MN, B_MN);
+    const uint32_t idesc = idesc_bf16_f32(256, BN, A_MN, B_MN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -516,7 +523,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
+      const uint32_t d_tmem = tmem_base + acc * 256;
       for (int it = 0; it < k_iters; ++it) {
         if (!mbar_wait(&full[stage], phase, args.err, kErrTimeoutMma, abort_flag)) {
           ok = false;
@@ -551,7 +558,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp & 3;
-    const int c_begin = ((warp - 2) >> 2) * (BN / 64);
+    const int nch = BN / 32, half = (nch + 1) / 2;  // 32-column chunks, split over 2 warp sets
+    const int c_begin = ((warp - 2) >> 2) ? half : 0;
+    const int c_end = ((warp - 2) >> 2) ? nch : half;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -563,9 +572,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = c_begin; c < c_begin + BN / 64; ++c) {
+      for (int c = c_begin; c < c_end; ++c) {
         float v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN + c * 32,
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256 + c * 32,
                            v);
         const int n0 = tc.nb * BN + c * 32;
         if (row < args.M && n0 < args.Ng) {
@@ -665,7 +674,7 @@ cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
 
 template <bool A_MN, bool B_MN, int EPI>
 cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                             int num_sms, cudaStream_t stream) {
+                             int num_sms, int bn, cudaStream_t stream) {
   auto kern = gemm_tc2_kernel<A_MN, B_MN, EPI>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -675,31 +684,53 @@ cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const
     attr_done = true;
   }
   const int num_m2 = (a.M + 255) / 256;
-  const int num_n = (a.Ng + 255) / 256;
+  const int num_n = (a.Ng + bn - 1) / bn;
   const int tiles = a.NG * num_m2 * num_n;
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  kern<<<2 * pairs, kThreads, kPairSmem, stream>>>(ta, tb, a, num_m2, num_n);
+  kern<<<2 * pairs, kThreads, kPairSmem, stream>>>(ta, tb, a, num_m2, num_n, bn);
   return cudaGetLastError();
 }
 
 template <bool A_MN, bool B_MN>
 cudaError_t launch_pair_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                            int num_sms, cudaStream_t s) {
+                            int num_sms, int bn, cudaStream_t s) {
   switch (a.epi) {
-    case kEpiStoreF32: return launch_pair_inst<A_MN, B_MN, kEpiStoreF32>(ta, tb, a, num_sms, s);
-    case kEpiBf16: return launch_pair_inst<A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, s);
-    case kEpiGelu: return launch_pair_inst<A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, s);
-    case kEpiDGelu: return launch_pair_inst<A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, s);
+    case kEpiStoreF32:
+      return launch_pair_inst<A_MN, B_MN, kEpiStoreF32>(ta, tb, a, num_sms, bn, s);
+    case kEpiBf16: return launch_pair_inst<A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, bn, s);
+    case kEpiGelu: return launch_pair_inst<A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, bn, s);
+    case kEpiDGelu: return launch_pair_inst<A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, bn, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                        int num_sms, cudaStream_t s) {
-  if (!a.a_mn && !a.b_mn) return launch_pair_epi<false, false>(ta, tb, a, num_sms, s);
-  if (!a.a_mn && a.b_mn) return launch_pair_epi<false, true>(ta, tb, a, num_sms, s);
-  if (a.a_mn && !a.b_mn) return launch_pair_epi<true, false>(ta, tb, a, num_sms, s);
-  return launch_pair_epi<true, true>(ta, tb, a, num_sms, s);
+                        int num_sms, int bn, cudaStream_t s) {
+  if (!a.a_mn && !a.b_mn) return launch_pair_epi<false, false>(ta, tb, a, num_sms, bn, s);
+  if (!a.a_mn && a.b_mn) return launch_pair_epi<false, true>(ta, tb, a, num_sms, bn, s);
+  if (a.a_mn && !a.b_mn) return launch_pair_epi<true, false>(ta, tb, a, num_sms, bn, s);
+  return launch_pair_epi<true, true>(ta, tb, a, num_sms, bn, s);
+}
+
+// N tile of the pair kernel: the width (multiple of 32, <= 256) that minimises the number of
+// tile rounds over the pairs times the tile width (+ a fixed per-tile cost), so the last round
+// is as full as possible. MN-major B loads 64-wide chunks per CTA half, so it keeps 256.
+int pick_pair_bn(const GemmArgs& a, int num_sms) {
+  if (a.b_mn) return 256;
+  const int pairs = num_sms / 2;
+  const long long m2 = (a.M + 255) / 256;
+  int best = 256;
+  long long best_cost = -1;
+  for (int bn = 256; bn >= 128; bn -= 32) {
+    const long long tiles = (long long)a.NG * m2 * ((a.Ng + bn - 1) / bn);
+    const long long rounds = (tiles + pairs - 1) / pairs;
+    const long long cost = rounds * (bn + 48);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
 }
 
 template <int BN>
@@ -718,10 +749,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
   if (a.M <= 0 || a.Ng <= 0 || a.NG <= 0 || a.Kg <= 0 || a.KG <= 0) return cudaErrorInvalidValue;
   if ((a.a_mn && a.KG != 1) || (a.b_mn && a.KG != 1) || (!a.b_mn && a.NG != 1))
     return cudaErrorInvalidValue;
-  // Wide tiles run on CTA pairs (cta_group::2, 256 x 256 per pair); narrow N on one CTA.
+  // Wide tiles run on CTA pairs (cta_group::2, 256 x BN per pair); narrow N on one CTA.
   const bool pair = a.Ng > 128 && num_sms >= 2;
   const int BN = (a.Ng <= 128) ? 128 : 256;
-  const int b_rows = pair ? 128 : BN;  // B rows per CTA per k-step
+  const int pair_bn = pair ? pick_pair_bn(a, num_sms) : BN;
+  const int b_rows = pair ? pair_bn / 2 : BN;  // B rows per CTA per k-step
   CUtensorMap ta, tb;
   {
     uint64_t dims[3], str[2];
@@ -754,7 +786,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
     }
     if (!make_map(&tb, a.B, dims, str, box)) return cudaErrorInvalidValue;
   }
-  if (pair) return launch_pair(ta, tb, a, num_sms, stream);
+  if (pair) return launch_pair(ta, tb, a, num_sms, pair_bn, stream);
   if (BN == 128) return launch_bn<128>(ta, tb, a, num_sms, stream);
   return launch_bn<256>(ta, tb, a, num_sms, stream);
 }

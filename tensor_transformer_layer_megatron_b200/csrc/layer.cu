@@ -114,7 +114,7 @@ void layout(mgt_layer* L) {
                                    T * h * e,
                                    bHs * 4,
                                    0,
-                                   nblk * 2 * h * 4};
+                                   nblk * 3 * h * 4};
   off = 0;
   for (int i = 0; i < MGT_WS_COUNT - 64; ++i) {
     L->ws[i].off = off;
@@ -271,7 +271,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   char* ln2 = sp(saved, L->saved[MGT_SAVED_LN2]);
   float* mu2 = reinterpret_cast<float*>(sp(saved, L->saved[MGT_SAVED_LN2_MEAN]));
   float* rs2 = reinterpret_cast<float*>(sp(saved, L->saved[MGT_SAVED_LN2_RSTD]));
-  char* u = sp(saved, L->saved[MGT_SAVED_FC1_U]);
+  char* gd = sp(saved, L->saved[MGT_SAVED_FC1_DGELU]);
   char* act = sp(saved, L->saved[MGT_SAVED_FC1_A]);
   const double ln_bytes = (double)T * h * 2 * e + 8.0 * h;
 
@@ -307,11 +307,11 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     return launch_ln_fwd(dt, T, h, L->cfg.ln_eps, h1, (const float*)P->ln2_g,
                          (const float*)P->ln2_b, ln2, mu2, rs2, s);
   }));
-  // 6. fc1, column-parallel, + b1, GeLU (stores u and a)
+  // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and GeLU'(u) for the backward)
   {
     GemmArgs a = gemm_base(T, f, 1, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
-    a.epi = kEpiGelu; a.out = act; a.out2 = u; a.ldc = f; a.bias = P->b1;
+    a.epi = kEpiGelu; a.out = act; a.out2 = gd; a.ldc = f; a.bias = P->b1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   }
@@ -354,7 +354,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   const char* ln2 = sp(saved, L->saved[MGT_SAVED_LN2]);
   const float* mu2 = reinterpret_cast<const float*>(sp(saved, L->saved[MGT_SAVED_LN2_MEAN]));
   const float* rs2 = reinterpret_cast<const float*>(sp(saved, L->saved[MGT_SAVED_LN2_RSTD]));
-  const char* u = sp(saved, L->saved[MGT_SAVED_FC1_U]);
+  const char* gd = sp(saved, L->saved[MGT_SAVED_FC1_DGELU]);
   const char* act = sp(saved, L->saved[MGT_SAVED_FC1_A]);
   char* du = sp(workspace, L->ws[MGT_WS_DU - 64]);
   char* dln2 = sp(workspace, L->ws[MGT_WS_DLN2 - 64]);
@@ -369,15 +369,14 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, s,
                [&] { return launch_colsum(dt, T, cols, src, (float*)out, s); });
   };
-  const double lnb_bytes = (double)T * h * 4 * e + 2.0 * nblk * h * 4 * 2;
+  const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
 
-  // B1. fc2: db2, dgrad fused with GeLU' -> du, wgrad
-  MGT_TRY(colsum(dy, h, G->b2));
+  // B1. fc2: dgrad fused with GeLU' -> du, wgrad (db2 = sum dy comes with the LN2 backward)
   {
     GemmArgs a = gemm_base(T, f / p, p, h, 1);  // N grouped by shard
     a.b_mn = 1; a.A = dy; a.lda = h; a.B = P->w2; a.ldb = f / p;
     a.b_ngs = (long long)h * (f / p);
-    a.epi = kEpiDGelu; a.out = du; a.ldc = f; a.aux = u; a.ld_aux = f;
+    a.epi = kEpiDGelu; a.out = du; a.ldc = f; a.aux = gd; a.ld_aux = f;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc2_dgrad", a, s));
   }
@@ -404,11 +403,11 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   }
   // B4. LN2 backward + residual gradient dy -> dh1
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
+    // dres = dy, so the residual-gradient sum it also returns is db2
     return launch_ln_bwd(dt, T, h, dln2, dy, h1, (const float*)P->ln2_g, mu2, rs2, dh1, part,
-                         nblk, (float*)G->ln2_g, (float*)G->ln2_b, s);
+                         nblk, (float*)G->ln2_g, (float*)G->ln2_b, (float*)G->b2, s);
   }));
-  // B5. out-proj: db_o, dgrad (N grouped by shard) -> dO, wgrad
-  MGT_TRY(colsum(dh1, h, G->b_o));
+  // B5. out-proj: dgrad (N grouped by shard) -> dO, wgrad (db_o = sum dh1 comes with LN1 bwd)
   {
     GemmArgs a = gemm_base(T, h / p, p, h, 1);
     a.b_mn = 1; a.A = dh1; a.lda = h; a.B = P->w_o; a.ldb = h / p;
@@ -446,8 +445,9 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   }
   // B8. LN1 backward + residual gradient dh1 -> dx
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
+    // dres = dh1, so the residual-gradient sum it also returns is db_o
     return launch_ln_bwd(dt, T, h, dln1, dh1, x, (const float*)P->ln1_g, mu1, rs1, dx, part,
-                         nblk, (float*)G->ln1_g, (float*)G->ln1_b, s);
+                         nblk, (float*)G->ln1_g, (float*)G->ln1_b, (float*)G->b_o, s);
   }));
   return MGT_OK;
 }

@@ -48,6 +48,17 @@ struct Vec<float> {
   }
 };
 
+// V consecutive fp32 parameters (gamma or beta) with 16-byte loads; the column index is a
+// multiple of V, so the address is 16-byte aligned.
+template <int V>
+__device__ __forceinline__ void load_param(const float* __restrict__ p, int c, float (&v)[V]) {
+#pragma unroll
+  for (int j = 0; j < V; j += 4) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(p + c + j));
+    v[j] = w.x; v[j + 1] = w.y; v[j + 2] = w.z; v[j + 3] = w.w;
+  }
+}
+
 // ---------------------------------------------------------------------------- row groups
 // A row is owned by a group of W warps (W*32 threads); a 256-thread CTA holds 8/W groups. Sums
 // over the row are warp shuffles, then (W > 1) a named barrier private to the group, so groups
@@ -121,12 +132,11 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(long long rows, int h, floa
   for (int i = 0; i < VPL; ++i) {
     const int vi = t + i * GT;
     if (vi < nvec) {
-      float o[V];
+      float o[V], gv[V], bv[V];
+      load_param<V>(gamma, vi * V, gv);
+      load_param<V>(beta, vi * V, bv);
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const int c = vi * V + j;
-        o[j] = (v[i][j] - mu) * rs * __ldg(gamma + c) + __ldg(beta + c);
-      }
+      for (int j = 0; j < V; ++j) o[j] = (v[i][j] - mu) * rs * gv[j] + bv[j];
       Vec<T>::store(yr + vi * V, o);
     }
   }
@@ -163,13 +173,14 @@ __global__ void __launch_bounds__(256) ln_bwd_dx_kernel(long long rows, int h,
   for (int i = 0; i < VPL; ++i) {
     const int vi = t + i * GT;
     if (valid && vi < nvec) {
-      float xv[V], dv[V];
+      float xv[V], dv[V], gv[V];
       Vec<T>::load(x + r * h + vi * V, xv);
       Vec<T>::load(dy + r * h + vi * V, dv);
+      load_param<V>(gamma, vi * V, gv);
 #pragma unroll
       for (int j = 0; j < V; ++j) {
         xh[i][j] = (xv[j] - mu) * rs;
-        g[i][j] = dv[j] * __ldg(gamma + vi * V + j);
+        g[i][j] = dv[j] * gv[j];
         s1 += g[i][j];
         s2 += g[i][j] * xh[i][j];
       }
@@ -196,25 +207,28 @@ __global__ void __launch_bounds__(256) ln_bwd_dx_kernel(long long rows, int h,
   }
 }
 
-// Partial dgamma = sum dy*xhat and dbeta = sum dy over one slice of rows. Block = 32 x 8
-// threads covering 32*VEC columns; blockIdx.y is the slice; the 8 row lanes are combined in
-// shared memory and written to partial[slice][2][h] (no atomics: deterministic).
-template <typename T>
+// Partial dgamma = sum dy*xhat and dbeta = sum dy over one slice of rows, and with NSUM = 3 also
+// sum dres (the residual gradient: a bias gradient of the layer for free, as the LayerNorm
+// backward reads it anyway). Block = 32 x 8 threads covering 32*VEC columns; blockIdx.y is the
+// slice; the 8 row lanes are combined in shared memory and written to partial[slice][NSUM][h]
+// (no atomics: deterministic).
+template <typename T, int NSUM>
 __global__ void __launch_bounds__(256) ln_bwd_param_kernel(long long rows, int h,
                                                            const T* __restrict__ dy,
                                                            const T* __restrict__ x,
+                                                           const T* __restrict__ dres,
                                                            const float* __restrict__ mean,
                                                            const float* __restrict__ rstd,
                                                            float* __restrict__ partial,
                                                            long long rows_per) {
   constexpr int V = Vec<T>::N;
-  __shared__ float red[2][8][32 * V + 1];
+  __shared__ float red[NSUM][8][32 * V + 1];
   const int c0 = (blockIdx.x * 32 + threadIdx.x) * V;
   const long long r0 = blockIdx.y * rows_per;
   const long long r1 = min(rows, r0 + rows_per);
-  float ag[V], ab[V];
+  float ag[V], ab[V], ar[V];
 #pragma unroll
-  for (int j = 0; j < V; ++j) ag[j] = ab[j] = 0.f;
+  for (int j = 0; j < V; ++j) ag[j] = ab[j] = ar[j] = 0.f;
   if (c0 < h) {
     long long r = r0 + threadIdx.y;
     for (; r + 8 < r1; r += 16) {  // two independent rows in flight per thread
@@ -229,6 +243,13 @@ __global__ void __launch_bounds__(256) ln_bwd_param_kernel(long long rows, int h
         ag[j] += d0[j] * ((x0[j] - mu0) * rs0) + d1[j] * ((x1[j] - mu1) * rs1);
         ab[j] += d0[j] + d1[j];
       }
+      if constexpr (NSUM == 3) {
+        float e0[V], e1[V];
+        Vec<T>::load(dres + r * h + c0, e0);
+        Vec<T>::load(dres + (r + 8) * h + c0, e1);
+#pragma unroll
+        for (int j = 0; j < V; ++j) ar[j] += e0[j] + e1[j];
+      }
     }
     for (; r < r1; r += 8) {
       float x0[V], d0[V];
@@ -240,17 +261,24 @@ __global__ void __launch_bounds__(256) ln_bwd_param_kernel(long long rows, int h
         ag[j] += d0[j] * ((x0[j] - mu0) * rs0);
         ab[j] += d0[j];
       }
+      if constexpr (NSUM == 3) {
+        float e0[V];
+        Vec<T>::load(dres + r * h + c0, e0);
+#pragma unroll
+        for (int j = 0; j < V; ++j) ar[j] += e0[j];
+      }
     }
   }
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     red[0][threadIdx.y][threadIdx.x * V + j] = ag[j];
     red[1][threadIdx.y][threadIdx.x * V + j] = ab[j];
+    if constexpr (NSUM == 3) red[2][threadIdx.y][threadIdx.x * V + j] = ar[j];
   }
   __syncthreads();
-  float* pg = partial + (long long)blockIdx.y * 2 * h;
+  float* pg = partial + (long long)blockIdx.y * NSUM * h;
   const int t = threadIdx.y * 32 + threadIdx.x;
-  for (int cc = t; cc < 2 * 32 * V; cc += 256) {
+  for (int cc = t; cc < NSUM * 32 * V; cc += 256) {
     const int which = cc / (32 * V), cl = cc % (32 * V);
     const int col = blockIdx.x * 32 * V + cl;
     if (col < h) {
@@ -262,28 +290,28 @@ __global__ void __launch_bounds__(256) ln_bwd_param_kernel(long long rows, int h
   }
 }
 
-// dgamma[c] = sum_b partial[b][0][c]; dbeta[c] = sum_b partial[b][1][c]. Block = 32 columns x
-// 8 slices of the partial rows; fixed summation order.
-__global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk,
+// dgamma[c] = sum_b partial[b][0][c], dbeta[c] = sum_b partial[b][1][c] and, when the partials
+// carry a third row, dres_sum[c] = sum_b partial[b][2][c]. Block = 32 columns x 8 slices of the
+// partial rows; fixed summation order.
+__global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, int nsum,
                                                               const float* __restrict__ partial,
                                                               float* __restrict__ dgamma,
-                                                              float* __restrict__ dbeta) {
+                                                              float* __restrict__ dbeta,
+                                                              float* __restrict__ dres_sum) {
   __shared__ float red[8][33];
   const int c = blockIdx.x * 32 + (threadIdx.x & 31);
   const int sl = threadIdx.x >> 5;
   float s = 0.f;
-  if (c < 2 * h)
-    for (int b = sl; b < nblk; b += 8) s += partial[(long long)b * 2 * h + c];
+  if (c < nsum * h)
+    for (int b = sl; b < nblk; b += 8) s += partial[(long long)b * nsum * h + c];
   red[sl][threadIdx.x & 31] = s;
   __syncthreads();
-  if (sl == 0 && c < 2 * h) {
+  if (sl == 0 && c < nsum * h) {
     float tot = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) tot += red[k][threadIdx.x & 31];
-    if (c < h)
-      dgamma[c] = tot;
-    else
-      dbeta[c - h] = tot;
+    float* out = c < h ? dgamma : (c < 2 * h ? dbeta : dres_sum);
+    out[c % h] = tot;
   }
 }
 
@@ -372,13 +400,14 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
     }
     case kEpiGelu: {
       if (bias) acc += bias[col];
-      reinterpret_cast<float*>(a.out2)[off] = acc;
-      out[off] = gelu_f(acc, a.gelu_tanh);
+      float g, dg;
+      gelu_and_grad_f(acc, a.gelu_tanh, g, dg);
+      reinterpret_cast<float*>(a.out2)[off] = dg;
+      out[off] = g;
       break;
     }
     case kEpiDGelu: {
-      const float u = reinterpret_cast<const float*>(a.aux)[(long long)m * a.ld_aux + col];
-      out[off] = acc * gelu_grad_f(u, a.gelu_tanh);
+      out[off] = acc * reinterpret_cast<const float*>(a.aux)[(long long)m * a.ld_aux + col];
       break;
     }
   }
@@ -422,7 +451,7 @@ template <typename T>
 cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* dres,
                             const void* x, const float* g, const float* mean, const float* rstd,
                             void* dx, float* partial, int nblk, float* dgamma, float* dbeta,
-                            cudaStream_t s) {
+                            float* dres_sum, cudaStream_t s) {
   const int nvec = h / Vec<T>::N;
   cudaError_t e;
   if (nvec <= 64)
@@ -446,12 +475,18 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
   if (slices < 1) slices = 1;
   const long long rows_per = (rows + slices - 1) / slices;
   slices = (rows + rows_per - 1) / rows_per;
-  ln_bwd_param_kernel<T><<<dim3(cb, (unsigned)slices), dim3(32, 8), 0, s>>>(
-      rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x), mean, rstd,
-      partial, rows_per);
+  const int nsum = (dres_sum && dres) ? 3 : 2;
+  if (nsum == 3)
+    ln_bwd_param_kernel<T, 3><<<dim3(cb, (unsigned)slices), dim3(32, 8), 0, s>>>(
+        rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x),
+        reinterpret_cast<const T*>(dres), mean, rstd, partial, rows_per);
+  else
+    ln_bwd_param_kernel<T, 2><<<dim3(cb, (unsigned)slices), dim3(32, 8), 0, s>>>(
+        rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x), nullptr, mean,
+        rstd, partial, rows_per);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ln_param_reduce_kernel<<<(2 * h + 31) / 32, 256, 0, s>>>(h, (int)slices, partial, dgamma,
-                                                          dbeta);
+  ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
+                                                             dgamma, dbeta, dres_sum);
   return cudaGetLastError();
 }
 
@@ -474,12 +509,12 @@ int ln_bwd_blocks(long long rows, int num_sms) {
 cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, const void* dres,
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk, float* dgamma,
-                          float* dbeta, cudaStream_t s) {
+                          float* dbeta, float* dres_sum, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   return dtype ? ln_bwd_dispatch<__nv_bfloat16>(rows, h, dy, dres, x, gamma, mean, rstd, dx,
-                                                partial, nblk, dgamma, dbeta, s)
+                                                partial, nblk, dgamma, dbeta, dres_sum, s)
                : ln_bwd_dispatch<float>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial,
-                                        nblk, dgamma, dbeta, s);
+                                        nblk, dgamma, dbeta, dres_sum, s);
 }
 
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,

@@ -324,6 +324,19 @@ __device__ __forceinline__ float gelu_f(float u, int tanh_form) {
   }
   return 0.5f * u * (1.0f + erff(u * 0.7071067811865476f));
 }
+// GeLU(u) and GeLU'(u) together (the erf / tanh is shared).
+__device__ __forceinline__ void gelu_and_grad_f(float u, int tanh_form, float& g, float& dg) {
+  if (tanh_form) {
+    const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);
+    const float t = tanhf(z);
+    g = 0.5f * u * (1.0f + t);
+    dg = 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * 0.7978845608028654f * (1.0f + 0.134145f * u * u);
+    return;
+  }
+  const float cdf = 0.5f * (1.0f + erff(u * 0.7071067811865476f));
+  g = u * cdf;
+  dg = cdf + u * 0.3989422804014327f * expf(-0.5f * u * u);
+}
 __device__ __forceinline__ float gelu_grad_f(float u, int tanh_form) {
   if (tanh_form) {
     const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);

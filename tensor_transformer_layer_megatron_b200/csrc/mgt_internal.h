@@ -20,8 +20,8 @@ enum DeviceError : int {
 enum Epilogue : int {
   kEpiStoreF32 = 0,  // out (fp32) = acc                     (weight gradients)
   kEpiBf16 = 1,      // out (act) = acc [+ bias] [+ residual] (QKV, out-proj, fc2, dgrads)
-  kEpiGelu = 2,      // u = acc + bias -> out2; out = GeLU(u) (fc1)
-  kEpiDGelu = 3,     // out = acc * GeLU'(aux)                (fc2 dgrad -> du)
+  kEpiGelu = 2,      // u = acc + bias; out = GeLU(u), out2 = GeLU'(u) (fc1)
+  kEpiDGelu = 3,     // out = acc * aux, aux = GeLU'(u)        (fc2 dgrad -> du)
 };
 
 // One GEMM  C[m, col] = sum_{kg < KG} sum_{kk < Kg} A(m, kg, kk) * B(ng, n, kg, kk)
@@ -41,10 +41,10 @@ struct GemmArgs {
   // Epilogue.
   int epi;
   void* out; long long ldc; int out_ng; long long out_gs;
-  void* out2;                           // kEpiGelu: pre-activation u (same addressing as out)
+  void* out2;                           // kEpiGelu: GeLU'(u) (same addressing as out)
   const void* bias;                     // indexed by col; nullable
   const void* res; long long ldr;       // residual, res[m*ldr + col]; nullable
-  const void* aux; long long ld_aux;    // kEpiDGelu: u[m*ld_aux + col]
+  const void* aux; long long ld_aux;    // kEpiDGelu: GeLU'(u)[m*ld_aux + col]
   int gelu_tanh;
   int* err;                             // device status word
 };
@@ -64,13 +64,14 @@ cudaError_t launch_gemm_simt_f32(const GemmArgs& args, cudaStream_t stream);
 cudaError_t launch_ln_fwd(int dtype, long long rows, int h, float eps, const void* x,
                           const float* gamma, const float* beta, void* y, float* mean,
                           float* rstd, cudaStream_t stream);
-// dx = dres + LN'^T(dy); per-block partial dgamma/dbeta into `partial` [nblk][2][h], then a
-// second kernel reduces them into dgamma/dbeta. Returns the number of blocks used in *nblk.
+// dx = dres + LN'^T(dy); dgamma, dbeta and (if dres_sum and dres are given) dres_sum =
+// sum over rows of dres, through per-slice partials in `partial`, which must hold
+// nblk * (dres_sum ? 3 : 2) * h floats; at most nblk slices are used.
 int ln_bwd_blocks(long long rows, int num_sms);
 cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, const void* dres,
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk,
-                          float* dgamma, float* dbeta, cudaStream_t stream);
+                          float* dgamma, float* dbeta, float* dres_sum, cudaStream_t stream);
 
 // Column sums of a [rows, cols] activation matrix into fp32 (bias gradients).
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,

@@ -53,7 +53,7 @@ def gpu_intermediates(cfg, layer, run):
         lse=v(run.saved, "attn_lse", torch.float32, (cfg.micro_batch, H, cfg.seq)),
         h1=v(run.saved, "h1", act, (T, h)),
         ln2=v(run.saved, "ln2", act, (T, h)),
-        u=v(run.saved, "fc1_u", act, (T, p, f // p)),
+        gelu_grad=v(run.saved, "fc1_dgelu", act, (T, p, f // p)),
         a=v(run.saved, "fc1_a", act, (T, p, f // p)),
         du=v(run.ws, "du", act, (T, p, f // p)),
         dln2=v(run.ws, "dln2", act, (T, h)),
@@ -78,7 +78,8 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
     if intermediates:
         gi = gpu_intermediates(cfg, layer, run)
         ref = dict(ln1=saved["ln1"], qkv=saved["qkv"], O=saved["O"], lse=saved["lse"],
-                   h1=saved["h1"], ln2=saved["ln2"], u=saved["u"], a=saved["a"], **inter)
+                   h1=saved["h1"], ln2=saved["ln2"], a=saved["a"],
+                   gelu_grad=oracle.gelu_grad(saved["u"], cfg.gelu_tanh), **inter)
         for k in gi:
             errs[k] = rel_err(gi[k], ref[k])
     return errs

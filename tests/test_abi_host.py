@@ -88,7 +88,7 @@ def test_region_layout(cfg):
     saved, ws = L.sizes()
     T, h, f, e = cfg.tokens, cfg.hidden, cfg.ffn, 2 if cfg.dtype == "bf16" else 4
     expect = {"ln1": T * h * e, "qkv": 3 * T * h * e, "attn_o": T * h * e,
-              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_u": T * f * e,
+              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_dgelu": T * f * e,
               "fc1_a": T * f * e, "du": T * f * e, "dqkv": 3 * T * h * e}
     spans = []
     for name, rid in mgt.REGIONS.items():

@@ -13,8 +13,9 @@ def ceil8(v):
     return (v + 7) // 8 * 8
 
 
+# (2048, 12288, 64) selects the 224-wide pair tile for K-major B, the others 128 or 256.
 SHAPES = [(128, 256, 64), (200, 300, 136), (1, 8, 8), (1000, 520, 1000), (256, 384, 4096),
-          (129, 129, 72)]
+          (129, 129, 72), (2048, 12288, 64)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
