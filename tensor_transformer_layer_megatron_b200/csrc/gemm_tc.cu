@@ -18,6 +18,7 @@
 // the epilogue of tile i overlaps the main loop of tile i+1.
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "mgt_device.cuh"
@@ -400,13 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairStages = 6;
 constexpr int kPairAB = BM * BK * 2;            // 16 KB: this CTA's A rows or B half
 constexpr int kPairStageBytes = 2 * kPairAB;    // 32 KB per CTA per stage
-constexpr int kPairSmem = kPairStages * kPairStageBytes + 256 + 1024;
+constexpr int kStageOut = 32 * 32 * 4;          // fp32 store staging: 32 rows x 32 columns
+// stages | barriers (padded to 1 KB) | fp32 staging (fp32 epilogue only) | 1 KB alignment slack
+constexpr int pair_smem(int epi) {
+  return kPairStages * kPairStageBytes + 1024 + (epi == kEpiStoreF32 ? kEpiWarps * kStageOut : 0) +
+         1024;
+}
+static_assert(pair_smem(kEpiStoreF32) <= 232448, "shared memory per CTA");
 
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args, int num_m2,
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const GemmArgs args, int num_m2,
                     int num_n, int BN) {
+  // tmC (fp32 epilogue only): output viewed as {out_ng, M, groups}; each epilogue warp stages
+  // a 32 x 32 fp32 chunk in a 128B-swizzled shared buffer and stores it with one TMA bulk
+  // tensor store (coalesced full lines; rows past M and columns past N are clipped).
   // BN: the pair's N tile, a multiple of 32 up to 256 (256 when B is MN-major); each CTA
   // loads BN/2 rows of B. Accumulator buffers stay 256 columns apart in TMEM.
   const uint32_t b_bytes = (uint32_t)(BN / 2) * BK * 2;
@@ -422,6 +433,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* stage_out = smem + kPairStages * kPairStageBytes + 1024;  // 1024-aligned
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -446,6 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI == kEpiStoreF32) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -577,7 +590,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256 + c * 32,
                            v);
         const int n0 = tc.nb * BN + c * 32;
-        if (row < args.M && n0 < args.Ng) {
+        if constexpr (EPI == kEpiStoreF32) {
+          const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
+          // Whole chunks go through TMA; a chunk straddling N is written element by element
+          // (the bulk store clips the inner dimension only at 16-byte granularity).
+          if (n0 < args.Ng && n0 + 32 > args.Ng) {
+            if (row < args.M) epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, args.Ng - n0, v);
+          } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
+            uint8_t* buf = stage_out + (warp - 2) * kStageOut;
+            if (lane == 0) bulk_wait_read0();  // the previous chunk's store has read the buffer
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const int col = tc.ng * args.Ng + n0;
+              tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
+              bulk_commit();
+            }
+          }
+        } else if (row < args.M && n0 < args.Ng) {
           const int count = min(32, args.Ng - n0);
           epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, count, v);
         }
@@ -592,6 +627,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (EPI == kEpiStoreF32 && warp >= 2 && lane == 0) bulk_wait0();
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while its peer may still touch its barriers or TMEM
@@ -672,22 +708,43 @@ cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
   return cudaErrorInvalidValue;
 }
 
+// fp32 output viewed as {out_ng, M, groups} with a 32 x 32 box (128-byte rows, swizzled).
+bool make_out_map_f32(CUtensorMap* m, const GemmArgs& a) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const long long ncols = (long long)a.Ng * a.NG;
+  const long long groups = (ncols + a.out_ng - 1) / a.out_ng;
+  cuuint64_t gd[3] = {(cuuint64_t)(ncols < a.out_ng ? ncols : a.out_ng), (cuuint64_t)a.M,
+                      (cuuint64_t)groups};
+  cuuint64_t gs[2] = {(cuuint64_t)a.ldc * 4,
+                      (cuuint64_t)(groups > 1 ? a.out_gs : a.ldc * a.M) * 4};
+  cuuint32_t bd[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.out, gd, gs, bd, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool A_MN, bool B_MN, int EPI>
 cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                              int num_sms, int bn, cudaStream_t stream) {
   auto kern = gemm_tc2_kernel<A_MN, B_MN, EPI>;
+  constexpr int smem_bytes = pair_smem(EPI);
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
+  CUtensorMap tc;
+  std::memset(&tc, 0, sizeof(tc));
+  if (EPI == kEpiStoreF32 && !make_out_map_f32(&tc, a)) return cudaErrorInvalidValue;
   const int num_m2 = (a.M + 255) / 256;
   const int num_n = (a.Ng + bn - 1) / bn;
   const int tiles = a.NG * num_m2 * num_n;
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  kern<<<2 * pairs, kThreads, kPairSmem, stream>>>(ta, tb, a, num_m2, num_n, bn);
+  kern<<<2 * pairs, kThreads, smem_bytes, stream>>>(ta, tb, tc, a, num_m2, num_n, bn);
   return cudaGetLastError();
 }
 
