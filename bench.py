@@ -138,25 +138,46 @@ def run_mgt(args):
     run.check()
     torch.cuda.synchronize()
 
-    # ---- timed region: device events, per-kernel events inside the C ABI
-    layer.profile(True)
-    layer.profile_read()  # reset totals
+    # ---- timed region. With --graph (default) one step (fwd + bwd, 26 kernel launches through
+    # the C ABI) is captured once into a CUDA graph and replayed K times; otherwise the C ABI is
+    # called eagerly. Per-kernel CUDA events are recorded by the C ABI around every launch of
+    # the eager steps (in graph mode: an eager pass of K steps right after the timed replays).
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            run.step()
+        graph.replay()
+        torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
+    if not args.graph:
+        layer.profile(True)
+        layer.profile_read()  # reset totals
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        run.step()
+        if graph is not None:
+            graph.replay()
+        else:
+            run.step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    if args.graph:  # per-kernel breakdown from an eager pass of the same K steps
+        layer.profile(True)
+        layer.profile_read()
+        for _ in range(args.steps):
+            run.step()
+        torch.cuda.synchronize()
     prof = layer.profile_read()
     layer.profile(False)
     run.check()
+    del graph
     if world > 1:
         tt = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
@@ -261,6 +282,11 @@ def run_mgt(args):
                     "what": "x, dy pinned host -> device; fwd+bwd via the C ABI; y, dx -> host"},
             "roofline": roof,
             "kernels": kernels,
+            "kernels_timing": ("CUDA events around every launch, eager pass of the same K steps "
+                               "right after the timed graph replays" if args.graph else
+                               "CUDA events around every launch inside the timed region"),
+            "timed_region": ("CUDA-graph replay of the step (fwd+bwd through the C ABI)"
+                             if args.graph else "eager C-ABI calls"),
             "gemm_sites": gemm_sites,
             "gpu_launches": launches,
             "clocks": clk,
@@ -328,6 +354,10 @@ def main():
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="time CUDA-graph replays of the step (default)")
+    ap.add_argument("--eager", dest="graph", action="store_false",
+                    help="time eager C-ABI calls instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -25,7 +25,6 @@
 namespace mgt {
 namespace {
 
-constexpr int kAttnThreads = 192;
 constexpr float kLog2eF = 1.4426950408889634f;
 constexpr float kLn2F = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -39,9 +38,14 @@ struct FwdLayout {
   static constexpr int V_OFF = K_OFF + 2 * TILE; // 2 stages
   static constexpr int P_OFF = V_OFF + 2 * TILE; // [128 q][128 keys] bf16, 2 chunks
   static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
-  static constexpr int BYTES = BAR_OFF + 256 + 1024;
+  static constexpr int RED_OFF = BAR_OFF + 256;  // float [3][2 halves][128 rows]: max x2, sum
+  static constexpr int BYTES = RED_OFF + 3 * 2 * 128 * 4 + 1024;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
 };
+
+// Every attention CTA: warps 0-7 do the elementwise work on TMEM rows (warp w: TMEM lane
+// quarter w%4, column half w/4), warp 8 is the TMA producer, warp 9 owns TMEM and issues MMAs.
+constexpr int kFwdThreads = 320;
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
@@ -51,7 +55,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a,
                        float scale_log2) {
   using L = FwdLayout<D>;
@@ -61,12 +65,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* k_empty = bars + 5;   // [2]: released as soon as S of that block has read K
   uint64_t* s_full = bars + 7;    // [2]
   uint64_t* p_full = bars + 9;
   uint64_t* pv_done = bars + 10;
   uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* v_empty = bars + 12;  // [2]: released once PV of that block has read V
+  uint64_t* xchg = bars + 14;     // [4 quarters][2 parities]: row-max exchange of a warp pair
+  uint64_t* xsum = bars + 22;     // [4 quarters]: final row-sum exchange
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -82,17 +89,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
     }
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&xchg[i], 64);
+    for (int i = 0; i < 4; ++i) mbar_init(&xsum[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -101,38 +111,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
       mbar_arrive_expect_tx(q_full, L::TILE);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c)
         tma_load_3d(&tm, q_full, smem + L::Q_OFF + c * 16384, col_q + c * 64, qb * 128, b);
-      int issued = 0;
+      int issued_k = 0, issued_v = 0;
       for (int kb = 0; kb < nkv; ++kb) {
         const int st = kb & 1;
-        if (!mbar_wait(&kv_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+        if (!mbar_wait(&k_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
           break;
         mbar_arrive_expect_tx(&k_full[st], L::TILE);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c)
           tma_load_3d(&tm, &k_full[st], smem + L::K_OFF + st * L::TILE + c * 16384,
                       col_k + c * 64, kb * 128, b);
+        issued_k = kb + 1;
+        if (!mbar_wait(&v_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
         mbar_arrive_expect_tx(&v_full[st], L::TILE);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c)
           tma_load_3d(&tm, &v_full[st], smem + L::V_OFF + st * L::TILE + c * 16384,
                       col_v + c * 64, kb * 128, b);
-        issued = kb + 1;
+        issued_v = kb + 1;
       }
       // every issued load lands before the CTA can exit
       mbar_wait(q_full, 0, a.err, kErrTimeoutDrain, nullptr);
-      for (int kb = issued - 2 < 0 ? 0 : issued - 2; kb < issued; ++kb) {
+      for (int kb = issued_k - 2 < 0 ? 0 : issued_k - 2; kb < issued_k; ++kb)
         mbar_wait(&k_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+      for (int kb = issued_v - 2 < 0 ? 0 : issued_v - 2; kb < issued_v; ++kb)
         mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
-      }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
@@ -154,6 +167,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[st]);
+        tc_commit(&k_empty[st]);  // K is free once this S has been computed
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -172,17 +186,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      (kb > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(pv_done);
-        tc_commit(&kv_empty[kb & 1]);
+        tc_commit(&v_empty[kb & 1]);
       }
       tc_commit(drain);
       mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
-    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int quarter = warp & 3, hf = warp >> 2;  // TMEM lane quarter, key-column half
+    const int r = quarter * 32 + lane;             // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t p_addr = smem_u32(smem + L::P_OFF);
-    float m_run = -INFINITY, l_run = 0.f;
+    float* red = reinterpret_cast<float*>(smem + L::RED_OFF);  // [3][2][128]
+    float m_run = -INFINITY, l_part = 0.f;
     bool ok = true;
     for (int kb = 0; kb < nkv; ++kb) {
       const int st = kb & 1;
@@ -192,33 +208,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[128];
+      float sv[64];
+      {
+        uint32_t raw[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float tmp[32];
-        tmem_ld_32x32b_x32(lane_base + (st ? L::TMEM_S1 : L::TMEM_S0) + c * 32, tmp);
+        for (int c = 0; c < 2; ++c)
+          tmem_ld_32x32b_x32_nw(lane_base + (st ? L::TMEM_S1 : L::TMEM_S0) + hf * 64 + c * 32,
+                                raw[c]);
+        tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = tmp[i];
+        for (int c = 0; c < 2; ++c) {
+          reg_fence(raw[c]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[c][i]);
+        }
       }
-      float mx = -INFINITY;
+      if (kb == qb) {  // diagonal block: keys after this query are masked
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float v = sv[i] * scale_log2;
-        if (kb == qb && i > r) v = -INFINITY;  // causal mask on the diagonal block
-        sv[i] = v;
-        mx = fmaxf(mx, v);
+        for (int i = 0; i < 64; ++i)
+          if (hf * 64 + i > r) sv[i] = -INFINITY;
       }
-      const bool need = mx > m_run + kRescaleThreshold;
-      const float alpha = need ? exp2f(m_run - mx) : 1.f;
+      // row max over both halves (raw scores; the scale is positive)
+      float mx = sv[0];
+#pragma unroll
+      for (int i = 1; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+      // exchange with the other half's warp (same rows) through a bounded mbarrier wait
+      red[(st * 2 + hf) * 128 + r] = mx;
+      mbar_arrive(&xchg[quarter * 2 + st]);
+      ok = mbar_wait(&xchg[quarter * 2 + st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, red[(st * 2 + (hf ^ 1)) * 128 + r]) * scale_log2;
+      const bool need = mx > m_run + kRescaleThreshold;  // identical in both halves
+      const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
       float rs = 0.f;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const float p = exp2f(sv[i] - m_run);
+      for (int i = 0; i < 64; ++i) {
+        const float p = ex2_approx(fmaf(sv[i], scale_log2, -m_run));
         sv[i] = p;
         rs += p;
       }
-      l_run = l_run * alpha + rs;
+      l_part = l_part * alpha + rs;
       if (kb > 0) {
         // PV of the previous block must be done before O is rescaled or P overwritten.
         ok = mbar_wait(pv_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
@@ -227,31 +260,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        if (__any_sync(0xffffffffu, need)) {  // this half rescales its half of O
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             float o[32];
-            tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+            const uint32_t ta = lane_base + L::TMEM_O + hf * (D / 2) + c * 32;
+            tmem_ld_32x32b_x32(ta, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+            tmem_st_32x32b_x32(ta, o);
           }
         }
       }
-      // P (bf16) -> shared memory, K-major 128B-swizzled: row r, 16-byte chunk c16
+      // P (bf16) -> shared memory, K-major 128B-swizzled: this half owns one 64-key atom
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        const uint32_t addr = p_addr + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(sv[c16 * 8 + 0], sv[c16 * 8 + 1]),
-                     pack_bf16x2(sv[c16 * 8 + 2], sv[c16 * 8 + 3]),
-                     pack_bf16x2(sv[c16 * 8 + 4], sv[c16 * 8 + 5]),
-                     pack_bf16x2(sv[c16 * 8 + 6], sv[c16 * 8 + 7]));
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t addr = p_addr + hf * 16384 + r * 128 + ((j ^ (r & 7)) << 4);
+        st_shared_v4(addr, pack_bf16x2(sv[j * 8 + 0], sv[j * 8 + 1]),
+                     pack_bf16x2(sv[j * 8 + 2], sv[j * 8 + 3]),
+                     pack_bf16x2(sv[j * 8 + 4], sv[j * 8 + 5]),
+                     pack_bf16x2(sv[j * 8 + 6], sv[j * 8 + 7]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // combine the two halves' row sums (own slot: the max slots may still be read)
+    if (ok) {
+      red[(4 + hf) * 128 + r] = l_part;
+      mbar_arrive(&xsum[quarter]);
+      ok = mbar_wait(&xsum[quarter], 0, a.err, kErrTimeoutAttn, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    const float l_run = ok ? l_part + red[(4 + (hf ^ 1)) * 128 + r] : 1.f;
     if (ok) {
       ok = mbar_wait(pv_done, (nkv - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
@@ -259,11 +301,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int qrow = qb * 128 + r;
         const float inv = 1.f / l_run;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                              ((long long)b * S + qrow) * H * D + (long long)n * D;
+                              ((long long)b * S + qrow) * H * D + (long long)n * D + hf * (D / 2);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           float o[32];
-          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + hf * (D / 2) + c * 32, o);
           if (qrow < S) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -276,14 +318,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
           }
         }
-        if (qrow < S) a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
+        if (qrow < S && hf == 0)
+          a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -314,10 +357,12 @@ struct BwdLayout {
   static constexpr int B_BAR = 6 * TILE;
   static constexpr int B_BYTES = B_BAR + 256 + 1024;
   static constexpr int T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+  // dQ kernel: two S buffers so the next block's S overlaps this block's dS computation.
+  static constexpr int Q_S0 = 0, Q_S1 = 128, Q_DP = 256, Q_DQ = 384;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                             const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
                             float scale_log2, float scale) {
@@ -332,7 +377,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* p_full = bars + 6;
   uint64_t* mm_done = bars + 7;
   uint64_t* drain = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* stat_bar = bars + 9;  // [2]: per-query stats of a block staged by the 4 warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* lse_s = reinterpret_cast<float*>(smem + L::A_STAT);  // [2][128], log2 units
   float* dsum_s = lse_s + 256;                                 // [2][128]
@@ -352,15 +398,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&q_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(mm_done, 1);
     mbar_init(drain, 1);
+    mbar_init(&stat_bar[0], 256);
+    mbar_init(&stat_bar[1], 256);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -369,7 +417,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
@@ -397,7 +445,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int it = issued - 2 < 0 ? 0 : issued - 2; it < issued; ++it)
         mbar_wait(&q_full[it & 1], (it >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
@@ -444,19 +492,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ P^T, dS^T and the output
-    const int r = warp * 32 + lane;  // key row within the block = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // warp w: TMEM lane quarter w%4 (key rows), query-column half w/4 (64 queries)
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // key row within the block = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float* lse_g = a.lse + ((long long)b * H + n) * S;
     const float* dsum_g = a.Dsum + ((long long)b * H + n) * S;
     bool ok = true;
+    // Per-query stats of the next block are fetched one iteration ahead (registers); half 0
+    // stages lse, half 1 stages D, each for query r of the block.
+    const float* stat_g = hf ? dsum_g : lse_g;
+    float* stat_s = hf ? dsum_s : lse_s;
+    auto fetch = [&](int qi) -> float {
+      const int q = qi * 128 + r;  // padded queries get lse = +inf, hence P = 0
+      if (hf == 0) return q < S ? stat_g[q] * kLog2eF : INFINITY;
+      return q < S ? stat_g[q] : 0.f;
+    };
+    float nv = niter > 0 ? fetch(kb) : 0.f;
     for (int it = 0; it < niter; ++it) {
       const int st = it & 1, qi = kb + it;
-      {
-        const int q = qi * 128 + r;  // padded queries get lse = +inf, hence P = 0
-        lse_s[st * 128 + r] = q < S ? lse_g[q] * kLog2eF : INFINITY;
-        dsum_s[st * 128 + r] = q < S ? dsum_g[q] : 0.f;
+      stat_s[st * 128 + r] = nv;
+      if (it + 1 < niter) nv = fetch(qi + 1);
+      mbar_arrive(&stat_bar[st]);
+      ok = mbar_wait(&stat_bar[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
       ok = mbar_wait(s_full, it & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
@@ -465,28 +527,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       const float* ls = lse_s + st * 128;
       const float* ds_ = dsum_s + st * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32], dp[32];
-        tmem_ld_32x32b_x32(lane_base + L::T_S + c * 32, sv);
-        tmem_ld_32x32b_x32(lane_base + L::T_DP + c * 32, dp);
-        uint32_t pw[16], dw[16];
+      {
+        const int c2 = hf * 2;  // this half's two 32-column chunks of S and dP
+        uint32_t sr[2][32], dr[2][32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = c * 32 + i + e;
-            float p = exp2f(sv[i + e] * scale_log2 - ls[col]);
-            if (qi == kb && col < r) p = 0.f;  // key > query
-            p2[e] = p;
-            d2[e] = p * (dp[i + e] - ds_[col]);
-          }
-          pw[i >> 1] = pack_bf16x2(p2[0], p2[1]);
-          dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+        for (int u = 0; u < 2; ++u) {
+          tmem_ld_32x32b_x32_nw(lane_base + L::T_S + (c2 + u) * 32, sr[u]);
+          tmem_ld_32x32b_x32_nw(lane_base + L::T_DP + (c2 + u) * 32, dr[u]);
         }
-        tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, pw);
-        tmem_st_32x32b_x16(lane_base + L::T_DP + c * 16, dw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          reg_fence(sr[u]);
+          reg_fence(dr[u]);
+          const int c = c2 + u;
+          if (qi == kb) {  // diagonal block: queries before this key see nothing of it
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i < r) sr[u][i] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pw[16], dw[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + i);
+            const float4 d4 = *reinterpret_cast<const float4*>(ds_ + c * 32 + i);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+            float p4[4], q4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              p4[e] = ex2_approx(fmaf(__uint_as_float(sr[u][i + e]), scale_log2, -lv[e]));
+              q4[e] = p4[e] * (__uint_as_float(dr[u][i + e]) - dv[e]);
+            }
+            pw[i >> 1] = pack_bf16x2(p4[0], p4[1]);
+            pw[(i >> 1) + 1] = pack_bf16x2(p4[2], p4[3]);
+            dw[i >> 1] = pack_bf16x2(q4[0], q4[1]);
+            dw[(i >> 1) + 1] = pack_bf16x2(q4[2], q4[3]);
+          }
+          tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, pw);
+          tmem_st_32x32b_x16(lane_base + L::T_DP + c * 16, dw);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -503,10 +582,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             (long long)t * 3 * hp * D + (long long)jh * D + (long long)hp * D;
         __nv_bfloat16* dv = dk + (long long)hp * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32], k[32];
+        for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {  // this half of d
+          float v[32], kk[32];
           tmem_ld_32x32b_x32(lane_base + L::T_ACC0 + c * 32, v);
-          tmem_ld_32x32b_x32(lane_base + L::T_ACC1 + c * 32, k);
+          tmem_ld_32x32b_x32(lane_base + L::T_ACC1 + c * 32, kk);
           if (key < S) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -515,10 +594,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               wv.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
               wv.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
               wv.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              wk.x = pack_bf16x2(k[q * 8 + 0] * scale, k[q * 8 + 1] * scale);
-              wk.y = pack_bf16x2(k[q * 8 + 2] * scale, k[q * 8 + 3] * scale);
-              wk.z = pack_bf16x2(k[q * 8 + 4] * scale, k[q * 8 + 5] * scale);
-              wk.w = pack_bf16x2(k[q * 8 + 6] * scale, k[q * 8 + 7] * scale);
+              wk.x = pack_bf16x2(kk[q * 8 + 0] * scale, kk[q * 8 + 1] * scale);
+              wk.y = pack_bf16x2(kk[q * 8 + 2] * scale, kk[q * 8 + 3] * scale);
+              wk.z = pack_bf16x2(kk[q * 8 + 4] * scale, kk[q * 8 + 5] * scale);
+              wk.w = pack_bf16x2(kk[q * 8 + 6] * scale, kk[q * 8 + 7] * scale);
               *reinterpret_cast<uint4*>(dv + c * 32 + q * 8) = wv;
               *reinterpret_cast<uint4*>(dk + c * 32 + q * 8) = wk;
             }
@@ -530,14 +609,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                           const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
                           float scale_log2, float scale) {
@@ -570,7 +649,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(mm_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -578,7 +657,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -587,7 +666,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * L::TILE);
 #pragma unroll
@@ -614,49 +693,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int kb = issued - 2 < 0 ? 0 : issued - 2; kb < issued; ++kb)
         mbar_wait(&kv_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(smem + L::B_Q), do_addr = smem_u32(smem + L::B_DO);
-      bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag);
-      for (int kb = 0; kb < nkv && ok; ++kb) {
-        const int st = kb & 1;
-        if (kb > 0 && !mbar_wait(mm_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
-          break;
-        if (!mbar_wait(&kv_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::B_K + st * L::TILE);
-        const uint32_t v_addr = smem_u32(smem + L::B_V + st * L::TILE);
+      // S_kb -> S buffer kb&1; dP_kb -> the single dP buffer; dQ += dS_kb K_kb with dS_kb in
+      // S buffer kb&1. S_{kb+1} is issued before waiting for this block's dS, so it overlaps
+      // the softmax warps; dP_{kb+1} waits until they have read dP_kb.
+      auto issue_s = [&](int kb) {
+        const uint32_t k_addr = smem_u32(smem + L::B_K + (kb & 1) * L::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_f16(tmem + L::T_S, smem_desc_sw128(q_addr + off, 16, 1024),
+          tc_mma_f16(tmem + ((kb & 1) ? L::Q_S1 : L::Q_S0),
+                     smem_desc_sw128(q_addr + off, 16, 1024),
                      smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int kb) {
+        const uint32_t v_addr = smem_u32(smem + L::B_V + (kb & 1) * L::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_f16(tmem + L::T_DP, smem_desc_sw128(do_addr + off, 16, 1024),
+          tc_mma_f16(tmem + L::Q_DP, smem_desc_sw128(do_addr + off, 16, 1024),
                      smem_desc_sw128(v_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag) &&
+                mbar_wait(&kv_full[0], 0, a.err, kErrTimeoutAttn, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
         tc_commit(s_full);
+      }
+      for (int kb = 0; kb < nkv && ok; ++kb) {
+        const bool more = kb + 1 < nkv;
+        if (more) {
+          // S buffer (kb+1)&1 was last read (as dS) by the dQ MMA of block kb-1
+          if (kb >= 1 && !mbar_wait(mm_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+            break;
+          if (!mbar_wait(&kv_full[(kb + 1) & 1], ((kb + 1) >> 1) & 1, a.err, kErrTimeoutAttn,
+                         abort_flag))
+            break;
+          tc_fence_after();
+          issue_s(kb + 1);
+        }
         if (!mbar_wait(p_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
         tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::B_K + (kb & 1) * L::TILE);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA; dS sits in the S columns
-          tc_mma_f16_tmem_a(tmem + L::T_ACC0, tmem + L::T_S + kk * 8,
+        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA; dS sits in S buffer kb&1
+          tc_mma_f16_tmem_a(tmem + L::Q_DQ, tmem + ((kb & 1) ? L::Q_S1 : L::Q_S0) + kk * 8,
                             smem_desc_sw128(k_addr + kk * 2048, 16384, 1024), idesc_acc,
                             (kb > 0 || kk > 0) ? 1u : 0u);
         tc_commit(mm_done);
-        tc_commit(&kv_empty[st]);
+        tc_commit(&kv_empty[kb & 1]);
+        if (more) {
+          issue_dp(kb + 1);
+          tc_commit(s_full);
+        }
       }
       tc_commit(drain);
       mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
     }
   } else {
-    const int r = warp * 32 + lane;  // query row within the block = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // warp w: TMEM lane quarter w%4 (query rows), key-column half w/4 (64 keys)
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row within the block = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int q = qb * 128 + r;
     const float lse2 = q < S ? a.lse[((long long)b * H + n) * S + q] * kLog2eF : INFINITY;
     const float dq_sum = q < S ? a.Dsum[((long long)b * H + n) * S + q] : 0.f;
@@ -668,25 +774,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32], dp[32];
-        tmem_ld_32x32b_x32(lane_base + L::T_S + c * 32, sv);
-        tmem_ld_32x32b_x32(lane_base + L::T_DP + c * 32, dp);
-        uint32_t dw[16];
+      const uint32_t s_col = (kb & 1) ? L::Q_S1 : L::Q_S0;
+      {
+        const int c2 = hf * 2;  // this half's two 32-column chunks of S and dP
+        uint32_t sr[2][32], dr[2][32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = c * 32 + i + e;
-            float p = exp2f(sv[i + e] * scale_log2 - lse2);
-            if (kb == qb && col > r) p = 0.f;  // key > query
-            d2[e] = p * (dp[i + e] - dq_sum);
-          }
-          dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+        for (int u = 0; u < 2; ++u) {
+          tmem_ld_32x32b_x32_nw(lane_base + s_col + (c2 + u) * 32, sr[u]);
+          tmem_ld_32x32b_x32_nw(lane_base + L::Q_DP + (c2 + u) * 32, dr[u]);
         }
-        tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, dw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          reg_fence(sr[u]);
+          reg_fence(dr[u]);
+          const int c = c2 + u;
+          uint32_t dw[16];
+          if (kb == qb) {  // diagonal block: keys after this query are masked
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > r) sr[u][i] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float d2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float p = ex2_approx(fmaf(__uint_as_float(sr[u][i + e]), scale_log2, -lse2));
+              d2[e] = p * (__uint_as_float(dr[u][i + e]) - dq_sum);
+            }
+            dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
+          }
+          tmem_st_32x32b_x16(lane_base + s_col + c * 16, dw);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -701,9 +821,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + ((long long)b * S + q) * ld +
                             (long long)t * 3 * hp * D + (long long)jh * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {  // this half of d
           float v[32];
-          tmem_ld_32x32b_x32(lane_base + L::T_ACC0 + c * 32, v);
+          tmem_ld_32x32b_x32(lane_base + L::Q_DQ + c * 32, v);
           if (q < S) {
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
@@ -722,7 +842,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -756,11 +876,11 @@ cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
   }
   const float scale = 1.f / sqrtf((float)D);
   dim3 grid((a.s + 127) / 128, a.b * a.H);
-  attn_bwd_dkdv_tc_kernel<D><<<grid, kAttnThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kFwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                     kLog2eF * scale, scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_tc_kernel<D><<<grid, kAttnThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
+  attn_bwd_dq_tc_kernel<D><<<grid, kFwdThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                   kLog2eF * scale, scale);
   return cudaGetLastError();
 }
@@ -783,7 +903,7 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
   dim3 grid((a.s + 127) / 128, a.b * a.H);
-  attn_fwd_tc_kernel<D><<<grid, kAttnThreads, L::BYTES, s>>>(tm, a, kLog2eF / sqrtf((float)D));
+  attn_fwd_tc_kernel<D><<<grid, kFwdThreads, L::BYTES, s>>>(tm, a, kLog2eF / sqrtf((float)D));
   return cudaGetLastError();
 }
 
