@@ -184,6 +184,18 @@ mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major,
                          int32_t b_mn_major, const void* A, int64_t lda, const void* B,
                          int64_t ldb, float* C, int64_t ldc, int32_t* status, void* stream);
 
+/* Failure-path probe (diagnostics and tests; no counterpart in the pages). Launches one thread
+ * that waits on a device barrier nothing ever arrives on, through the same bounded wait that
+ * every pipelined kernel of this library uses; after limit_ns (0 < limit_ns <= 1e9) it gives
+ * up, records a non-zero code in the int32 device word `status` and returns. Demonstrates that a
+ * device wait which runs out ends in a readable status, not a hang or trap, and that the context
+ * stays usable. Point `status` at a layer's status word (mgt_layer_status_word) to make
+ * mgt_layer_get_error report MGT_ETIMEOUT. */
+mgt_status mgt_debug_bounded_wait(int64_t limit_ns, int32_t* status, void* stream);
+
+/* Device address of the status word inside `workspace` (the first bytes of the workspace). */
+mgt_status mgt_layer_status_word(mgt_layer* layer, void* workspace, int32_t** word);
+
 /* LayerNorm backward that allocates nothing -- the pages have no counterpart; it exists for
  * callers that cannot call cudaMalloc where they run the backward (frameworks that own all
  * device memory through their own pool allocator, hot loops where an allocation would

@@ -84,6 +84,10 @@ def load_library():
                                   ctypes.c_int64, vp, ctypes.c_int64, vp, vp]
     lib.mgt_layernorm_bwd_noalloc.argtypes = [i32, ctypes.c_int64, i32, vp, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp]
+    lib.mgt_debug_bounded_wait.argtypes = [ctypes.c_int64, vp, vp]
+    lib.mgt_layer_status_word.argtypes = [vp, vp, ctypes.POINTER(vp)]
+    lib.mgt_debug_bounded_wait.restype = ctypes.c_int
+    lib.mgt_layer_status_word.restype = ctypes.c_int
     for name in ("mgt_layer_init", "mgt_layer_sizes", "mgt_layer_region", "mgt_layer_fwd",
                  "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
                  "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc"):
@@ -200,6 +204,13 @@ class Layer:
     def get_error(self, workspace, stream=None) -> int:
         return self.lib.mgt_layer_get_error(self.handle, _ptr(workspace), _stream_handle(stream))
 
+    def status_word_ptr(self, workspace) -> int:
+        """Device address of the status word inside `workspace`."""
+        w = ctypes.c_void_p()
+        _check(self.lib.mgt_layer_status_word(self.handle, _ptr(workspace), ctypes.byref(w)),
+               "mgt_layer_status_word")
+        return w.value
+
     def profile(self, enable=True):
         _check(self.lib.mgt_layer_profile(self.handle, 1 if enable else 0), "mgt_layer_profile")
 
@@ -240,3 +251,11 @@ def layernorm_bwd_noalloc(dtype, rows, h, dy, dres, x, gamma, mean, rstd, dx, dg
                                          _ptr(dres), _ptr(x), _ptr(gamma), _ptr(mean),
                                          _ptr(rstd), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
                                          _stream_handle(stream)), "mgt_layernorm_bwd_noalloc")
+
+
+def debug_bounded_wait(limit_ns, status_ptr, stream=None):
+    """Run the bounded-wait failure probe (see mgt_debug_bounded_wait); status_ptr is a device
+    address of an int32 status word."""
+    lib = load_library()
+    _check(lib.mgt_debug_bounded_wait(int(limit_ns), ctypes.c_void_p(status_ptr),
+                                      _stream_handle(stream)), "mgt_debug_bounded_wait")

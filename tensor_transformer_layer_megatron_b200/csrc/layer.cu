@@ -519,6 +519,19 @@ void mgt_layer_destroy(mgt_layer* L) {
   delete L;
 }
 
+mgt_status mgt_debug_bounded_wait(int64_t limit_ns, int32_t* status, void* stream) {
+  if (!status || limit_ns <= 0 || limit_ns > 1000000000LL) return MGT_EINVAL;
+  return cuda_status(launch_bounded_wait_probe(reinterpret_cast<int*>(status),
+                                               (unsigned long long)limit_ns,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+mgt_status mgt_layer_status_word(mgt_layer* L, void* workspace, int32_t** word) {
+  if (!L || !workspace || !word) return MGT_EINVAL;
+  *word = reinterpret_cast<int32_t*>(sp(workspace, L->ws[MGT_WS_STATUS - 64]));
+  return MGT_OK;
+}
+
 mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major, int32_t b_mn_major,
                          const void* A, int64_t lda, const void* B, int64_t ldb, float* C,
                          int64_t ldc, int32_t* status, void* stream) {

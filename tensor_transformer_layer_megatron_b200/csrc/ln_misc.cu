@@ -537,6 +537,24 @@ cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, fl
   return cudaGetLastError();
 }
 
+// One thread waits on an mbarrier that nothing ever arrives on, through the same bounded
+// wait every pipelined kernel uses: it gives up after limit_ns, records kErrTimeoutProbe in
+// the status word and returns, leaving the context usable.
+__global__ void bounded_wait_probe_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, status, kErrTimeoutProbe, nullptr, limit_ns);
+}
+
+cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns, cudaStream_t s) {
+  bounded_wait_probe_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_simt_f32(const GemmArgs& a, cudaStream_t s) {
   const long long total = (long long)a.NG * a.M * a.Ng;
   if (total <= 0) return cudaSuccess;

@@ -68,9 +68,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Bounded: returns false (and
-// records `code` in *err) after kWaitLimitNs, or at once if *abort becomes non-zero.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code,
-                                          volatile int* abort) {
+// records `code` in *err) after limit_ns, or at once if *abort becomes non-zero.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* err,
+                                                int code, volatile int* abort,
+                                                uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -79,12 +80,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(addr, parity)) return true;
     if (abort && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       record_error(err, code);
       if (abort) *abort = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code,
+                                          volatile int* abort) {
+  return mbar_wait_limit(bar, parity, err, code, abort, kWaitLimitNs);
 }
 
 // ----------------------------------------------------------------------------- TMA

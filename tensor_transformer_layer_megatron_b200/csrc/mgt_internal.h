@@ -14,6 +14,7 @@ enum DeviceError : int {
   kErrTimeoutEpilogue = 0x102,  // epilogue waited too long for an accumulator
   kErrTimeoutDrain = 0x103,     // unwinding after a timeout waited too long
   kErrTimeoutAttn = 0x110,
+  kErrTimeoutProbe = 0x1F0,     // the bounded-wait probe (mgt_debug_bounded_wait) gave up
 };
 
 // Epilogue applied to each fp32 accumulator tile of the GEMM.
@@ -72,6 +73,10 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk,
                           float* dgamma, float* dbeta, float* dres_sum, cudaStream_t stream);
+
+// Device-side failure-path probe (see mgt_debug_bounded_wait).
+cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
+                                      cudaStream_t stream);
 
 // Column sums of a [rows, cols] activation matrix into fp32 (bias gradients).
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
