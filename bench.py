@@ -7,7 +7,8 @@ rank runs its own replica on its own batch (data parallel, no collective on the 
 weak scaling, value = tokens of all ranks / max-over-ranks time.
 
 Prints ONE JSON line (rank 0). --impl reference times the fp64 CPU oracle instead, on a bounded
-sample of the same workload, on this host's cores.
+sample of the same workload, on this host's cores. --impl torch times the same layer in eager
+PyTorch on the GPU (cuBLAS + flash SDPA), as context.
 """
 from __future__ import annotations
 
@@ -112,6 +113,22 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(ms, world, device):
+    """The job's time is the slowest rank's: all-reduce MAX of this rank's device-timed ms."""
+    if world == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, ms_total, steps):
+    """Whole-job tokens/s (all ranks' tokens over the max-over-ranks time) and ms per step."""
+    ms_step = ms_total / steps
+    return tokens_per_rank * world / (ms_step / 1e3), ms_step
+
+
 def run_mgt(args):
     import torch
 
@@ -178,13 +195,9 @@ def run_mgt(args):
     layer.profile(False)
     run.check()
     del graph
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
-    ms_step = ms / args.steps
+    ms = max_over_ranks(ms, world, dev)
     tokens = cfg.tokens * world
-    value = tokens / (ms_step / 1e3)
+    value, ms_step = job_throughput(cfg.tokens, world, ms, args.steps)
     flops_step = cfg.model_flops() * world
     tflops = flops_step / (ms_step / 1e3) / 1e12
 
@@ -206,12 +219,8 @@ def run_mgt(args):
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = tokens / (e2e_ms / args.steps / 1e3)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
+    e2e_value, _ = job_throughput(cfg.tokens, world, e2e_ms, args.steps)
     h2d = (x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size())
     d2h = (y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size())
 
@@ -297,6 +306,80 @@ def run_mgt(args):
         torch.distributed.destroy_process_group()
 
 
+def run_torch(args):
+    """Context comparator: the same layer in eager PyTorch on the GPU (cuBLAS GEMMs through
+    F.linear on the full unsharded weights, which is what logical TP on one GPU computes;
+    flash scaled_dot_product_attention; F.layer_norm; autograd backward with bf16 weight
+    gradients). Same inputs, same K/W, CUDA events on the stream. Not the product path."""
+    import torch
+    import torch.nn.functional as F
+
+    from mgt_inputs import config_by_name, make_inputs
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = config_by_name(args.config)
+    t = make_inputs(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    h, H, d, b, s = cfg.hidden, cfg.heads, cfg.head_dim, cfg.micro_batch, cfg.seq
+    names = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o", "ln2_g", "ln2_b", "w1", "b1",
+             "w2", "b2")
+    P = {k: t[k].to(dev, dt).requires_grad_(True) for k in names}
+    x = t["x"].to(dev, dt).requires_grad_(True)
+    dy = t["dy"].to(dev, dt)
+    approx = "tanh" if cfg.gelu_tanh else "none"
+
+    def step():
+        for v in P.values():
+            v.grad = None
+        x.grad = None
+        ln1 = F.layer_norm(x, (h,), P["ln1_g"], P["ln1_b"], cfg.ln_eps)
+        q, k, v = F.linear(ln1, P["w_qkv"], P["b_qkv"]).view(b, s, 3, H, d).unbind(2)
+        o = F.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2),
+                                           v.transpose(1, 2), is_causal=True)
+        h1 = x + F.linear(o.transpose(1, 2).reshape(b, s, h), P["w_o"], P["b_o"])
+        ln2 = F.layer_norm(h1, (h,), P["ln2_g"], P["ln2_b"], cfg.ln_eps)
+        a = F.gelu(F.linear(ln2, P["w1"], P["b1"]), approximate=approx)
+        y = h1 + F.linear(a, P["w2"], P["b2"])
+        y.backward(dy)
+        return y
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    value, ms_step = job_throughput(cfg.tokens, world, ms, args.steps)
+    tflops = cfg.model_flops() * world / (ms_step / 1e3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "impl": "torch-eager", "metric": METRIC, "value": round(value, 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+            "data": "synthetic (same seeded inputs as the main arm)",
+            "tflops": round(tflops, 1),
+            "what": "context comparator: eager torch (cuBLAS F.linear on unsharded weights, "
+                    "flash SDPA, F.layer_norm, autograd; bf16 weight grads)",
+            "config": {"workload": cfg.name, "tokens_per_gpu": cfg.tokens},
+            "clocks": clk}), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def cpu_baseline(cfg, tokens):
     """The fp64 oracle, as it stands, on a bounded sample: one sequence of `tokens` tokens of
     the same layer (weights of the full shape), forward + backward, on this host's cores."""
@@ -350,7 +433,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", default="mgt", choices=["mgt", "reference"])
+    ap.add_argument("--impl", default="mgt", choices=["mgt", "reference", "torch"])
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -363,6 +446,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.impl == "torch":
+        run_torch(args)
     else:
         run_mgt(args)
 
