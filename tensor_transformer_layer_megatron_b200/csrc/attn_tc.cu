@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.s, H = a.H, hp = H / a.p;
   const int nqb = (S + 127) / 128;
-  const int qb = nqb - 1 - blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  // Heads vary fastest in the launch order and query blocks run from the longest rows down,
+  // so every head's longest tiles start in the first wave (longest-processing-time order).
+  const int qb = nqb - 1 - blockIdx.y;
+  const int bh = blockIdx.x, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
   const int nkv = qb + 1;
 
@@ -385,8 +387,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.s, H = a.H, hp = H / a.p;
-  const int kb = blockIdx.x;  // key block; kb = 0 has the most query blocks: launched first
-  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  // Key block; kb = 0 sees the most query blocks. Heads vary fastest in the launch order, so
+  // the longest tiles of every head go first.
+  const int kb = blockIdx.y;
+  const int bh = blockIdx.x, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
   const int nq = (S + 127) / 128;
   const int niter = nq - kb;  // query blocks qi = kb .. nq-1 see keys of this block
@@ -637,8 +641,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.s, H = a.H, hp = H / a.p;
   const int nqb = (S + 127) / 128;
-  const int qb = nqb - 1 - blockIdx.x;
-  const int bh = blockIdx.y, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const int qb = nqb - 1 - blockIdx.y;  // longest rows first, heads fastest (as above)
+  const int bh = blockIdx.x, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
   const int nkv = qb + 1;
 
@@ -875,7 +879,7 @@ cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
     if (!make_tensor_map_bf16_3d(&tm_do, a.dO, dims, strides, box)) return cudaErrorInvalidValue;
   }
   const float scale = 1.f / sqrtf((float)D);
-  dim3 grid((a.s + 127) / 128, a.b * a.H);
+  dim3 grid(a.b * a.H, (a.s + 127) / 128);
   attn_bwd_dkdv_tc_kernel<D><<<grid, kFwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                     kLog2eF * scale, scale);
   cudaError_t e = cudaGetLastError();
@@ -902,7 +906,7 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   const uint64_t strides[2] = {three_h, three_h * a.s};
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
-  dim3 grid((a.s + 127) / 128, a.b * a.H);
+  dim3 grid(a.b * a.H, (a.s + 127) / 128);
   attn_fwd_tc_kernel<D><<<grid, kFwdThreads, L::BYTES, s>>>(tm, a, kLog2eF / sqrtf((float)D));
   return cudaGetLastError();
 }

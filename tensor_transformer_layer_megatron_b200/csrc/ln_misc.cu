@@ -27,6 +27,14 @@ struct Vec<__nv_bfloat16> {
       v[2 * j + 1] = bf16_hi(ww[j]);
     }
   }
+  __device__ static void unpack(const uint4& w, float (&v)[8]) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = bf16_lo(ww[j]);
+      v[2 * j + 1] = bf16_hi(ww[j]);
+    }
+  }
   __device__ static void store(__nv_bfloat16* p, const float (&v)[8]) {
     uint4 w;
     w.x = pack_bf16x2(v[0], v[1]);
@@ -42,6 +50,10 @@ struct Vec<float> {
   __device__ static void load(const float* p, float (&v)[4]) {
     const float4 w = *reinterpret_cast<const float4*>(p);
     v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+  }
+  __device__ static void unpack(const uint4& w, float (&v)[4]) {
+    v[0] = __uint_as_float(w.x); v[1] = __uint_as_float(w.y);
+    v[2] = __uint_as_float(w.z); v[3] = __uint_as_float(w.w);
   }
   __device__ static void store(float* p, const float (&v)[4]) {
     *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -203,6 +215,144 @@ __global__ void __launch_bounds__(256) ln_bwd_dx_kernel(long long rows, int h,
 #pragma unroll
       for (int j = 0; j < V; ++j) o[j] = rs * (g[i][j] - m1 - xh[i][j] * m2) + rv[j];
       Vec<T>::store(dx + r * h + vi * V, o);
+    }
+  }
+}
+
+// dx and the parameter partials in one pass over x, dy and dres (rows up to 512 16-byte vectors).
+// The block walks a contiguous slice of rows one row at a time with all 256 threads (thread t
+// owns the column vectors t, t + 256, ...), loading the next row's x, dy, dres and statistics
+// while it reduces the current one. Every column belongs to one thread, so dgamma = sum dy*xhat,
+// dbeta = sum dy and (NSUM = 3) sum dres accumulate in registers and leave as one partial row
+// set per block, partial[slice][NSUM][h], for ln_param_reduce_kernel (fixed order).
+template <typename T, int VPL, int NSUM>
+__global__ void __launch_bounds__(256, 2) ln_bwd_fused_kernel(long long rows, int h,
+                                                           const T* __restrict__ dy,
+                                                           const T* __restrict__ dres,
+                                                           const T* __restrict__ x,
+                                                           const float* __restrict__ gamma,
+                                                           const float* __restrict__ mean,
+                                                           const float* __restrict__ rstd,
+                                                           T* __restrict__ dx,
+                                                           float* __restrict__ partial,
+                                                           long long rows_per) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float2 red[2][8];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nvec = h / V;
+  const long long r0 = (long long)blockIdx.x * rows_per;
+  const long long r1 = min(rows, r0 + rows_per);
+  const float inv_h = 1.f / (float)h;
+  // gamma is re-read (from L1) at each use rather than held: registers go to the accumulators
+  // and the prefetched row.
+  float ag[VPL][V], ab[VPL][V], ar[VPL][V];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+#pragma unroll
+    for (int j = 0; j < V; ++j) ag[i][j] = ab[i][j] = ar[i][j] = 0.f;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  uint4 cx[VPL], cd[VPL], cr[VPL];
+  float cmu = 0.f, crs = 0.f;
+  auto load_row = [&](long long r, uint4 (&px)[VPL], uint4 (&pd)[VPL], uint4 (&pr)[VPL],
+                      float& mu, float& rs) {
+    mu = mean[r];
+    rs = rstd[r];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = t + i * 256;
+      const bool ok = vi < nvec;
+      px[i] = ok ? *reinterpret_cast<const uint4*>(x + r * h + vi * V) : zero;
+      pd[i] = ok ? *reinterpret_cast<const uint4*>(dy + r * h + vi * V) : zero;
+      pr[i] = (ok && dres) ? *reinterpret_cast<const uint4*>(dres + r * h + vi * V) : zero;
+    }
+  };
+  if (r0 < r1) load_row(r0, cx, cd, cr, cmu, crs);
+  int par = 0;
+  for (long long r = r0; r < r1; ++r, par ^= 1) {
+    uint4 nx[VPL], nd[VPL], nr[VPL];
+    float nmu = 0.f, nrs = 0.f;
+    if (r + 1 < r1) load_row(r + 1, nx, nd, nr, nmu, nrs);
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = t + i * 256;
+      float xv[V], dv[V], gv[V];
+      Vec<T>::unpack(cx[i], xv);
+      Vec<T>::unpack(cd[i], dv);
+      if (vi < nvec) {
+        load_param<V>(gamma, vi * V, gv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < V; ++j) gv[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
+        s1 += g;
+        s2 += g * xh;
+        ag[i][j] += dv[j] * xh;
+        ab[i][j] += dv[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    // Two buffers by row parity: a buffer is rewritten two rows later, after every thread has
+    // passed the next row's barrier and so has finished reading it.
+    if (lane == 0) red[par][warp] = make_float2(s1, s2);
+    __syncthreads();
+    float S1 = 0.f, S2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 v = red[par][k];
+      S1 += v.x;
+      S2 += v.y;
+    }
+    const float m1 = S1 * inv_h, m2 = S2 * inv_h;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = t + i * 256;
+      if (vi < nvec) {
+        float xv[V], dv[V], rv[V], gv[V], o[V];
+        Vec<T>::unpack(cx[i], xv);
+        Vec<T>::unpack(cd[i], dv);
+        Vec<T>::unpack(cr[i], rv);
+        load_param<V>(gamma, vi * V, gv);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
+          o[j] = crs * (g - m1 - xh * m2) + rv[j];
+          if constexpr (NSUM == 3) ar[i][j] += rv[j];
+        }
+        Vec<T>::store(dx + r * h + vi * V, o);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      cx[i] = nx[i];
+      cd[i] = nd[i];
+      cr[i] = nr[i];
+    }
+    cmu = nmu;
+    crs = nrs;
+  }
+  float* pg = partial + (long long)blockIdx.x * NSUM * h;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = t + i * 256;
+    if (vi < nvec) {
+#pragma unroll
+      for (int j = 0; j < V; j += 4) {
+        *reinterpret_cast<float4*>(pg + vi * V + j) =
+            make_float4(ag[i][j], ag[i][j + 1], ag[i][j + 2], ag[i][j + 3]);
+        *reinterpret_cast<float4*>(pg + h + vi * V + j) =
+            make_float4(ab[i][j], ab[i][j + 1], ab[i][j + 2], ab[i][j + 3]);
+        if constexpr (NSUM == 3)
+          *reinterpret_cast<float4*>(pg + 2 * h + vi * V + j) =
+              make_float4(ar[i][j], ar[i][j + 1], ar[i][j + 2], ar[i][j + 3]);
+      }
     }
   }
 }
@@ -453,7 +603,38 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
                             void* dx, float* partial, int nblk, float* dgamma, float* dbeta,
                             float* dres_sum, cudaStream_t s) {
   const int nvec = h / Vec<T>::N;
+  const int nsum = (dres_sum && dres) ? 3 : 2;
   cudaError_t e;
+  if (nvec <= 512) {  // one pass: dx and the parameter partials together
+    long long slices = nblk < rows ? nblk : rows;
+    const long long rows_per = (rows + slices - 1) / slices;
+    slices = (rows + rows_per - 1) / rows_per;
+    const T* pdy = reinterpret_cast<const T*>(dy);
+    const T* pdr = reinterpret_cast<const T*>(dres);
+    const T* px = reinterpret_cast<const T*>(x);
+    T* pdx = reinterpret_cast<T*>(dx);
+    const unsigned gs = (unsigned)slices;
+    if (nvec <= 256) {
+      if (nsum == 3)
+        ln_bwd_fused_kernel<T, 1, 3><<<gs, 256, 0, s>>>(rows, h, pdy, pdr, px, g, mean, rstd,
+                                                        pdx, partial, rows_per);
+      else
+        ln_bwd_fused_kernel<T, 1, 2><<<gs, 256, 0, s>>>(rows, h, pdy, pdr, px, g, mean, rstd,
+                                                        pdx, partial, rows_per);
+    } else {
+      if (nsum == 3)
+        ln_bwd_fused_kernel<T, 2, 3><<<gs, 256, 0, s>>>(rows, h, pdy, pdr, px, g, mean, rstd,
+                                                        pdx, partial, rows_per);
+      else
+        ln_bwd_fused_kernel<T, 2, 2><<<gs, 256, 0, s>>>(rows, h, pdy, pdr, px, g, mean, rstd,
+                                                        pdx, partial, rows_per);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
+                                                               dgamma, dbeta, dres_sum);
+    return cudaGetLastError();
+  }
+  // Wider rows: a dx kernel, then a parameter-partial kernel over slices of rows.
   if (nvec <= 64)
     e = ln_bwd_dx_inst<T, 1, 2>(rows, h, dy, dres, x, g, mean, rstd, dx, s);
   else if (nvec <= 128)
@@ -475,7 +656,6 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
   if (slices < 1) slices = 1;
   const long long rows_per = (rows + slices - 1) / slices;
   slices = (rows + rows_per - 1) / rows_per;
-  const int nsum = (dres_sum && dres) ? 3 : 2;
   if (nsum == 3)
     ln_bwd_param_kernel<T, 3><<<dim3(cb, (unsigned)slices), dim3(32, 8), 0, s>>>(
         rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x),
