@@ -58,6 +58,8 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n) 
 }
 
 // ---------------------------------------------------------------------------- epilogue
+// Every loop over the 32 accumulator values is unrolled with compile-time indices (ragged chunks
+// are predicated, not shortened), so v stays in registers instead of local memory.
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int col,
                                                int count, float (&v)[32]) {
@@ -70,7 +72,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
       for (int i = 0; i < 32; i += 4)
         *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     } else {
-      for (int i = 0; i < count; ++i) o[i] = v[i];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < count) o[i] = v[i];
     }
     return;
   } else {
@@ -91,7 +95,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
             }
           }
         } else {
-          for (int i = 0; i < count; ++i) v[i] += __bfloat162float(bias[col + i]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < count) v[i] += __bfloat162float(bias[col + i]);
         }
       }
     }
@@ -110,7 +116,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
           }
         }
       } else {
-        for (int i = 0; i < count; ++i) v[i] += __bfloat162float(r[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < count) v[i] += __bfloat162float(r[i]);
       }
     }
     if (EPI == kEpiDGelu) {  // aux holds GeLU'(u), stored by the forward epilogue
@@ -128,7 +136,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
           }
         }
       } else {
-        for (int i = 0; i < count; ++i) v[i] *= __bfloat162float(g[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < count) v[i] *= __bfloat162float(g[i]);
       }
     }
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + off;
@@ -153,11 +163,14 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
           *reinterpret_cast<uint4*>(o + q * 8) = wa;
         }
       } else {
-        for (int i = 0; i < count; ++i) {
-          float ga, gd;
-          gelu_and_grad_f(v[i], a.gelu_tanh, ga, gd);
-          o2[i] = __float2bfloat16_rn(gd);
-          o[i] = __float2bfloat16_rn(ga);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i < count) {
+            float ga, gd;
+            gelu_and_grad_f(v[i], a.gelu_tanh, ga, gd);
+            o2[i] = __float2bfloat16_rn(gd);
+            o[i] = __float2bfloat16_rn(ga);
+          }
         }
       }
       return;
@@ -173,7 +186,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
         *reinterpret_cast<uint4*>(o + q * 8) = w;
       }
     } else {
-      for (int i = 0; i < count; ++i) o[i] = __float2bfloat16_rn(v[i]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < count) o[i] = __float2bfloat16_rn(v[i]);
     }
   }
 }
