@@ -17,10 +17,16 @@ Packed layouts (row-major, weights stored nn.Linear-style [out, in], y = x W^T +
     w_o    [p][h][h/p]         shard t owns input columns t*h/p .. (t+1)*h/p-1
     w1     [p][f/p][h]         shard t owns output rows t*f/p .. (t+1)*f/p-1
     b1     [p][f/p]
+    (SwiGLU: w1 [p][2][f/p][h], b1 [p][2][f/p]: shard t's gate rows, then its up rows; the
+     full matrix is [2f, h] with all gate rows first, then all up rows)
     w2     [p][h][f/p]
     b_o, b2, ln gammas/betas   replicated [h]
 Activations: x, y [b, s, h]; qkv [b*s][p][3][H/p][d]; attention output [b*s][p][H/p][d]
 (= head-major [b*s, h]); u, a [b*s][p][f/p] (= [b*s, f]).
+
+Variants (the trdm.cn page, section 3.3, lists them as launch flags): swiglu=1 replaces GeLU by
+SwiGLU, a = silu(gate) * up, fc1 producing gate and up (2f outputs); disable_bias_linear=1
+drops the biases of all four linear layers (the LayerNorm affine parameters stay).
 """
 from __future__ import annotations
 
@@ -31,12 +37,13 @@ from typing import Dict
 import torch
 
 __all__ = [
-    "LayerConfig", "CONFIGS", "config_by_name", "make_inputs", "pack_params", "unpack_params",
-    "PARAM_NAMES",
+    "LayerConfig", "CONFIGS", "VARIANTS", "config_by_name", "make_inputs", "pack_params",
+    "unpack_params", "PARAM_NAMES", "BIAS_NAMES",
 ]
 
 PARAM_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
+BIAS_NAMES = ("b_qkv", "b_o", "b1", "b2")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -55,6 +62,8 @@ class LayerConfig:
     ln_eps: float = 1e-5
     gelu_tanh: int = 0
     causal: int = 1
+    swiglu: int = 0               # 1: a = silu(gate) * up instead of GeLU(u)
+    disable_bias_linear: int = 0  # 1: no biases in the QKV, out-proj, fc1, fc2 layers
 
     @property
     def head_dim(self) -> int:
@@ -64,13 +73,19 @@ class LayerConfig:
     def tokens(self) -> int:
         return self.seq * self.micro_batch
 
+    @property
+    def fc1_rows(self) -> int:
+        """Output width of fc1: f, or 2f (gate and up) with SwiGLU."""
+        return 2 * self.ffn if self.swiglu else self.ffn
+
     def replace(self, **kw) -> "LayerConfig":
         return dataclasses.replace(self, **kw)
 
     def model_flops(self) -> float:
         """fwd+bwd model FLOPs: 3 x forward, causal attention counted as half of s^2."""
         T, h, f = self.tokens, self.hidden, self.ffn
-        fwd = 2.0 * T * (4 * h * h + 2 * h * f) + 2.0 * self.micro_batch * self.seq ** 2 * h
+        mlp = (3 if self.swiglu else 2) * h * f  # fc1 (f or 2f outputs) + fc2
+        fwd = 2.0 * T * (4 * h * h + mlp) + 2.0 * self.micro_batch * self.seq ** 2 * h
         return 3.0 * fwd
 
 
@@ -85,8 +100,17 @@ CONFIGS = (
 )
 
 
+# The MLP/bias variants: a tiny fp32 SwiGLU layer and the h=4096 layer in its LLaMA form
+# (SwiGLU over the same f = 11008, no linear biases).
+VARIANTS = (
+    LayerConfig("tiny-h64-tp2-f32-swiglu", 64, 4, 256, 32, 2, 2, "f32", 1005, swiglu=1),
+    LayerConfig("llama-h4096-tp2-bf16-swiglu-nobias", 4096, 32, 11008, 2048, 1, 2, "bf16", 1006,
+                swiglu=1, disable_bias_linear=1),
+)
+
+
 def config_by_name(name: str) -> LayerConfig:
-    for c in CONFIGS:
+    for c in CONFIGS + VARIANTS:
         if c.name == name:
             return c
     raise KeyError(name)
@@ -109,6 +133,7 @@ def make_inputs(cfg: LayerConfig, nonzero_affine: bool = False, dy_scale: float 
 
     Full-layout tensors: x, dy [b, s, h]; w_qkv [3h, h] with rows [Q heads | K heads | V heads]
     (head n of Q = rows n*d..(n+1)*d-1); w_o [h, h]; w1 [f, h]; w2 [h, f]; b_qkv [3h]; b1 [f].
+    SwiGLU: w1 [2f, h], b1 [2f] (gate rows, then up rows). disable_bias_linear: no b_* keys.
     """
     h, f, b, s = cfg.hidden, cfg.ffn, cfg.micro_batch, cfg.seq
     g = torch.Generator("cpu").manual_seed(cfg.seed)
@@ -116,7 +141,7 @@ def make_inputs(cfg: LayerConfig, nonzero_affine: bool = False, dy_scale: float 
     t["x"] = _randn(g, (b, s, h), 1.0)
     t["w_qkv"] = _randn(g, (3 * h, h), cfg.init_std)
     t["w_o"] = _randn(g, (h, h), cfg.out_init_std)
-    t["w1"] = _randn(g, (f, h), cfg.init_std)
+    t["w1"] = _randn(g, (cfg.fc1_rows, h), cfg.init_std)
     t["w2"] = _randn(g, (h, f), cfg.out_init_std)
     t["dy"] = _randn(g, (b, s, h), dy_scale)
     if nonzero_affine:
@@ -126,7 +151,7 @@ def make_inputs(cfg: LayerConfig, nonzero_affine: bool = False, dy_scale: float 
         t["b_o"] = _randn(g, (h,), 0.05)
         t["ln2_g"] = 1.0 + _randn(g, (h,), 0.1)
         t["ln2_b"] = _randn(g, (h,), 0.1)
-        t["b1"] = _randn(g, (f,), 0.05)
+        t["b1"] = _randn(g, (cfg.fc1_rows,), 0.05)
         t["b2"] = _randn(g, (h,), 0.05)
     else:
         t["ln1_g"] = torch.ones(h)
@@ -135,12 +160,15 @@ def make_inputs(cfg: LayerConfig, nonzero_affine: bool = False, dy_scale: float 
         t["b_o"] = torch.zeros(h)
         t["ln2_g"] = torch.ones(h)
         t["ln2_b"] = torch.zeros(h)
-        t["b1"] = torch.zeros(f)
+        t["b1"] = torch.zeros(cfg.fc1_rows)
         t["b2"] = torch.zeros(h)
     if cfg.dtype == "bf16":
         # LN parameters stay fp32 on the device; everything else is a bf16 tensor there.
         for k in ("x", "dy", "w_qkv", "w_o", "w1", "w2", "b_qkv", "b_o", "b1", "b2"):
             t[k] = t[k].to(torch.bfloat16).to(torch.float32)
+    if cfg.disable_bias_linear:  # drawn above all the same, so the other tensors do not move
+        for k in BIAS_NAMES:
+            del t[k]
     return t
 
 
@@ -152,14 +180,22 @@ def pack_params(cfg: LayerConfig, full: Dict[str, torch.Tensor]) -> Dict[str, to
     # [3][H][d][h] -> [3][p][H/p][d][h] -> [p][3][H/p][d][h]
     out["w_qkv"] = (full["w_qkv"].reshape(3, p, H // p, d, h).permute(1, 0, 2, 3, 4)
                     .contiguous())
-    out["b_qkv"] = full["b_qkv"].reshape(3, p, H // p, d).permute(1, 0, 2, 3).contiguous()
+    if "b_qkv" in full:
+        out["b_qkv"] = full["b_qkv"].reshape(3, p, H // p, d).permute(1, 0, 2, 3).contiguous()
     # [h][p][h/p] -> [p][h][h/p]
     out["w_o"] = full["w_o"].reshape(h, p, h // p).permute(1, 0, 2).contiguous()
-    out["w1"] = full["w1"].reshape(p, f // p, h).contiguous()
-    out["b1"] = full["b1"].reshape(p, f // p).contiguous()
+    if cfg.swiglu:  # [2][p][f/p][h] (gate rows, then up rows) -> [p][2][f/p][h]
+        out["w1"] = full["w1"].reshape(2, p, f // p, h).permute(1, 0, 2, 3).contiguous()
+        if "b1" in full:
+            out["b1"] = full["b1"].reshape(2, p, f // p).permute(1, 0, 2).contiguous()
+    else:
+        out["w1"] = full["w1"].reshape(p, f // p, h).contiguous()
+        if "b1" in full:
+            out["b1"] = full["b1"].reshape(p, f // p).contiguous()
     out["w2"] = full["w2"].reshape(h, p, f // p).permute(1, 0, 2).contiguous()
     for k in ("ln1_g", "ln1_b", "b_o", "ln2_g", "ln2_b", "b2"):
-        out[k] = full[k].clone()
+        if k in full:
+            out[k] = full[k].clone()
     return out
 
 
@@ -170,11 +206,21 @@ def unpack_params(cfg: LayerConfig, packed: Dict[str, torch.Tensor]) -> Dict[str
     out = {}
     out["w_qkv"] = (packed["w_qkv"].reshape(p, 3, H // p, d, h).permute(1, 0, 2, 3, 4)
                     .reshape(3 * h, h).contiguous())
-    out["b_qkv"] = packed["b_qkv"].reshape(p, 3, H // p, d).permute(1, 0, 2, 3).reshape(3 * h)
+    if "b_qkv" in packed:
+        out["b_qkv"] = (packed["b_qkv"].reshape(p, 3, H // p, d).permute(1, 0, 2, 3)
+                        .reshape(3 * h))
     out["w_o"] = packed["w_o"].reshape(p, h, h // p).permute(1, 0, 2).reshape(h, h).contiguous()
-    out["w1"] = packed["w1"].reshape(f, h).contiguous()
-    out["b1"] = packed["b1"].reshape(f).contiguous()
+    if cfg.swiglu:
+        out["w1"] = (packed["w1"].reshape(p, 2, f // p, h).permute(1, 0, 2, 3)
+                     .reshape(2 * f, h).contiguous())
+        if "b1" in packed:
+            out["b1"] = packed["b1"].reshape(p, 2, f // p).permute(1, 0, 2).reshape(2 * f)
+    else:
+        out["w1"] = packed["w1"].reshape(f, h).contiguous()
+        if "b1" in packed:
+            out["b1"] = packed["b1"].reshape(f).contiguous()
     out["w2"] = packed["w2"].reshape(p, h, f // p).permute(1, 0, 2).reshape(h, f).contiguous()
     for k in ("ln1_g", "ln1_b", "b_o", "ln2_g", "ln2_b", "b2"):
-        out[k] = packed[k].clone()
+        if k in packed:
+            out[k] = packed[k].clone()
     return out

@@ -11,5 +11,5 @@ only primitive. No blocking, fusion or reordering beyond what the definition sta
 from .layer import (  # noqa: F401
     layer_norm, layer_norm_grad, gelu, gelu_grad, causal_softmax, attention_head_fwd,
     attention_head_bwd, attention_fwd, attention_bwd, layer_fwd, layer_bwd, layer_fwd_full,
-    layer_bwd_full, gather_grads,
+    layer_bwd_full, gather_grads, sigmoid, silu, silu_grad, swiglu, swiglu_grad,
 )

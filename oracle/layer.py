@@ -18,6 +18,8 @@ Sources (web pages about Megatron-LM; they print no formulas, so each reading is
   [ACT]  the trdm.cn page, section 3.3 (launch flags): GeLU is the default MLP activation.
   [RC]   the trdm.cn page, section 4.1 (checkpointing / recompute): only the layer input is
          kept and intermediates are recomputed in backward -- mathematically the identity.
+  [VAR]  the trdm.cn page, section 3.3 (launch flags): --swiglu replaces GeLU by SwiGLU, and
+         --disable-bias-linear removes the biases of the linear layers.
 
 Readings where the pages are silent (each also listed in the design notes):
   * LayerNorm: biased variance (divide by h), eps inside the square root, affine gamma/beta.
@@ -29,6 +31,10 @@ Readings where the pages are silent (each also listed in the design notes):
   * GeLU exact: u * Phi(u); the tanh form is selected by gelu_tanh=1.
   * QKV packing: shard-major, then [Q|K|V], then head, then head_dim.
   * No dropout.
+  * SwiGLU: fc1 gives two halves per shard, gate then up (each f/p wide); a = silu(gate)*up
+    with silu(z) = z*sigmoid(z); fc2 is unchanged (input width f).
+  * disable_bias_linear: b_qkv, b_o, b1, b2 are absent (not zero) and get no gradient; the
+    LayerNorm affine parameters stay.
 """
 from __future__ import annotations
 
@@ -159,7 +165,39 @@ def attention_bwd(qkv, dO, b, s, heads, tp):
     return dqkv
 
 
+# ----------------------------------------------------------------------------- SwiGLU ([VAR])
+def sigmoid(z):
+    """Logistic function 1/(1+exp(-z)), written as (1 + tanh(z/2))/2 (the same function,
+    without overflow for large |z|)."""
+    return 0.5 * (1.0 + np.tanh(0.5 * z))
+
+
+def silu(z):
+    """SiLU (swish): z * sigmoid(z)."""
+    return z * sigmoid(z)
+
+
+def silu_grad(z):
+    """d/dz [z*sigmoid(z)] = sigmoid(z) * (1 + z*(1 - sigmoid(z)))."""
+    sg = sigmoid(z)
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def swiglu(gate, up):
+    """SwiGLU activation: silu(gate) * up, elementwise."""
+    return silu(gate) * up
+
+
+def swiglu_grad(gate, up, da):
+    """Reverse of swiglu for the upstream grad da: (d gate, d up)."""
+    return da * up * silu_grad(gate), da * silu(gate)
+
+
 # ----------------------------------------------------------------------------- the layer
+def _flags(cfg):
+    return bool(getattr(cfg, "swiglu", 0)), bool(getattr(cfg, "disable_bias_linear", 0))
+
+
 def _np(a):
     if hasattr(a, "detach"):
         a = a.detach().cpu().to(dtype=__import__("torch").float64).numpy()
@@ -169,13 +207,16 @@ def _np(a):
 def layer_fwd(cfg, params, x):
     """Forward of the layer on packed per-shard parameters (the TP path).
 
-    cfg: object with hidden, heads, ffn, seq, micro_batch, tp_size, ln_eps, gelu_tanh.
+    cfg: object with hidden, heads, ffn, seq, micro_batch, tp_size, ln_eps, gelu_tanh and
+    optionally swiglu, disable_bias_linear.
     params: dict of packed arrays (layouts in the mgt_inputs docstring). x: [b, s, h].
     Returns (y [b, s, h], saved dict of every intermediate)."""
     h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
     b, s = cfg.micro_batch, cfg.seq
     T, d, hp = b * s, h // H, H // p
+    sw, nb = _flags(cfg)
     P = {k: _np(v) for k, v in params.items()}
+    bias = (lambda key: 0.0) if nb else (lambda key: P[key])  # noqa: E731
     x2 = _np(x).reshape(T, h)
 
     ln1, mu1, rstd1, xhat1 = layer_norm(x2, P["ln1_g"], P["ln1_b"], cfg.ln_eps)
@@ -184,7 +225,8 @@ def layer_fwd(cfg, params, x):
     qkv = np.empty((T, p, 3, hp, d))
     for t in range(p):
         w_t = P["w_qkv"][t].reshape(3 * hp * d, h)
-        qkv[:, t] = (ln1 @ w_t.T + P["b_qkv"][t].reshape(-1)).reshape(T, 3, hp, d)
+        b_t = 0.0 if nb else P["b_qkv"][t].reshape(-1)
+        qkv[:, t] = (ln1 @ w_t.T + b_t).reshape(T, 3, hp, d)
     O, lse = attention_fwd(qkv, b, s, H, p)
     # Row-parallel out-proj ([TP]): shard t multiplies its slice of the attention output by
     # its input-column block of W_o; the partials are summed (the AllReduce), then b_o is
@@ -192,17 +234,24 @@ def layer_fwd(cfg, params, x):
     acc = np.zeros((T, h))
     for t in range(p):
         acc += O[:, t].reshape(T, h // p) @ P["w_o"][t].T
-    h1 = x2 + P["b_o"] + acc
+    h1 = x2 + bias("b_o") + acc
     ln2, mu2, rstd2, xhat2 = layer_norm(h1, P["ln2_g"], P["ln2_b"], cfg.ln_eps)
-    # Column-parallel fc1 + GeLU, row-parallel fc2 with shard sum, bias once, residual.
-    u = np.empty((T, p, f // p))
-    for t in range(p):
-        u[:, t] = ln2 @ P["w1"][t].T + P["b1"][t]
-    a = gelu(u, cfg.gelu_tanh)
+    # Column-parallel fc1 + activation, row-parallel fc2 with shard sum, bias once, residual.
+    if sw:  # u [T][p][2][f/p]: each shard's gate half, then its up half
+        u = np.empty((T, p, 2, f // p))
+        for t in range(p):
+            for c in range(2):
+                u[:, t, c] = ln2 @ P["w1"][t, c].T + (0.0 if nb else P["b1"][t, c])
+        a = swiglu(u[:, :, 0], u[:, :, 1])
+    else:
+        u = np.empty((T, p, f // p))
+        for t in range(p):
+            u[:, t] = ln2 @ P["w1"][t].T + (0.0 if nb else P["b1"][t])
+        a = gelu(u, cfg.gelu_tanh)
     acc2 = np.zeros((T, h))
     for t in range(p):
         acc2 += a[:, t] @ P["w2"][t].T
-    y = h1 + P["b2"] + acc2
+    y = h1 + bias("b2") + acc2
     saved = dict(x=x2, ln1=ln1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, qkv=qkv, O=O, lse=lse,
                  h1=h1, ln2=ln2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, u=u, a=a)
     return y.reshape(b, s, h), saved
@@ -214,30 +263,40 @@ def layer_bwd(cfg, params, saved, dy):
     h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
     b, s = cfg.micro_batch, cfg.seq
     T, d, hp = b * s, h // H, H // p
+    sw, nb = _flags(cfg)
     P = {k: _np(v) for k, v in params.items()}
     dy2 = _np(dy).reshape(T, h)
     g = {}
     # fc2 (row-parallel): y = h1 + b2 + sum_t a_t W2_t^T
-    g["b2"] = dy2.sum(axis=0)
+    if not nb:
+        g["b2"] = dy2.sum(axis=0)
     g["w2"] = np.empty((p, h, f // p))
     da = np.empty((T, p, f // p))
     for t in range(p):
         g["w2"][t] = dy2.T @ saved["a"][:, t]
         da[:, t] = dy2 @ P["w2"][t]
-    du = da * gelu_grad(saved["u"], cfg.gelu_tanh)
+    u = saved["u"]
+    if sw:
+        du = np.stack(swiglu_grad(u[:, :, 0], u[:, :, 1], da), axis=2)  # [T][p][2][f/p]
+    else:
+        du = da * gelu_grad(u, cfg.gelu_tanh)
     # fc1 (column-parallel): the input ln2 was broadcast to every shard, so its gradient is
     # the sum of the shards' contributions.
-    g["b1"] = du.sum(axis=0)
-    g["w1"] = np.empty((p, f // p, h))
+    if not nb:
+        g["b1"] = du.sum(axis=0)
+    rows = (2 if sw else 1) * (f // p)  # fc1 output rows per shard
+    g["w1"] = np.empty((p,) + P["w1"].shape[1:])
     dln2 = np.zeros((T, h))
     for t in range(p):
-        g["w1"][t] = du[:, t].T @ saved["ln2"]
-        dln2 += du[:, t] @ P["w1"][t]
+        du_t = du[:, t].reshape(T, rows)
+        g["w1"][t] = (du_t.T @ saved["ln2"]).reshape(P["w1"].shape[1:])
+        dln2 += du_t @ P["w1"][t].reshape(rows, h)
     d_ln, g["ln2_g"], g["ln2_b"] = layer_norm_grad(dln2, saved["xhat2"], saved["rstd2"],
                                                    P["ln2_g"])
     dh1 = dy2 + d_ln
     # out-proj (row-parallel)
-    g["b_o"] = dh1.sum(axis=0)
+    if not nb:
+        g["b_o"] = dh1.sum(axis=0)
     g["w_o"] = np.empty((p, h, h // p))
     dO = np.empty((T, p, hp, d))
     for t in range(p):
@@ -245,12 +304,14 @@ def layer_bwd(cfg, params, saved, dy):
         dO[:, t] = (dh1 @ P["w_o"][t]).reshape(T, hp, d)
     dqkv = attention_bwd(saved["qkv"], dO, b, s, H, p)
     # QKV (column-parallel)
-    g["b_qkv"] = np.empty((p, 3, hp, d))
+    if not nb:
+        g["b_qkv"] = np.empty((p, 3, hp, d))
     g["w_qkv"] = np.empty((p, 3, hp, d, h))
     dln1 = np.zeros((T, h))
     for t in range(p):
         dq_t = dqkv[:, t].reshape(T, 3 * hp * d)
-        g["b_qkv"][t] = dq_t.sum(axis=0).reshape(3, hp, d)
+        if not nb:
+            g["b_qkv"][t] = dq_t.sum(axis=0).reshape(3, hp, d)
         g["w_qkv"][t] = (dq_t.T @ saved["ln1"]).reshape(3, hp, d, h)
         dln1 += dq_t @ P["w_qkv"][t].reshape(3 * hp * d, h)
     d_ln1, g["ln1_g"], g["ln1_b"] = layer_norm_grad(dln1, saved["xhat1"], saved["rstd1"],
@@ -262,15 +323,18 @@ def layer_bwd(cfg, params, saved, dy):
 
 def layer_fwd_full(cfg, params, x):
     """The same layer on full, unsharded matrices (no tensor parallelism): w_qkv [3h, h] with
-    rows [Q | K | V], head n of each at rows n*d..(n+1)*d-1; w_o [h, h]; w1 [f, h]; w2 [h, f].
+    rows [Q | K | V], head n of each at rows n*d..(n+1)*d-1; w_o [h, h]; w1 [f, h] (SwiGLU:
+    [2f, h], gate rows then up rows); w2 [h, f].
     Used to check that the sharded computation equals the unsharded one."""
-    h, H = cfg.hidden, cfg.heads
+    h, H, f = cfg.hidden, cfg.heads, cfg.ffn
     b, s = cfg.micro_batch, cfg.seq
     T, d = b * s, h // H
+    sw, nb = _flags(cfg)
     P = {k: _np(v) for k, v in params.items()}
+    bias = (lambda key: 0.0) if nb else (lambda key: P[key])  # noqa: E731
     x2 = _np(x).reshape(T, h)
     ln1, mu1, rstd1, xhat1 = layer_norm(x2, P["ln1_g"], P["ln1_b"], cfg.ln_eps)
-    qkv = ln1 @ P["w_qkv"].T + P["b_qkv"]
+    qkv = ln1 @ P["w_qkv"].T + bias("b_qkv")
     O = np.empty((T, h))
     for bi in range(b):
         rows = slice(bi * s, (bi + 1) * s)
@@ -279,11 +343,11 @@ def layer_fwd_full(cfg, params, x):
             o, _, _ = attention_head_fwd(qkv[rows, c], qkv[rows, h:][:, c],
                                          qkv[rows, 2 * h:][:, c])
             O[rows, c] = o
-    h1 = x2 + O @ P["w_o"].T + P["b_o"]
+    h1 = x2 + O @ P["w_o"].T + bias("b_o")
     ln2, mu2, rstd2, xhat2 = layer_norm(h1, P["ln2_g"], P["ln2_b"], cfg.ln_eps)
-    u = ln2 @ P["w1"].T + P["b1"]
-    a = gelu(u, cfg.gelu_tanh)
-    y = h1 + a @ P["w2"].T + P["b2"]
+    u = ln2 @ P["w1"].T + bias("b1")
+    a = swiglu(u[:, :f], u[:, f:]) if sw else gelu(u, cfg.gelu_tanh)
+    y = h1 + a @ P["w2"].T + bias("b2")
     saved = dict(x=x2, ln1=ln1, xhat1=xhat1, rstd1=rstd1, qkv=qkv, O=O, h1=h1, ln2=ln2,
                  xhat2=xhat2, rstd2=rstd2, u=u, a=a)
     return y.reshape(b, s, h), saved
@@ -291,21 +355,30 @@ def layer_fwd_full(cfg, params, x):
 
 def layer_bwd_full(cfg, params, saved, dy):
     """Reverse of layer_fwd_full. Returns (dx, grads in the full layout)."""
-    h, H = cfg.hidden, cfg.heads
+    h, H, f = cfg.hidden, cfg.heads, cfg.ffn
     b, s = cfg.micro_batch, cfg.seq
     T, d = b * s, h // H
+    sw, nb = _flags(cfg)
     P = {k: _np(v) for k, v in params.items()}
     dy2 = _np(dy).reshape(T, h)
     g = {}
-    g["b2"] = dy2.sum(axis=0)
+    if not nb:
+        g["b2"] = dy2.sum(axis=0)
     g["w2"] = dy2.T @ saved["a"]
-    du = (dy2 @ P["w2"]) * gelu_grad(saved["u"], cfg.gelu_tanh)
-    g["b1"] = du.sum(axis=0)
+    da = dy2 @ P["w2"]
+    u = saved["u"]
+    if sw:
+        du = np.concatenate(swiglu_grad(u[:, :f], u[:, f:], da), axis=1)
+    else:
+        du = da * gelu_grad(u, cfg.gelu_tanh)
+    if not nb:
+        g["b1"] = du.sum(axis=0)
     g["w1"] = du.T @ saved["ln2"]
     d_ln, g["ln2_g"], g["ln2_b"] = layer_norm_grad(du @ P["w1"], saved["xhat2"],
                                                    saved["rstd2"], P["ln2_g"])
     dh1 = dy2 + d_ln
-    g["b_o"] = dh1.sum(axis=0)
+    if not nb:
+        g["b_o"] = dh1.sum(axis=0)
     g["w_o"] = dh1.T @ saved["O"]
     dO = dh1 @ P["w_o"]
     qkv = saved["qkv"]
@@ -320,7 +393,8 @@ def layer_bwd_full(cfg, params, saved, dy):
             dqkv[rows, n * d:(n + 1) * d] = dq
             dqkv[rows, h + n * d:h + (n + 1) * d] = dk
             dqkv[rows, 2 * h + n * d:2 * h + (n + 1) * d] = dv
-    g["b_qkv"] = dqkv.sum(axis=0)
+    if not nb:
+        g["b_qkv"] = dqkv.sum(axis=0)
     g["w_qkv"] = dqkv.T @ saved["ln1"]
     d_ln1, g["ln1_g"], g["ln1_b"] = layer_norm_grad(dqkv @ P["w_qkv"], saved["xhat1"],
                                                     saved["rstd1"], P["ln1_g"])
@@ -333,13 +407,23 @@ def gather_grads(cfg, g):
     packing), so sharded results can be compared with layer_bwd_full."""
     h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
     d, hp = h // H, H // p
+    sw, _ = _flags(cfg)
     out = dict(g)
     out["w_qkv"] = np.asarray(g["w_qkv"]).reshape(p, 3, hp, d, h).transpose(1, 0, 2, 3, 4) \
         .reshape(3 * h, h)
-    out["b_qkv"] = np.asarray(g["b_qkv"]).reshape(p, 3, hp, d).transpose(1, 0, 2, 3) \
-        .reshape(3 * h)
+    if "b_qkv" in g:
+        out["b_qkv"] = np.asarray(g["b_qkv"]).reshape(p, 3, hp, d).transpose(1, 0, 2, 3) \
+            .reshape(3 * h)
     out["w_o"] = np.asarray(g["w_o"]).reshape(p, h, h // p).transpose(1, 0, 2).reshape(h, h)
-    out["w1"] = np.asarray(g["w1"]).reshape(f, h)
-    out["b1"] = np.asarray(g["b1"]).reshape(f)
+    if sw:  # [p][2][f/p] -> [2][p][f/p]: all gate rows, then all up rows
+        out["w1"] = np.asarray(g["w1"]).reshape(p, 2, f // p, h).transpose(1, 0, 2, 3) \
+            .reshape(2 * f, h)
+        if "b1" in g:
+            out["b1"] = np.asarray(g["b1"]).reshape(p, 2, f // p).transpose(1, 0, 2) \
+                .reshape(2 * f)
+    else:
+        out["w1"] = np.asarray(g["w1"]).reshape(f, h)
+        if "b1" in g:
+            out["b1"] = np.asarray(g["b1"]).reshape(f)
     out["w2"] = np.asarray(g["w2"]).reshape(p, h, f // p).transpose(1, 0, 2).reshape(h, f)
     return out

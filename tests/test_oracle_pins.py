@@ -115,22 +115,32 @@ def torch_layer(cfg, full, x):
     h, H = cfg.hidden, cfg.heads
     d = h // H
     b, s = cfg.micro_batch, cfg.seq
+    bias = lambda k: full.get(k)  # noqa: E731  (absent under disable_bias_linear)
     ln1 = F.layer_norm(x, (h,), full["ln1_g"], full["ln1_b"], cfg.ln_eps)
-    qkv = F.linear(ln1, full["w_qkv"], full["b_qkv"])
+    qkv = F.linear(ln1, full["w_qkv"], bias("b_qkv"))
     q, k, v = qkv.split(h, dim=-1)
     heads = lambda t: t.reshape(b, s, H, d).transpose(1, 2)  # noqa: E731
     o = F.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=True)
     o = o.transpose(1, 2).reshape(b, s, h)
-    h1 = x + F.linear(o, full["w_o"], full["b_o"])
+    h1 = x + F.linear(o, full["w_o"], bias("b_o"))
     ln2 = F.layer_norm(h1, (h,), full["ln2_g"], full["ln2_b"], cfg.ln_eps)
-    a = F.gelu(F.linear(ln2, full["w1"], full["b1"]),
-               approximate="tanh" if cfg.gelu_tanh else "none")
-    return h1 + F.linear(a, full["w2"], full["b2"])
+    u = F.linear(ln2, full["w1"], bias("b1"))
+    if cfg.swiglu:
+        gate, up = u.chunk(2, dim=-1)
+        a = F.silu(gate) * up
+    else:
+        a = F.gelu(u, approximate="tanh" if cfg.gelu_tanh else "none")
+    return h1 + F.linear(a, full["w2"], bias("b2"))
 
 
-@pytest.mark.parametrize("gelu_tanh", [0, 1])
-def test_layer_vs_torch_composition(gelu_tanh):
-    cfg = tiny(p=2, gelu_tanh=gelu_tanh)
+VARIANT_KW = {"gelu": {}, "gelu_tanh": {"gelu_tanh": 1}, "swiglu": {"swiglu": 1},
+              "nobias": {"disable_bias_linear": 1},
+              "swiglu_nobias": {"swiglu": 1, "disable_bias_linear": 1}}
+
+
+@pytest.mark.parametrize("variant", list(VARIANT_KW))
+def test_layer_vs_torch_composition(variant):
+    cfg = tiny(p=2, **VARIANT_KW[variant])
     t = make_inputs(cfg, nonzero_affine=True)
     full = {k: v.double() for k, v in t.items()}
     y, saved = oracle.layer_fwd(cfg, pack_params(cfg, full), full["x"])
@@ -138,7 +148,8 @@ def test_layer_vs_torch_composition(gelu_tanh):
     g = oracle.gather_grads(cfg, g)
     leaves = {k: full[k].clone().requires_grad_(True) for k in
               ("x", "ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o", "ln2_g", "ln2_b", "w1",
-               "b1", "w2", "b2")}
+               "b1", "w2", "b2") if k in full}
+    assert set(g) == set(leaves) - {"x"}
     yt = torch_layer(cfg, leaves, leaves["x"])
     assert rel(y, yt.detach().numpy()) < 1e-13
     yt.backward(full["dy"])
@@ -147,11 +158,13 @@ def test_layer_vs_torch_composition(gelu_tanh):
         assert rel(g[k], leaves[k].grad.numpy()) < 1e-11, k
 
 
-@pytest.mark.parametrize("p", [2, 4])
-def test_sharded_equals_unsharded(p):
+@pytest.mark.parametrize("p,variant", [(2, "gelu"), (4, "gelu"), (2, "swiglu"),
+                                       (4, "swiglu_nobias")])
+def test_sharded_equals_unsharded(p, variant):
     """Column-split QKV/fc1 and row-split out-proj/fc2 with summed partials give the result of
-    the unsplit layer (the partitioning claim of the trdm.cn page, section 2.1)."""
-    cfg = tiny(p=p, hidden=32, heads=4, ffn=64)
+    the unsplit layer (the partitioning claim of the trdm.cn page, section 2.1). With SwiGLU
+    each shard holds matching gate and up rows, so the activation stays shard-local."""
+    cfg = tiny(p=p, hidden=32, heads=4, ffn=64, **VARIANT_KW[variant])
     t = make_inputs(cfg, nonzero_affine=True)
     full = {k: v.double() for k, v in t.items()}
     y_s, sv_s = oracle.layer_fwd(cfg, pack_params(cfg, full), full["x"])
@@ -187,11 +200,12 @@ def test_seq1_attention_is_v_projection():
     assert rel(saved["h1"], expect) < 1e-13
 
 
-def test_backward_central_finite_differences():
+@pytest.mark.parametrize("variant", ["gelu", "swiglu", "swiglu_nobias"])
+def test_backward_central_finite_differences(variant):
     """Central differences of L = <y, dy> along random directions, for x and every
     parameter: relative error <= 1e-6. The step 1e-5 balances truncation (O(eps^2)) against
     rounding (1e-16*|L|/eps); both stay near 1e-10 here."""
-    cfg = tiny(p=2, hidden=8, heads=2, ffn=16, seq=5)
+    cfg = tiny(p=2, hidden=8, heads=2, ffn=16, seq=5, **VARIANT_KW[variant])
     t = make_inputs(cfg, nonzero_affine=True)
     full = {k: v.double() for k, v in t.items()}
     packed = {k: v.numpy() for k, v in pack_params(cfg, full).items()}
@@ -234,3 +248,67 @@ def test_pack_unpack_roundtrip():
         assert torch.equal(pk["w_qkv"][n // hp, 0, n % hp], t["w_qkv"][n * d:(n + 1) * d])
         assert torch.equal(pk["w_qkv"][n // hp, 2, n % hp],
                            t["w_qkv"][2 * cfg.hidden + n * d:2 * cfg.hidden + (n + 1) * d])
+
+
+# ------------------------------------------------------------------ SwiGLU and no-bias
+def test_silu_and_sigmoid_vs_torch():
+    z = torch.linspace(-60.0, 60.0, 4001, dtype=torch.float64)
+    zn = z.numpy()
+    assert rel(oracle.sigmoid(zn), torch.sigmoid(z).numpy()) < 1e-15
+    assert rel(oracle.silu(zn), F.silu(z).numpy()) < 1e-15
+    zz = z.clone().requires_grad_(True)
+    F.silu(zz).sum().backward()
+    assert rel(oracle.silu_grad(zn), zz.grad.numpy()) < 1e-14
+
+
+def test_swiglu_closed_forms_and_grad():
+    rng = np.random.default_rng(3)
+    gate, up, da = rng.normal(size=(3, 50, 20)) * 3.0
+    # silu(0) = 0, so a zero gate gives a = 0 and no gradient to up; large gates pass through
+    assert np.all(oracle.swiglu(np.zeros(5), np.arange(5.0)) == 0.0)
+    assert rel(oracle.swiglu(np.full(3, 40.0), up[0, :3]), 40.0 * up[0, :3]) < 1e-15
+    assert np.max(np.abs(oracle.swiglu(np.full(3, -40.0), up[0, :3]))) < 1e-15
+    tg = torch.tensor(gate, requires_grad=True)
+    tu = torch.tensor(up, requires_grad=True)
+    (F.silu(tg) * tu).backward(torch.tensor(da))
+    dg, du = oracle.swiglu_grad(gate, up, da)
+    assert rel(dg, tg.grad.numpy()) < 1e-14
+    assert rel(du, tu.grad.numpy()) < 1e-14
+
+
+@pytest.mark.parametrize("swiglu", [0, 1])
+def test_no_bias_equals_zero_bias(swiglu):
+    """Dropping the linear biases is the layer with those biases fixed at zero: identical y,
+    dx and weight/LN gradients, and no bias gradients at all."""
+    cfg = tiny(p=2, swiglu=swiglu)
+    cfg_nb = cfg.replace(disable_bias_linear=1)
+    t = make_inputs(cfg, nonzero_affine=True)
+    full = {k: v.double() for k, v in t.items()}
+    for k in ("b_qkv", "b_o", "b1", "b2"):
+        full[k] = torch.zeros_like(full[k])
+    full_nb = {k: v for k, v in full.items() if k not in ("b_qkv", "b_o", "b1", "b2")}
+    y0, s0 = oracle.layer_fwd(cfg, pack_params(cfg, full), full["x"])
+    y1, s1 = oracle.layer_fwd(cfg_nb, pack_params(cfg_nb, full_nb), full["x"])
+    assert np.array_equal(y0, y1)
+    dx0, g0, _ = oracle.layer_bwd(cfg, pack_params(cfg, full), s0, full["dy"])
+    dx1, g1, _ = oracle.layer_bwd(cfg_nb, pack_params(cfg_nb, full_nb), s1, full["dy"])
+    assert np.array_equal(dx0, dx1)
+    assert set(g1) == set(g0) - {"b_qkv", "b_o", "b1", "b2"}
+    for k in g1:
+        assert np.array_equal(g0[k], g1[k]), k
+
+
+def test_swiglu_packing_pairs_gate_and_up():
+    """Shard t of the packed SwiGLU fc1 holds gate rows t*f/p.. and the up rows with the same
+    indices, so gate j and up j meet on one shard."""
+    cfg = tiny(p=4, hidden=32, heads=8, ffn=64, swiglu=1)
+    t = make_inputs(cfg, nonzero_affine=True)
+    pk = pack_params(cfg, t)
+    f, fp = cfg.ffn, cfg.ffn // cfg.tp_size
+    for j in range(f):
+        assert torch.equal(pk["w1"][j // fp, 0, j % fp], t["w1"][j])
+        assert torch.equal(pk["w1"][j // fp, 1, j % fp], t["w1"][f + j])
+        assert pk["b1"][j // fp, 1, j % fp] == t["b1"][f + j]
+    back = unpack_params(cfg, pk)
+    for k in back:
+        assert torch.equal(back[k], t[k]), k
