@@ -149,7 +149,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
         for (int q = 0; q < 4; ++q) {
           float ga[8], gd[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) gelu_and_grad_f(v[q * 8 + j], a.gelu_tanh, ga[j], gd[j]);
+          for (int j = 0; j < 8; ++j) gelu_and_grad_bf16out(v[q * 8 + j], a.gelu_tanh, ga[j], gd[j]);
           uint4 wd, wa;
           wd.x = pack_bf16x2(gd[0], gd[1]);
           wd.y = pack_bf16x2(gd[2], gd[3]);
@@ -167,7 +167,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
         for (int i = 0; i < 32; ++i) {
           if (i < count) {
             float ga, gd;
-            gelu_and_grad_f(v[i], a.gelu_tanh, ga, gd);
+            gelu_and_grad_bf16out(v[i], a.gelu_tanh, ga, gd);
             o2[i] = __float2bfloat16_rn(gd);
             o[i] = __float2bfloat16_rn(ga);
           }
@@ -190,6 +190,66 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
       for (int i = 0; i < 32; ++i)
         if (i < count) o[i] = __float2bfloat16_rn(v[i]);
     }
+  }
+}
+
+// Values of one whole 32-column chunk of a bf16 epilogue, packed as bf16 pairs for a staged
+// (TMA) store: w holds out, w2 out2 (kEpiGelu only). Rows at or past M (row_ok false) read no
+// residual or aux; the store clips them.
+template <int EPI>
+__device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int col, bool row_ok,
+                                                float (&v)[32], uint32_t (&w)[16],
+                                                uint32_t (&w2)[16]) {
+  const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+  if ((EPI == kEpiBf16 || EPI == kEpiGelu) && bias) {
+    const uint4* bp = reinterpret_cast<const uint4*>(bias + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u4 = __ldg(bp + q);
+      const uint32_t ww[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[q * 8 + 2 * j] += bf16_lo(ww[j]);
+        v[q * 8 + 2 * j + 1] += bf16_hi(ww[j]);
+      }
+    }
+  }
+  if ((EPI == kEpiBf16 && a.res) || EPI == kEpiDGelu) {
+    const __nv_bfloat16* src =
+        EPI == kEpiDGelu
+            ? reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col
+            : reinterpret_cast<const __nv_bfloat16*>(a.res) + (long long)row * a.ldr + col;
+    uint4 r4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      r4[q] = row_ok ? *reinterpret_cast<const uint4*>(src + q * 8) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t ww[4] = {r4[q].x, r4[q].y, r4[q].z, r4[q].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (EPI == kEpiDGelu) {  // aux holds GeLU'(u), stored by the forward epilogue
+          v[q * 8 + 2 * j] *= bf16_lo(ww[j]);
+          v[q * 8 + 2 * j + 1] *= bf16_hi(ww[j]);
+        } else {
+          v[q * 8 + 2 * j] += bf16_lo(ww[j]);
+          v[q * 8 + 2 * j + 1] += bf16_hi(ww[j]);
+        }
+      }
+    }
+  }
+  if constexpr (EPI == kEpiGelu) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float g0, d0, g1, d1;
+      gelu_and_grad_bf16out(v[2 * i], a.gelu_tanh, g0, d0);
+      gelu_and_grad_bf16out(v[2 * i + 1], a.gelu_tanh, g1, d1);
+      w[i] = pack_bf16x2(g0, g1);
+      w2[i] = pack_bf16x2(d0, d1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
   }
 }
 
@@ -416,11 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairStages = 6;
 constexpr int kPairAB = BM * BK * 2;            // 16 KB: this CTA's A rows or B half
 constexpr int kPairStageBytes = 2 * kPairAB;    // 32 KB per CTA per stage
-constexpr int kStageOut = 32 * 32 * 4;          // fp32 store staging: 32 rows x 32 columns
-// stages | barriers (padded to 1 KB) | fp32 staging (fp32 epilogue only) | 1 KB alignment slack
-constexpr int pair_smem(int epi) {
-  return kPairStages * kPairStageBytes + 1024 + (epi == kEpiStoreF32 ? kEpiWarps * kStageOut : 0) +
-         1024;
+// Output staging per epilogue warp: one 32 x 32 fp32 chunk (128-byte rows), or up to two
+// 32 x 32 bf16 chunks (64-byte rows; out and, for kEpiGelu, out2 2 KB further on).
+constexpr int kStageOut = 32 * 32 * 4;
+// stages | barriers (padded to 1 KB) | output staging | 1 KB alignment slack
+constexpr int pair_smem(int) {
+  return kPairStages * kPairStageBytes + 1024 + kEpiWarps * kStageOut + 1024;
 }
 static_assert(pair_smem(kEpiStoreF32) <= 232448, "shared memory per CTA");
 
@@ -428,11 +489,15 @@ template <bool A_MN, bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, const GemmArgs args, int num_m2,
-                    int num_n, int BN) {
-  // tmC (fp32 epilogue only): output viewed as {out_ng, M, groups}; each epilogue warp stages
-  // a 32 x 32 fp32 chunk in a 128B-swizzled shared buffer and stores it with one TMA bulk
-  // tensor store (coalesced full lines; rows past M and columns past N are clipped).
+                    const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmC2, const GemmArgs args, int num_m2,
+                    int num_n, int BN, int staged) {
+  // tmC (tmC2: out2 of kEpiGelu): output viewed as {out_ng, M, groups}; each epilogue warp
+  // stages a 32 x 32 chunk in a swizzled shared buffer (128-byte rows for fp32, 64-byte rows
+  // for bf16) and stores it with one TMA bulk tensor store (full lines, coalesced; rows past M
+  // are clipped). A chunk that straddles N is written element by element instead, and so is
+  // every chunk when `staged` is 0 (the host found a column offset that is not a multiple of
+  // 16 bytes, which a TMA store cannot start at).
   // BN: the pair's N tile, a multiple of 32 up to 256 (256 when B is MN-major); each CTA
   // loads BN/2 rows of B. Accumulator buffers stay 256 columns apart in TMEM.
   const uint32_t b_bytes = (uint32_t)(BN / 2) * BK * 2;
@@ -473,7 +538,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI == kEpiStoreF32) tma_prefetch_desc(&tmC);
+    if (staged) {
+      tma_prefetch_desc(&tmC);
+      if (EPI == kEpiGelu) tma_prefetch_desc(&tmC2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -605,31 +673,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256 + c * 32,
                            v);
         const int n0 = tc.nb * BN + c * 32;
-        if constexpr (EPI == kEpiStoreF32) {
-          const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
-          // Whole chunks go through TMA; a chunk straddling N is written element by element
-          // (the bulk store clips the inner dimension only at 16-byte granularity).
-          if (n0 < args.Ng && n0 + 32 > args.Ng) {
-            if (row < args.M) epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, args.Ng - n0, v);
-          } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
-            uint8_t* buf = stage_out + (warp - 2) * kStageOut;
+        const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
+        const int col = tc.ng * args.Ng + n0;
+        // Whole chunks go through TMA; a chunk straddling N is written element by element
+        // (the bulk store clips the inner dimension only at 16-byte granularity).
+        if (n0 < args.Ng && (n0 + 32 > args.Ng || !staged)) {
+          if (row < args.M) epilogue_chunk<EPI>(args, row, col, min(32, args.Ng - n0), v);
+        } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
+          uint8_t* buf = stage_out + (warp - 2) * kStageOut;
+          if constexpr (EPI == kEpiStoreF32) {
             if (lane == 0) bulk_wait_read0();  // the previous chunk's store has read the buffer
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            fence_proxy_async_smem();
+          } else {
+            uint32_t w[16], w2[16];
+            epi_values_bf16<EPI>(args, row, col, row < args.M, v, w, w2);
+            if (lane == 0) bulk_wait_read0();
             __syncwarp();
-            if (lane == 0) {
-              const int col = tc.ng * args.Ng + n0;
-              tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
-              bulk_commit();
+            // 64-byte rows, 64-byte swizzle: 16-byte unit j of row r sits at unit
+            // j ^ ((r >> 1) & 3), so the 32 lanes' stores fill whole 128-byte wavefronts.
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) =
+                  make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              if (EPI == kEpiGelu)
+                *reinterpret_cast<uint4*>(buf + 2048 + lane * 64 + ((j ^ sw) << 4)) =
+                    make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
             }
           }
-        } else if (row < args.M && n0 < args.Ng) {
-          const int count = min(32, args.Ng - n0);
-          epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, count, v);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
+            if (EPI == kEpiGelu)
+              tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, row0, col / args.out_ng);
+            bulk_commit();
+          }
         }
       }
       tc_fence_before();
@@ -642,7 +725,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (EPI == kEpiStoreF32 && warp >= 2 && lane == 0) bulk_wait0();
+  if (warp >= 2 && lane == 0) bulk_wait0();  // staged stores have finished reading smem
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while its peer may still touch its barriers or TMEM
@@ -724,19 +807,23 @@ cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
 }
 
 // fp32 output viewed as {out_ng, M, groups} with a 32 x 32 box (128-byte rows, swizzled).
-bool make_out_map_f32(CUtensorMap* m, const GemmArgs& a) {
+// Output tensor map for the staged epilogue store: {out_ng, M, groups}, box 32 x 32; fp32 with
+// 128-byte swizzle (128-byte rows), bf16 with 64-byte swizzle (64-byte rows).
+bool make_out_map(CUtensorMap* m, const GemmArgs& a, void* base, bool f32) {
   auto fn = get_encode_fn();
   if (!fn) return false;
+  const long long esz = f32 ? 4 : 2;
   const long long ncols = (long long)a.Ng * a.NG;
   const long long groups = (ncols + a.out_ng - 1) / a.out_ng;
   cuuint64_t gd[3] = {(cuuint64_t)(ncols < a.out_ng ? ncols : a.out_ng), (cuuint64_t)a.M,
                       (cuuint64_t)groups};
-  cuuint64_t gs[2] = {(cuuint64_t)a.ldc * 4,
-                      (cuuint64_t)(groups > 1 ? a.out_gs : a.ldc * a.M) * 4};
+  cuuint64_t gs[2] = {(cuuint64_t)(a.ldc * esz),
+                      (cuuint64_t)((groups > 1 ? a.out_gs : a.ldc * a.M) * esz)};
   cuuint32_t bd[3] = {32, 32, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.out, gd, gs, bd, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+            gd, gs, bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -752,14 +839,26 @@ cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  CUtensorMap tc;
+  CUtensorMap tc, tc2;
   std::memset(&tc, 0, sizeof(tc));
-  if (EPI == kEpiStoreF32 && !make_out_map_f32(&tc, a)) return cudaErrorInvalidValue;
+  std::memset(&tc2, 0, sizeof(tc2));
+  // A staged store covers output columns col .. col+31, col = ng*Ng + n0 with n0 a multiple of
+  // 32, at inner coordinate col % out_ng. It needs col to be a multiple of 16 bytes' worth of
+  // elements (true for one group, else Ng must be) and must not run across an out_ng boundary
+  // (true if one out_ng block holds every column, else out_ng must be a multiple of 32).
+  // Tensor-map encoding also needs 16-byte aligned bases and strides.
+  const int vec = EPI == kEpiStoreF32 ? 4 : 8;
+  const bool cols_ok = (a.NG == 1 || a.Ng % vec == 0) &&
+                       ((long long)a.out_ng >= (long long)a.Ng * a.NG || a.out_ng % 32 == 0);
+  int staged = cols_ok ? 1 : 0;
+  if (staged && !make_out_map(&tc, a, a.out, EPI == kEpiStoreF32)) staged = 0;
+  if (staged && EPI == kEpiGelu && !make_out_map(&tc2, a, a.out2, false)) staged = 0;
   const int num_m2 = (a.M + 255) / 256;
   const int num_n = (a.Ng + bn - 1) / bn;
   const int tiles = a.NG * num_m2 * num_n;
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  kern<<<2 * pairs, kThreads, smem_bytes, stream>>>(ta, tb, tc, a, num_m2, num_n, bn);
+  kern<<<2 * pairs, kThreads, smem_bytes, stream>>>(ta, tb, tc, tc2, a, num_m2, num_n, bn,
+                                                     staged);
   return cudaGetLastError();
 }
 

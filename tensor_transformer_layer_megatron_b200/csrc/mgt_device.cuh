@@ -394,6 +394,45 @@ __device__ __forceinline__ void gelu_and_grad_f(float u, int tanh_form, float& g
   g = u * cdf;
   dg = cdf + u * 0.3989422804014327f * expf(-0.5f * u * u);
 }
+// GeLU(u) and GeLU'(u) for the bf16 GEMM epilogue, whose outputs are rounded to bf16 (relative
+// step 2^-8): erf from the rational approximation of Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (after Hastings), |error| <= 1.5e-7 for x >= 0, odd
+// extension for x < 0. Its factor e^{-x^2} with x = u/sqrt(2) is the Gaussian density's
+// exponent, so GeLU' = Phi(u) + u * e^{-u^2/2} / sqrt(2 pi) reuses it. The tanh form uses the
+// hardware tanh (tanh.approx.f32, relative error about 2^-11).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void gelu_and_grad_bf16out(float u, int tanh_form, float& g,
+                                                      float& dg) {
+  if (tanh_form) {
+    const float u2 = u * u;
+    const float t = tanh_approx(0.7978845608028654f * fmaf(0.044715f * u2, u, u));
+    const float half1pt = fmaf(0.5f, t, 0.5f);
+    g = u * half1pt;
+    dg = fmaf(0.5f * u * fmaf(-t, t, 1.0f), 0.7978845608028654f * fmaf(0.134145f, u2, 1.0f),
+              half1pt);
+    return;
+  }
+  const float x = u * 0.7071067811865476f;
+  const float ax = fabsf(x);
+  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
+  const float e = ex2_approx(-1.4426950408889634f * x * x);  // e^{-x^2} = e^{-u^2/2}
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f),
+                       -0.284496736f), 0.254829592f);
+  const float erf_ax = fmaf(-poly, e, 1.0f);
+  const float cdf = fmaf(0.5f, copysignf(erf_ax, x), 0.5f);
+  g = u * cdf;
+  dg = fmaf(u * 0.3989422804014327f, e, cdf);
+}
 __device__ __forceinline__ float gelu_grad_f(float u, int tanh_form) {
   if (tanh_form) {
     const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);
