@@ -279,6 +279,9 @@ def run_mgt(args):
             "frac_of_measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
             "frac_of_measured_burst": round(tflops / peaks["bf16_tflops"], 4),
             "config": {"workload": cfg.name, "hidden": cfg.hidden, "heads": cfg.heads,
+                       "mlp": "swiglu" if cfg.swiglu else ("gelu-tanh" if cfg.gelu_tanh
+                                                           else "gelu"),
+                       "linear_bias": not cfg.disable_bias_linear,
                        "ffn": cfg.ffn, "seq_len": cfg.seq, "micro_batch": cfg.micro_batch,
                        "tp_size": cfg.tp_size, "tokens_per_gpu": cfg.tokens,
                        "global_batch": cfg.micro_batch * world,
@@ -325,7 +328,7 @@ def run_torch(args):
     h, H, d, b, s = cfg.hidden, cfg.heads, cfg.head_dim, cfg.micro_batch, cfg.seq
     names = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o", "ln2_g", "ln2_b", "w1", "b1",
              "w2", "b2")
-    P = {k: t[k].to(dev, dt).requires_grad_(True) for k in names}
+    P = {k: t[k].to(dev, dt).requires_grad_(True) for k in names if k in t}
     x = t["x"].to(dev, dt).requires_grad_(True)
     dy = t["dy"].to(dev, dt)
     approx = "tanh" if cfg.gelu_tanh else "none"
@@ -335,13 +338,18 @@ def run_torch(args):
             v.grad = None
         x.grad = None
         ln1 = F.layer_norm(x, (h,), P["ln1_g"], P["ln1_b"], cfg.ln_eps)
-        q, k, v = F.linear(ln1, P["w_qkv"], P["b_qkv"]).view(b, s, 3, H, d).unbind(2)
+        q, k, v = F.linear(ln1, P["w_qkv"], P.get("b_qkv")).view(b, s, 3, H, d).unbind(2)
         o = F.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2),
                                            v.transpose(1, 2), is_causal=True)
-        h1 = x + F.linear(o.transpose(1, 2).reshape(b, s, h), P["w_o"], P["b_o"])
+        h1 = x + F.linear(o.transpose(1, 2).reshape(b, s, h), P["w_o"], P.get("b_o"))
         ln2 = F.layer_norm(h1, (h,), P["ln2_g"], P["ln2_b"], cfg.ln_eps)
-        a = F.gelu(F.linear(ln2, P["w1"], P["b1"]), approximate=approx)
-        y = h1 + F.linear(a, P["w2"], P["b2"])
+        u = F.linear(ln2, P["w1"], P.get("b1"))
+        if cfg.swiglu:
+            gate, up = u.chunk(2, dim=-1)
+            a = F.silu(gate) * up
+        else:
+            a = F.gelu(u, approximate=approx)
+        y = h1 + F.linear(a, P["w2"], P.get("b2"))
         y.backward(dy)
         return y
 

@@ -11,6 +11,10 @@
  *   a   = GeLU(ln2 W1^T + b1)         column-parallel
  *   y   = h1 + b2 + sum_t a_t W2,t^T      row-parallel
  *
+ * Variants (launch flags on the trdm.cn page, section 3.3): swiglu = 1 gives the MLP
+ * a = silu(gate) * up with [gate | up] = ln2 W1^T + b1 (fc1 has 2*ffn outputs, each shard its
+ * own gate and up halves); disable_bias_linear = 1 drops b_qkv, b_o, b1 and b2.
+ *
  * Sources: the page "Megatron-LM 3D并行原理与万亿参数训练实战指南" (trdm.cn), section 2.1
  * (tensor parallelism: W_q/W_k/W_v split by output columns with x broadcast and no
  * communication; W_o split by input rows with partial outputs summed by AllReduce), section 3.2
@@ -29,6 +33,7 @@
  *         w_qkv [p][3][H/p][d][h]   b_qkv [p][3][H/p][d]
  *         w_o   [p][h][h/p]         b_o   [h]
  *         w1    [p][f/p][h]         b1    [p][f/p]
+ *         (swiglu: w1 [p][2][f/p][h], b1 [p][2][f/p]: shard t's gate rows, then its up rows)
  *         w2    [p][h][f/p]         b2    [h]
  *         ln1_g, ln1_b, ln2_g, ln2_b [h]
  *   - x, y, dx, dy: [b, s, h], tokens flattened as T = b*s with s fastest.
@@ -75,7 +80,9 @@ typedef enum mgt_dtype { MGT_F32 = 0, MGT_BF16 = 1 } mgt_dtype;
  * ffn % tp_size == 0; head_dim in {64, 128} for bf16, <= 64 for f32; for bf16 also
  * hidden/tp_size and ffn/tp_size multiples of 64. causal must be 1 (the GPT mask);
  * recompute_attn is accepted for either value -- attention probabilities are never stored,
- * the backward always recomputes them from the saved log-sum-exp. */
+ * the backward always recomputes them from the saved log-sum-exp. swiglu and
+ * disable_bias_linear are 0 or 1 (a zero-filled tail keeps the GeLU layer with biases);
+ * gelu_tanh has no effect with swiglu. */
 typedef struct mgt_layer_config {
   int32_t hidden;
   int32_t heads;
@@ -88,9 +95,12 @@ typedef struct mgt_layer_config {
   float ln_eps;           /* LayerNorm epsilon, added to the biased variance */
   int32_t recompute_attn; /* informational; see above */
   int32_t gelu_tanh;      /* 0: exact erf GeLU; 1: tanh approximation */
+  int32_t swiglu;         /* 0: GeLU MLP; 1: SwiGLU, a = silu(gate) * up (fc1: 2*ffn outputs) */
+  int32_t disable_bias_linear; /* 1: no biases in QKV, out-proj, fc1, fc2 (b_* may be NULL) */
 } mgt_layer_config;
 
-/* Parameters (device pointers, packed layouts above). */
+/* Parameters (device pointers, packed layouts above). With disable_bias_linear the four b_*
+ * pointers are ignored and may be NULL; likewise their gradients. */
 typedef struct mgt_layer_params {
   const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o;
   const void *ln2_g, *ln2_b, *w1, *b1, *w2, *b2;
@@ -124,11 +134,12 @@ typedef enum mgt_region {
   MGT_SAVED_LN2 = 7,        /* ACT [T, h]                                              */
   MGT_SAVED_LN2_MEAN = 8,   /* F32 [T]                                                 */
   MGT_SAVED_LN2_RSTD = 9,   /* F32 [T]                                                 */
-  MGT_SAVED_FC1_DGELU = 10, /* ACT [T][p][f/p]     GeLU'(u), u = fc1 pre-activation    */
-  MGT_SAVED_FC1_A = 11,     /* ACT [T][p][f/p]     GeLU(u)                             */
+  MGT_SAVED_FC1_DGELU = 10, /* ACT [T][p][f/p]     GeLU'(u), u = fc1 pre-activation;
+                               swiglu: ACT [T][p][2][f/p], u = [gate | up] itself       */
+  MGT_SAVED_FC1_A = 11,     /* ACT [T][p][f/p]     GeLU(u) (swiglu: silu(gate) * up)   */
   MGT_SAVED_COUNT = 12,
   MGT_WS_STATUS = 64,       /* int32 device status word (first 256 bytes)              */
-  MGT_WS_DU = 65,           /* ACT [T, f]   dL/du                                      */
+  MGT_WS_DU = 65,           /* ACT [T, f]   dL/du (swiglu: [T][p][2][f/p], d gate | d up) */
   MGT_WS_DLN2 = 66,         /* ACT [T, h]   dL/d ln2 (shard contributions summed)      */
   MGT_WS_DH1 = 67,          /* ACT [T, h]   dL/d h1                                    */
   MGT_WS_DO = 68,           /* ACT [T, h]   dL/d attention output                      */
@@ -143,8 +154,9 @@ mgt_status mgt_layer_region(const mgt_layer* layer, int region, size_t* offset, 
 
 /* Forward. Reads x [b,s,h]; writes y [b,s,h] and every region of `saved`.
  * Launch order on `stream`: LN1, QKV GEMM(+bias), attention, out-proj GEMM (+shard sum,
- * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores a and GeLU'(u)), fc2 GEMM (+shard sum, +b2,
- * +h1). */
+ * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores a and GeLU'(u); swiglu: each tile holds a
+ * shard's gate and up columns for the same outputs and stores a and [gate | up]), fc2 GEMM
+ * (+shard sum, +b2, +h1). */
 mgt_status mgt_layer_fwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
                          void* y, void* saved, void* workspace, void* stream);
 

@@ -41,7 +41,8 @@ class _Config(ctypes.Structure):
                 ("seq", ctypes.c_int32), ("micro_batch", ctypes.c_int32),
                 ("tp_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("ln_eps", ctypes.c_float),
-                ("recompute_attn", ctypes.c_int32), ("gelu_tanh", ctypes.c_int32)]
+                ("recompute_attn", ctypes.c_int32), ("gelu_tanh", ctypes.c_int32),
+                ("swiglu", ctypes.c_int32), ("disable_bias_linear", ctypes.c_int32)]
 
 
 class _Params(ctypes.Structure):
@@ -119,11 +120,13 @@ class Layer:
     per-shard layouts of include/mgt_layer.h (see PARAM_ORDER)."""
 
     def __init__(self, hidden, heads, ffn, seq, micro_batch, tp_size=1, dtype="bf16",
-                 ln_eps=1e-5, gelu_tanh=0, causal=1):
+                 ln_eps=1e-5, gelu_tanh=0, causal=1, swiglu=0, disable_bias_linear=0):
         self.lib = load_library()
         self.cfg = _Config(hidden, heads, ffn, seq, micro_batch, tp_size,
-                           1 if dtype == "bf16" else 0, causal, ln_eps, 1, gelu_tanh)
+                           1 if dtype == "bf16" else 0, causal, ln_eps, 1, gelu_tanh, swiglu,
+                           disable_bias_linear)
         self.dtype = dtype
+        self.has_bias = not disable_bias_linear
         h = ctypes.c_void_p()
         _check(self.lib.mgt_layer_init(ctypes.byref(self.cfg), ctypes.byref(h)), "mgt_layer_init")
         self.handle = h
@@ -131,9 +134,10 @@ class Layer:
     @classmethod
     def from_config(cls, cfg):
         """Build from any object with hidden, heads, ffn, seq, micro_batch, tp_size, dtype,
-        ln_eps, gelu_tanh attributes."""
+        ln_eps, gelu_tanh (and optionally swiglu, disable_bias_linear) attributes."""
         return cls(cfg.hidden, cfg.heads, cfg.ffn, cfg.seq, cfg.micro_batch, cfg.tp_size,
-                   cfg.dtype, cfg.ln_eps, cfg.gelu_tanh)
+                   cfg.dtype, cfg.ln_eps, cfg.gelu_tanh, swiglu=getattr(cfg, "swiglu", 0),
+                   disable_bias_linear=getattr(cfg, "disable_bias_linear", 0))
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -173,12 +177,16 @@ class Layer:
     # ------------------------------------------------------------------ compute
     @staticmethod
     def _params(p: Dict) -> _Params:
-        return _Params(*[_ptr(p[n]) for n in PARAM_ORDER])
+        """Pointers in PARAM_ORDER; an absent entry (a bias of a layer built with
+        disable_bias_linear) is passed as NULL."""
+        return _Params(*[_ptr(p.get(n)) for n in PARAM_ORDER])
 
     def _check_types(self, params, acts, grads=None):
         import torch
         act = torch.bfloat16 if self.dtype == "bf16" else torch.float32
         for n in PARAM_ORDER:
+            if n not in params and not self.has_bias and n.startswith("b"):
+                continue
             want = torch.float32 if n.startswith("ln") else act
             if params[n].dtype != want:
                 raise TypeError("parameter %s must be %s" % (n, want))

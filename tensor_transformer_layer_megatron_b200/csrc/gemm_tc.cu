@@ -77,6 +77,23 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
         if (i < count) o[i] = v[i];
     }
     return;
+  } else if constexpr (EPI == kEpiDSwiglu) {
+    // The chunk lies inside one group ng (tiles never cross groups).
+    const int ng = col / a.Ng, n = col - ng * a.Ng;
+    const long long zo = (long long)row * a.ld_aux + 2LL * ng * a.Ng + n;
+    const long long oo = (long long)row * a.ldc + 2LL * ng * a.Ng + n;
+    const __nv_bfloat16* zg = reinterpret_cast<const __nv_bfloat16*>(a.aux) + zo;
+    __nv_bfloat16* og = reinterpret_cast<__nv_bfloat16*>(a.out) + oo;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i < count) {
+        float sl, ds;
+        silu_and_grad_bf16out(__bfloat162float(zg[i]), sl, ds);
+        og[i] = __float2bfloat16_rn(v[i] * __bfloat162float(zg[a.Ng + i]) * ds);
+        og[a.Ng + i] = __float2bfloat16_rn(v[i] * sl);
+      }
+    }
+    return;
   } else {
     // bias / residual / aux come in the activation dtype (bf16)
     const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
@@ -238,6 +255,33 @@ __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int 
       }
     }
   }
+  if constexpr (EPI == kEpiDSwiglu) {  // w: d gate, w2: d up (aux = [g | u] of this group)
+    const int ng = col / a.Ng, n = col - ng * a.Ng;
+    const __nv_bfloat16* zg = reinterpret_cast<const __nv_bfloat16*>(a.aux) +
+                              (long long)row * a.ld_aux + 2LL * ng * a.Ng + n;
+    uint4 g4[4], u4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      g4[q] = row_ok ? *reinterpret_cast<const uint4*>(zg + q * 8) : make_uint4(0, 0, 0, 0);
+      u4[q] = row_ok ? *reinterpret_cast<const uint4*>(zg + a.Ng + q * 8)
+                     : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t gg[4] = {g4[q].x, g4[q].y, g4[q].z, g4[q].w};
+      const uint32_t uu[4] = {u4[q].x, u4[q].y, u4[q].z, u4[q].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float s0, s1, d0, d1;
+        silu_and_grad_bf16out(bf16_lo(gg[j]), s0, d0);
+        silu_and_grad_bf16out(bf16_hi(gg[j]), s1, d1);
+        const float a0 = v[q * 8 + 2 * j], a1 = v[q * 8 + 2 * j + 1];
+        w[q * 4 + j] = pack_bf16x2(a0 * bf16_lo(uu[j]) * d0, a1 * bf16_hi(uu[j]) * d1);
+        w2[q * 4 + j] = pack_bf16x2(a0 * s0, a1 * s1);
+      }
+    }
+    return;
+  }
   if constexpr (EPI == kEpiGelu) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -250,6 +294,66 @@ __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int 
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  }
+}
+
+// SwiGLU forward, element by element (ragged chunks): gate and up accumulators of output
+// columns ng*Ng + n0 .. + count-1.
+__device__ __forceinline__ void swiglu_chunk_elem(const GemmArgs& a, int row, int ng, int n0,
+                                                  int count, const float (&vg)[32],
+                                                  const float (&vu)[32]) {
+  const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+  const long long brow = 2LL * ng * a.Ng + n0;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (long long)row * a.ldc +
+                     (long long)ng * a.Ng + n0;
+  __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(a.out2) + (long long)row * a.ldc2 + brow;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i < count) {
+      float g = vg[i], u = vu[i];
+      if (bias) {
+        g += __bfloat162float(bias[brow + i]);
+        u += __bfloat162float(bias[brow + a.Ng + i]);
+      }
+      float sl, ds;
+      silu_and_grad_bf16out(g, sl, ds);
+      o[i] = __float2bfloat16_rn(sl * u);
+      z[i] = __float2bfloat16_rn(g);
+      z[a.Ng + i] = __float2bfloat16_rn(u);
+    }
+  }
+}
+
+// SwiGLU forward for a whole chunk, packed for staged stores: w = silu(g)*u, w2 = g, w3 = u.
+__device__ __forceinline__ void swiglu_values(const GemmArgs& a, int ng, int n0, float (&vg)[32],
+                                              float (&vu)[32], uint32_t (&w)[16],
+                                              uint32_t (&w2)[16], uint32_t (&w3)[16]) {
+  const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+  if (bias) {
+    const long long brow = 2LL * ng * a.Ng + n0;
+    const uint4* bg = reinterpret_cast<const uint4*>(bias + brow);
+    const uint4* bu = reinterpret_cast<const uint4*>(bias + brow + a.Ng);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 g4 = __ldg(bg + q), u4 = __ldg(bu + q);
+      const uint32_t gg[4] = {g4.x, g4.y, g4.z, g4.w}, uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        vg[q * 8 + 2 * j] += bf16_lo(gg[j]);
+        vg[q * 8 + 2 * j + 1] += bf16_hi(gg[j]);
+        vu[q * 8 + 2 * j] += bf16_lo(uu[j]);
+        vu[q * 8 + 2 * j + 1] += bf16_hi(uu[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float s0, s1, d0, d1;
+    silu_and_grad_bf16out(vg[2 * i], s0, d0);
+    silu_and_grad_bf16out(vg[2 * i + 1], s1, d1);
+    w[i] = pack_bf16x2(s0 * vu[2 * i], s1 * vu[2 * i + 1]);
+    w2[i] = pack_bf16x2(vg[2 * i], vg[2 * i + 1]);
+    w3[i] = pack_bf16x2(vu[2 * i], vu[2 * i + 1]);
   }
 }
 
@@ -473,17 +577,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // `tfull` in both CTAs; both CTAs' epilogue warps arrive on the leader's `tempty` (count 8).
 // A cluster barrier after initialisation and another before exit bracket all cross-CTA
 // traffic; every wait in between is bounded.
-constexpr int kPairStages = 6;
+// Six 32 KB stages; the SwiGLU forward keeps five to make room for its three staged outputs.
+constexpr int pair_stages(int epi) { return epi == kEpiSwiglu ? 5 : 6; }
+constexpr int stage_out_bytes(int epi) { return epi == kEpiSwiglu ? 6144 : 4096; }
 constexpr int kPairAB = BM * BK * 2;            // 16 KB: this CTA's A rows or B half
 constexpr int kPairStageBytes = 2 * kPairAB;    // 32 KB per CTA per stage
-// Output staging per epilogue warp: one 32 x 32 fp32 chunk (128-byte rows), or up to two
-// 32 x 32 bf16 chunks (64-byte rows; out and, for kEpiGelu, out2 2 KB further on).
-constexpr int kStageOut = 32 * 32 * 4;
+// Output staging per epilogue warp: one 32 x 32 fp32 chunk (128-byte rows), or up to three
+// 32 x 32 bf16 chunks (64-byte rows, 2 KB apart: out, then out2 / the second GLU half).
 // stages | barriers (padded to 1 KB) | output staging | 1 KB alignment slack
-constexpr int pair_smem(int) {
-  return kPairStages * kPairStageBytes + 1024 + kEpiWarps * kStageOut + 1024;
+constexpr int pair_smem(int epi) {
+  return pair_stages(epi) * kPairStageBytes + 1024 + kEpiWarps * stage_out_bytes(epi) + 1024;
 }
 static_assert(pair_smem(kEpiStoreF32) <= 232448, "shared memory per CTA");
+static_assert(pair_smem(kEpiSwiglu) <= 232448, "shared memory per CTA");
 
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -500,20 +606,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // 16 bytes, which a TMA store cannot start at).
   // BN: the pair's N tile, a multiple of 32 up to 256 (256 when B is MN-major); each CTA
   // loads BN/2 rows of B. Accumulator buffers stay 256 columns apart in TMEM.
+  constexpr int STAGES = pair_stages(EPI);
+  constexpr int kStageOut = stage_out_bytes(EPI);
+  constexpr bool kGlu = EPI == kEpiSwiglu;
   const uint32_t b_bytes = (uint32_t)(BN / 2) * BK * 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kPairStages * kPairAB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
+  uint8_t* sB = smem + STAGES * kPairAB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * kPairStageBytes);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kPairStages;
-  uint64_t* tfull = bars + 2 * kPairStages;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* stage_out = smem + kPairStages * kPairStageBytes + 1024;  // 1024-aligned
+  uint8_t* stage_out = smem + STAGES * kPairStageBytes + 1024;  // 1024-aligned
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -525,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int num_tiles = args.NG * num_m2 * num_n;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -540,7 +649,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB);
     if (staged) {
       tma_prefetch_desc(&tmC);
-      if (EPI == kEpiGelu) tma_prefetch_desc(&tmC2);
+      if (EPI == kEpiGelu || kGlu) tma_prefetch_desc(&tmC2);
     }
   }
   if (warp == 1) {
@@ -578,13 +687,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_3d_pair(&tmA, fb, a_dst, m0, kt * BK, 0);
             tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, kt * BK, 0);
           }
-          if constexpr (!B_MN) {
+          if constexpr (kGlu) {
+            // GLU tile: this CTA's half of B is the gate (rank 0) or up (rank 1) block of
+            // group ng, rows nb*BN/2 ..; the map views B as {K, Ng, 2*NG}.
+            tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, tc.nb * (BN / 2), 2 * tc.ng + rank);
+          } else if constexpr (!B_MN) {
             tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, n0, kg);
           } else {
             tma_load_3d_pair(&tmB, fb, b_dst, n0, kt * BK, tc.ng);
             tma_load_3d_pair(&tmB, fb, b_dst + kChunkBytes, n0 + 64, kt * BK, tc.ng);
           }
-          if (++stage == kPairStages) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -595,11 +708,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // land; the peer relies on the end-of-kernel cluster barrier, which the leader reaches
     // only after its MMA issuer consumed (or gave up on) every stage.
     if (leader) {
-      for (int i = 1; i <= kPairStages; ++i) {
+      for (int i = 1; i <= STAGES; ++i) {
         int s = stage - i;
         uint32_t ph = phase;
         if (s < 0) {
-          s += kPairStages;
+          s += STAGES;
           ph ^= 1;
         }
         mbar_wait(&full[s], ph, args.err, kErrTimeoutDrain, nullptr);
@@ -637,7 +750,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_mma_f16_pair(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit_pair_mc(&empty[stage], 0x3);  // frees the slot in both CTAs
-        if (++stage == kPairStages) {
+        if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
@@ -654,7 +767,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp & 3;
-    const int nch = BN / 32, half = (nch + 1) / 2;  // 32-column chunks, split over 2 warp sets
+    // 32-column chunks, split over 2 warp sets; a GLU tile yields BN/64 output chunks, each
+    // from one gate chunk and the up chunk BN/2 columns further on.
+    const int nch = kGlu ? BN / 64 : BN / 32, half = (nch + 1) / 2;
     const int c_begin = ((warp - 2) >> 2) ? half : 0;
     const int c_end = ((warp - 2) >> 2) ? nch : half;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
@@ -667,6 +782,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      if constexpr (kGlu) {
+#pragma unroll 1
+        for (int c = c_begin; c < c_end; ++c) {
+          float vg[32], vu[32];
+          const uint32_t t0 = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256;
+          tmem_ld_32x32b_x32(t0 + c * 32, vg);
+          tmem_ld_32x32b_x32(t0 + BN / 2 + c * 32, vu);
+          const int n0 = tc.nb * (BN / 2) + c * 32;
+          const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
+          if (n0 < args.Ng && (n0 + 32 > args.Ng || !staged)) {
+            if (row < args.M)
+              swiglu_chunk_elem(args, row, tc.ng, n0, min(32, args.Ng - n0), vg, vu);
+          } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
+            uint8_t* buf = stage_out + (warp - 2) * kStageOut;
+            uint32_t w[16], w2[16], w3[16];
+            swiglu_values(args, tc.ng, n0, vg, vu, w, w2, w3);
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+            const int sw = (lane >> 1) & 3;  // 64-byte swizzle, as below
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int o = lane * 64 + ((j ^ sw) << 4);
+              *reinterpret_cast<uint4*>(buf + o) =
+                  make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              *reinterpret_cast<uint4*>(buf + 2048 + o) =
+                  make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
+              *reinterpret_cast<uint4*>(buf + 4096 + o) =
+                  make_uint4(w3[4 * j], w3[4 * j + 1], w3[4 * j + 2], w3[4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmC, buf, tc.ng * args.Ng + n0, row0, 0);
+              tma_store_3d(&tmC2, buf + 2048, n0, row0, 2 * tc.ng);
+              tma_store_3d(&tmC2, buf + 4096, n0, row0, 2 * tc.ng + 1);
+              bulk_commit();
+            }
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = c_begin; c < c_end; ++c) {
         float v[32];
@@ -691,6 +846,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           } else {
             uint32_t w[16], w2[16];
             epi_values_bf16<EPI>(args, row, col, row < args.M, v, w, w2);
+            constexpr bool two = EPI == kEpiGelu || EPI == kEpiDSwiglu;
             if (lane == 0) bulk_wait_read0();
             __syncwarp();
             // 64-byte rows, 64-byte swizzle: 16-byte unit j of row r sits at unit
@@ -700,7 +856,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 4; ++j) {
               *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) =
                   make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-              if (EPI == kEpiGelu)
+              if (two)
                 *reinterpret_cast<uint4*>(buf + 2048 + lane * 64 + ((j ^ sw) << 4)) =
                     make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
             }
@@ -708,13 +864,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
-            if (EPI == kEpiGelu)
-              tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, row0, col / args.out_ng);
+            if constexpr (EPI == kEpiDSwiglu) {  // tmC views dz as {Ng, M, 2*NG}
+              tma_store_3d(&tmC, buf, n0, row0, 2 * tc.ng);
+              tma_store_3d(&tmC, buf + 2048, n0, row0, 2 * tc.ng + 1);
+            } else {
+              tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
+              if (EPI == kEpiGelu)
+                tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, row0, col / args.out_ng);
+            }
             bulk_commit();
           }
         }
       }
+      }  // kGlu
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
@@ -802,11 +964,14 @@ cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
     case kEpiBf16: return launch_inst<BN, A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, s);
     case kEpiGelu: return launch_inst<BN, A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, s);
     case kEpiDGelu: return launch_inst<BN, A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, s);
+    case kEpiDSwiglu:
+      if constexpr (!A_MN && B_MN)
+        return launch_inst<BN, A_MN, B_MN, kEpiDSwiglu>(ta, tb, a, num_sms, s);
+      break;
   }
   return cudaErrorInvalidValue;
 }
 
-// fp32 output viewed as {out_ng, M, groups} with a 32 x 32 box (128-byte rows, swizzled).
 // Output tensor map for the staged epilogue store: {out_ng, M, groups}, box 32 x 32; fp32 with
 // 128-byte swizzle (128-byte rows), bf16 with 64-byte swizzle (64-byte rows).
 bool make_out_map(CUtensorMap* m, const GemmArgs& a, void* base, bool f32) {
@@ -824,6 +989,20 @@ bool make_out_map(CUtensorMap* m, const GemmArgs& a, void* base, bool f32) {
   return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
             gd, gs, bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 view {Ng, M, 2*NG} of a [M][NG][2][Ng] buffer with row stride ld (elements): group
+// 2*ng is the gate half of group ng, 2*ng + 1 its up half. Box 32 x 32, 64-byte swizzle.
+bool make_glu_map(CUtensorMap* m, const GemmArgs& a, void* base, long long ld) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3] = {(cuuint64_t)a.Ng, (cuuint64_t)a.M, 2 * (cuuint64_t)a.NG};
+  cuuint64_t gs[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)a.Ng * 2};
+  cuuint32_t bd[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, gd, gs, bd, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -847,14 +1026,29 @@ cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const
   // elements (true for one group, else Ng must be) and must not run across an out_ng boundary
   // (true if one out_ng block holds every column, else out_ng must be a multiple of 32).
   // Tensor-map encoding also needs 16-byte aligned bases and strides.
+  // The SwiGLU epilogues store [gate | up] halves through a view {Ng, M, 2*NG} of their
+  // buffer (row stride ldc2 / ldc, group stride Ng), at inner coordinate n0: they need Ng to
+  // be a multiple of 32 (whole chunks inside a group) and the SwiGLU forward also stores a at
+  // column ng*Ng + n0 of out.
   const int vec = EPI == kEpiStoreF32 ? 4 : 8;
-  const bool cols_ok = (a.NG == 1 || a.Ng % vec == 0) &&
-                       ((long long)a.out_ng >= (long long)a.Ng * a.NG || a.out_ng % 32 == 0);
-  int staged = cols_ok ? 1 : 0;
-  if (staged && !make_out_map(&tc, a, a.out, EPI == kEpiStoreF32)) staged = 0;
-  if (staged && EPI == kEpiGelu && !make_out_map(&tc2, a, a.out2, false)) staged = 0;
+  int staged;
+  if (EPI == kEpiSwiglu || EPI == kEpiDSwiglu) {
+    staged = a.Ng % 32 == 0 ? 1 : 0;
+    if (staged && !make_glu_map(&(EPI == kEpiSwiglu ? tc2 : tc), a,
+                                EPI == kEpiSwiglu ? a.out2 : a.out,
+                                EPI == kEpiSwiglu ? a.ldc2 : a.ldc))
+      staged = 0;
+    if (staged && EPI == kEpiSwiglu && !make_out_map(&tc, a, a.out, false)) staged = 0;
+  } else {
+    const bool cols_ok = (a.NG == 1 || a.Ng % vec == 0) &&
+                         ((long long)a.out_ng >= (long long)a.Ng * a.NG || a.out_ng % 32 == 0);
+    staged = cols_ok ? 1 : 0;
+    if (staged && !make_out_map(&tc, a, a.out, EPI == kEpiStoreF32)) staged = 0;
+    if (staged && EPI == kEpiGelu && !make_out_map(&tc2, a, a.out2, false)) staged = 0;
+  }
   const int num_m2 = (a.M + 255) / 256;
-  const int num_n = (a.Ng + bn - 1) / bn;
+  const int tile_cols = EPI == kEpiSwiglu ? bn / 2 : bn;  // outputs per tile and group
+  const int num_n = (a.Ng + tile_cols - 1) / tile_cols;
   const int tiles = a.NG * num_m2 * num_n;
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
   kern<<<2 * pairs, kThreads, smem_bytes, stream>>>(ta, tb, tc, tc2, a, num_m2, num_n, bn,
@@ -871,6 +1065,14 @@ cudaError_t launch_pair_epi(const CUtensorMap& ta, const CUtensorMap& tb, const 
     case kEpiBf16: return launch_pair_inst<A_MN, B_MN, kEpiBf16>(ta, tb, a, num_sms, bn, s);
     case kEpiGelu: return launch_pair_inst<A_MN, B_MN, kEpiGelu>(ta, tb, a, num_sms, bn, s);
     case kEpiDGelu: return launch_pair_inst<A_MN, B_MN, kEpiDGelu>(ta, tb, a, num_sms, bn, s);
+    case kEpiSwiglu:
+      if constexpr (!A_MN && !B_MN)
+        return launch_pair_inst<A_MN, B_MN, kEpiSwiglu>(ta, tb, a, num_sms, bn, s);
+      break;
+    case kEpiDSwiglu:
+      if constexpr (!A_MN && B_MN)
+        return launch_pair_inst<A_MN, B_MN, kEpiDSwiglu>(ta, tb, a, num_sms, bn, s);
+      break;
   }
   return cudaErrorInvalidValue;
 }
@@ -888,12 +1090,14 @@ cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const Gemm
 // is as full as possible. MN-major B loads 64-wide chunks per CTA half, so it keeps 256.
 int pick_pair_bn(const GemmArgs& a, int num_sms) {
   if (a.b_mn) return 256;
+  const bool glu = a.epi == kEpiSwiglu;  // a GLU tile covers bn/2 outputs (gate + up halves)
   const int pairs = num_sms / 2;
   const long long m2 = (a.M + 255) / 256;
   int best = 256;
   long long best_cost = -1;
-  for (int bn = 256; bn >= 128; bn -= 32) {
-    const long long tiles = (long long)a.NG * m2 * ((a.Ng + bn - 1) / bn);
+  for (int bn = 256; bn >= (glu ? 64 : 128); bn -= (glu ? 64 : 32)) {
+    const int cols = glu ? bn / 2 : bn;
+    const long long tiles = (long long)a.NG * m2 * ((a.Ng + cols - 1) / cols);
     const long long rounds = (tiles + pairs - 1) / pairs;
     const long long cost = rounds * (bn + 48);
     if (best_cost < 0 || cost < best_cost) {
@@ -918,10 +1122,14 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   // Shape rules of the tensor maps (checked by the callers too).
   if (a.M <= 0 || a.Ng <= 0 || a.NG <= 0 || a.Kg <= 0 || a.KG <= 0) return cudaErrorInvalidValue;
-  if ((a.a_mn && a.KG != 1) || (a.b_mn && a.KG != 1) || (!a.b_mn && a.NG != 1))
+  const bool glu = a.epi == kEpiSwiglu;
+  if ((a.a_mn && a.KG != 1) || (a.b_mn && a.KG != 1) || (!a.b_mn && a.NG != 1 && !glu))
     return cudaErrorInvalidValue;
-  // Wide tiles run on CTA pairs (cta_group::2, 256 x BN per pair); narrow N on one CTA.
-  const bool pair = a.Ng > 128 && num_sms >= 2;
+  if (glu && (a.a_mn || a.b_mn || a.KG != 1 || num_sms < 2)) return cudaErrorInvalidValue;
+  if (a.epi == kEpiDSwiglu && (a.a_mn || !a.b_mn)) return cudaErrorInvalidValue;
+  // Wide tiles run on CTA pairs (cta_group::2, 256 x BN per pair); narrow N on one CTA. GLU
+  // tiles (gate and up halves from the two CTAs) exist only on pairs.
+  const bool pair = (a.Ng > 128 || glu) && num_sms >= 2;
   const int BN = (a.Ng <= 128) ? 128 : 256;
   const int pair_bn = pair ? pick_pair_bn(a, num_sms) : BN;
   const int b_rows = pair ? pair_bn / 2 : BN;  // B rows per CTA per k-step
@@ -944,7 +1152,12 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
   {
     uint64_t dims[3], str[2];
     uint32_t box[3];
-    if (!a.b_mn) {
+    if (glu) {  // B rows [NG][2][Ng] (gate block, up block per group) viewed as {K, Ng, 2*NG}
+      dims[0] = a.Kg; dims[1] = a.Ng; dims[2] = 2 * (uint64_t)a.NG;
+      str[0] = a.ldb;
+      str[1] = (uint64_t)a.Ng * a.ldb;
+      box[0] = BK; box[1] = b_rows; box[2] = 1;
+    } else if (!a.b_mn) {
       dims[0] = a.Kg; dims[1] = a.Ng; dims[2] = a.KG;
       str[0] = a.ldb;
       str[1] = a.KG > 1 ? (uint64_t)a.b_kgs : (uint64_t)a.ldb;

@@ -74,6 +74,8 @@ mgt_status validate(const mgt_layer_config* c) {
       c->ffn % c->tp_size)
     return MGT_EINVAL;
   if (!(c->ln_eps >= 0.f)) return MGT_EINVAL;
+  if (c->swiglu != 0 && c->swiglu != 1) return MGT_EINVAL;
+  if (c->disable_bias_linear != 0 && c->disable_bias_linear != 1) return MGT_EINVAL;
   if (c->causal != 1) return MGT_EUNSUPPORTED;
   const long long T = (long long)c->seq * c->micro_batch;
   if (T > (1LL << 30) || (long long)c->ffn * 3 > (1LL << 30) || (long long)c->hidden * 3 > (1LL << 30))
@@ -94,9 +96,10 @@ mgt_status validate(const mgt_layer_config* c) {
 
 void layout(mgt_layer* L) {
   const size_t T = L->T, h = L->h, f = L->f, e = L->esz;
+  const size_t f1 = L->cfg.swiglu ? 2 * f : f;  // fc1 outputs: [gate | up] with SwiGLU
   const size_t bHs = (size_t)L->cfg.micro_batch * L->H * L->cfg.seq;
   size_t sz[MGT_SAVED_COUNT] = {T * h * e, T * 4, T * 4, T * 3 * h * e, T * h * e, bHs * 4,
-                                T * h * e, T * h * e, T * 4, T * 4, T * f * e, T * f * e};
+                                T * h * e, T * h * e, T * 4, T * 4, T * f1 * e, T * f * e};
   size_t off = 0;
   for (int i = 0; i < MGT_SAVED_COUNT; ++i) {
     L->saved[i].off = off;
@@ -106,7 +109,7 @@ void layout(mgt_layer* L) {
   L->saved_bytes = off;
   const size_t nblk = T < (size_t)kMaxLnBlocks ? T : (size_t)kMaxLnBlocks;
   size_t wsz[MGT_WS_COUNT - 64] = {256,
-                                   T * f * e,
+                                   T * f1 * e,
                                    T * h * e,
                                    T * h * e,
                                    T * h * e,
@@ -154,7 +157,9 @@ GemmArgs gemm_base(int M, int Ng, int NG, int Kg, int KG) {
 
 // `site` names the call ("gemm_tc/fc1_fwd", ...): profiling groups launches by this name.
 cudaError_t gemm(mgt_layer* L, const char* site, const GemmArgs& a, cudaStream_t s) {
-  const double flops = 2.0 * a.M * (double)a.Ng * a.NG * (double)a.Kg * a.KG;
+  // A SwiGLU fc1 tile computes a gate and an up product per output.
+  const double flops = 2.0 * a.M * (double)a.Ng * a.NG * (double)a.Kg * a.KG *
+                       (a.epi == kEpiSwiglu ? 2 : 1);
   if (L->cfg.dtype == MGT_BF16)
     return run(L, site, flops, 0, s, [&] { return launch_gemm_tc(a, L->num_sms, s); });
   return run(L, "gemm_simt", flops, 0, s, [&] { return launch_gemm_simt_f32(a, s); });
@@ -188,6 +193,18 @@ mgt_status ensure_device(mgt_layer* L) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Every parameter (and gradient) pointer must be set and 16-byte aligned, except the four
+// linear biases of a layer without them, which are ignored.
+mgt_status check_param_ptrs(const mgt_layer* L, const void* const* q) {
+  for (int i = 0; i < 12; ++i) {
+    const bool is_bias = i == 3 || i == 5 || i == 9 || i == 11;  // b_qkv, b_o, b1, b2
+    if (is_bias && L->cfg.disable_bias_linear) continue;
+    if (!q[i]) return MGT_EINVAL;
+    if (!aligned16(q[i])) return MGT_EUNSUPPORTED;
+  }
+  return MGT_OK;
+}
 
 }  // namespace
 
@@ -251,11 +268,11 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   if (!L || !P || !x || !y || !saved || !workspace) return MGT_EINVAL;
   const void* ptrs[] = {P->ln1_g, P->ln1_b, P->w_qkv, P->b_qkv, P->w_o, P->b_o,
                         P->ln2_g, P->ln2_b, P->w1, P->b1, P->w2, P->b2};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return q ? MGT_EUNSUPPORTED : MGT_EINVAL;
+  mgt_status st = check_param_ptrs(L, ptrs);
+  if (st != MGT_OK) return st;
   if (!aligned16(x) || !aligned16(y) || ((uintptr_t)saved & 255) || ((uintptr_t)workspace & 255))
     return MGT_EUNSUPPORTED;
-  mgt_status st = ensure_device(L);
+  st = ensure_device(L);
   if (st != MGT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = L->T, h = L->h, f = L->f, p = L->p, dt = L->cfg.dtype == MGT_BF16 ? 1 : 0;
@@ -274,6 +291,11 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   char* gd = sp(saved, L->saved[MGT_SAVED_FC1_DGELU]);
   char* act = sp(saved, L->saved[MGT_SAVED_FC1_A]);
   const double ln_bytes = (double)T * h * 2 * e + 8.0 * h;
+  const bool nb = L->cfg.disable_bias_linear;
+  const void* b_qkv = nb ? nullptr : P->b_qkv;
+  const void* b_o = nb ? nullptr : P->b_o;
+  const void* b1 = nb ? nullptr : P->b1;
+  const void* b2 = nb ? nullptr : P->b2;
 
   // 1. LN1
   MGT_TRY(run(L, "ln_fwd", 0, ln_bytes, s, [&] {
@@ -284,7 +306,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   {
     GemmArgs a = gemm_base(T, 3 * h, 1, h, 1);
     a.A = ln1; a.lda = h; a.B = P->w_qkv; a.ldb = h;
-    a.epi = kEpiBf16; a.out = qkv; a.ldc = 3 * h; a.bias = P->b_qkv; a.err = err;
+    a.epi = kEpiBf16; a.out = qkv; a.ldc = 3 * h; a.bias = b_qkv; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/qkv_fwd", a, s));
   }
   // 3. causal attention per head (each shard's heads are local)
@@ -299,7 +321,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   {
     GemmArgs a = gemm_base(T, h, 1, h / p, p);
     a.A = O; a.lda = h; a.B = P->w_o; a.ldb = h / p; a.b_kgs = (long long)h * (h / p);
-    a.epi = kEpiBf16; a.out = h1; a.ldc = h; a.bias = P->b_o; a.res = x; a.ldr = h; a.err = err;
+    a.epi = kEpiBf16; a.out = h1; a.ldc = h; a.bias = b_o; a.res = x; a.ldr = h; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/outproj_fwd", a, s));
   }
   // 5. LN2
@@ -307,11 +329,19 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     return launch_ln_fwd(dt, T, h, L->cfg.ln_eps, h1, (const float*)P->ln2_g,
                          (const float*)P->ln2_b, ln2, mu2, rs2, s);
   }));
-  // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and GeLU'(u) for the backward)
-  {
+  // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and GeLU'(u) for the backward).
+  //    SwiGLU: shard t's gate and up rows go to the two halves of one tile; the epilogue stores
+  //    a = silu(gate) * up and [gate | up] for the backward.
+  if (L->cfg.swiglu) {
+    GemmArgs a = gemm_base(T, f / p, p, h, 1);
+    a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
+    a.epi = kEpiSwiglu; a.out = act; a.ldc = f; a.out2 = gd; a.ldc2 = 2LL * f; a.bias = b1;
+    a.err = err;
+    MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
+  } else {
     GemmArgs a = gemm_base(T, f, 1, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
-    a.epi = kEpiGelu; a.out = act; a.out2 = gd; a.ldc = f; a.bias = P->b1;
+    a.epi = kEpiGelu; a.out = act; a.out2 = gd; a.ldc = f; a.bias = b1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   }
@@ -319,7 +349,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   {
     GemmArgs a = gemm_base(T, h, 1, f / p, p);
     a.A = act; a.lda = f; a.B = P->w2; a.ldb = f / p; a.b_kgs = (long long)h * (f / p);
-    a.epi = kEpiBf16; a.out = y; a.ldc = h; a.bias = P->b2; a.res = h1; a.ldr = h; a.err = err;
+    a.epi = kEpiBf16; a.out = y; a.ldc = h; a.bias = b2; a.res = h1; a.ldr = h; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc2_fwd", a, s));
   }
   return MGT_OK;
@@ -330,15 +360,16 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
                          void* workspace, void* stream) {
   if (!L || !P || !x || !saved || !dy || !dx || !G || !workspace) return MGT_EINVAL;
   const void* ptrs[] = {P->ln1_g, P->ln1_b, P->w_qkv, P->b_qkv, P->w_o, P->b_o,
-                        P->ln2_g, P->ln2_b, P->w1, P->b1, P->w2, P->b2,
-                        G->ln1_g, G->ln1_b, G->w_qkv, G->b_qkv, G->w_o, G->b_o,
-                        G->ln2_g, G->ln2_b, G->w1, G->b1, G->w2, G->b2};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return q ? MGT_EUNSUPPORTED : MGT_EINVAL;
+                        P->ln2_g, P->ln2_b, P->w1, P->b1, P->w2, P->b2};
+  const void* gptrs[] = {G->ln1_g, G->ln1_b, G->w_qkv, G->b_qkv, G->w_o, G->b_o,
+                         G->ln2_g, G->ln2_b, G->w1, G->b1, G->w2, G->b2};
+  mgt_status st = check_param_ptrs(L, ptrs);
+  if (st == MGT_OK) st = check_param_ptrs(L, gptrs);
+  if (st != MGT_OK) return st;
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || ((uintptr_t)saved & 255) ||
       ((uintptr_t)workspace & 255))
     return MGT_EUNSUPPORTED;
-  mgt_status st = ensure_device(L);
+  st = ensure_device(L);
   if (st != MGT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = L->T, h = L->h, f = L->f, p = L->p, dt = L->cfg.dtype == MGT_BF16 ? 1 : 0;
@@ -370,13 +401,16 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
                [&] { return launch_colsum(dt, T, cols, src, (float*)out, s); });
   };
   const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
+  const bool nb = L->cfg.disable_bias_linear, sw = L->cfg.swiglu;
+  const int f1 = sw ? 2 * f : f;  // fc1 output columns (gate and up with SwiGLU)
 
-  // B1. fc2: dgrad fused with GeLU' -> du, wgrad (db2 = sum dy comes with the LN2 backward)
+  // B1. fc2: dgrad fused with GeLU' -> du (SwiGLU: with the SwiGLU backward -> d[gate | up]),
+  //     wgrad (db2 = sum dy comes with the LN2 backward)
   {
     GemmArgs a = gemm_base(T, f / p, p, h, 1);  // N grouped by shard
     a.b_mn = 1; a.A = dy; a.lda = h; a.B = P->w2; a.ldb = f / p;
     a.b_ngs = (long long)h * (f / p);
-    a.epi = kEpiDGelu; a.out = du; a.ldc = f; a.aux = gd; a.ld_aux = f;
+    a.epi = sw ? kEpiDSwiglu : kEpiDGelu; a.out = du; a.ldc = f1; a.aux = gd; a.ld_aux = f1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc2_dgrad", a, s));
   }
@@ -387,17 +421,17 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.out_gs = (long long)h * (f / p); a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, s));
   }
-  // B3. fc1: db1, dgrad (sum over shards = K loop over f), wgrad
-  MGT_TRY(colsum(du, f, G->b1));
+  // B3. fc1: db1, dgrad (sum over shards = K loop over all fc1 outputs), wgrad
+  if (!nb) MGT_TRY(colsum(du, f1, G->b1));
   {
-    GemmArgs a = gemm_base(T, h, 1, f, 1);
-    a.b_mn = 1; a.A = du; a.lda = f; a.B = P->w1; a.ldb = h;
+    GemmArgs a = gemm_base(T, h, 1, f1, 1);
+    a.b_mn = 1; a.A = du; a.lda = f1; a.B = P->w1; a.ldb = h;
     a.epi = kEpiBf16; a.out = dln2; a.ldc = h; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc1_dgrad", a, s));
   }
   {
-    GemmArgs a = gemm_base(f, h, 1, T, 1);
-    a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f; a.B = ln2; a.ldb = h;
+    GemmArgs a = gemm_base(f1, h, 1, T, 1);
+    a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f1; a.B = ln2; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, s));
   }
@@ -405,7 +439,8 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
     // dres = dy, so the residual-gradient sum it also returns is db2
     return launch_ln_bwd(dt, T, h, dln2, dy, h1, (const float*)P->ln2_g, mu2, rs2, dh1, part,
-                         nblk, (float*)G->ln2_g, (float*)G->ln2_b, (float*)G->b2, s);
+                         nblk, (float*)G->ln2_g, (float*)G->ln2_b,
+                         nb ? nullptr : (float*)G->b2, s);
   }));
   // B5. out-proj: dgrad (N grouped by shard) -> dO, wgrad (db_o = sum dh1 comes with LN1 bwd)
   {
@@ -430,7 +465,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     MGT_TRY(run(L, "attn_bwd", fl, 0, s, [&] { return launch_attn_bwd(dt, a, s); }));
   }
   // B7. QKV: db_qkv, dgrad (sum over shards = K loop over 3h), wgrad
-  MGT_TRY(colsum(dqkv, 3 * h, G->b_qkv));
+  if (!nb) MGT_TRY(colsum(dqkv, 3 * h, G->b_qkv));
   {
     GemmArgs a = gemm_base(T, h, 1, 3 * h, 1);
     a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = P->w_qkv; a.ldb = h;
@@ -447,7 +482,8 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
     // dres = dh1, so the residual-gradient sum it also returns is db_o
     return launch_ln_bwd(dt, T, h, dln1, dh1, x, (const float*)P->ln1_g, mu1, rs1, dx, part,
-                         nblk, (float*)G->ln1_g, (float*)G->ln1_b, (float*)G->b_o, s);
+                         nblk, (float*)G->ln1_g, (float*)G->ln1_b,
+                         nb ? nullptr : (float*)G->b_o, s);
   }));
   return MGT_OK;
 }

@@ -525,6 +525,28 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
   const int m = (int)(r / a.Ng), n = (int)(r % a.Ng);
   const float* A = reinterpret_cast<const float*>(a.A);
   const float* B = reinterpret_cast<const float*>(a.B);
+  float* out = reinterpret_cast<float*>(a.out);
+  const float* bias = reinterpret_cast<const float*>(a.bias);
+  if (a.epi == kEpiSwiglu) {  // gate row ng*2Ng + n and up row + Ng of K-major B
+    const long long rg = 2LL * ng * a.Ng + n, ru = rg + a.Ng;
+    float g = 0.f, u = 0.f;
+    for (int k = 0; k < a.Kg; ++k) {
+      const float av = A[(long long)m * a.lda + k];
+      g = fmaf(av, B[rg * a.ldb + k], g);
+      u = fmaf(av, B[ru * a.ldb + k], u);
+    }
+    if (bias) {
+      g += bias[rg];
+      u += bias[ru];
+    }
+    float sl, ds;
+    silu_and_grad_f(g, sl, ds);
+    out[(long long)m * a.ldc + (long long)ng * a.Ng + n] = sl * u;
+    float* z = reinterpret_cast<float*>(a.out2) + (long long)m * a.ldc2;
+    z[rg] = g;
+    z[ru] = u;
+    return;
+  }
   float acc = 0.f;
   for (int kg = 0; kg < a.KG; ++kg) {
     for (int kk = 0; kk < a.Kg; ++kk) {
@@ -538,8 +560,6 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
   const int col = ng * a.Ng + n;
   const long long off = (long long)(col / a.out_ng) * a.out_gs + (long long)m * a.ldc +
                         col % a.out_ng;
-  float* out = reinterpret_cast<float*>(a.out);
-  const float* bias = reinterpret_cast<const float*>(a.bias);
   switch (a.epi) {
     case kEpiStoreF32: out[off] = acc; break;
     case kEpiBf16: {
@@ -558,6 +578,16 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
     }
     case kEpiDGelu: {
       out[off] = acc * reinterpret_cast<const float*>(a.aux)[(long long)m * a.ld_aux + col];
+      break;
+    }
+    case kEpiDSwiglu: {  // acc = dA(m, ng*Ng + n); aux and out laid out [M][NG][2][Ng]
+      const long long zo = 2LL * ng * a.Ng + n;
+      const float* z = reinterpret_cast<const float*>(a.aux) + (long long)m * a.ld_aux;
+      float sl, ds;
+      silu_and_grad_f(z[zo], sl, ds);
+      float* o = out + (long long)m * a.ldc;
+      o[zo] = acc * z[zo + a.Ng] * ds;
+      o[zo + a.Ng] = acc * sl;
       break;
     }
   }

@@ -23,6 +23,15 @@ enum Epilogue : int {
   kEpiBf16 = 1,      // out (act) = acc [+ bias] [+ residual] (QKV, out-proj, fc2, dgrads)
   kEpiGelu = 2,      // u = acc + bias; out = GeLU(u), out2 = GeLU'(u) (fc1)
   kEpiDGelu = 3,     // out = acc * aux, aux = GeLU'(u)        (fc2 dgrad -> du)
+  // SwiGLU fc1 (GLU tiles): group ng holds Ng outputs; B rows ng*2Ng + n (gate) and
+  // ng*2Ng + Ng + n (up) feed output (m, ng*Ng + n). out[m*ldc + ng*Ng + n] = silu(g) * u;
+  // out2[m*ldc2 + ng*2Ng + n] = g, out2[... + Ng] = u (g, u include the bias, indexed like
+  // the B rows). Pair kernel only, K-major operands.
+  kEpiSwiglu = 4,
+  // SwiGLU backward on the fc2 dgrad: acc = dA(m, ng*Ng + n); aux = [g | u] as stored above
+  // (row stride ld_aux); out[m*ldc + ng*2Ng + n] = dA * u * silu'(g), out[... + Ng] =
+  // dA * silu(g).
+  kEpiDSwiglu = 5,
 };
 
 // One GEMM  C[m, col] = sum_{kg < KG} sum_{kk < Kg} A(m, kg, kk) * B(ng, n, kg, kk)
@@ -43,6 +52,7 @@ struct GemmArgs {
   int epi;
   void* out; long long ldc; int out_ng; long long out_gs;
   void* out2;                           // kEpiGelu: GeLU'(u) (same addressing as out)
+  long long ldc2;                       // kEpiSwiglu: row stride of out2
   const void* bias;                     // indexed by col; nullable
   const void* res; long long ldr;       // residual, res[m*ldr + col]; nullable
   const void* aux; long long ld_aux;    // kEpiDGelu: GeLU'(u)[m*ld_aux + col]

@@ -18,11 +18,13 @@ class LayerRun:
         self.layer = layer
         act = torch.bfloat16 if layer.dtype == "bf16" else torch.float32
         self.act = act
+        # Biases are absent from `packed` for a layer without linear biases.
+        names = [k for k in PARAM_ORDER if k in packed]
         self.params = {k: packed[k].to(device=device,
                                        dtype=torch.float32 if k in LN_PARAMS else act)
-                       .contiguous() for k in PARAM_ORDER}
+                       .contiguous() for k in names}
         self.grads = {k: torch.empty(packed[k].shape, dtype=torch.float32, device=device)
-                      for k in PARAM_ORDER}
+                      for k in names}
         self.x = x.to(device=device, dtype=act).contiguous()
         self.dy = dy.to(device=device, dtype=act).contiguous()
         self.y = torch.empty_like(self.x)

@@ -53,15 +53,19 @@ def gpu_intermediates(cfg, layer, run):
         lse=v(run.saved, "attn_lse", torch.float32, (cfg.micro_batch, H, cfg.seq)),
         h1=v(run.saved, "h1", act, (T, h)),
         ln2=v(run.saved, "ln2", act, (T, h)),
-        gelu_grad=v(run.saved, "fc1_dgelu", act, (T, p, f // p)),
         a=v(run.saved, "fc1_a", act, (T, p, f // p)),
-        du=v(run.ws, "du", act, (T, p, f // p)),
         dln2=v(run.ws, "dln2", act, (T, h)),
         dh1=v(run.ws, "dh1", act, (T, h)),
         dO=v(run.ws, "dO", act, (T, p, H // p, d)),
         dqkv=v(run.ws, "dqkv", act, (T, p, 3, H // p, d)),
         dln1=v(run.ws, "dln1", act, (T, h)),
     )
+    if getattr(cfg, "swiglu", 0):  # the fc1 pre-activations [gate | up] and their gradient
+        out["u"] = v(run.saved, "fc1_dgelu", act, (T, p, 2, f // p))
+        out["du"] = v(run.ws, "du", act, (T, p, 2, f // p))
+    else:
+        out["gelu_grad"] = v(run.saved, "fc1_dgelu", act, (T, p, f // p))
+        out["du"] = v(run.ws, "du", act, (T, p, f // p))
     return out
 
 
@@ -73,13 +77,19 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
     y_ref, saved = oracle.layer_fwd(cfg, packed, t["x"])
     dx_ref, g_ref, inter = oracle.layer_bwd(cfg, packed, saved, t["dy"])
     errs = {"y": rel_err(to_np(run.y), y_ref), "dx": rel_err(to_np(run.dx), dx_ref)}
+    # a layer without linear biases has no bias gradients on either side
+    assert set(run.grads) == set(g_ref), (sorted(run.grads), sorted(g_ref))
     for k in GRAD_NAMES:
-        errs["d_" + k] = rel_err(to_np(run.grads[k]), g_ref[k])
+        if k in g_ref:
+            errs["d_" + k] = rel_err(to_np(run.grads[k]), g_ref[k])
     if intermediates:
         gi = gpu_intermediates(cfg, layer, run)
         ref = dict(ln1=saved["ln1"], qkv=saved["qkv"], O=saved["O"], lse=saved["lse"],
-                   h1=saved["h1"], ln2=saved["ln2"], a=saved["a"],
-                   gelu_grad=oracle.gelu_grad(saved["u"], cfg.gelu_tanh), **inter)
+                   h1=saved["h1"], ln2=saved["ln2"], a=saved["a"], **inter)
+        if getattr(cfg, "swiglu", 0):
+            ref["u"] = saved["u"]
+        else:
+            ref["gelu_grad"] = oracle.gelu_grad(saved["u"], cfg.gelu_tanh)
         for k in gi:
             errs[k] = rel_err(gi[k], ref[k])
     return errs

@@ -8,7 +8,7 @@ import re
 import pytest
 
 import tensor_transformer_layer_megatron_b200 as mgt
-from mgt_inputs import CONFIGS
+from mgt_inputs import CONFIGS, VARIANTS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -29,7 +29,8 @@ def test_library_exports_every_declared_symbol():
 
 def _init(**kw):
     base = dict(hidden=64, heads=4, ffn=256, seq=32, micro_batch=2, tp_size=2, dtype=0,
-                causal=1, ln_eps=1e-5, recompute_attn=1, gelu_tanh=0)
+                causal=1, ln_eps=1e-5, recompute_attn=1, gelu_tanh=0, swiglu=0,
+                disable_bias_linear=0)
     base.update(kw)
     lib = mgt.load_library()
     cfg = mgt._Config(*[base[f] for f, _ in mgt._Config._fields_])
@@ -63,6 +64,7 @@ def test_golden_tp_divisibility():
     (dict(dtype=1), 2),                   # bf16 needs head_dim 64/128 (here 16)
     (dict(dtype=1, hidden=128, heads=2, tp_size=2, ffn=200), 2),      # f/p = 100, not a multiple of 64
     (dict(hidden=512, heads=4), 2),       # fp32 head_dim 128 > 64
+    (dict(swiglu=2), 1), (dict(disable_bias_linear=-1), 1),           # flags are 0 or 1
 ])
 def test_init_rejects(kw, code):
     assert _init(**kw) == code
@@ -82,14 +84,15 @@ def test_null_handle_and_status_strings():
     assert lib.mgt_status_string(4) == b"device wait timed out"
 
 
-@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", CONFIGS + VARIANTS, ids=lambda c: c.name)
 def test_region_layout(cfg):
     L = mgt.Layer.from_config(cfg)
     saved, ws = L.sizes()
     T, h, f, e = cfg.tokens, cfg.hidden, cfg.ffn, 2 if cfg.dtype == "bf16" else 4
+    f1 = cfg.fc1_rows  # SwiGLU keeps [gate | up] and its gradient: 2f columns
     expect = {"ln1": T * h * e, "qkv": 3 * T * h * e, "attn_o": T * h * e,
-              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_dgelu": T * f * e,
-              "fc1_a": T * f * e, "du": T * f * e, "dqkv": 3 * T * h * e}
+              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_dgelu": T * f1 * e,
+              "fc1_a": T * f * e, "du": T * f1 * e, "dqkv": 3 * T * h * e}
     spans = []
     for name, rid in mgt.REGIONS.items():
         o, n = L.region(name)

@@ -1,7 +1,8 @@
 """Parity at the full workload sizes, in the launch configuration the benchmark times.
 
-h=1024 and h=4096 layers: the whole layer (y, dx, all 12 parameter gradients and every saved or
-workspace intermediate) against the fp64 oracle on the benchmark's own seeded inputs.
+h=1024 and h=4096 layers (and the h=4096 layer in its SwiGLU, no-bias form): the whole layer
+(y, dx, every parameter gradient and every saved or workspace intermediate) against the fp64
+oracle on the benchmark's own seeded inputs.
 
 h=6144 and h=12288 layers (too large for a whole-layer fp64 run in a test): the GPU runs the full
 layer with the benchmark's inputs except that the upstream gradient dy is zero beyond the first m
@@ -29,7 +30,8 @@ def _log(name, errs):
             f.write(json.dumps({"config": name, "errors": errs}) + "\n")
 
 
-@pytest.mark.parametrize("name", ["gpt-h1024-bf16", "gpt-h4096-tp2-bf16"])
+@pytest.mark.parametrize("name", ["gpt-h1024-bf16", "gpt-h4096-tp2-bf16",
+                                  "llama-h4096-tp2-bf16-swiglu-nobias"])
 def test_full_layer_parity_at_full_size(name):
     cfg = config_by_name(name)
     errs = full_parity(cfg, nonzero_affine=False, intermediates=True)

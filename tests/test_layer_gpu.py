@@ -1,6 +1,7 @@
 """Layer parity of the CUDA path against the fp64 oracle, through the C ABI, on seeded inputs:
 small layers spanning several tiles with ragged tails (tokens, sequence, ffn per shard),
-tp_size 1/2/4, head_dim 64/128, both GeLU forms, and the fp32 correctness layer."""
+tp_size 1/2/4, head_dim 64/128, both GeLU forms, the SwiGLU and no-bias variants, and the
+fp32 correctness layer."""
 import pytest
 
 from mgt_inputs import LayerConfig, config_by_name
@@ -27,6 +28,19 @@ SMALL = [
     small("h128-d64-p1-s1", hidden=128, heads=2, ffn=256, seq=1, micro_batch=4, tp_size=1),
 ]
 
+# SwiGLU (fc1 tiles pair a shard's gate and up rows) and no-bias layers. f/p = 128 sends the
+# fc2 dgrad (SwiGLU backward epilogue) to the one-CTA kernel, wider f/p to the CTA pairs.
+VARIANTS = [
+    small("h128-d64-p2-swiglu-s80-b2", hidden=128, heads=2, ffn=256, seq=80, micro_batch=2,
+          tp_size=2, swiglu=1),
+    small("h256-d128-p2-swiglu-s200", hidden=256, heads=2, ffn=512, seq=200, micro_batch=1,
+          tp_size=2, swiglu=1),
+    small("h512-d64-p4-swiglu-nobias-s130-b3", hidden=512, heads=8, ffn=1536, seq=130,
+          micro_batch=3, tp_size=4, swiglu=1, disable_bias_linear=1),
+    small("h256-d64-p1-nobias-s64", hidden=256, heads=4, ffn=768, seq=64, micro_batch=1,
+          tp_size=1, disable_bias_linear=1),
+]
+
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_layer_bf16_small(cfg):
@@ -38,6 +52,22 @@ def test_layer_bf16_small(cfg):
 @pytest.mark.parametrize("affine", [False, True])
 def test_layer_f32_tiny(affine):
     cfg = config_by_name("tiny-h64-tp2-f32")
+    errs = full_parity(cfg, nonzero_affine=affine)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("cfg", VARIANTS, ids=lambda c: c.name)
+def test_layer_bf16_variants(cfg):
+    errs = full_parity(cfg)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("nobias", [0, 1])
+@pytest.mark.parametrize("affine", [False, True])
+def test_layer_f32_tiny_swiglu(affine, nobias):
+    cfg = config_by_name("tiny-h64-tp2-f32-swiglu").replace(disable_bias_linear=nobias)
     errs = full_parity(cfg, nonzero_affine=affine)
     bad = {k: v for k, v in errs.items() if v > tol(cfg)}
     assert not bad, (bad, errs)
