@@ -4,9 +4,8 @@
 // heads without communication). Softmax arithmetic is fp32 (section 3.2,
 // attention_softmax_in_fp32). Scale 1/sqrt(d); key j visible to query i iff j <= i.
 //
-// bf16 path: forward and backward run on tcgen05 (attn_tc.cu); this file holds the pass that
-// forms D = rowsum(dO * O) for the backward. The backward recomputes the probabilities from
-// the saved log-sum-exp (the page's section 4.1 recompute).
+// bf16 path: forward and backward run on tcgen05 (attn_tc.cu). The backward recomputes the
+// probabilities from the saved log-sum-exp (the page's section 4.1 recompute).
 // fp32 path: plain per-row kernels (tiny shapes only).
 #include "mgt_device.cuh"
 
@@ -89,41 +88,6 @@ __global__ void attn_bwd_f32_kernel(AttnArgs a) {
   for (int c = 0; c < d; ++c) dbase[(long long)i * ld + c] = dq[c] * scale;
 }
 
-// ============================================================================ bf16 backward
-// D[b][n][q] = sum_c dO[q, n*d + c] * O[q, n*d + c]; one warp per (token, head).
-template <int D>
-__global__ void attn_bwd_pre_kernel(AttnArgs a) {
-  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long long total = (long long)a.b * a.s * a.H;
-  if (w >= total) return;
-  const int n = (int)(w % a.H);
-  const long long tok = w / a.H;
-  const int b = (int)(tok / a.s), q = (int)(tok % a.s);
-  constexpr int E = D / 32;  // 2 or 4 elements per lane
-  const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(a.o) + tok * a.H * D + n * D;
-  const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(a.dO) + tok * a.H * D + n * D;
-  float s = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; e += 2) {
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + lane * E + e);
-    const uint32_t dv = *reinterpret_cast<const uint32_t*>(dO + lane * E + e);
-    s += bf16_lo(ov) * bf16_lo(dv) + bf16_hi(ov) * bf16_hi(dv);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) a.Dsum[((long long)b * a.H + n) * a.s + q] = s;
-}
-
-template <int D>
-cudaError_t bwd_bf16(const AttnArgs& a, cudaStream_t s) {
-  const long long warps = (long long)a.b * a.s * a.H;
-  attn_bwd_pre_kernel<D><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_attn_bwd_tc(a, s);  // dK/dV and dQ kernels on tcgen05 (attn_tc.cu)
-}
-
 }  // namespace
 
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t s) {
@@ -144,9 +108,7 @@ cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t s) {
     attn_bwd_f32_kernel<64><<<(total + 127) / 128, 128, 0, s>>>(a);
     return cudaGetLastError();
   }
-  if (a.d == 64) return bwd_bf16<64>(a, s);
-  if (a.d == 128) return bwd_bf16<128>(a, s);
-  return cudaErrorInvalidValue;
+  return launch_attn_bwd_tc(a, s);  // dQ (with D) then dK/dV kernels on tcgen05 (attn_tc.cu)
 }
 
 

@@ -336,11 +336,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 // ============================================================================ backward
 // Two kernels, both on tcgen05 with the probabilities recomputed from the saved log-sum-exp:
-//   dK/dV kernel, one CTA per 128-key block (key-stationary), looping over query blocks:
-//     S^T = K Q^T and dP^T = V dO^T in TMEM; one thread per key row forms
-//     P^T = exp2(S^T*scale*log2e - lse*log2e) and dS^T = P^T * (dP^T - D) (D = rowsum(dO*O))
-//     and writes both back into TMEM as packed bf16; then dV += P^T dO and dK += dS^T Q run with
-//     the A operand read from TMEM and dO, Q read N-major from their TMA tiles.
+//   dK/dV kernel, one CTA per 128-key block (key-stationary), looping over query blocks in
+//     64-query sub-blocks with double-buffered TMEM: S^T = K Q^T and dP^T = V dO^T; one
+//     thread per key row forms P^T = exp2(S^T*scale*log2e - lse*log2e) and
+//     dS^T = P^T * (dP^T - D) (D = rowsum(dO*O)) and writes both back into TMEM as packed
+//     bf16; then dV += P^T dO and dK += dS^T Q run with the A operand read from TMEM and dO, Q
+//     read N-major from their TMA tiles. The next sub-block's S^T, dP^T are computed while the
+//     softmax warps work on this one.
 //   dQ kernel, one CTA per 128-query block (query-stationary), looping over key blocks:
 //     S = Q K^T, dP = dO V^T, dS = P * (dP - D) per query row, dQ += dS K.
 // dQ therefore needs no atomics and is written once, in bf16, scaled by 1/sqrt(d); the cost is
@@ -357,8 +359,12 @@ struct BwdLayout {
   // dQ kernel: Q, dO resident; K and V double-buffered.
   static constexpr int B_Q = 0, B_DO = TILE, B_K = 2 * TILE, B_V = 4 * TILE;
   static constexpr int B_BAR = 6 * TILE;
-  static constexpr int B_BYTES = B_BAR + 256 + 1024;
-  static constexpr int T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+  static constexpr int B_RED = B_BAR + 256;  // float [2 halves][128 rows]: partial rowsum(dO*O)
+  static constexpr int B_BYTES = B_RED + 1024 + 1024;
+  // dK/dV kernel: each 128-query block runs as two 64-query sub-blocks; sub-block g uses
+  // buffer x = g & 1 with S^T in columns x*128 .. +63 and dP^T in x*128 + 64 .. +63; the dV
+  // and dK accumulators follow.
+  static constexpr int T_SUB = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
   // dQ kernel: two S buffers so the next block's S overlaps this block's dS computation.
   static constexpr int Q_S0 = 0, Q_S1 = 128, Q_DP = 256, Q_DQ = 384;
 };
@@ -375,12 +381,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;   // [2]: Q and dO of one query block
   uint64_t* q_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* mm_done = bars + 7;
-  uint64_t* drain = bars + 8;
-  uint64_t* stat_bar = bars + 9;  // [2]: per-query stats of a block staged by the 4 warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* s_full = bars + 5;   // [2]: S^T, dP^T of a sub-block in buffer x
+  uint64_t* p_full = bars + 7;   // [2]: P^T, dS^T of a sub-block written back
+  uint64_t* mm_done = bars + 9;  // [2]: dV, dK MMAs of a sub-block done (buffer x free)
+  uint64_t* drain = bars + 11;
+  uint64_t* stat_bar = bars + 12;  // [2]: per-query stats of a block staged by the 8 warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* lse_s = reinterpret_cast<float*>(smem + L::A_STAT);  // [2][128], log2 units
   float* dsum_s = lse_s + 256;                                 // [2][128]
@@ -401,9 +407,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
-    mbar_init(mm_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&mm_done[i], 1);
+    }
     mbar_init(drain, 1);
     mbar_init(&stat_bar[0], 256);
     mbar_init(&stat_bar[1], 256);
@@ -452,59 +460,81 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == 9) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      // Sub-block g (query block it = g/2, half j = g%2) in TMEM buffer x = g%2:
+      //   S^T = K Q_j^T and dP^T = V dO_j^T (M=128 keys, N=64 queries), then, once the
+      //   softmax warps have written P^T and dS^T back, dV += P^T dO_j and dK += dS^T Q_j
+      //   (K=64 queries, A from TMEM). S^T, dP^T of g+1 are issued before waiting for the
+      //   softmax of g, so the tensor pipe and the softmax warps overlap.
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
       const uint32_t k_addr = smem_u32(smem + L::A_K), v_addr = smem_u32(smem + L::A_V);
-      bool ok = mbar_wait(kv_full, 0, a.err, kErrTimeoutAttn, abort_flag);
-      for (int it = 0; it < niter && ok; ++it) {
-        const int st = it & 1;
-        // the previous block's dV/dK MMAs read P and dS from the S/dP columns: wait for them
-        if (it > 0 && !mbar_wait(mm_done, (it - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
-          break;
-        if (!mbar_wait(&q_full[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+      const int G = 2 * niter;
+      auto issue_sd = [&](int g) -> bool {
+        const int it = g >> 1, j = g & 1, st = it & 1;
+        const uint32_t x = (g & 1) * L::T_SUB;
+        if (j == 0 && !mbar_wait(&q_full[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + L::A_Q + st * L::TILE);
-        const uint32_t do_addr = smem_u32(smem + L::A_DO + st * L::TILE);
+        const uint32_t q_addr = smem_u32(smem + L::A_Q + st * L::TILE) + j * 8192;
+        const uint32_t do_addr = smem_u32(smem + L::A_DO + st * L::TILE) + j * 8192;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_f16(tmem + L::T_S, smem_desc_sw128(k_addr + off, 16, 1024),
+          tc_mma_f16(tmem + x, smem_desc_sw128(k_addr + off, 16, 1024),
                      smem_desc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_f16(tmem + L::T_DP, smem_desc_sw128(v_addr + off, 16, 1024),
+          tc_mma_f16(tmem + x + 64, smem_desc_sw128(v_addr + off, 16, 1024),
                      smem_desc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(s_full);
-        if (!mbar_wait(p_full, it & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        tc_commit(&s_full[g & 1]);
+        return true;
+      };
+      bool ok = mbar_wait(kv_full, 0, a.err, kErrTimeoutAttn, abort_flag);
+      if (ok && G > 0) ok = issue_sd(0);
+      for (int g = 0; g < G && ok; ++g) {
+        if (g + 1 < G) {
+          // buffer (g+1)&1 was last read (P^T, dS^T as A operands) by the MMAs of g-1
+          if (g >= 1 && !mbar_wait(&mm_done[(g + 1) & 1], ((g - 1) >> 1) & 1, a.err,
+                                   kErrTimeoutAttn, abort_flag))
+            break;
+          if (!issue_sd(g + 1)) break;
+        }
+        if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
         tc_fence_after();
+        const int it = g >> 1, j = g & 1, st = it & 1;
+        const uint32_t x = (g & 1) * L::T_SUB;
+        const uint32_t q_addr = smem_u32(smem + L::A_Q + st * L::TILE) + j * 8192;
+        const uint32_t do_addr = smem_u32(smem + L::A_DO + st * L::TILE) + j * 8192;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 128 queries, 16 per MMA
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          tc_mma_f16_tmem_a(tmem + L::T_ACC0, tmem + L::T_S + kk * 8,
+        for (int kk = 0; kk < 4; ++kk) {  // 64 queries, 16 per MMA
+          const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
+          // packed P^T / dS^T: queries 0-31 in columns 0-15, queries 32-63 in 32-47
+          const uint32_t pc = kk * 8 + (kk >= 2 ? 16 : 0);
+          tc_mma_f16_tmem_a(tmem + L::T_ACC0, tmem + x + pc,
                             smem_desc_sw128(do_addr + kk * 2048, 16384, 1024), idesc_acc, acc);
-          tc_mma_f16_tmem_a(tmem + L::T_ACC1, tmem + L::T_DP + kk * 8,
+          tc_mma_f16_tmem_a(tmem + L::T_ACC1, tmem + x + 64 + pc,
                             smem_desc_sw128(q_addr + kk * 2048, 16384, 1024), idesc_acc, acc);
         }
-        tc_commit(mm_done);
-        tc_commit(&q_empty[st]);
+        tc_commit(&mm_done[g & 1]);
+        if (j == 1) tc_commit(&q_empty[st]);
       }
       tc_commit(drain);
       mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
     }
   } else {
     // ------------------------------------------------------------ P^T, dS^T and the output
-    // warp w: TMEM lane quarter w%4 (key rows), query-column half w/4 (64 queries)
+    // warp w: TMEM lane quarter w%4 (key rows), 32-query half w/4 of each 64-query sub-block
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // key row within the block = TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float* lse_g = a.lse + ((long long)b * H + n) * S;
     const float* dsum_g = a.Dsum + ((long long)b * H + n) * S;
     bool ok = true;
-    // Per-query stats of the next block are fetched one iteration ahead (registers); half 0
-    // stages lse, half 1 stages D, each for query r of the block.
+    // Per-query stats of the next block are fetched one block ahead (registers); warps of
+    // half 0 stage lse, half 1 stage D, each for query r of the block.
     const float* stat_g = hf ? dsum_g : lse_g;
     float* stat_s = hf ? dsum_s : lse_s;
     auto fetch = [&](int qi) -> float {
@@ -513,71 +543,68 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       return q < S ? stat_g[q] : 0.f;
     };
     float nv = niter > 0 ? fetch(kb) : 0.f;
-    for (int it = 0; it < niter; ++it) {
-      const int st = it & 1, qi = kb + it;
-      stat_s[st * 128 + r] = nv;
-      if (it + 1 < niter) nv = fetch(qi + 1);
-      mbar_arrive(&stat_bar[st]);
-      ok = mbar_wait(&stat_bar[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
+    for (int g = 0; g < 2 * niter; ++g) {
+      const int it = g >> 1, j = g & 1, st = it & 1, qi = kb + it;
+      if (j == 0) {
+        stat_s[st * 128 + r] = nv;
+        if (it + 1 < niter) nv = fetch(qi + 1);
+        mbar_arrive(&stat_bar[st]);
+        ok = mbar_wait(&stat_bar[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
       }
-      ok = mbar_wait(s_full, it & 1, a.err, kErrTimeoutAttn, abort_flag);
+      ok = mbar_wait(&s_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* ls = lse_s + st * 128;
-      const float* ds_ = dsum_s + st * 128;
-      {
-        const int c2 = hf * 2;  // this half's two 32-column chunks of S and dP
-        uint32_t sr[2][32], dr[2][32];
+      const uint32_t x = (g & 1) * L::T_SUB;
+      const int q0 = j * 64 + hf * 32;  // first query (within the block) of this warp's columns
+      const float* ls = lse_s + st * 128 + q0;
+      const float* ds_ = dsum_s + st * 128 + q0;
+      uint32_t sr[32], dr[32];
+      tmem_ld_32x32b_x32_nw(lane_base + x + hf * 32, sr);
+      tmem_ld_32x32b_x32_nw(lane_base + x + 64 + hf * 32, dr);
+      tmem_ld_wait();
+      reg_fence(sr);
+      reg_fence(dr);
+      if (qi == kb) {  // diagonal block: queries before this key see nothing of it
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          tmem_ld_32x32b_x32_nw(lane_base + L::T_S + (c2 + u) * 32, sr[u]);
-          tmem_ld_32x32b_x32_nw(lane_base + L::T_DP + (c2 + u) * 32, dr[u]);
-        }
-        tmem_ld_wait();
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          reg_fence(sr[u]);
-          reg_fence(dr[u]);
-          const int c = c2 + u;
-          if (qi == kb) {  // diagonal block: queries before this key see nothing of it
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i < r) sr[u][i] = __float_as_uint(-INFINITY);
-          }
-          uint32_t pw[16], dw[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + i);
-            const float4 d4 = *reinterpret_cast<const float4*>(ds_ + c * 32 + i);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-            float p4[4], q4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              p4[e] = ex2_approx(fmaf(__uint_as_float(sr[u][i + e]), scale_log2, -lv[e]));
-              q4[e] = p4[e] * (__uint_as_float(dr[u][i + e]) - dv[e]);
-            }
-            pw[i >> 1] = pack_bf16x2(p4[0], p4[1]);
-            pw[(i >> 1) + 1] = pack_bf16x2(p4[2], p4[3]);
-            dw[i >> 1] = pack_bf16x2(q4[0], q4[1]);
-            dw[(i >> 1) + 1] = pack_bf16x2(q4[2], q4[3]);
-          }
-          tmem_st_32x32b_x16(lane_base + L::T_S + c * 16, pw);
-          tmem_st_32x32b_x16(lane_base + L::T_DP + c * 16, dw);
-        }
+        for (int i = 0; i < 32; ++i)
+          if (q0 + i < r) sr[i] = __float_as_uint(-INFINITY);
       }
+      uint32_t pw[16], dw[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(ls + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(ds_ + i);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float p4[4], q4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          p4[e] = ex2_approx(fmaf(__uint_as_float(sr[i + e]), scale_log2, -lv[e]));
+          q4[e] = p4[e] * (__uint_as_float(dr[i + e]) - dv[e]);
+        }
+        pw[i >> 1] = pack_bf16x2(p4[0], p4[1]);
+        pw[(i >> 1) + 1] = pack_bf16x2(p4[2], p4[3]);
+        dw[i >> 1] = pack_bf16x2(q4[0], q4[1]);
+        dw[(i >> 1) + 1] = pack_bf16x2(q4[2], q4[3]);
+      }
+      // Packed into the first half of the 32 columns this warp itself read, so the other
+      // warp of the quarter (reading its own 32 columns) is never overwritten.
+      tmem_st_32x32b_x16(lane_base + x + hf * 32, pw);
+      tmem_st_32x32b_x16(lane_base + x + 64 + hf * 32, dw);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[g & 1]);
     }
     if (ok && niter > 0) {
-      ok = mbar_wait(mm_done, (niter - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      const int gl = 2 * niter - 1;  // last sub-block
+      ok = mbar_wait(&mm_done[gl & 1], (gl >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int key = kb * 128 + r;
@@ -635,7 +662,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_full = bars + 6;
   uint64_t* mm_done = bars + 7;
   uint64_t* drain = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* dsum_bar = bars + 9;  // [4 quarters]: the two halves of D = rowsum(dO*O)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -656,6 +684,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(p_full, 8);
     mbar_init(mm_done, 1);
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&dsum_bar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -746,18 +775,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if (!mbar_wait(p_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::B_K + (kb & 1) * L::TILE);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA; dS sits in S buffer kb&1
-          tc_mma_f16_tmem_a(tmem + L::Q_DQ, tmem + ((kb & 1) ? L::Q_S1 : L::Q_S0) + kk * 8,
-                            smem_desc_sw128(k_addr + kk * 2048, 16384, 1024), idesc_acc,
-                            (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(mm_done);
-        tc_commit(&kv_empty[kb & 1]);
+        // The softmax warps are done with dP_kb: dP_{kb+1} goes first, so they can start on
+        // the next block while the tensor pipe still works on dQ += dS_kb K_kb.
         if (more) {
           issue_dp(kb + 1);
           tc_commit(s_full);
         }
+        const uint32_t k_addr = smem_u32(smem + L::B_K + (kb & 1) * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA; dS sits in S buffer kb&1
+          tc_mma_f16_tmem_a(tmem + L::Q_DQ,
+                            tmem + ((kb & 1) ? L::Q_S1 : L::Q_S0) + kk * 8 + (kk >= 4 ? 32 : 0),
+                            smem_desc_sw128(k_addr + kk * 2048, 16384, 1024), idesc_acc,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(mm_done);
+        tc_commit(&kv_empty[kb & 1]);
       }
       tc_commit(drain);
       mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
@@ -769,9 +801,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int q = qb * 128 + r;
     const float lse2 = q < S ? a.lse[((long long)b * H + n) * S + q] * kLog2eF : INFINITY;
-    const float dq_sum = q < S ? a.Dsum[((long long)b * H + n) * S + q] : 0.f;
-    bool ok = true;
-    for (int kb = 0; kb < nkv; ++kb) {
+    // D = rowsum(dO * O) of this query row, each warp of the quarter pair summing half of d
+    // while the first tiles load; the dK/dV kernel, launched next, reads it from a.Dsum.
+    float dpart = 0.f;
+    if (q < S) {
+      const long long off = ((long long)b * S + q) * H * D + (long long)n * D + hf * (D / 2);
+      const __nv_bfloat16* orow = reinterpret_cast<const __nv_bfloat16*>(a.o) + off;
+      const __nv_bfloat16* drow = reinterpret_cast<const __nv_bfloat16*>(a.dO) + off;
+#pragma unroll
+      for (int i = 0; i < D / 2; i += 8) {
+        const uint4 ov = *reinterpret_cast<const uint4*>(orow + i);
+        const uint4 dv = *reinterpret_cast<const uint4*>(drow + i);
+        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw4[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dpart += bf16_lo(ow[e]) * bf16_lo(dw4[e]) + bf16_hi(ow[e]) * bf16_hi(dw4[e]);
+      }
+    }
+    float* dred = reinterpret_cast<float*>(smem + L::B_RED);  // [2][128]
+    dred[hf * 128 + r] = dpart;
+    mbar_arrive(&dsum_bar[quarter]);
+    bool ok = mbar_wait(&dsum_bar[quarter], 0, a.err, kErrTimeoutAttn, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    const float dq_sum = ok ? dpart + dred[(hf ^ 1) * 128 + r] : 0.f;
+    if (ok && hf == 0 && q < S) a.Dsum[((long long)b * H + n) * S + q] = dq_sum;
+    for (int kb = 0; kb < nkv && ok; ++kb) {
       ok = mbar_wait(s_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
@@ -809,7 +863,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             dw[i >> 1] = pack_bf16x2(d2[0], d2[1]);
           }
-          tmem_st_32x32b_x16(lane_base + s_col + c * 16, dw);
+          // packed into the first half of this warp's own 64 columns (see the dK/dV kernel)
+          tmem_st_32x32b_x16(lane_base + s_col + hf * 64 + u * 16, dw);
         }
       }
       tmem_wait_st();
@@ -880,12 +935,13 @@ cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
   }
   const float scale = 1.f / sqrtf((float)D);
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
-  attn_bwd_dkdv_tc_kernel<D><<<grid, kFwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
-                                                                    kLog2eF * scale, scale);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // The dQ kernel goes first: it also forms D = rowsum(dO * O), which the dK/dV kernel reads.
   attn_bwd_dq_tc_kernel<D><<<grid, kFwdThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                   kLog2eF * scale, scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kFwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
+                                                                    kLog2eF * scale, scale);
   return cudaGetLastError();
 }
 

@@ -482,14 +482,14 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
   if (c0 < cols) {
     long long r = r0 + threadIdx.y;
-    for (; r + 24 < r1; r += 32) {  // four independent rows in flight per thread
-      float v0[V], v1[V], v2[V], v3[V];
-      Vec<T>::load(x + r * cols + c0, v0);
-      Vec<T>::load(x + (r + 8) * cols + c0, v1);
-      Vec<T>::load(x + (r + 16) * cols + c0, v2);
-      Vec<T>::load(x + (r + 24) * cols + c0, v3);
+    for (; r + 56 < r1; r += 64) {  // eight independent rows in flight per thread
+      float v[8][V];
 #pragma unroll
-      for (int j = 0; j < V; ++j) acc[j] += (v0[j] + v1[j]) + (v2[j] + v3[j]);
+      for (int u = 0; u < 8; ++u) Vec<T>::load(x + (r + 8 * u) * cols + c0, v[u]);
+#pragma unroll
+      for (int j = 0; j < V; ++j)
+        acc[j] += ((v[0][j] + v[1][j]) + (v[2][j] + v[3][j])) +
+                  ((v[4][j] + v[5][j]) + (v[6][j] + v[7][j]));
     }
     for (; r < r1; r += 8) {
       float v[V];
@@ -733,7 +733,7 @@ cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, fl
   if (e != cudaSuccess || rows <= 0) return e;
   const int V = dtype ? 8 : 4;
   const int cb = (cols + 32 * V - 1) / (32 * V);
-  long long splits = (2 * 148 + cb - 1) / cb;  // aim for >= 2 blocks per SM
+  long long splits = (4 * 148 + cb - 1) / cb;  // aim for ~4 blocks per SM
   if (splits > (rows + 7) / 8) splits = (rows + 7) / 8;
   if (splits < 1) splits = 1;
   const long long rows_per = (rows + splits - 1) / splits;

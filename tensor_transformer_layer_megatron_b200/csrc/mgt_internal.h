@@ -101,7 +101,8 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t stream);  // bf16, d in {64, 128}
-// bf16 backward: dK/dV kernel then dQ kernel, both tcgen05; needs a.Dsum = rowsum(dO * O).
+// bf16 backward: dQ kernel (which also writes a.Dsum = rowsum(dO * O)) then dK/dV kernel,
+// both tcgen05.
 cudaError_t launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 
