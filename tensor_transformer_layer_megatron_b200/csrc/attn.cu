@@ -12,8 +12,6 @@
 namespace mgt {
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
-
 // ============================================================================ fp32 kernels
 // One thread per (batch, head, query): online softmax over keys 0..i.
 template <int DMAX>

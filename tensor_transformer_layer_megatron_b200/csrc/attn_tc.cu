@@ -230,10 +230,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < 64; ++i)
           if (hf * 64 + i > r) sv[i] = -INFINITY;
       }
-      // row max over both halves (raw scores; the scale is positive)
-      float mx = sv[0];
+      // row max over both halves (raw scores; the scale is positive): eight independent
+      // chains, then a tree
+      float m8[8];
 #pragma unroll
-      for (int i = 1; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+      for (int k = 0; k < 8; ++k) m8[k] = sv[k];
+#pragma unroll
+      for (int i = 8; i < 64; i += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], sv[i + k]);
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       // exchange with the other half's warp (same rows) through a bounded mbarrier wait
       red[(st * 2 + hf) * 128 + r] = mx;
       mbar_arrive(&xchg[quarter * 2 + st]);
@@ -246,13 +253,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool need = mx > m_run + kRescaleThreshold;  // identical in both halves
       const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
-      float rs = 0.f;
+      // eight partial sums (short dependency chains)
+      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const float p = ex2_approx(fmaf(sv[i], scale_log2, -m_run));
         sv[i] = p;
-        rs += p;
+        r8[i & 7] += p;
       }
+      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l_part = l_part * alpha + rs;
       if (kb > 0) {
         // PV of the previous block must be done before O is rescaled or P overwritten.
@@ -383,8 +392,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* q_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;   // [2]: S^T, dP^T of a sub-block in buffer x
   uint64_t* p_full = bars + 7;   // [2]: P^T, dS^T of a sub-block written back
-  uint64_t* mm_done = bars + 9;  // [2]: dV, dK MMAs of a sub-block done (buffer x free)
-  uint64_t* drain = bars + 11;
+  uint64_t* drain = bars + 11;   // every MMA done (the output reads dV, dK after it)
   uint64_t* stat_bar = bars + 12;  // [2]: per-query stats of a block staged by the 8 warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -410,7 +418,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 8);
-      mbar_init(&mm_done[i], 1);
     }
     mbar_init(drain, 1);
     mbar_init(&stat_bar[0], 256);
@@ -495,13 +502,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = mbar_wait(kv_full, 0, a.err, kErrTimeoutAttn, abort_flag);
       if (ok && G > 0) ok = issue_sd(0);
       for (int g = 0; g < G && ok; ++g) {
-        if (g + 1 < G) {
-          // buffer (g+1)&1 was last read (P^T, dS^T as A operands) by the MMAs of g-1
-          if (g >= 1 && !mbar_wait(&mm_done[(g + 1) & 1], ((g - 1) >> 1) & 1, a.err,
-                                   kErrTimeoutAttn, abort_flag))
-            break;
-          if (!issue_sd(g + 1)) break;
-        }
+        // Buffer (g+1)&1 was last read (P^T, dS^T as A operands) by the dV/dK MMAs of g-1,
+        // issued earlier by this thread: MMAs of one thread execute in issue order, so those
+        // reads precede the S^T, dP^T writes of g+1 and no wait is needed. (The softmax
+        // warps' own reads of that buffer finished before they signalled p_full of g-1.)
+        if (g + 1 < G && !issue_sd(g + 1)) break;
         if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
         tc_fence_after();
         const int it = g >> 1, j = g & 1, st = it & 1;
@@ -518,7 +523,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tc_mma_f16_tmem_a(tmem + L::T_ACC1, tmem + x + 64 + pc,
                             smem_desc_sw128(q_addr + kk * 2048, 16384, 1024), idesc_acc, acc);
         }
-        tc_commit(&mm_done[g & 1]);
         if (j == 1) tc_commit(&q_empty[st]);
       }
       tc_commit(drain);
@@ -603,8 +607,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[g & 1]);
     }
     if (ok && niter > 0) {
-      const int gl = 2 * niter - 1;  // last sub-block
-      ok = mbar_wait(&mm_done[gl & 1], (gl >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
+      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int key = kb * 128 + r;
@@ -660,7 +664,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
-  uint64_t* mm_done = bars + 7;
   uint64_t* drain = bars + 8;
   uint64_t* dsum_bar = bars + 9;  // [4 quarters]: the two halves of D = rowsum(dO*O)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
@@ -682,7 +685,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, 8);
-    mbar_init(mm_done, 1);
     mbar_init(drain, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&dsum_bar[i], 64);
     *abort_flag = 0;
@@ -764,9 +766,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int kb = 0; kb < nkv && ok; ++kb) {
         const bool more = kb + 1 < nkv;
         if (more) {
-          // S buffer (kb+1)&1 was last read (as dS) by the dQ MMA of block kb-1
-          if (kb >= 1 && !mbar_wait(mm_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
-            break;
+          // S buffer (kb+1)&1 was last read (as dS) by the dQ MMAs of block kb-1, issued
+          // earlier by this thread: MMAs execute in issue order, so no wait is needed.
           if (!mbar_wait(&kv_full[(kb + 1) & 1], ((kb + 1) >> 1) & 1, a.err, kErrTimeoutAttn,
                          abort_flag))
             break;
@@ -788,7 +789,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             tmem + ((kb & 1) ? L::Q_S1 : L::Q_S0) + kk * 8 + (kk >= 4 ? 32 : 0),
                             smem_desc_sw128(k_addr + kk * 2048, 16384, 1024), idesc_acc,
                             (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(mm_done);
         tc_commit(&kv_empty[kb & 1]);
       }
       tc_commit(drain);
@@ -873,7 +873,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (lane == 0) mbar_arrive(p_full);
     }
     if (ok) {
-      ok = mbar_wait(mm_done, (nkv - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
+      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const long long ld = 3LL * H * D;
