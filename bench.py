@@ -129,15 +129,27 @@ def job_throughput(tokens_per_rank, world, ms_total, steps):
     return tokens_per_rank * world / (ms_step / 1e3), ms_step
 
 
-def e2e_steps(run, host, steps, stream):
+def e2e_steps(run, host, steps, stream, graph=True):
     """K steps through the C ABI with host buffers; returns the device-timed ms. Every step
     copies its own x, dy from pinned host memory and its y, dx back. The device buffers are
     double-buffered and the copies run on two copy streams, so step i+1's inputs arrive and
-    step i-1's results leave while step i computes (a training loop with prefetch)."""
+    step i-1's results leave while step i computes (a training loop with prefetch). With
+    `graph`, the C-ABI calls of a step (which allocate nothing and never synchronise) are
+    captured once per buffer set into a CUDA graph and replayed; the copies stay outside."""
     import torch
     x_h, dy_h, y_h, dx_h = host
     first = (run.x, run.dy, run.y, run.dx)
     bufs = [first, tuple(torch.empty_like(t) for t in first)]
+    graphs = [None, None]
+    if graph:
+        for b in range(2):
+            run.x, run.dy, run.y, run.dx = bufs[b]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run.step()
+            graphs[b] = g
+        run.x, run.dy, run.y, run.dx = first
+        torch.cuda.synchronize()
     s_in, s_out = torch.cuda.Stream(run.x.device), torch.cuda.Stream(run.x.device)
     in_ready = [torch.cuda.Event(), torch.cuda.Event()]
     comp_done = [torch.cuda.Event(), torch.cuda.Event()]
@@ -157,8 +169,11 @@ def e2e_steps(run, host, steps, stream):
         stream.wait_event(in_ready[b])
         if i >= 2:
             stream.wait_event(out_done[b])  # step i-2's y[b], dx[b] have been copied out
-        run.x, run.dy, run.y, run.dx = x, dy, y, dx
-        run.step(stream)
+        if graphs[b] is not None:
+            graphs[b].replay()
+        else:
+            run.x, run.dy, run.y, run.dx = x, dy, y, dx
+            run.step(stream)
         comp_done[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[b])
@@ -251,8 +266,8 @@ def run_mgt(args):
     dx_h = torch.empty_like(x_h).pin_memory()
     barrier()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e2e_steps(run, (x_h, dy_h, y_h, dx_h), args.steps, stream), world,
-                            dev)
+    e2e_ms = max_over_ranks(e2e_steps(run, (x_h, dy_h, y_h, dx_h), args.steps, stream,
+                                      graph=args.graph), world, dev)
     barrier()
     # the pipelined copies delivered what the device computed (same inputs every step; the
     # layer's y and dx are deterministic)
@@ -334,10 +349,11 @@ def run_mgt(args):
                              "630 MB + activations) exceeds the 126 MB L2"},
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "what": "every step: x, dy pinned host -> device, fwd+bwd via the C ABI, "
-                            "y, dx -> pinned host; copies on two copy streams into "
+                    "what": "every step: x, dy pinned host -> device, fwd+bwd via the C ABI "
+                            "(%s), y, dx -> pinned host; copies on two copy streams into "
                             "double-buffered device tensors, overlapping the neighbouring "
-                            "steps' compute"},
+                            "steps' compute" % ("CUDA-graph replay of the calls" if args.graph
+                                                else "eager calls")},
             "roofline": roof,
             "kernels": kernels,
             "kernels_timing": ("CUDA events around every launch, eager pass of the same K steps "

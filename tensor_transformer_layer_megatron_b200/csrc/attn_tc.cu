@@ -9,13 +9,14 @@
 // Per key block of 128 (double-buffered K/V tiles from TMA):
 //   S = Q K^T            tcgen05.mma M=128 N=128, fp32 in TMEM (two S buffers, so the next
 //                        block's S is computed while the softmax works on this one)
-//   softmax warps        one thread per query row reads its 128 scores with tcgen05.ld, so
-//                        the row max and sum need no shuffles; P = exp2(S*scale*log2e - m)
-//                        goes to shared memory as bf16 in the 128B-swizzled K-major layout
-//   O += P V             tcgen05.mma M=128 N=d, V read N-major straight from its TMA tile
+//   softmax warps        one thread per query row reads all 128 of its scores with tcgen05.ld,
+//                        so the row max and sum need no exchange between threads;
+//                        P = exp2(S*scale*log2e - m) is packed to bf16 and written back into the
+//                        first 64 columns of the same S buffer
+//   O += P V             tcgen05.mma M=128 N=d with A = P read from TMEM and V read N-major
+//                        straight from its TMA tile
 // The running max is updated lazily: O and the row sum are rescaled only when a row's max grows
-// by more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16), and the
-// rescale of O in TMEM is done by whole warps (tcgen05.ld/st are warp-collective).
+// by more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16).
 // Finally O / l is written in bf16 and lse = (m + log2 l) * ln 2.
 //
 // Warps 0-3: softmax + output (warp w owns TMEM lanes 32w..32w+31, i.e. query rows);
@@ -36,26 +37,19 @@ struct FwdLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = TILE;             // 2 stages
   static constexpr int V_OFF = K_OFF + 2 * TILE; // 2 stages
-  static constexpr int P_OFF = V_OFF + 2 * TILE; // [128 q][128 keys] bf16, 2 chunks
-  static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
-  static constexpr int RED_OFF = BAR_OFF + 256;  // float [3][2 halves][128 rows]: max x2, sum
-  static constexpr int BYTES = RED_OFF + 3 * 2 * 128 * 4 + 1024;
+  static constexpr int BAR_OFF = V_OFF + 2 * TILE;
+  static constexpr int BYTES = BAR_OFF + 256 + 1024;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
 };
 
-// Every attention CTA: warps 0-7 do the elementwise work on TMEM rows (warp w: TMEM lane
-// quarter w%4, column half w/4), warp 8 is the TMA producer, warp 9 owns TMEM and issues MMAs.
+// Forward CTA: warps 0-3 softmax (one TMEM lane quarter each), warp 4 TMA, warp 5 MMA.
+constexpr int kAttnFwdThreads = 192;
+// Backward CTAs: warps 0-7 do the elementwise work on TMEM rows (warp w: TMEM lane quarter w%4,
+// column half w/4), warp 8 is the TMA producer, warp 9 owns TMEM and issues MMAs.
 constexpr int kFwdThreads = 320;
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kAttnFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a,
                        float scale_log2) {
   using L = FwdLayout<D>;
@@ -66,14 +60,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* k_empty = bars + 5;   // [2]: released as soon as S of that block has read K
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint64_t* v_empty = bars + 12;  // [2]: released once PV of that block has read V
-  uint64_t* xchg = bars + 14;     // [4 quarters][2 parities]: row-max exchange of a warp pair
-  uint64_t* xsum = bars + 22;     // [4 quarters]: final row-sum exchange
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
+  uint64_t* v_empty = bars + 7;   // [2]: released once PV of that block has read V
+  uint64_t* s_full = bars + 9;    // [2]
+  uint64_t* p_full = bars + 11;   // [2]: P of the block written into its S buffer
+  uint64_t* pv_done = bars + 13;
+  uint64_t* drain = bars + 14;    // every MMA done (one-shot: the output waits on it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -94,17 +86,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
     }
-    mbar_init(p_full, 8);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&xchg[i], 64);
-    for (int i = 0; i < 4; ++i) mbar_init(&xsum[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
   }
-  if (warp == 9) {
+  if (warp == 5) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -113,7 +103,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 4) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
       mbar_arrive_expect_tx(q_full, L::TILE);
@@ -147,13 +137,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int kb = issued_v - 2 < 0 ? 0 : issued_v - 2; kb < issued_v; ++kb)
         mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
     }
-  } else if (warp == 9) {
+  } else if (warp == 5) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
-      const uint32_t p_addr = smem_u32(smem + L::P_OFF);
       bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag);
       auto issue_s = [&](int kb) -> bool {
         const int st = kb & 1;
@@ -174,19 +163,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       if (ok) ok = issue_s(0);
       for (int kb = 0; kb < nkv && ok; ++kb) {
+        // S buffer (kb+1)&1 held block kb-1: its softmax finished reading it (p_full of kb-1
+        // was waited for below, one iteration ago) and its PV, which read P from it, was
+        // issued before this S by this thread (MMAs execute in issue order).
         if (kb + 1 < nkv && !issue_s(kb + 1)) break;
-        if (!mbar_wait(p_full, kb & 1, a.err, kErrTimeoutAttn, abort_flag)) break;
+        if (!mbar_wait(&p_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
         if (!mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
           break;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + L::V_OFF + (kb & 1) * L::TILE);
+        const uint32_t p_tmem = tmem + ((kb & 1) ? L::TMEM_S1 : L::TMEM_S0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
-          const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_f16(tmem + L::TMEM_O, smem_desc_sw128(p_addr + a_off, 16, 1024),
-                     smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                     (kb > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA (8 packed P columns)
+          tc_mma_f16_tmem_a(tmem + L::TMEM_O, p_tmem + kk * 8,
+                            smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
         tc_commit(pv_done);
         tc_commit(&v_empty[kb & 1]);
       }
@@ -195,31 +187,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + output
-    const int quarter = warp & 3, hf = warp >> 2;  // TMEM lane quarter, key-column half
-    const int r = quarter * 32 + lane;             // query row within the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t p_addr = smem_u32(smem + L::P_OFF);
-    float* red = reinterpret_cast<float*>(smem + L::RED_OFF);  // [3][2][128]
-    float m_run = -INFINITY, l_part = 0.f;
+    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int kb = 0; kb < nkv; ++kb) {
       const int st = kb & 1;
+      const uint32_t s_col = st ? L::TMEM_S1 : L::TMEM_S0;
       ok = mbar_wait(&s_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sv[64];
+      float sv[128];
       {
-        uint32_t raw[2][32];
+        uint32_t raw[4][32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tmem_ld_32x32b_x32_nw(lane_base + (st ? L::TMEM_S1 : L::TMEM_S0) + hf * 64 + c * 32,
-                                raw[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, raw[c]);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           reg_fence(raw[c]);
 #pragma unroll
           for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[c][i]);
@@ -227,55 +215,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (kb == qb) {  // diagonal block: keys after this query are masked
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (hf * 64 + i > r) sv[i] = -INFINITY;
+        for (int i = 0; i < 128; ++i)
+          if (i > r) sv[i] = -INFINITY;
       }
-      // row max over both halves (raw scores; the scale is positive): eight independent
-      // chains, then a tree
+      // row max (raw scores; the scale is positive): eight independent chains, then a tree
       float m8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) m8[k] = sv[k];
 #pragma unroll
-      for (int i = 8; i < 64; i += 8)
+      for (int i = 8; i < 128; i += 8)
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], sv[i + k]);
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      // exchange with the other half's warp (same rows) through a bounded mbarrier wait
-      red[(st * 2 + hf) * 128 + r] = mx;
-      mbar_arrive(&xchg[quarter * 2 + st]);
-      ok = mbar_wait(&xchg[quarter * 2 + st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      mx = fmaxf(mx, red[(st * 2 + (hf ^ 1)) * 128 + r]) * scale_log2;
-      const bool need = mx > m_run + kRescaleThreshold;  // identical in both halves
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;
+      const bool need = mx > m_run + kRescaleThreshold;
       const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
-      // eight partial sums (short dependency chains)
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
+      for (int i = 0; i < 128; ++i) {
         const float p = ex2_approx(fmaf(sv[i], scale_log2, -m_run));
         sv[i] = p;
         r8[i & 7] += p;
       }
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      l_part = l_part * alpha + rs;
+      l_run = l_run * alpha +
+              (((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7])));
       if (kb > 0) {
-        // PV of the previous block must be done before O is rescaled or P overwritten.
+        // PV of the previous block must be done before O is rescaled (waited every block,
+        // so the barrier's phases are followed one by one).
         ok = mbar_wait(pv_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {  // this half rescales its half of O
+        if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            const uint32_t ta = lane_base + L::TMEM_O + hf * (D / 2) + c * 32;
+            const uint32_t ta = lane_base + L::TMEM_O + c * 32;
             tmem_ld_32x32b_x32(ta, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
@@ -283,40 +261,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      // P (bf16) -> shared memory, K-major 128B-swizzled: this half owns one 64-key atom
+      // P (bf16 pairs) into the first 64 columns of this block's S buffer: this thread's own
+      // row, read completely above, so nothing else is overwritten.
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t addr = p_addr + hf * 16384 + r * 128 + ((j ^ (r & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(sv[j * 8 + 0], sv[j * 8 + 1]),
-                     pack_bf16x2(sv[j * 8 + 2], sv[j * 8 + 3]),
-                     pack_bf16x2(sv[j * 8 + 4], sv[j * 8 + 5]),
-                     pack_bf16x2(sv[j * 8 + 6], sv[j * 8 + 7]));
+      for (int c = 0; c < 2; ++c) {
+        float pw[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          pw[j] = __uint_as_float(pack_bf16x2(sv[c * 64 + 2 * j], sv[c * 64 + 2 * j + 1]));
+        tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[st]);
     }
-    // combine the two halves' row sums (own slot: the max slots may still be read)
     if (ok) {
-      red[(4 + hf) * 128 + r] = l_part;
-      mbar_arrive(&xsum[quarter]);
-      ok = mbar_wait(&xsum[quarter], 0, a.err, kErrTimeoutAttn, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    const float l_run = ok ? l_part + red[(4 + (hf ^ 1)) * 128 + r] : 1.f;
-    if (ok) {
-      ok = mbar_wait(pv_done, (nkv - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
+      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int qrow = qb * 128 + r;
         const float inv = 1.f / l_run;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                              ((long long)b * S + qrow) * H * D + (long long)n * D + hf * (D / 2);
+                              ((long long)b * S + qrow) * H * D + (long long)n * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + hf * (D / 2) + c * 32, o);
+          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
           if (qrow < S) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -329,15 +301,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
           }
         }
-        if (qrow < S && hf == 0)
-          a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
+        if (qrow < S) a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -964,7 +935,8 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
-  attn_fwd_tc_kernel<D><<<grid, kFwdThreads, L::BYTES, s>>>(tm, a, kLog2eF / sqrtf((float)D));
+  attn_fwd_tc_kernel<D><<<grid, kAttnFwdThreads, L::BYTES, s>>>(tm, a,
+                                                                kLog2eF / sqrtf((float)D));
   return cudaGetLastError();
 }
 
