@@ -33,6 +33,31 @@ KERNELS_PER_LAUNCH = {"gemm_tc": 1, "gemm_simt": 1, "attn_fwd": 1, "attn_bwd": 2
                       "ln_bwd": 2, "colsum": 1}
 
 
+GEMM_SOURCES = ("csrc/gemm_tc.cu", "csrc/mgt_device.cuh", "csrc/mgt_internal.h")
+GEMM_TRAFFIC = os.path.join(ROOT, "profiles", "gemm_tc_dram_h4096.md")
+
+
+def gemm_traffic(cfg_name):
+    """Average DRAM bytes per GEMM launch from the committed ncu summary, for the workload it
+    was captured on and only while the GEMM sources still hash to what was captured."""
+    import hashlib
+    if cfg_name != DEFAULT_WORKLOAD or not os.path.exists(GEMM_TRAFFIC):
+        return None, "no capture for this workload"
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "tensor_transformer_layer_megatron_b200", f), "rb") as fh:
+            h.update(fh.read())
+    vals = {}
+    for line in open(GEMM_TRAFFIC):
+        if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch", "sources_sha256"):
+            k, v = line.split(":", 1)
+            vals[k] = v.strip()
+    if vals.get("sources_sha256") != h.hexdigest():
+        return None, "GEMM sources changed since the ncu capture"
+    return int(vals["traffic_bytes_per_launch"]), "ncu dram__bytes_read.sum + dram__bytes_write.sum, " \
+        "average over the 12 GEMM launches of one step (profiles/gemm_tc_dram_h4096.md)"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -289,6 +314,7 @@ def run_mgt(args):
     prof = families
     fam = max(prof.items(), key=lambda kv: kv[1]["ms"]) if prof else (None, None)
     roof = None
+    traffic, traffic_src = gemm_traffic(cfg.name)
     if fam[0] is not None:
         name, st = fam
         if st["flops"] > 0:
@@ -298,7 +324,7 @@ def run_mgt(args):
                     "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
                     "peak_source": peak_src + " bf16_tflops_sustained (kernel timed inside "
                                    "the step)",
-                    "traffic": None,
+                    "traffic": traffic, "traffic_source": traffic_src,
                     "launches": st["launches"], "avg_launch_ms": round(st["ms"] / st["launches"], 4),
                     "share_of_step": round(st["ms"] / ms, 4)}
         else:
