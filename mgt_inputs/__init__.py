@@ -27,6 +27,11 @@ Activations: x, y [b, s, h]; qkv [b*s][p][3][H/p][d]; attention output [b*s][p][
 Variants (the trdm.cn page, section 3.3, lists them as launch flags): swiglu=1 replaces GeLU by
 SwiGLU, a = silu(gate) * up, fc1 producing gate and up (2f outputs); disable_bias_linear=1
 drops the biases of all four linear layers (the LayerNorm affine parameters stay).
+
+Sequence parallelism (sequence_parallel=1): the tensors outside the tensor-parallel regions
+(x, y, dx, dy and the LayerNorm / residual activations) are split along the sequence, shard t
+owning positions t*s/p .. (t+1)*s/p - 1 of every sequence, and laid out shard-major:
+[p][b][s/p][h] (to_sp / from_sp convert from / to [b, s, h]).
 """
 from __future__ import annotations
 
@@ -38,7 +43,7 @@ import torch
 
 __all__ = [
     "LayerConfig", "CONFIGS", "VARIANTS", "config_by_name", "make_inputs", "pack_params",
-    "unpack_params", "PARAM_NAMES", "BIAS_NAMES",
+    "unpack_params", "PARAM_NAMES", "BIAS_NAMES", "to_sp", "from_sp",
 ]
 
 PARAM_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
@@ -64,6 +69,7 @@ class LayerConfig:
     causal: int = 1
     swiglu: int = 0               # 1: a = silu(gate) * up instead of GeLU(u)
     disable_bias_linear: int = 0  # 1: no biases in the QKV, out-proj, fc1, fc2 layers
+    sequence_parallel: int = 0    # 1: x, y, dx, dy (and LN/residual regions) sequence-sharded
 
     @property
     def head_dim(self) -> int:
@@ -106,7 +112,23 @@ VARIANTS = (
     LayerConfig("tiny-h64-tp2-f32-swiglu", 64, 4, 256, 32, 2, 2, "f32", 1005, swiglu=1),
     LayerConfig("llama-h4096-tp2-bf16-swiglu-nobias", 4096, 32, 11008, 2048, 1, 2, "bf16", 1006,
                 swiglu=1, disable_bias_linear=1),
+    # sequence-parallel layer with two sequences per micro-batch, so that the shard-major layout
+    # is a real permutation of the token order
+    LayerConfig("gpt-h4096-tp2-sp-b2-bf16", 4096, 32, 11008, 1024, 2, 2, "bf16", 1007,
+                sequence_parallel=1),
 )
+
+
+def to_sp(cfg: LayerConfig, t: torch.Tensor) -> torch.Tensor:
+    """[b, s, h] -> the sequence-parallel layout [p][b][s/p][h] (a permutation of rows)."""
+    b, s, p = cfg.micro_batch, cfg.seq, cfg.tp_size
+    return t.reshape(b, p, s // p, -1).permute(1, 0, 2, 3).contiguous()
+
+
+def from_sp(cfg: LayerConfig, t: torch.Tensor) -> torch.Tensor:
+    """Inverse of to_sp: [p][b][s/p][h] -> [b, s, h]."""
+    b, s, p = cfg.micro_batch, cfg.seq, cfg.tp_size
+    return t.reshape(p, b, s // p, -1).permute(1, 0, 2, 3).reshape(b, s, -1).contiguous()
 
 
 def config_by_name(name: str) -> LayerConfig:

@@ -12,4 +12,5 @@ from .layer import (  # noqa: F401
     layer_norm, layer_norm_grad, gelu, gelu_grad, causal_softmax, attention_head_fwd,
     attention_head_bwd, attention_fwd, attention_bwd, layer_fwd, layer_bwd, layer_fwd_full,
     layer_bwd_full, gather_grads, sigmoid, silu, silu_grad, swiglu, swiglu_grad,
+    all_gather_seq, reduce_scatter_seq, layer_fwd_sp, layer_bwd_sp,
 )

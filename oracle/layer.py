@@ -20,6 +20,10 @@ Sources (web pages about Megatron-LM; they print no formulas, so each reading is
          kept and intermediates are recomputed in backward -- mathematically the identity.
   [VAR]  the trdm.cn page, section 3.3 (launch flags): --swiglu replaces GeLU by SwiGLU, and
          --disable-bias-linear removes the biases of the linear layers.
+  [SP]   "Megatron-LM：NVIDIA大模型训练框架" (second-brain-czx), sequence-parallel section: the
+         LayerNorm / dropout / residual regions are split along the sequence across the tensor-
+         parallel ranks, an all-gather precedes the column-parallel layer and a reduce-scatter
+         replaces the all-reduce after the row-parallel one.
 
 Readings where the pages are silent (each also listed in the design notes):
   * LayerNorm: biased variance (divide by h), eps inside the square root, affine gamma/beta.
@@ -35,6 +39,10 @@ Readings where the pages are silent (each also listed in the design notes):
     with silu(z) = z*sigmoid(z); fc2 is unchanged (input width f).
   * disable_bias_linear: b_qkv, b_o, b1, b2 are absent (not zero) and get no gradient; the
     LayerNorm affine parameters stay.
+  * sequence_parallel: shard t owns positions t*s/p .. (t+1)*s/p - 1 of every sequence of x, y,
+    dx, dy and of the LN/residual activations, held shard-major as [p][b][s/p][h]; in the
+    backward the all-gather's adjoint is a reduce-scatter and the reduce-scatter's an
+    all-gather, and the replicated LayerNorm parameters' gradients are summed over shards.
 """
 from __future__ import annotations
 
@@ -205,12 +213,15 @@ def _np(a):
 
 
 def layer_fwd(cfg, params, x):
-    """Forward of the layer on packed per-shard parameters (the TP path).
+    """Forward of the layer on packed per-shard parameters (the TP path); with
+    cfg.sequence_parallel, x and y are in the sequence-parallel layout (layer_fwd_sp).
 
     cfg: object with hidden, heads, ffn, seq, micro_batch, tp_size, ln_eps, gelu_tanh and
     optionally swiglu, disable_bias_linear.
     params: dict of packed arrays (layouts in the mgt_inputs docstring). x: [b, s, h].
     Returns (y [b, s, h], saved dict of every intermediate)."""
+    if getattr(cfg, "sequence_parallel", 0):
+        return layer_fwd_sp(cfg, params, x)
     h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
     b, s = cfg.micro_batch, cfg.seq
     T, d, hp = b * s, h // H, H // p
@@ -259,7 +270,10 @@ def layer_fwd(cfg, params, x):
 
 def layer_bwd(cfg, params, saved, dy):
     """Hand-written reverse of layer_fwd (packed TP path). Returns (dx [b,s,h], grads in the
-    packed parameter layout, intermediate grads)."""
+    packed parameter layout, intermediate grads); with cfg.sequence_parallel, dy and dx are in
+    the sequence-parallel layout (layer_bwd_sp)."""
+    if getattr(cfg, "sequence_parallel", 0):
+        return layer_bwd_sp(cfg, params, saved, dy)
     h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
     b, s = cfg.micro_batch, cfg.seq
     T, d, hp = b * s, h // H, H // p
@@ -319,6 +333,162 @@ def layer_bwd(cfg, params, saved, dy):
     dx = dh1 + d_ln1
     inter = dict(du=du, dln2=dln2, dh1=dh1, dO=dO, dqkv=dqkv, dln1=dln1)
     return dx.reshape(b, s, h), g, inter
+
+
+# ----------------------------------------------------------------------------- sequence parallel
+def all_gather_seq(xs, b, s, p):
+    """Sequence all-gather: the shards' pieces [p][b][s/p][n] -> the whole [b*s, n] in token
+    order, shard t's piece at positions t*s/p .. (t+1)*s/p - 1 of every sequence ([SP])."""
+    sp = s // p
+    full = np.empty((b, s, xs.shape[-1]))
+    for t in range(p):
+        full[:, t * sp:(t + 1) * sp] = xs[t]
+    return full.reshape(b * s, -1)
+
+
+def reduce_scatter_seq(parts, b, s, p):
+    """Sequence reduce-scatter: the p shards' partial sums over all tokens ([b*s, n] each) are
+    added, and shard t keeps its positions: -> [p][b][s/p][n] ([SP])."""
+    sp = s // p
+    total = np.zeros_like(parts[0])
+    for q in parts:
+        total = total + q
+    full = total.reshape(b, s, -1)
+    return np.stack([full[:, t * sp:(t + 1) * sp] for t in range(p)])
+
+
+def layer_fwd_sp(cfg, params, x_sp):
+    """The layer with sequence parallelism ([SP]): x_sp [p][b][s/p][h]. Each shard normalises
+    its own positions; the column-parallel layers run on the all-gathered LayerNorm output;
+    the row-parallel partial sums are reduce-scattered back to the sequence shards before the
+    bias and the residual. Returns (y [p][b][s/p][h], saved)."""
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    b, s = cfg.micro_batch, cfg.seq
+    T, d, hp, sp = b * s, h // H, H // p, s // p
+    sw, nb = _flags(cfg)
+    P = {k: _np(v) for k, v in params.items()}
+    bias = (lambda key: 0.0) if nb else (lambda key: P[key])  # noqa: E731
+    xs = _np(x_sp).reshape(p, b, sp, h)
+
+    def shard_ln(src, g, be):
+        out = np.empty_like(src)
+        xhat = np.empty_like(src)
+        rstd = np.empty((p, b * sp))
+        for t in range(p):
+            y_, _, r_, xh_ = layer_norm(src[t].reshape(b * sp, h), g, be, cfg.ln_eps)
+            out[t] = y_.reshape(b, sp, h)
+            xhat[t] = xh_.reshape(b, sp, h)
+            rstd[t] = r_
+        return out, xhat, rstd
+
+    ln1_s, xhat1, rstd1 = shard_ln(xs, P["ln1_g"], P["ln1_b"])
+    ln1 = all_gather_seq(ln1_s, b, s, p)
+    qkv = np.empty((T, p, 3, hp, d))
+    for t in range(p):
+        w_t = P["w_qkv"][t].reshape(3 * hp * d, h)
+        b_t = 0.0 if nb else P["b_qkv"][t].reshape(-1)
+        qkv[:, t] = (ln1 @ w_t.T + b_t).reshape(T, 3, hp, d)
+    O, lse = attention_fwd(qkv, b, s, H, p)
+    z = reduce_scatter_seq([O[:, t].reshape(T, h // p) @ P["w_o"][t].T for t in range(p)],
+                           b, s, p)
+    h1_s = xs + bias("b_o") + z
+    ln2_s, xhat2, rstd2 = shard_ln(h1_s, P["ln2_g"], P["ln2_b"])
+    ln2 = all_gather_seq(ln2_s, b, s, p)
+    if sw:
+        u = np.empty((T, p, 2, f // p))
+        for t in range(p):
+            for c in range(2):
+                u[:, t, c] = ln2 @ P["w1"][t, c].T + (0.0 if nb else P["b1"][t, c])
+        a = swiglu(u[:, :, 0], u[:, :, 1])
+    else:
+        u = np.empty((T, p, f // p))
+        for t in range(p):
+            u[:, t] = ln2 @ P["w1"][t].T + (0.0 if nb else P["b1"][t])
+        a = gelu(u, cfg.gelu_tanh)
+    z2 = reduce_scatter_seq([a[:, t] @ P["w2"][t].T for t in range(p)], b, s, p)
+    y_s = h1_s + bias("b2") + z2
+    # the layout-held activations in the shard-major row order ([p][b][s/p] flattened)
+    saved = dict(x=xs, ln1=ln1_s.reshape(T, h), ln1_full=ln1, xhat1=xhat1, rstd1=rstd1,
+                 qkv=qkv, O=O, lse=lse, h1=h1_s.reshape(T, h), ln2=ln2_s.reshape(T, h),
+                 ln2_full=ln2, xhat2=xhat2, rstd2=rstd2, u=u, a=a)
+    return y_s, saved
+
+
+def layer_bwd_sp(cfg, params, saved, dy_sp):
+    """Reverse of layer_fwd_sp: the all-gathers' adjoints are reduce-scatters and vice versa;
+    LayerNorm parameter gradients are summed over the shards. Returns (dx [p][b][s/p][h],
+    grads, intermediate grads with the sequence-parallel ones in the shard-major row order)."""
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    b, s = cfg.micro_batch, cfg.seq
+    T, d, hp, sp = b * s, h // H, H // p, s // p
+    sw, nb = _flags(cfg)
+    P = {k: _np(v) for k, v in params.items()}
+    dys = _np(dy_sp).reshape(p, b, sp, h)
+    g = {}
+    dy = all_gather_seq(dys, b, s, p)  # adjoint of the reduce-scatter after fc2
+    if not nb:
+        g["b2"] = dy.sum(axis=0)
+    g["w2"] = np.empty((p, h, f // p))
+    da = np.empty((T, p, f // p))
+    for t in range(p):
+        g["w2"][t] = dy.T @ saved["a"][:, t]
+        da[:, t] = dy @ P["w2"][t]
+    u = saved["u"]
+    if sw:
+        du = np.stack(swiglu_grad(u[:, :, 0], u[:, :, 1], da), axis=2)
+    else:
+        du = da * gelu_grad(u, cfg.gelu_tanh)
+    if not nb:
+        g["b1"] = du.sum(axis=0)
+    rows = (2 if sw else 1) * (f // p)
+    g["w1"] = np.empty((p,) + P["w1"].shape[1:])
+    parts = []
+    for t in range(p):
+        du_t = du[:, t].reshape(T, rows)
+        g["w1"][t] = (du_t.T @ saved["ln2_full"]).reshape(P["w1"].shape[1:])
+        parts.append(du_t @ P["w1"][t].reshape(rows, h))
+    dln2_s = reduce_scatter_seq(parts, b, s, p)  # adjoint of the all-gather before fc1
+
+    def shard_ln_grad(dsrc, xhat, rstd, gam):
+        dx_ = np.empty_like(dsrc)
+        dg, dbe = np.zeros(h), np.zeros(h)
+        for t in range(p):
+            a_, g_, b_ = layer_norm_grad(dsrc[t].reshape(b * sp, h),
+                                         xhat[t].reshape(b * sp, h), rstd[t], gam)
+            dx_[t] = a_.reshape(b, sp, h)
+            dg += g_
+            dbe += b_
+        return dx_, dg, dbe
+
+    d_ln, g["ln2_g"], g["ln2_b"] = shard_ln_grad(dln2_s, saved["xhat2"], saved["rstd2"],
+                                                 P["ln2_g"])
+    dh1_s = dys + d_ln
+    if not nb:
+        g["b_o"] = dh1_s.reshape(T, h).sum(axis=0)
+    dh1 = all_gather_seq(dh1_s, b, s, p)  # adjoint of the reduce-scatter after out-proj
+    g["w_o"] = np.empty((p, h, h // p))
+    dO = np.empty((T, p, hp, d))
+    for t in range(p):
+        g["w_o"][t] = dh1.T @ saved["O"][:, t].reshape(T, h // p)
+        dO[:, t] = (dh1 @ P["w_o"][t]).reshape(T, hp, d)
+    dqkv = attention_bwd(saved["qkv"], dO, b, s, H, p)
+    if not nb:
+        g["b_qkv"] = np.empty((p, 3, hp, d))
+    g["w_qkv"] = np.empty((p, 3, hp, d, h))
+    parts = []
+    for t in range(p):
+        dq_t = dqkv[:, t].reshape(T, 3 * hp * d)
+        if not nb:
+            g["b_qkv"][t] = dq_t.sum(axis=0).reshape(3, hp, d)
+        g["w_qkv"][t] = (dq_t.T @ saved["ln1_full"]).reshape(3, hp, d, h)
+        parts.append(dq_t @ P["w_qkv"][t].reshape(3 * hp * d, h))
+    dln1_s = reduce_scatter_seq(parts, b, s, p)  # adjoint of the all-gather before QKV
+    d_ln1, g["ln1_g"], g["ln1_b"] = shard_ln_grad(dln1_s, saved["xhat1"], saved["rstd1"],
+                                                  P["ln1_g"])
+    dx_s = dh1_s + d_ln1
+    inter = dict(du=du, dln2=dln2_s.reshape(T, h), dh1=dh1_s.reshape(T, h), dO=dO, dqkv=dqkv,
+                 dln1=dln1_s.reshape(T, h))
+    return dx_s, g, inter
 
 
 def layer_fwd_full(cfg, params, x):

@@ -312,3 +312,82 @@ def test_swiglu_packing_pairs_gate_and_up():
     back = unpack_params(cfg, pk)
     for k in back:
         assert torch.equal(back[k], t[k]), k
+
+
+# ------------------------------------------------------------------ sequence parallelism
+def test_sequence_collectives_are_adjoint():
+    """<reduce_scatter(u_0..u_p-1), v> = sum_t <u_t, all_gather(v)>: the reduce-scatter after a
+    row-parallel layer and the all-gather before a column-parallel one are each other's
+    adjoints, which is what the backward relies on; and gather(scatter-of-one) is the identity
+    on the shard layout."""
+    rng = np.random.default_rng(5)
+    b, s, p, n = 3, 12, 4, 5
+    parts = [rng.normal(size=(b * s, n)) for _ in range(p)]
+    v = rng.normal(size=(p, b, s // p, n))
+    lhs = float(np.sum(oracle.reduce_scatter_seq(parts, b, s, p) * v))
+    g = oracle.all_gather_seq(v, b, s, p)
+    rhs = float(sum(np.sum(u * g) for u in parts))
+    assert abs(lhs - rhs) <= 1e-12 * abs(rhs)
+    one = [g] + [np.zeros_like(g)] * (p - 1)
+    assert np.array_equal(oracle.reduce_scatter_seq(one, b, s, p), v)
+    # token (bb, pos) of the gathered tensor is shard pos // (s/p), row (bb, pos % (s/p))
+    for bb in range(b):
+        for pos in range(s):
+            assert np.array_equal(g[bb * s + pos], v[pos // (s // p), bb, pos % (s // p)])
+
+
+@pytest.mark.parametrize("variant", ["gelu", "swiglu_nobias"])
+def test_sequence_parallel_equals_plain_layer(variant):
+    """Sharding the LayerNorm/residual regions along the sequence (all-gather before QKV and
+    fc1, reduce-scatter after out-proj and fc2) computes the same layer: y and dx equal the
+    plain layer's in the shard-major layout, every gradient is equal."""
+    from mgt_inputs import to_sp
+    cfg = tiny(p=2, hidden=16, heads=4, ffn=32, seq=8, micro_batch=3, **VARIANT_KW[variant])
+    cfg_sp = cfg.replace(sequence_parallel=1)
+    t = make_inputs(cfg, nonzero_affine=True)
+    full = {k: v.double() for k, v in t.items()}
+    pk = pack_params(cfg, full)
+    y, sv = oracle.layer_fwd(cfg, pk, full["x"])
+    dx, g, inter = oracle.layer_bwd(cfg, pk, sv, full["dy"])
+    y_sp, sv_sp = oracle.layer_fwd(cfg_sp, pk, to_sp(cfg, full["x"]))
+    dx_sp, g_sp, inter_sp = oracle.layer_bwd(cfg_sp, pk, sv_sp, to_sp(cfg, full["dy"]))
+    assert rel(y_sp, to_sp(cfg, torch.tensor(y)).numpy()) < 1e-12
+    assert rel(dx_sp, to_sp(cfg, torch.tensor(dx)).numpy()) < 1e-12
+    assert set(g) == set(g_sp)
+    for k in g:
+        assert rel(g_sp[k], g[k]) < 1e-12, k
+    # token-parallel intermediates are unchanged; sequence-parallel ones are permuted
+    assert rel(inter_sp["dqkv"], inter["dqkv"]) < 1e-12
+    sp_rows = lambda a: to_sp(cfg, torch.tensor(a).reshape(cfg.micro_batch, cfg.seq, -1))  # noqa
+    assert rel(inter_sp["dh1"], sp_rows(inter["dh1"]).reshape(-1, cfg.hidden).numpy()) < 1e-12
+
+
+def test_sequence_parallel_finite_differences():
+    """The sequence-parallel backward against central differences on x (given in the
+    shard-major layout) and two parameters."""
+    from mgt_inputs import to_sp
+    cfg = tiny(p=2, hidden=8, heads=2, ffn=16, seq=6, micro_batch=2, sequence_parallel=1)
+    t = make_inputs(cfg.replace(sequence_parallel=0), nonzero_affine=True)
+    full = {k: v.double() for k, v in t.items()}
+    packed = {k: v.numpy() for k, v in pack_params(cfg, full).items()}
+    x = to_sp(cfg, full["x"]).numpy()
+    dy = to_sp(cfg, full["dy"]).numpy()
+    _, saved = oracle.layer_fwd(cfg, packed, x)
+    dx, g, _ = oracle.layer_bwd(cfg, packed, saved, dy)
+
+    def loss(pk, xx):
+        y, _ = oracle.layer_fwd(cfg, pk, xx)
+        return float(np.sum(y * dy))
+
+    rng = np.random.default_rng(13)
+    eps = 1e-5
+    for name in ("x", "ln1_g", "w1"):
+        vdir = rng.normal(size=(x if name == "x" else packed[name]).shape)
+        if name == "x":
+            lp, lm, an = loss(packed, x + eps * vdir), loss(packed, x - eps * vdir), np.sum(dx * vdir)
+        else:
+            pp = dict(packed); pp[name] = packed[name] + eps * vdir
+            pm = dict(packed); pm[name] = packed[name] - eps * vdir
+            lp, lm, an = loss(pp, x), loss(pm, x), np.sum(g[name] * vdir)
+        fd = (lp - lm) / (2 * eps)
+        assert abs(fd - an) <= 1e-6 * max(abs(an), 1e-3), (name, fd, an)
