@@ -216,7 +216,7 @@ def run_mgt(args):
     import torch
 
     import tensor_transformer_layer_megatron_b200 as mgt
-    from mgt_inputs import config_by_name, make_inputs, pack_params
+    from mgt_inputs import config_by_name, make_inputs, pack_params, to_sp
     from tensor_transformer_layer_megatron_b200.runner import LayerRun
 
     world, rank, local = dist_setup()
@@ -226,7 +226,10 @@ def run_mgt(args):
     t = make_inputs(cfg)
     packed = pack_params(cfg, t)
     layer = mgt.Layer.from_config(cfg)
-    run = LayerRun(layer, packed, t["x"], t["dy"], device=dev)
+    x, dy = t["x"], t["dy"]
+    if cfg.sequence_parallel:  # x, dy (and y, dx) in the shard-major sequence-parallel layout
+        x, dy = to_sp(cfg, x), to_sp(cfg, dy)
+    run = LayerRun(layer, packed, x, dy, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
@@ -366,6 +369,7 @@ def run_mgt(args):
                        "mlp": "swiglu" if cfg.swiglu else ("gelu-tanh" if cfg.gelu_tanh
                                                            else "gelu"),
                        "linear_bias": not cfg.disable_bias_linear,
+                       "sequence_parallel": bool(cfg.sequence_parallel),
                        "ffn": cfg.ffn, "seq_len": cfg.seq, "micro_batch": cfg.micro_batch,
                        "tp_size": cfg.tp_size, "tokens_per_gpu": cfg.tokens,
                        "global_batch": cfg.micro_batch * world,
@@ -482,13 +486,16 @@ def cpu_baseline(cfg, tokens):
     import torch
 
     import oracle
-    from mgt_inputs import make_inputs, pack_params
+    from mgt_inputs import make_inputs, pack_params, to_sp
     sub = cfg.replace(seq=tokens, micro_batch=1)
     t = make_inputs(sub)
     packed = pack_params(sub, t)
+    x, dy = t["x"], t["dy"]
+    if sub.sequence_parallel:
+        x, dy = to_sp(sub, x), to_sp(sub, dy)
     t0 = time.time()
-    _, saved = oracle.layer_fwd(sub, packed, t["x"])
-    oracle.layer_bwd(sub, packed, saved, t["dy"])
+    _, saved = oracle.layer_fwd(sub, packed, x)
+    oracle.layer_bwd(sub, packed, saved, dy)
     dt = time.time() - t0
     return {"value": round(tokens / dt, 3), "unit": "tokens/s",
             "cores": torch.get_num_threads(), "kind": "oracle",

@@ -14,6 +14,11 @@
  * Variants (launch flags on the trdm.cn page, section 3.3): swiglu = 1 gives the MLP
  * a = silu(gate) * up with [gate | up] = ln2 W1^T + b1 (fc1 has 2*ffn outputs, each shard its
  * own gate and up halves); disable_bias_linear = 1 drops b_qkv, b_o, b1 and b2.
+ * sequence_parallel = 1 (the second-brain-czx page's sequence parallelism): x, y, dx, dy and
+ * the LayerNorm / residual activations are split along the sequence, shard t owning
+ * positions t*s/p .. (t+1)*s/p - 1 of every sequence, laid out shard-major [p][b][s/p][h];
+ * the all-gather before QKV / fc1 and the reduce-scatter after out-proj / fc2 are realised
+ * as the row order in which the GEMMs read and write those tensors.
  *
  * Sources: the page "Megatron-LM 3D并行原理与万亿参数训练实战指南" (trdm.cn), section 2.1
  * (tensor parallelism: W_q/W_k/W_v split by output columns with x broadcast and no
@@ -36,7 +41,8 @@
  *         (swiglu: w1 [p][2][f/p][h], b1 [p][2][f/p]: shard t's gate rows, then its up rows)
  *         w2    [p][h][f/p]         b2    [h]
  *         ln1_g, ln1_b, ln2_g, ln2_b [h]
- *   - x, y, dx, dy: [b, s, h], tokens flattened as T = b*s with s fastest.
+ *   - x, y, dx, dy: [b, s, h], tokens flattened as T = b*s with s fastest (sequence_parallel:
+ *     [p][b][s/p][h]; so are the regions ln1, h1, ln2, their statistics, dln2, dh1, dln1).
  *   - dtype MGT_BF16: activations, weights and biases are bf16; LN gamma/beta are fp32.
  *     dtype MGT_F32: everything fp32. All gradients of parameters are written in fp32 and
  *     OVERWRITTEN (not accumulated); dx is in the activation dtype.
@@ -82,7 +88,8 @@ typedef enum mgt_dtype { MGT_F32 = 0, MGT_BF16 = 1 } mgt_dtype;
  * recompute_attn is accepted for either value -- attention probabilities are never stored,
  * the backward always recomputes them from the saved log-sum-exp. swiglu and
  * disable_bias_linear are 0 or 1 (a zero-filled tail keeps the GeLU layer with biases);
- * gelu_tanh has no effect with swiglu. */
+ * gelu_tanh has no effect with swiglu. sequence_parallel is 0 or 1 and needs seq % tp_size
+ * == 0 and, for bf16, (seq / tp_size) % 128 == 0. */
 typedef struct mgt_layer_config {
   int32_t hidden;
   int32_t heads;
@@ -97,6 +104,7 @@ typedef struct mgt_layer_config {
   int32_t gelu_tanh;      /* 0: exact erf GeLU; 1: tanh approximation */
   int32_t swiglu;         /* 0: GeLU MLP; 1: SwiGLU, a = silu(gate) * up (fc1: 2*ffn outputs) */
   int32_t disable_bias_linear; /* 1: no biases in QKV, out-proj, fc1, fc2 (b_* may be NULL) */
+  int32_t sequence_parallel;   /* 1: sequence-sharded [p][b][s/p][h] LN/residual regions */
 } mgt_layer_config;
 
 /* Parameters (device pointers, packed layouts above). With disable_bias_linear the four b_*

@@ -42,7 +42,8 @@ class _Config(ctypes.Structure):
                 ("tp_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("ln_eps", ctypes.c_float),
                 ("recompute_attn", ctypes.c_int32), ("gelu_tanh", ctypes.c_int32),
-                ("swiglu", ctypes.c_int32), ("disable_bias_linear", ctypes.c_int32)]
+                ("swiglu", ctypes.c_int32), ("disable_bias_linear", ctypes.c_int32),
+                ("sequence_parallel", ctypes.c_int32)]
 
 
 class _Params(ctypes.Structure):
@@ -120,11 +121,12 @@ class Layer:
     per-shard layouts of include/mgt_layer.h (see PARAM_ORDER)."""
 
     def __init__(self, hidden, heads, ffn, seq, micro_batch, tp_size=1, dtype="bf16",
-                 ln_eps=1e-5, gelu_tanh=0, causal=1, swiglu=0, disable_bias_linear=0):
+                 ln_eps=1e-5, gelu_tanh=0, causal=1, swiglu=0, disable_bias_linear=0,
+                 sequence_parallel=0):
         self.lib = load_library()
         self.cfg = _Config(hidden, heads, ffn, seq, micro_batch, tp_size,
                            1 if dtype == "bf16" else 0, causal, ln_eps, 1, gelu_tanh, swiglu,
-                           disable_bias_linear)
+                           disable_bias_linear, sequence_parallel)
         self.dtype = dtype
         self.has_bias = not disable_bias_linear
         h = ctypes.c_void_p()
@@ -134,10 +136,12 @@ class Layer:
     @classmethod
     def from_config(cls, cfg):
         """Build from any object with hidden, heads, ffn, seq, micro_batch, tp_size, dtype,
-        ln_eps, gelu_tanh (and optionally swiglu, disable_bias_linear) attributes."""
+        ln_eps, gelu_tanh (and optionally swiglu, disable_bias_linear, sequence_parallel)
+        attributes."""
         return cls(cfg.hidden, cfg.heads, cfg.ffn, cfg.seq, cfg.micro_batch, cfg.tp_size,
                    cfg.dtype, cfg.ln_eps, cfg.gelu_tanh, swiglu=getattr(cfg, "swiglu", 0),
-                   disable_bias_linear=getattr(cfg, "disable_bias_linear", 0))
+                   disable_bias_linear=getattr(cfg, "disable_bias_linear", 0),
+                   sequence_parallel=getattr(cfg, "sequence_parallel", 0))
 
     def __del__(self):
         h = getattr(self, "handle", None)

@@ -424,13 +424,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           uint8_t* a_dst = sA + stage * C::A_BYTES;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
+          // token coordinates go through the sequence-parallel row map where set
+          const int ka = args.a_sp ? seq_row(args, kt * BK) : kt * BK;
+          const int kb = args.b_sp ? seq_row(args, kt * BK) : kt * BK;
           if constexpr (!A_MN) {
-            tma_load_3d(&tmA, &full[stage], a_dst, kt * BK, kg, tc.mb * BM);
+            const int ma = args.a_sp ? seq_row(args, tc.mb * BM) : tc.mb * BM;
+            tma_load_3d(&tmA, &full[stage], a_dst, kt * BK, kg, ma);
           } else {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
               tma_load_3d(&tmA, &full[stage], a_dst + c * kChunkBytes, tc.mb * BM + c * 64,
-                          kt * BK, 0);
+                          ka, 0);
           }
           if constexpr (!B_MN) {
             tma_load_3d(&tmB, &full[stage], b_dst, kt * BK, tc.nb * BN, kg);
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < BN / 64; ++c)
               tma_load_3d(&tmB, &full[stage], b_dst + c * kChunkBytes, tc.nb * BN + c * 64,
-                          kt * BK, tc.ng);
+                          kb, tc.ng);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -540,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = tc.nb * BN + c * 32;
         if (row < args.M && n0 < args.Ng) {
           const int count = min(32, args.Ng - n0);
-          epilogue_chunk<EPI>(args, row, tc.ng * args.Ng + n0, count, v);
+          epilogue_chunk<EPI>(args, args.out_sp ? seq_row(args, row) : row,
+                              tc.ng * args.Ng + n0, count, v);
         }
       }
       if (k_iters > 0) {
@@ -681,11 +686,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kPairAB;
           uint8_t* b_dst = sB + stage * kPairAB;
+          // token coordinates go through the sequence-parallel row map where set
+          const int ka = args.a_sp ? seq_row(args, kt * BK) : kt * BK;
+          const int kb = args.b_sp ? seq_row(args, kt * BK) : kt * BK;
           if constexpr (!A_MN) {
-            tma_load_3d_pair(&tmA, fb, a_dst, kt * BK, kg, m0);
+            tma_load_3d_pair(&tmA, fb, a_dst, kt * BK, kg, args.a_sp ? seq_row(args, m0) : m0);
           } else {
-            tma_load_3d_pair(&tmA, fb, a_dst, m0, kt * BK, 0);
-            tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, kt * BK, 0);
+            tma_load_3d_pair(&tmA, fb, a_dst, m0, ka, 0);
+            tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, ka, 0);
           }
           if constexpr (kGlu) {
             // GLU tile: this CTA's half of B is the gate (rank 0) or up (rank 1) block of
@@ -694,8 +702,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           } else if constexpr (!B_MN) {
             tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, n0, kg);
           } else {
-            tma_load_3d_pair(&tmB, fb, b_dst, n0, kt * BK, tc.ng);
-            tma_load_3d_pair(&tmB, fb, b_dst + kChunkBytes, n0 + 64, kt * BK, tc.ng);
+            tma_load_3d_pair(&tmB, fb, b_dst, n0, kb, tc.ng);
+            tma_load_3d_pair(&tmB, fb, b_dst + kChunkBytes, n0 + 64, kb, tc.ng);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -830,10 +838,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n0 = tc.nb * BN + c * 32;
         const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
         const int col = tc.ng * args.Ng + n0;
+        // output (and residual) rows in the sequence-parallel layout where set; the 32 rows of
+        // a warp stay contiguous there (the shard length is a multiple of 128)
+        const int orow = args.out_sp ? seq_row(args, row) : row;
+        const int orow0 = args.out_sp ? seq_row(args, row0) : row0;
         // Whole chunks go through TMA; a chunk straddling N is written element by element
         // (the bulk store clips the inner dimension only at 16-byte granularity).
         if (n0 < args.Ng && (n0 + 32 > args.Ng || !staged)) {
-          if (row < args.M) epilogue_chunk<EPI>(args, row, col, min(32, args.Ng - n0), v);
+          if (row < args.M) epilogue_chunk<EPI>(args, orow, col, min(32, args.Ng - n0), v);
         } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
           uint8_t* buf = stage_out + (warp - 2) * kStageOut;
           if constexpr (EPI == kEpiStoreF32) {
@@ -845,7 +857,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           } else {
             uint32_t w[16], w2[16];
-            epi_values_bf16<EPI>(args, row, col, row < args.M, v, w, w2);
+            epi_values_bf16<EPI>(args, orow, col, row < args.M, v, w, w2);
             constexpr bool two = EPI == kEpiGelu || EPI == kEpiDSwiglu;
             if (lane == 0) bulk_wait_read0();
             __syncwarp();
@@ -865,12 +877,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) {
             if constexpr (EPI == kEpiDSwiglu) {  // tmC views dz as {Ng, M, 2*NG}
-              tma_store_3d(&tmC, buf, n0, row0, 2 * tc.ng);
-              tma_store_3d(&tmC, buf + 2048, n0, row0, 2 * tc.ng + 1);
+              tma_store_3d(&tmC, buf, n0, orow0, 2 * tc.ng);
+              tma_store_3d(&tmC, buf + 2048, n0, orow0, 2 * tc.ng + 1);
             } else {
-              tma_store_3d(&tmC, buf, col % args.out_ng, row0, col / args.out_ng);
+              tma_store_3d(&tmC, buf, col % args.out_ng, orow0, col / args.out_ng);
               if (EPI == kEpiGelu)
-                tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, row0, col / args.out_ng);
+                tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, orow0, col / args.out_ng);
             }
             bulk_commit();
           }

@@ -76,6 +76,11 @@ mgt_status validate(const mgt_layer_config* c) {
   if (!(c->ln_eps >= 0.f)) return MGT_EINVAL;
   if (c->swiglu != 0 && c->swiglu != 1) return MGT_EINVAL;
   if (c->disable_bias_linear != 0 && c->disable_bias_linear != 1) return MGT_EINVAL;
+  if (c->sequence_parallel != 0 && c->sequence_parallel != 1) return MGT_EINVAL;
+  if (c->sequence_parallel && c->seq % c->tp_size) return MGT_EINVAL;
+  // sequence-parallel tiles: 128 tokens of a GEMM tile stay inside one shard's positions
+  if (c->sequence_parallel && c->dtype == MGT_BF16 && (c->seq / c->tp_size) % 128)
+    return MGT_EUNSUPPORTED;
   if (c->causal != 1) return MGT_EUNSUPPORTED;
   const long long T = (long long)c->seq * c->micro_batch;
   if (T > (1LL << 30) || (long long)c->ffn * 3 > (1LL << 30) || (long long)c->hidden * 3 > (1LL << 30))
@@ -156,7 +161,17 @@ GemmArgs gemm_base(int M, int Ng, int NG, int Kg, int KG) {
 }
 
 // `site` names the call ("gemm_tc/fc1_fwd", ...): profiling groups launches by this name.
-cudaError_t gemm(mgt_layer* L, const char* site, const GemmArgs& a, cudaStream_t s) {
+// With sequence parallelism the row map of the shard-major layout is filled in here; the call
+// sites set which operand or output lives in it (a_sp, b_sp, out_sp).
+cudaError_t gemm(mgt_layer* L, const char* site, const GemmArgs& a_in, cudaStream_t s) {
+  GemmArgs a = a_in;
+  if (!L->cfg.sequence_parallel) {
+    a.a_sp = a.b_sp = a.out_sp = 0;
+  } else {
+    a.sp_seq = L->cfg.seq;
+    a.sp_len = L->cfg.seq / L->cfg.tp_size;
+    a.sp_b = L->cfg.micro_batch;
+  }
   // A SwiGLU fc1 tile computes a gate and an up product per output.
   const double flops = 2.0 * a.M * (double)a.Ng * a.NG * (double)a.Kg * a.KG *
                        (a.epi == kEpiSwiglu ? 2 : 1);
@@ -307,6 +322,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, 3 * h, 1, h, 1);
     a.A = ln1; a.lda = h; a.B = P->w_qkv; a.ldb = h;
     a.epi = kEpiBf16; a.out = qkv; a.ldc = 3 * h; a.bias = b_qkv; a.err = err;
+    a.a_sp = 1;  // sequence parallel: the all-gather of ln1 is this row map
     MGT_TRY(gemm(L, "gemm_tc/qkv_fwd", a, s));
   }
   // 3. causal attention per head (each shard's heads are local)
@@ -322,6 +338,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, h / p, p);
     a.A = O; a.lda = h; a.B = P->w_o; a.ldb = h / p; a.b_kgs = (long long)h * (h / p);
     a.epi = kEpiBf16; a.out = h1; a.ldc = h; a.bias = b_o; a.res = x; a.ldr = h; a.err = err;
+    a.out_sp = 1;  // sequence parallel: the reduce-scatter of the shard sum is this row map
     MGT_TRY(gemm(L, "gemm_tc/outproj_fwd", a, s));
   }
   // 5. LN2
@@ -336,13 +353,13 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, f / p, p, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
     a.epi = kEpiSwiglu; a.out = act; a.ldc = f; a.out2 = gd; a.ldc2 = 2LL * f; a.bias = b1;
-    a.err = err;
+    a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   } else {
     GemmArgs a = gemm_base(T, f, 1, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
     a.epi = kEpiGelu; a.out = act; a.out2 = gd; a.ldc = f; a.bias = b1;
-    a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
+    a.gelu_tanh = L->cfg.gelu_tanh; a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   }
   // 7. fc2, row-parallel with shard sum, + b2, + residual h1
@@ -350,6 +367,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, f / p, p);
     a.A = act; a.lda = f; a.B = P->w2; a.ldb = f / p; a.b_kgs = (long long)h * (f / p);
     a.epi = kEpiBf16; a.out = y; a.ldc = h; a.bias = b2; a.res = h1; a.ldr = h; a.err = err;
+    a.out_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc2_fwd", a, s));
   }
   return MGT_OK;
@@ -412,13 +430,14 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.b_ngs = (long long)h * (f / p);
     a.epi = sw ? kEpiDSwiglu : kEpiDGelu; a.out = du; a.ldc = f1; a.aux = gd; a.ld_aux = f1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
+    a.a_sp = 1;  // dy is sequence-parallel: its all-gather (adjoint of the reduce-scatter)
     MGT_TRY(gemm(L, "gemm_tc/fc2_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(h, f, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dy; a.lda = h; a.B = act; a.ldb = f;
     a.epi = kEpiStoreF32; a.out = G->w2; a.ldc = f / p; a.out_ng = f / p;
-    a.out_gs = (long long)h * (f / p); a.err = err;
+    a.out_gs = (long long)h * (f / p); a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, s));
   }
   // B3. fc1: db1, dgrad (sum over shards = K loop over all fc1 outputs), wgrad
@@ -427,12 +446,13 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h, 1, f1, 1);
     a.b_mn = 1; a.A = du; a.lda = f1; a.B = P->w1; a.ldb = h;
     a.epi = kEpiBf16; a.out = dln2; a.ldc = h; a.err = err;
+    a.out_sp = 1;  // the reduce-scatter of dln2 (adjoint of the all-gather of ln2)
     MGT_TRY(gemm(L, "gemm_tc/fc1_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(f1, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f1; a.B = ln2; a.ldb = h;
-    a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err;
+    a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err; a.b_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, s));
   }
   // B4. LN2 backward + residual gradient dy -> dh1
@@ -447,12 +467,12 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, h / p, p, h, 1);
     a.b_mn = 1; a.A = dh1; a.lda = h; a.B = P->w_o; a.ldb = h / p;
     a.b_ngs = (long long)h * (h / p);
-    a.epi = kEpiBf16; a.out = dO; a.ldc = h; a.err = err;
+    a.epi = kEpiBf16; a.out = dO; a.ldc = h; a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/outproj_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(h, h, 1, T, 1);
-    a.a_mn = 1; a.b_mn = 1; a.A = dh1; a.lda = h; a.B = O; a.ldb = h;
+    a.a_mn = 1; a.b_mn = 1; a.A = dh1; a.lda = h; a.B = O; a.ldb = h; a.a_sp = 1;
     a.epi = kEpiStoreF32; a.out = G->w_o; a.ldc = h / p; a.out_ng = h / p;
     a.out_gs = (long long)h * (h / p); a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/outproj_wgrad", a, s));
@@ -469,13 +489,13 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   {
     GemmArgs a = gemm_base(T, h, 1, 3 * h, 1);
     a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = P->w_qkv; a.ldb = h;
-    a.epi = kEpiBf16; a.out = dln1; a.ldc = h; a.err = err;
+    a.epi = kEpiBf16; a.out = dln1; a.ldc = h; a.err = err; a.out_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/qkv_dgrad", a, s));
   }
   {
     GemmArgs a = gemm_base(3 * h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = ln1; a.ldb = h;
-    a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err;
+    a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err; a.b_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/qkv_wgrad", a, s));
   }
   // B8. LN1 backward + residual gradient dh1 -> dx

@@ -527,11 +527,14 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
   const float* B = reinterpret_cast<const float*>(a.B);
   float* out = reinterpret_cast<float*>(a.out);
   const float* bias = reinterpret_cast<const float*>(a.bias);
+  // token indices of operands / outputs held in the sequence-parallel layout
+  const int ma = a.a_sp ? seq_row(a, m) : m;
+  const int mo = a.out_sp ? seq_row(a, m) : m;
   if (a.epi == kEpiSwiglu) {  // gate row ng*2Ng + n and up row + Ng of K-major B
     const long long rg = 2LL * ng * a.Ng + n, ru = rg + a.Ng;
     float g = 0.f, u = 0.f;
     for (int k = 0; k < a.Kg; ++k) {
-      const float av = A[(long long)m * a.lda + k];
+      const float av = A[(long long)ma * a.lda + k];
       g = fmaf(av, B[rg * a.ldb + k], g);
       u = fmaf(av, B[ru * a.ldb + k], u);
     }
@@ -551,20 +554,22 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
   for (int kg = 0; kg < a.KG; ++kg) {
     for (int kk = 0; kk < a.Kg; ++kk) {
       const long long k = (long long)kg * a.Kg + kk;
-      const float av = a.a_mn ? A[k * a.lda + m] : A[(long long)m * a.lda + k];
-      const float bv = a.b_mn ? B[(long long)ng * a.b_ngs + k * a.ldb + n]
+      const long long kt_a = a.a_sp ? seq_row(a, (int)k) : k;  // token K of an MN-major A
+      const long long kt_b = a.b_sp ? seq_row(a, (int)k) : k;  // token K of an MN-major B
+      const float av = a.a_mn ? A[kt_a * a.lda + m] : A[(long long)ma * a.lda + k];
+      const float bv = a.b_mn ? B[(long long)ng * a.b_ngs + kt_b * a.ldb + n]
                               : B[(long long)kg * a.b_kgs + (long long)n * a.ldb + kk];
       acc = fmaf(av, bv, acc);
     }
   }
   const int col = ng * a.Ng + n;
-  const long long off = (long long)(col / a.out_ng) * a.out_gs + (long long)m * a.ldc +
+  const long long off = (long long)(col / a.out_ng) * a.out_gs + (long long)mo * a.ldc +
                         col % a.out_ng;
   switch (a.epi) {
     case kEpiStoreF32: out[off] = acc; break;
     case kEpiBf16: {
       if (bias) acc += bias[col];
-      if (a.res) acc += reinterpret_cast<const float*>(a.res)[(long long)m * a.ldr + col];
+      if (a.res) acc += reinterpret_cast<const float*>(a.res)[(long long)mo * a.ldr + col];
       out[off] = acc;
       break;
     }

@@ -58,7 +58,21 @@ struct GemmArgs {
   const void* aux; long long ld_aux;    // kEpiDGelu: GeLU'(u)[m*ld_aux + col]
   int gelu_tanh;
   int* err;                             // device status word
+  // Sequence-parallel layout: token m (= batch * seq + position) of an operand or output held
+  // shard-major lives at row seq_row(m) (see below). a_sp / b_sp remap A's / B's token
+  // coordinate (M of a K-major A; K of an MN-major A or B), out_sp the output rows and the
+  // residual rows read with them. Needs the shard length a multiple of 128.
+  int a_sp, b_sp, out_sp;
+  int sp_seq, sp_len, sp_b;             // sequence length, positions per shard, micro-batch
 };
+
+// Row of token m in the sequence-parallel layout [p][b][s/p]: shard t = pos / (s/p) owns
+// positions t*s/p .. of every sequence.
+__host__ __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
+  const int bb = m / a.sp_seq, pos = m - bb * a.sp_seq;
+  const int t = pos / a.sp_len;
+  return (t * a.sp_b + bb) * a.sp_len + (pos - t * a.sp_len);
+}
 
 // 3-D bf16 tensor map (128-byte swizzle, zero fill out of bounds); strides in elements.
 bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import tensor_transformer_layer_megatron_b200 as mgt
-from mgt_inputs import make_inputs, pack_params
+from mgt_inputs import make_inputs, pack_params, to_sp
 from tensor_transformer_layer_megatron_b200.runner import LayerRun
 
 GRAD_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o", "ln2_g", "ln2_b", "w1", "b1",
@@ -31,10 +31,19 @@ def to_np(t):
     return t.detach().float().cpu().double().numpy()
 
 
+def layer_io(cfg, t):
+    """x and dy as the layer takes them: [b, s, h], or the shard-major sequence-parallel
+    layout [p][b][s/p][h]."""
+    if getattr(cfg, "sequence_parallel", 0):
+        return to_sp(cfg, t["x"]), to_sp(cfg, t["dy"])
+    return t["x"], t["dy"]
+
+
 def run_gpu(cfg, t):
     packed = pack_params(cfg, t)
     layer = mgt.Layer.from_config(cfg)
-    run = LayerRun(layer, packed, t["x"], t["dy"])
+    x, dy = layer_io(cfg, t)
+    run = LayerRun(layer, packed, x, dy)
     run.step()
     run.check()
     torch.cuda.synchronize()
@@ -74,8 +83,9 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
     intermediate). Returns the dict of relative errors."""
     t = make_inputs(cfg, nonzero_affine=nonzero_affine)
     packed, layer, run = run_gpu(cfg, t)
-    y_ref, saved = oracle.layer_fwd(cfg, packed, t["x"])
-    dx_ref, g_ref, inter = oracle.layer_bwd(cfg, packed, saved, t["dy"])
+    x, dy = layer_io(cfg, t)
+    y_ref, saved = oracle.layer_fwd(cfg, packed, x)
+    dx_ref, g_ref, inter = oracle.layer_bwd(cfg, packed, saved, dy)
     errs = {"y": rel_err(to_np(run.y), y_ref), "dx": rel_err(to_np(run.dx), dx_ref)}
     # a layer without linear biases has no bias gradients on either side
     assert set(run.grads) == set(g_ref), (sorted(run.grads), sorted(g_ref))

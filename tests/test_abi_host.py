@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def _init(**kw):
     base = dict(hidden=64, heads=4, ffn=256, seq=32, micro_batch=2, tp_size=2, dtype=0,
                 causal=1, ln_eps=1e-5, recompute_attn=1, gelu_tanh=0, swiglu=0,
-                disable_bias_linear=0)
+                disable_bias_linear=0, sequence_parallel=0)
     base.update(kw)
     lib = mgt.load_library()
     cfg = mgt._Config(*[base[f] for f, _ in mgt._Config._fields_])
@@ -65,6 +65,9 @@ def test_golden_tp_divisibility():
     (dict(dtype=1, hidden=128, heads=2, tp_size=2, ffn=200), 2),      # f/p = 100, not a multiple of 64
     (dict(hidden=512, heads=4), 2),       # fp32 head_dim 128 > 64
     (dict(swiglu=2), 1), (dict(disable_bias_linear=-1), 1),           # flags are 0 or 1
+    (dict(sequence_parallel=3), 1),
+    (dict(sequence_parallel=1, seq=33), 1),                           # s % p
+    (dict(sequence_parallel=1, dtype=1, hidden=256, heads=2, ffn=512, seq=192), 2),  # s/p % 128
 ])
 def test_init_rejects(kw, code):
     assert _init(**kw) == code

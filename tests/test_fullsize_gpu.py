@@ -1,6 +1,7 @@
 """Parity at the full workload sizes, in the launch configuration the benchmark times.
 
-h=1024 and h=4096 layers (and the h=4096 layer in its SwiGLU, no-bias form): the whole layer
+h=1024 and h=4096 layers (and the h=4096 layer in its SwiGLU, no-bias form and with sequence
+parallelism over two sequences): the whole layer
 (y, dx, every parameter gradient and every saved or workspace intermediate) against the fp64
 oracle on the benchmark's own seeded inputs.
 
@@ -31,7 +32,8 @@ def _log(name, errs):
 
 
 @pytest.mark.parametrize("name", ["gpt-h1024-bf16", "gpt-h4096-tp2-bf16",
-                                  "llama-h4096-tp2-bf16-swiglu-nobias"])
+                                  "llama-h4096-tp2-bf16-swiglu-nobias",
+                                  "gpt-h4096-tp2-sp-b2-bf16"])
 def test_full_layer_parity_at_full_size(name):
     cfg = config_by_name(name)
     errs = full_parity(cfg, nonzero_affine=False, intermediates=True)

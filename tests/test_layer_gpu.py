@@ -39,6 +39,12 @@ VARIANTS = [
           micro_batch=3, tp_size=4, swiglu=1, disable_bias_linear=1),
     small("h256-d64-p1-nobias-s64", hidden=256, heads=4, ffn=768, seq=64, micro_batch=1,
           tp_size=1, disable_bias_linear=1),
+    # sequence parallelism: shard-major [p][b][s/p][h] LN/residual regions (a real permutation
+    # of the tokens with b > 1)
+    small("h256-d128-p2-sp-s256-b2", hidden=256, heads=2, ffn=512, seq=256, micro_batch=2,
+          tp_size=2, sequence_parallel=1),
+    small("h512-d64-p4-sp-swiglu-s512-b3", hidden=512, heads=8, ffn=1536, seq=512,
+          micro_batch=3, tp_size=4, sequence_parallel=1, swiglu=1),
 ]
 
 
@@ -68,6 +74,14 @@ def test_layer_bf16_variants(cfg):
 @pytest.mark.parametrize("affine", [False, True])
 def test_layer_f32_tiny_swiglu(affine, nobias):
     cfg = config_by_name("tiny-h64-tp2-f32-swiglu").replace(disable_bias_linear=nobias)
+    errs = full_parity(cfg, nonzero_affine=affine)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("affine", [False, True])
+def test_layer_f32_tiny_sequence_parallel(affine):
+    cfg = config_by_name("tiny-h64-tp2-f32").replace(sequence_parallel=1)
     errs = full_parity(cfg, nonzero_affine=affine)
     bad = {k: v for k, v in errs.items() if v > tol(cfg)}
     assert not bad, (bad, errs)
