@@ -14,3 +14,4 @@ from .layer import (  # noqa: F401
     layer_bwd_full, gather_grads, sigmoid, silu, silu_grad, swiglu, swiglu_grad,
     all_gather_seq, reduce_scatter_seq, layer_fwd_sp, layer_bwd_sp,
 )
+from .fp8 import E4M3_MAX, e4m3_round, quantize_e4m3, gemm_fp8  # noqa: F401
