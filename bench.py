@@ -401,6 +401,65 @@ def run_mgt(args):
         torch.distributed.destroy_process_group()
 
 
+def run_gemm_fp8(args):
+    """The FP8 (e4m3) GEMM next to the bf16 one on the h=4096 layer's forward GEMM shapes (fp32
+    outputs for both): operands quantised once on the device, then K timed launches of each
+    GEMM between CUDA events. Prints one JSON line (not the layer-step benchmark)."""
+    import torch
+
+    import tensor_transformer_layer_megatron_b200 as mgt
+    dev = torch.device("cuda", 0)
+    T, h, f = 2048, 4096, 11008
+    shapes = {"qkv_fwd": (T, 3 * h, h), "outproj_fwd": (T, h, h), "fc1_fwd": (T, f, h),
+              "fc2_fwd": (T, h, f)}
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(5)
+    res, tot = {}, {"fp8": [0.0, 0.0], "bf16": [0.0, 0.0]}
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, (M, N, K) in shapes.items():
+        a = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        b = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        qa = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        qb = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        sa = torch.zeros(2, device=dev)
+        sb = torch.zeros(2, device=dev)
+        mgt.fp8_quantize(a, qa, sa)
+        mgt.fp8_quantize(b, qb, sb)
+        c = torch.empty(M, N, device=dev)
+        runs = {"fp8": lambda: mgt.gemm_fp8(qa, qb, sa, sb, c, M, N, K, K, K, N, st),
+                "bf16": lambda: mgt.gemm_bf16(a, b, c, M, N, K, 0, 0, K, K, N, st)}
+        res[name] = {}
+        for kind, fn in runs.items():
+            for _ in range(max(args.warmup, 3)):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            fl = 2.0 * M * N * K
+            res[name][kind] = {"us": round(ms * 1e3, 1), "tflops": round(fl / ms / 1e9, 1)}
+            tot[kind][0] += fl
+            tot[kind][1] += ms
+    clk = clocks.stop()
+    if int(st.item()) != 0:
+        raise RuntimeError("device status %d" % int(st.item()))
+    fp8 = tot["fp8"][0] / tot["fp8"][1] / 1e9
+    bf16 = tot["bf16"][0] / tot["bf16"][1] / 1e9
+    print(json.dumps({
+        "metric": "FP8 (e4m3, per-tensor scaled) GEMM TFLOP/s on the h=4096 forward GEMM shapes",
+        "value": round(fp8, 1), "unit": "TFLOP/s", "higher_is_better": True,
+        "bf16_same_shapes_tflops": round(bf16, 1), "speedup_vs_bf16": round(fp8 / bf16, 3),
+        "steps": args.steps, "warmup": args.warmup, "dtype": "e4m3 x e4m3 -> f32",
+        "data": "synthetic", "per_shape": res, "clocks": clk,
+        "timing": "CUDA events around K back-to-back launches per shape; operands (<= 230 MB) "
+                  "partly L2-resident"}), flush=True)
+
+
 def run_torch(args):
     """Context comparator: the same layer in eager PyTorch on the GPU (cuBLAS GEMMs through
     F.linear on the full unsharded weights, which is what logical TP on one GPU computes;
@@ -537,6 +596,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mgt", choices=["mgt", "reference", "torch"])
+    ap.add_argument("--gemm-fp8", action="store_true",
+                    help="time the FP8 GEMM against the bf16 one on the forward GEMM shapes")
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -547,7 +608,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.gemm_fp8:
+        run_gemm_fp8(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.impl == "torch":
         run_torch(args)

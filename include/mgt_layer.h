@@ -204,6 +204,30 @@ mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major,
                          int32_t b_mn_major, const void* A, int64_t lda, const void* B,
                          int64_t ldb, float* C, int64_t ldc, int32_t* status, void* stream);
 
+/* FP8 (e4m3) with per-tensor scaling. The page "把大模型训练“摁”到规模化：NVIDIA Megatron-LM /
+ * Megatron Core 上手与理解" (section 0) lists FP8 among Megatron Core's mixed precisions and the
+ * trdm.cn page's inference section enables it (--enable-fp8); neither gives a recipe. Here:
+ *
+ * mgt_fp8_quantize: amax = max |x| over n elements of x (dtype MGT_F32 or MGT_BF16), then
+ *   q[i] = e4m3(x[i] * s), s = 448 / amax (1 if amax == 0), rounded to nearest even and
+ *   saturated to +-448 (the largest finite e4m3); scales (device, 2 floats) receives
+ *   {amax, amax / 448} (the second, 1 if amax == 0, is the dequantisation factor). q: n bytes,
+ *   2-byte aligned. Asynchronous on `stream`; MGT_EINVAL for n < 1 or null pointers.
+ *
+ * mgt_gemm_fp8: C[m, n] = (sum_k A[m*lda + k] * B[n*ldb + k]) * a_scales[1] * b_scales[1]
+ *   with A [M][K], B [N][K] e4m3 bytes (both K-major), products accumulated in fp32 on the
+ *   tensor cores (tcgen05 kind::f8f6f4); C row-major with leading dimension ldc in c_dtype
+ *   (MGT_F32 or MGT_BF16, round to nearest even). K, lda, ldb multiples of 16; ldc a
+ *   multiple of 4 (f32) or 8 (bf16); pointers 16-byte aligned; `status` an int32 device word
+ *   (zeroed by the caller) that receives timeout codes. MGT_EUNSUPPORTED when the alignment
+ *   rules fail. */
+mgt_status mgt_fp8_quantize(int32_t dtype, int64_t n, const void* x, uint8_t* q, float* scales,
+                            void* stream);
+mgt_status mgt_gemm_fp8(int32_t M, int32_t N, int32_t K, const uint8_t* A, int64_t lda,
+                        const uint8_t* B, int64_t ldb, const float* a_scales,
+                        const float* b_scales, void* C, int32_t c_dtype, int64_t ldc,
+                        int32_t* status, void* stream);
+
 /* Failure-path probe (diagnostics and tests; no counterpart in the pages). Launches one thread
  * that waits on a device barrier nothing ever arrives on, through the same bounded wait that
  * every pipelined kernel of this library uses; after limit_ns (0 < limit_ns <= 1e9) it gives

@@ -86,13 +86,17 @@ def load_library():
                                   ctypes.c_int64, vp, ctypes.c_int64, vp, vp]
     lib.mgt_layernorm_bwd_noalloc.argtypes = [i32, ctypes.c_int64, i32, vp, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp]
+    lib.mgt_fp8_quantize.argtypes = [i32, ctypes.c_int64, vp, vp, vp, vp]
+    lib.mgt_gemm_fp8.argtypes = [i32, i32, i32, vp, ctypes.c_int64, vp, ctypes.c_int64, vp, vp,
+                                 vp, i32, ctypes.c_int64, vp, vp]
     lib.mgt_debug_bounded_wait.argtypes = [ctypes.c_int64, vp, vp]
     lib.mgt_layer_status_word.argtypes = [vp, vp, ctypes.POINTER(vp)]
     lib.mgt_debug_bounded_wait.restype = ctypes.c_int
     lib.mgt_layer_status_word.restype = ctypes.c_int
     for name in ("mgt_layer_init", "mgt_layer_sizes", "mgt_layer_region", "mgt_layer_fwd",
                  "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
-                 "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc"):
+                 "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc",
+                 "mgt_fp8_quantize", "mgt_gemm_fp8"):
         getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -244,6 +248,32 @@ def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):
     lib = load_library()
     _check(lib.mgt_gemm_bf16(M, N, K, a_mn, b_mn, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
                              _ptr(status), _stream_handle(stream)), "mgt_gemm_bf16")
+
+
+def fp8_quantize(x, q, scales, stream=None):
+    """Per-tensor e4m3 quantisation (see mgt_fp8_quantize): x fp32 or bf16, q uint8 with
+    x.numel() bytes, scales a 2-float device tensor receiving {amax, amax / 448}."""
+    import torch
+    if x.dtype not in (torch.float32, torch.bfloat16) or q.dtype != torch.uint8 or \
+            scales.dtype != torch.float32 or scales.numel() < 2 or q.numel() < x.numel():
+        raise TypeError("fp8_quantize takes fp32/bf16 x, uint8 q, 2 fp32 scales")
+    lib = load_library()
+    _check(lib.mgt_fp8_quantize(1 if x.dtype == torch.bfloat16 else 0, x.numel(), _ptr(x),
+                                _ptr(q), _ptr(scales), _stream_handle(stream)),
+           "mgt_fp8_quantize")
+
+
+def gemm_fp8(A, B, a_scales, b_scales, C, M, N, K, lda, ldb, ldc, status, stream=None):
+    """C = (A B^T) * a_scales[1] * b_scales[1] with e4m3 bytes A [M][K], B [N][K] (see
+    mgt_gemm_fp8); C fp32 or bf16."""
+    import torch
+    if A.dtype != torch.uint8 or B.dtype != torch.uint8 or \
+            C.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("gemm_fp8 takes uint8 A, B and an fp32/bf16 C")
+    lib = load_library()
+    _check(lib.mgt_gemm_fp8(M, N, K, _ptr(A), lda, _ptr(B), ldb, _ptr(a_scales),
+                            _ptr(b_scales), _ptr(C), 0 if C.dtype == torch.float32 else 1, ldc,
+                            _ptr(status), _stream_handle(stream)), "mgt_gemm_fp8")
 
 
 def layernorm_bwd_noalloc(dtype, rows, h, dy, dres, x, gamma, mean, rstd, dx, dgamma, dbeta,

@@ -596,7 +596,7 @@ constexpr int pair_smem(int epi) {
 static_assert(pair_smem(kEpiStoreF32) <= 232448, "shared memory per CTA");
 static_assert(pair_smem(kEpiSwiglu) <= 232448, "shared memory per CTA");
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
@@ -614,6 +614,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   constexpr int STAGES = pair_stages(EPI);
   constexpr int kStageOut = stage_out_bytes(EPI);
   constexpr bool kGlu = EPI == kEpiSwiglu;
+  // K elements per stage: one 128-byte swizzle row per operand row (64 bf16 or 128 e4m3);
+  // either way a stage holds the same bytes and takes four MMAs of 32 bytes of K each.
+  constexpr int KE = F8 ? 128 : BK;
+  static_assert(!F8 || (!A_MN && !B_MN && !kGlu), "FP8 operands are K-major");
   const uint32_t b_bytes = (uint32_t)(BN / 2) * BK * 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -634,7 +638,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  const int kt_per_group = (args.Kg + BK - 1) / BK;
+  const int kt_per_group = (args.Kg + KE - 1) / KE;
   const int k_iters = args.KG * kt_per_group;
   const int num_tiles = args.NG * num_m2 * num_n;
 
@@ -690,7 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int ka = args.a_sp ? seq_row(args, kt * BK) : kt * BK;
           const int kb = args.b_sp ? seq_row(args, kt * BK) : kt * BK;
           if constexpr (!A_MN) {
-            tma_load_3d_pair(&tmA, fb, a_dst, kt * BK, kg, args.a_sp ? seq_row(args, m0) : m0);
+            tma_load_3d_pair(&tmA, fb, a_dst, kt * KE, kg, args.a_sp ? seq_row(args, m0) : m0);
           } else {
             tma_load_3d_pair(&tmA, fb, a_dst, m0, ka, 0);
             tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, ka, 0);
@@ -700,7 +704,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // group ng, rows nb*BN/2 ..; the map views B as {K, Ng, 2*NG}.
             tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, tc.nb * (BN / 2), 2 * tc.ng + rank);
           } else if constexpr (!B_MN) {
-            tma_load_3d_pair(&tmB, fb, b_dst, kt * BK, n0, kg);
+            tma_load_3d_pair(&tmB, fb, b_dst, kt * KE, n0, kg);
           } else {
             tma_load_3d_pair(&tmB, fb, b_dst, n0, kb, tc.ng);
             tma_load_3d_pair(&tmB, fb, b_dst + kChunkBytes, n0 + 64, kb, tc.ng);
@@ -728,7 +732,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (leader && warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer (leader only)
-    const uint32_t idesc = idesc_bf16_f32(256, BN, A_MN, B_MN);
+    const uint32_t idesc = F8 ? idesc_e4m3_f32(256, BN) : idesc_bf16_f32(256, BN, A_MN, B_MN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -755,7 +759,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                    : smem_desc_sw128(a_addr + k * 32, 16, 1024);
           const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * 2048, kChunkBytes, 1024)
                                    : smem_desc_sw128(b_addr + k * 32, 16, 1024);
-          tc_mma_f16_pair(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+          if constexpr (F8)
+            tc_mma_f8_pair(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+          else
+            tc_mma_f16_pair(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit_pair_mc(&empty[stage], 0x3);  // frees the slot in both CTAs
         if (++stage == STAGES) {
@@ -781,6 +788,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int c_begin = ((warp - 2) >> 2) ? half : 0;
     const int c_end = ((warp - 2) >> 2) ? nch : half;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    // FP8: dequantisation factor of the product (operand scales, device scalars)
+    const float dq = F8 ? __ldg(args.a_scale) * __ldg(args.b_scale) : 1.f;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
@@ -835,6 +844,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256 + c * 32,
                            v);
+        if constexpr (F8) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= dq;
+        }
         const int n0 = tc.nb * BN + c * 32;
         const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
         const int col = tc.ng * args.Ng + n0;
@@ -1018,10 +1031,10 @@ bool make_glu_map(CUtensorMap* m, const GemmArgs& a, void* base, long long ld) {
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                              int num_sms, int bn, cudaStream_t stream) {
-  auto kern = gemm_tc2_kernel<A_MN, B_MN, EPI>;
+  auto kern = gemm_tc2_kernel<A_MN, B_MN, EPI, F8>;
   constexpr int smem_bytes = pair_smem(EPI);
   static bool attr_done = false;
   if (!attr_done) {
@@ -1130,6 +1143,46 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
 }
 
 }  // namespace
+
+// FP8 GEMM: C = (A B^T) * (*a_scale) * (*b_scale) with e4m3 A [M][K] and B [N][K] (K-major,
+// strides lda / ldb bytes-as-elements), on the CTA-pair kernel with 128-element K stages.
+cudaError_t launch_gemm_fp8(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.M <= 0 || a.Ng <= 0 || a.Kg <= 0 || a.NG != 1 || a.KG != 1 || a.a_mn || a.b_mn ||
+      !a.a_scale || !a.b_scale || num_sms < 2 ||
+      (a.epi != kEpiStoreF32 && a.epi != kEpiBf16))
+    return cudaErrorInvalidValue;
+  auto fn = get_encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  const int bn = pick_pair_bn(a, num_sms);
+  auto map_u8 = [&](CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t ld, uint32_t box_rows) {
+    cuuint64_t gd[3] = {inner, 1, rows};
+    cuuint64_t gs[2] = {ld, ld};
+    cuuint32_t bd[3] = {128, 1, box_rows};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), gd, gs, bd, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+  };
+  // A viewed as {K, 1, M}: coordinates (k, 0, m) like a bf16 K-major A with one K group;
+  // B as {K, N, 1}: coordinates (k, n, 0).
+  CUtensorMap ta, tb;
+  if (!map_u8(&ta, a.A, a.Kg, a.M, a.lda, BM)) return cudaErrorInvalidValue;
+  {
+    cuuint64_t gd[3] = {(cuuint64_t)a.Kg, (cuuint64_t)a.Ng, 1};
+    cuuint64_t gs[2] = {(cuuint64_t)a.ldb, (cuuint64_t)a.ldb * a.Ng};
+    cuuint32_t bd[3] = {128, (cuuint32_t)(bn / 2), 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (fn(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.B), gd, gs, bd, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  if (a.epi == kEpiStoreF32)
+    return launch_pair_inst<false, false, kEpiStoreF32, true>(ta, tb, a, num_sms, bn, stream);
+  return launch_pair_inst<false, false, kEpiBf16, true>(ta, tb, a, num_sms, bn, stream);
+}
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   // Shape rules of the tensor maps (checked by the callers too).

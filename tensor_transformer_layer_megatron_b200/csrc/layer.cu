@@ -607,4 +607,38 @@ mgt_status mgt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t a_mn_major, in
   return cuda_status(launch_gemm_tc(a, nsm, static_cast<cudaStream_t>(stream)));
 }
 
+mgt_status mgt_fp8_quantize(int32_t dtype, int64_t n, const void* x, uint8_t* q, float* scales,
+                            void* stream) {
+  if (n < 1 || !x || !q || !scales) return MGT_EINVAL;
+  if (dtype != MGT_F32 && dtype != MGT_BF16) return MGT_EUNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(q) & 1) return MGT_EUNSUPPORTED;
+  return cuda_status(launch_fp8_quantize(dtype == MGT_BF16 ? 1 : 0, n, x, q, scales,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+mgt_status mgt_gemm_fp8(int32_t M, int32_t N, int32_t K, const uint8_t* A, int64_t lda,
+                        const uint8_t* B, int64_t ldb, const float* a_scales,
+                        const float* b_scales, void* C, int32_t c_dtype, int64_t ldc,
+                        int32_t* status, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || !A || !B || !C || !a_scales || !b_scales || !status)
+    return MGT_EINVAL;
+  if (c_dtype != MGT_F32 && c_dtype != MGT_BF16) return MGT_EUNSUPPORTED;
+  if (lda < K || ldb < K || ldc < N) return MGT_EINVAL;
+  // TMA: 16-byte aligned bases and row strides; the K coordinate steps by 128 bytes.
+  if (K % 16 || lda % 16 || ldb % 16 || ldc % (c_dtype == MGT_F32 ? 4 : 8) || !aligned16(A) ||
+      !aligned16(B) || !aligned16(C))
+    return MGT_EUNSUPPORTED;
+  int dev = 0, nsm = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MGT_ECUDA;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return MGT_EUNSUPPORTED;
+  GemmArgs a = gemm_base(M, N, 1, K, 1);
+  a.A = A; a.lda = lda; a.B = B; a.ldb = ldb;
+  a.f8 = 1; a.a_scale = a_scales + 1; a.b_scale = b_scales + 1;
+  a.epi = c_dtype == MGT_F32 ? kEpiStoreF32 : kEpiBf16;
+  a.out = C; a.ldc = ldc; a.err = status;
+  return cuda_status(launch_gemm_fp8(a, nsm, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -64,6 +64,12 @@ struct GemmArgs {
   // residual rows read with them. Needs the shard length a multiple of 128.
   int a_sp, b_sp, out_sp;
   int sp_seq, sp_len, sp_b;             // sequence length, positions per shard, micro-batch
+  // FP8 (f8 = 1): A and B are e4m3 bytes, both K-major; the accumulator is multiplied by
+  // (*a_scale) * (*b_scale) (device scalars: the operands' dequantisation factors) before the
+  // epilogue. Only kEpiStoreF32 and kEpiBf16, one group, no K groups.
+  int f8;
+  const float* a_scale;
+  const float* b_scale;
 };
 
 // Row of token m in the sequence-parallel layout [p][b][s/p]: shard t = pos / (s/p) owns
@@ -82,6 +88,8 @@ bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t di
 // Builds the tensor maps from the pointers in `args` (A, B, strides) and launches a persistent
 // kernel with one CTA per SM. Returns a CUDA error code.
 cudaError_t launch_gemm_tc(const GemmArgs& args, int num_sms, cudaStream_t stream);
+// The FP8 path of the CTA-pair kernel (args.f8 semantics; e4m3 A [M][K], B [N][K]).
+cudaError_t launch_gemm_fp8(const GemmArgs& args, int num_sms, cudaStream_t stream);
 // Plain FFMA GEMM with the same semantics for fp32 operands.
 cudaError_t launch_gemm_simt_f32(const GemmArgs& args, cudaStream_t stream);
 
@@ -97,6 +105,12 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk,
                           float* dgamma, float* dbeta, float* dres_sum, cudaStream_t stream);
+
+// FP8 quantisation with a per-tensor scale: amax = max |x| over n elements (dtype 0 fp32,
+// 1 bf16), then q = e4m3(x * 448 / amax) with round-to-nearest-even and saturation, and
+// scale_out = {amax, amax / 448} (the second is the dequantisation factor).
+cudaError_t launch_fp8_quantize(int dtype, long long n, const void* x, uint8_t* q,
+                                float* scale_out, cudaStream_t stream);
 
 // Device-side failure-path probe (see mgt_debug_bounded_wait).
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
