@@ -450,10 +450,18 @@ def run_gemm_fp8(args):
         raise RuntimeError("device status %d" % int(st.item()))
     fp8 = tot["fp8"][0] / tot["fp8"][1] / 1e9
     bf16 = tot["bf16"][0] / tot["bf16"][1] / 1e9
+    peaks, src = load_peaks()
+    # e4m3 peak = the bf16 burst figure (timed alone) x the nominal dense ratio 4.5 / 2.25
+    f8_peak = 2.0 * float(peaks["bf16_tflops"])
+    peak_src = "%s bf16_tflops (burst) x 2, the nominal e4m3:bf16 dense ratio" % src
     print(json.dumps({
         "metric": "FP8 (e4m3, per-tensor scaled) GEMM TFLOP/s on the h=4096 forward GEMM shapes",
         "value": round(fp8, 1), "unit": "TFLOP/s", "higher_is_better": True,
         "bf16_same_shapes_tflops": round(bf16, 1), "speedup_vs_bf16": round(fp8 / bf16, 3),
+        "roofline": {"kernel": "gemm_tc2 (e4m3)", "bound": "tensor", "achieved": round(fp8, 1),
+                     "peak": round(f8_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(fp8 / f8_peak, 4), "peak_source": peak_src,
+                     "traffic": None},
         "steps": args.steps, "warmup": args.warmup, "dtype": "e4m3 x e4m3 -> f32",
         "data": "synthetic", "per_shape": res, "clocks": clk,
         "timing": "CUDA events around K back-to-back launches per shape; operands (<= 230 MB) "

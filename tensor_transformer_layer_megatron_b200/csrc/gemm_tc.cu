@@ -413,8 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    SeqCursor cur{0, 0};
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, num_m, num_n);
+      // token coordinates go through the sequence-parallel row map where set: M of a
+      // K-major A once per tile, the K of an MN-major operand through the cursor
+      const int ma = (!A_MN && args.a_sp) ? seq_row(args, tc.mb * BM) : tc.mb * BM;
       for (int kg = 0; kg < args.KG && ok; ++kg) {
         for (int kt = 0; kt < kt_per_group; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.err, kErrTimeoutProducer, abort_flag)) {
@@ -424,11 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           uint8_t* a_dst = sA + stage * C::A_BYTES;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
-          // token coordinates go through the sequence-parallel row map where set
-          const int ka = args.a_sp ? seq_row(args, kt * BK) : kt * BK;
-          const int kb = args.b_sp ? seq_row(args, kt * BK) : kt * BK;
+          const int kk = ((A_MN && args.a_sp) || (B_MN && args.b_sp)) ? cur.row(args, kt * BK)
+                                                                       : kt * BK;
+          const int ka = args.a_sp ? kk : kt * BK;
+          const int kb = args.b_sp ? kk : kt * BK;
           if constexpr (!A_MN) {
-            const int ma = args.a_sp ? seq_row(args, tc.mb * BM) : tc.mb * BM;
             tma_load_3d(&tmA, &full[stage], a_dst, kt * BK, kg, ma);
           } else {
 #pragma unroll
@@ -676,10 +680,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    SeqCursor cur{0, 0};
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
       const TileCoord tc = tile_coord(tile, num_m2, num_n);
       const int m0 = tc.mb * 256 + rank * 128;
       const int n0 = tc.nb * BN + rank * (BN / 2);
+      // token coordinates go through the sequence-parallel row map where set: M of a
+      // K-major A once per tile, the K of an MN-major operand through the cursor
+      const int am0 = (!A_MN && args.a_sp) ? seq_row(args, m0) : m0;
       for (int kg = 0; kg < args.KG && ok; ++kg) {
         for (int kt = 0; kt < kt_per_group; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.err, kErrTimeoutProducer, abort_flag)) {
@@ -690,11 +698,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kPairAB;
           uint8_t* b_dst = sB + stage * kPairAB;
-          // token coordinates go through the sequence-parallel row map where set
-          const int ka = args.a_sp ? seq_row(args, kt * BK) : kt * BK;
-          const int kb = args.b_sp ? seq_row(args, kt * BK) : kt * BK;
+          const int kk = ((A_MN && args.a_sp) || (B_MN && args.b_sp)) ? cur.row(args, kt * BK)
+                                                                       : kt * BK;
+          const int ka = args.a_sp ? kk : kt * BK;
+          const int kb = args.b_sp ? kk : kt * BK;
           if constexpr (!A_MN) {
-            tma_load_3d_pair(&tmA, fb, a_dst, kt * KE, kg, args.a_sp ? seq_row(args, m0) : m0);
+            tma_load_3d_pair(&tmA, fb, a_dst, kt * KE, kg, am0);
           } else {
             tma_load_3d_pair(&tmA, fb, a_dst, m0, ka, 0);
             tma_load_3d_pair(&tmA, fb, a_dst + kChunkBytes, m0 + 64, ka, 0);

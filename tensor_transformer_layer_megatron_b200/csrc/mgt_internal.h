@@ -80,6 +80,20 @@ __host__ __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
   return (t * a.sp_b + bb) * a.sp_len + (pos - t * a.sp_len);
 }
 
+// seq_row along one sweep of a token coordinate k (K of an MN-major operand): a shard chunk
+// of sp_len consecutive tokens lies in one sequence and one shard, so seq_row(k) - k is
+// constant over it and one division per chunk replaces two per k step. `end` starts at 0.
+struct SeqCursor {
+  int end, off;
+  __host__ __device__ __forceinline__ int row(const GemmArgs& a, int k) {
+    if (k >= end || k < end - a.sp_len) {
+      off = seq_row(a, k) - k;
+      end = (k / a.sp_len + 1) * a.sp_len;
+    }
+    return k + off;
+  }
+};
+
 // 3-D bf16 tensor map (128-byte swizzle, zero fill out of bounds); strides in elements.
 bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
                              const uint64_t strides[2], const uint32_t box[3]);
