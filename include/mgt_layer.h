@@ -169,7 +169,14 @@ mgt_status mgt_layer_fwd(mgt_layer* layer, const mgt_layer_params* params, const
                          void* y, void* saved, void* workspace, void* stream);
 
 /* Backward. Reads x, saved (from the matching fwd) and dy; writes dx and every gradient in
- * `grads` (fp32, overwritten). Uses `workspace` for intermediate gradients. */
+ * `grads` (fp32, overwritten). Uses `workspace` for intermediate gradients.
+ * Ordering: all work is ordered after what `stream` held at the call, and everything the call
+ * writes is complete before later work on `stream` runs. Inside, the weight-gradient GEMMs
+ * and the bias column sums run on a second stream of the handle (forked from `stream` by
+ * events after the launch that produces their inputs, joined back at the end) so that they
+ * overlap the data-gradient chain; under stream capture this is a fork/join in the graph.
+ * The first call creates that stream and its events on the current device: make it outside
+ * a stream capture. With profiling on (mgt_layer_profile) everything runs on `stream`. */
 mgt_status mgt_layer_bwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
                          const void* saved, const void* dy, void* dx, const mgt_layer_grads* grads,
                          void* workspace, void* stream);

@@ -55,6 +55,10 @@ struct mgt_layer {
   Region ws[MGT_WS_COUNT - 64];
   size_t saved_bytes = 0, ws_bytes = 0;
   int num_sms = 0;
+  // second stream of the backward (weight gradients) and its fork / join events
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork[4] = {};
+  cudaEvent_t ev_join = nullptr;
   // profiling
   bool prof = false;
   std::vector<cudaEvent_t> ev_pool;
@@ -209,6 +213,16 @@ mgt_status ensure_device(mgt_layer* L) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// The backward's second stream (non-blocking) and its events, created on first use.
+cudaError_t ensure_side_stream(mgt_layer* L) {
+  if (L->side) return cudaSuccess;
+  cudaError_t e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    e = cudaEventCreateWithFlags(&L->ev_fork[i], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);
+  return e;
+}
+
 // Every parameter (and gradient) pointer must be set and 16-byte aligned, except the four
 // linear biases of a layer without them, which are ignored.
 mgt_status check_param_ptrs(const mgt_layer* L, const void* const* q) {
@@ -315,7 +329,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   // 1. LN1
   MGT_TRY(run(L, "ln_fwd", 0, ln_bytes, s, [&] {
     return launch_ln_fwd(dt, T, h, L->cfg.ln_eps, x, (const float*)P->ln1_g,
-                         (const float*)P->ln1_b, ln1, mu1, rs1, s);
+                         (const float*)P->ln1_b, ln1, mu1, rs1, err, s);
   }));
   // 2. QKV, column-parallel: the packed [p][3][H/p][d] rows are the GEMM's N dimension.
   {
@@ -344,7 +358,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   // 5. LN2
   MGT_TRY(run(L, "ln_fwd", 0, ln_bytes, s, [&] {
     return launch_ln_fwd(dt, T, h, L->cfg.ln_eps, h1, (const float*)P->ln2_g,
-                         (const float*)P->ln2_b, ln2, mu2, rs2, s);
+                         (const float*)P->ln2_b, ln2, mu2, rs2, err, s);
   }));
   // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and GeLU'(u) for the backward).
   //    SwiGLU: shard t's gate and up rows go to the two halves of one tile; the epilogue stores
@@ -414,9 +428,30 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   float* Dsum = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_ATTN_D - 64]));
   float* part = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_LN_PARTIAL - 64]));
   const int nblk = T < kMaxLnBlocks ? T : kMaxLnBlocks;
+  // Weight gradients and bias column sums feed nothing else in the backward: they run on a
+  // second stream `w`, forked after the launch that produces their inputs and joined into `s`
+  // at the end, so their tiles fill the SMs that the data-gradient chain's last partial waves
+  // leave idle. With profiling on, every launch stays on `s` and is timed alone.
+  const bool two = !L->prof;
+  if (two) MGT_TRY(ensure_side_stream(L));
+  cudaStream_t w = two ? L->side : s;
+  auto fork = [&](int k) -> cudaError_t {
+    if (!two) return cudaSuccess;
+    cudaError_t r = cudaEventRecord(L->ev_fork[k], s);
+    return r == cudaSuccess ? cudaStreamWaitEvent(w, L->ev_fork[k], 0) : r;
+  };
+  // joins `w` into `s` on every return path once the first fork has been made
+  struct Join {
+    mgt_layer* L;
+    cudaStream_t s, w;
+    bool on = false;
+    ~Join() {
+      if (on && cudaEventRecord(L->ev_join, w) == cudaSuccess) cudaStreamWaitEvent(s, L->ev_join, 0);
+    }
+  } join{L, s, w};
   auto colsum = [&](const void* src, int cols, void* out) {
-    return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, s,
-               [&] { return launch_colsum(dt, T, cols, src, (float*)out, s); });
+    return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, w,
+               [&] { return launch_colsum(dt, T, cols, src, (float*)out, w); });
   };
   const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
   const bool nb = L->cfg.disable_bias_linear, sw = L->cfg.swiglu;
@@ -424,6 +459,8 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
 
   // B1. fc2: dgrad fused with GeLU' -> du (SwiGLU: with the SwiGLU backward -> d[gate | up]),
   //     wgrad (db2 = sum dy comes with the LN2 backward)
+  MGT_TRY(fork(0));  // dy and the saved activation a are ready
+  join.on = two;
   {
     GemmArgs a = gemm_base(T, f / p, p, h, 1);  // N grouped by shard
     a.b_mn = 1; a.A = dy; a.lda = h; a.B = P->w2; a.ldb = f / p;
@@ -438,8 +475,9 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.a_mn = 1; a.b_mn = 1; a.A = dy; a.lda = h; a.B = act; a.ldb = f;
     a.epi = kEpiStoreF32; a.out = G->w2; a.ldc = f / p; a.out_ng = f / p;
     a.out_gs = (long long)h * (f / p); a.err = err; a.a_sp = 1;
-    MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, w));
   }
+  MGT_TRY(fork(1));  // du is ready (fc2 dgrad)
   // B3. fc1: db1, dgrad (sum over shards = K loop over all fc1 outputs), wgrad
   if (!nb) MGT_TRY(colsum(du, f1, G->b1));
   {
@@ -453,15 +491,16 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(f1, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f1; a.B = ln2; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err; a.b_sp = 1;
-    MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, s));
+    MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, w));
   }
   // B4. LN2 backward + residual gradient dy -> dh1
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
     // dres = dy, so the residual-gradient sum it also returns is db2
     return launch_ln_bwd(dt, T, h, dln2, dy, h1, (const float*)P->ln2_g, mu2, rs2, dh1, part,
                          nblk, (float*)G->ln2_g, (float*)G->ln2_b,
-                         nb ? nullptr : (float*)G->b2, s);
+                         nb ? nullptr : (float*)G->b2, err, s);
   }));
+  MGT_TRY(fork(2));  // dh1 is ready
   // B5. out-proj: dgrad (N grouped by shard) -> dO, wgrad (db_o = sum dh1 comes with LN1 bwd)
   {
     GemmArgs a = gemm_base(T, h / p, p, h, 1);
@@ -475,7 +514,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     a.a_mn = 1; a.b_mn = 1; a.A = dh1; a.lda = h; a.B = O; a.ldb = h; a.a_sp = 1;
     a.epi = kEpiStoreF32; a.out = G->w_o; a.ldc = h / p; a.out_ng = h / p;
     a.out_gs = (long long)h * (h / p); a.err = err;
-    MGT_TRY(gemm(L, "gemm_tc/outproj_wgrad", a, s));
+    MGT_TRY(gemm(L, "gemm_tc/outproj_wgrad", a, w));
   }
   // B6. attention backward (probabilities recomputed from the saved log-sum-exp)
   {
@@ -484,6 +523,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     const double fl = 2.5 * 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;  // model FLOPs incl. one recompute of S
     MGT_TRY(run(L, "attn_bwd", fl, 0, s, [&] { return launch_attn_bwd(dt, a, s); }));
   }
+  MGT_TRY(fork(3));  // dqkv is ready
   // B7. QKV: db_qkv, dgrad (sum over shards = K loop over 3h), wgrad
   if (!nb) MGT_TRY(colsum(dqkv, 3 * h, G->b_qkv));
   {
@@ -496,14 +536,14 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(3 * h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = ln1; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err; a.b_sp = 1;
-    MGT_TRY(gemm(L, "gemm_tc/qkv_wgrad", a, s));
+    MGT_TRY(gemm(L, "gemm_tc/qkv_wgrad", a, w));
   }
   // B8. LN1 backward + residual gradient dh1 -> dx
   MGT_TRY(run(L, "ln_bwd", 0, lnb_bytes, s, [&] {
     // dres = dh1, so the residual-gradient sum it also returns is db_o
     return launch_ln_bwd(dt, T, h, dln1, dh1, x, (const float*)P->ln1_g, mu1, rs1, dx, part,
                          nblk, (float*)G->ln1_g, (float*)G->ln1_b,
-                         nb ? nullptr : (float*)G->b_o, s);
+                         nb ? nullptr : (float*)G->b_o, err, s);
   }));
   return MGT_OK;
 }
@@ -572,6 +612,10 @@ mgt_status mgt_layer_profile_read(mgt_layer* L, mgt_kernel_stat* out, int cap, i
 void mgt_layer_destroy(mgt_layer* L) {
   if (!L) return;
   for (auto& ev : L->ev_pool) cudaEventDestroy(ev);
+  for (auto& ev : L->ev_fork)
+    if (ev) cudaEventDestroy(ev);
+  if (L->ev_join) cudaEventDestroy(L->ev_join);
+  if (L->side) cudaStreamDestroy(L->side);
   delete L;
 }
 

@@ -6,6 +6,8 @@
 // is replicated on every shard under the column/row split, so each shard's statistics already
 // are the global ones. The page's section 4.2 motivates one fused kernel per LayerNorm (launch
 // overhead of unfused norms at short sequences).
+#include <mutex>
+
 #include "mgt_device.cuh"
 
 namespace mgt {
@@ -357,6 +359,283 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_fused_kernel(long long rows, in
   }
 }
 
+// ---------------------------------------------------------------------------- row rings
+// Rows of 256 to 1024 16-byte vectors stream through a ring of S shared-memory stages filled
+// by plain bulk copies (cp.async.bulk, one mbarrier per stage): one thread keeps up to S rows
+// of every input in flight per block while all 256 threads reduce the current row, so far
+// more bytes are in flight per SM than the registers of a row-per-group kernel can hold.
+// Thread t owns the vectors t, t + 256, ... of every row. Every wait is bounded; on a timeout
+// the block records it, waits (bounded) for its copies in flight and leaves.
+constexpr int kRingStages = 4;
+
+// Wait for the copies of local rows [i, min(n, i + S)) that are still in flight.
+template <int S>
+__device__ __forceinline__ void ring_drain(uint64_t* full, long long i, long long n, int* err) {
+  for (long long j = i; j < n && j < i + S; ++j)
+    mbar_wait(&full[j % S], (uint32_t)((j / S) & 1), err, kErrTimeoutDrain, nullptr);
+}
+
+// LayerNorm forward, one row per block iteration; rows r = blockIdx.x + i * gridDim.x. gamma
+// and beta of the thread's columns are loaded once per block.
+template <typename T, int VPL, int S>
+__global__ void __launch_bounds__(256) ln_fwd_ring_kernel(long long rows, int h, float eps,
+                                                          const T* __restrict__ x,
+                                                          const float* __restrict__ gamma,
+                                                          const float* __restrict__ beta,
+                                                          T* __restrict__ y,
+                                                          float* __restrict__ mean,
+                                                          float* __restrict__ rstd, int* err) {
+  constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[S];
+  __shared__ float red[2][8];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nvec = h / V;
+  const uint32_t row_bytes = (uint32_t)h * sizeof(T);
+  const long long nloc =
+      (long long)blockIdx.x < rows ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (t == 0) {
+    for (int k = 0; k < S; ++k) mbar_init(&full[k], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](long long i) {
+    const int st = (int)(i % S);
+    const long long r = blockIdx.x + i * gridDim.x;
+    mbar_arrive_expect_tx(&full[st], row_bytes);
+    bulk_load_1d(ring + (size_t)st * row_bytes, x + r * h, row_bytes, &full[st]);
+  };
+  if (t == 0)
+    for (long long i = 0; i < S && i < nloc; ++i) issue(i);
+  float gv[VPL][V], bv[VPL][V];
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int vi = t + k * 256;
+    if (vi < nvec) {
+      load_param<V>(gamma, vi * V, gv[k]);
+      load_param<V>(beta, vi * V, bv[k]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < V; ++j) gv[k][j] = bv[k][j] = 0.f;
+    }
+  }
+  const float inv_h = 1.f / (float)h;
+  for (long long i = 0; i < nloc; ++i) {
+    const int st = (int)(i % S);
+    const bool ok = mbar_wait(&full[st], (uint32_t)((i / S) & 1), err, kErrTimeoutLn, nullptr);
+    const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t)st * row_bytes);
+    float v[VPL][V];
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = t + k * 256;
+      if (ok && vi < nvec) {
+        Vec<T>::unpack(src[vi], v[k]);
+#pragma unroll
+        for (int j = 0; j < V; ++j) sum += v[k][j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < V; ++j) v[k][j] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) red[0][warp] = sum;
+    if (__syncthreads_or(!ok)) {
+      if (t == 0) ring_drain<S>(full, i, nloc, err);
+      return;
+    }
+    // every thread has read this stage (before the barrier): refill it
+    if (t == 0 && i + S < nloc) issue(i + S);
+    float mu = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) mu += red[0][w];
+    mu *= inv_h;
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      if (t + k * 256 < nvec) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const float c = v[k][j] - mu;
+          q += c * c;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane == 0) red[1][warp] = q;
+    __syncthreads();
+    float var = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) var += red[1][w];
+    const float rs = rsqrtf(var * inv_h + eps);
+    const long long r = blockIdx.x + i * gridDim.x;
+    T* yr = y + r * h;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = t + k * 256;
+      if (vi < nvec) {
+        float o[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) o[j] = (v[k][j] - mu) * rs * gv[k][j] + bv[k][j];
+        Vec<T>::store(yr + vi * V, o);
+      }
+    }
+    if (t == 0) {
+      mean[r] = mu;
+      rstd[r] = rs;
+    }
+  }
+}
+
+// LayerNorm backward over a contiguous slice of rows per block (rows_per each): dx per row and
+// the parameter partials of the slice, as ln_bwd_fused_kernel, with x, dy and dres streamed
+// through the ring (one stage = the three rows) instead of prefetched into registers.
+template <typename T, int VPL, int NSUM, int S>
+__global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int h,
+                                                          const T* __restrict__ dy,
+                                                          const T* __restrict__ dres,
+                                                          const T* __restrict__ x,
+                                                          const float* __restrict__ gamma,
+                                                          const float* __restrict__ mean,
+                                                          const float* __restrict__ rstd,
+                                                          T* __restrict__ dx,
+                                                          float* __restrict__ partial,
+                                                          long long rows_per, int* err) {
+  constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[S];
+  __shared__ float2 red[2][8];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nvec = h / V;
+  const uint32_t row_bytes = (uint32_t)h * sizeof(T);
+  const uint32_t stage_bytes = (dres ? 3u : 2u) * row_bytes;
+  const long long r0 = (long long)blockIdx.x * rows_per;
+  const long long r1 = min(rows, r0 + rows_per);
+  const long long nloc = r1 > r0 ? r1 - r0 : 0;
+  if (t == 0) {
+    for (int k = 0; k < S; ++k) mbar_init(&full[k], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](long long i) {
+    const int st = (int)(i % S);
+    const long long r = r0 + i;
+    uint8_t* dst = ring + (size_t)st * stage_bytes;
+    mbar_arrive_expect_tx(&full[st], stage_bytes);
+    bulk_load_1d(dst, x + r * h, row_bytes, &full[st]);
+    bulk_load_1d(dst + row_bytes, dy + r * h, row_bytes, &full[st]);
+    if (dres) bulk_load_1d(dst + 2 * row_bytes, dres + r * h, row_bytes, &full[st]);
+  };
+  if (t == 0)
+    for (long long i = 0; i < S && i < nloc; ++i) issue(i);
+  const float inv_h = 1.f / (float)h;
+  float ag[VPL][V], ab[VPL][V], ar[VPL][V];
+#pragma unroll
+  for (int k = 0; k < VPL; ++k)
+#pragma unroll
+    for (int j = 0; j < V; ++j) ag[k][j] = ab[k][j] = ar[k][j] = 0.f;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  float cmu = nloc ? mean[r0] : 0.f, crs = nloc ? rstd[r0] : 0.f;
+  int par = 0;
+  for (long long i = 0; i < nloc; ++i, par ^= 1) {
+    const long long r = r0 + i;
+    const int st = (int)(i % S);
+    const float nmu = i + 1 < nloc ? mean[r + 1] : 0.f;
+    const float nrs = i + 1 < nloc ? rstd[r + 1] : 0.f;
+    const bool ok = mbar_wait(&full[st], (uint32_t)((i / S) & 1), err, kErrTimeoutLn, nullptr);
+    const uint4* sx = reinterpret_cast<const uint4*>(ring + (size_t)st * stage_bytes);
+    const uint4* sd = sx + row_bytes / 16;
+    const uint4* sr = sd + row_bytes / 16;
+    uint4 cx[VPL], cd[VPL], cr[VPL];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = t + k * 256;
+      const bool in = ok && vi < nvec;
+      cx[k] = in ? sx[vi] : zero;
+      cd[k] = in ? sd[vi] : zero;
+      cr[k] = (in && dres) ? sr[vi] : zero;
+      float xv[V], dv[V], gv[V];
+      Vec<T>::unpack(cx[k], xv);
+      Vec<T>::unpack(cd[k], dv);
+      if (vi < nvec) {
+        load_param<V>(gamma, vi * V, gv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < V; ++j) gv[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
+        s1 += g;
+        s2 += g * xh;
+        ag[k][j] += dv[j] * xh;
+        ab[k][j] += dv[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    // Two buffers by row parity: a buffer is rewritten two rows later, after every thread has
+    // passed the next row's barrier and so has finished reading it.
+    if (lane == 0) red[par][warp] = make_float2(s1, s2);
+    if (__syncthreads_or(!ok)) {
+      if (t == 0) ring_drain<S>(full, i, nloc, err);
+      return;
+    }
+    if (t == 0 && i + S < nloc) issue(i + S);  // the stage has been read into registers
+    float S1 = 0.f, S2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float2 v = red[par][w];
+      S1 += v.x;
+      S2 += v.y;
+    }
+    const float m1 = S1 * inv_h, m2 = S2 * inv_h;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int vi = t + k * 256;
+      if (vi < nvec) {
+        float xv[V], dv[V], rv[V], gv[V], o[V];
+        Vec<T>::unpack(cx[k], xv);
+        Vec<T>::unpack(cd[k], dv);
+        Vec<T>::unpack(cr[k], rv);
+        load_param<V>(gamma, vi * V, gv);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
+          o[j] = crs * (g - m1 - xh * m2) + rv[j];
+          if constexpr (NSUM == 3) ar[k][j] += rv[j];
+        }
+        Vec<T>::store(dx + r * h + vi * V, o);
+      }
+    }
+    cmu = nmu;
+    crs = nrs;
+  }
+  float* pg = partial + (long long)blockIdx.x * NSUM * h;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int vi = t + k * 256;
+    if (vi < nvec) {
+#pragma unroll
+      for (int j = 0; j < V; j += 4) {
+        *reinterpret_cast<float4*>(pg + vi * V + j) =
+            make_float4(ag[k][j], ag[k][j + 1], ag[k][j + 2], ag[k][j + 3]);
+        *reinterpret_cast<float4*>(pg + h + vi * V + j) =
+            make_float4(ab[k][j], ab[k][j + 1], ab[k][j + 2], ab[k][j + 3]);
+        if constexpr (NSUM == 3)
+          *reinterpret_cast<float4*>(pg + 2 * h + vi * V + j) =
+              make_float4(ar[k][j], ar[k][j + 1], ar[k][j + 2], ar[k][j + 3]);
+      }
+    }
+  }
+}
+
 // Partial dgamma = sum dy*xhat and dbeta = sum dy over one slice of rows, and with NSUM = 3 also
 // sum dres (the residual gradient: a bias gradient of the layer for free, as the LayerNorm
 // backward reads it anyway). Block = 32 x 8 threads covering 32*VEC columns; blockIdx.y is the
@@ -452,8 +731,21 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
   const int c = blockIdx.x * 32 + (threadIdx.x & 31);
   const int sl = threadIdx.x >> 5;
   float s = 0.f;
-  if (c < nsum * h)
-    for (int b = sl; b < nblk; b += 8) s += partial[(long long)b * nsum * h + c];
+  if (c < nsum * h) {
+    // four loads in flight per thread; the additions keep the order b = sl, sl + 8, ...
+    const long long step = (long long)nsum * h;
+    int b = sl;
+    for (; b + 24 < nblk; b += 32) {
+      const float p0 = __ldg(partial + b * step + c), p1 = __ldg(partial + (b + 8) * step + c);
+      const float p2 = __ldg(partial + (b + 16) * step + c);
+      const float p3 = __ldg(partial + (b + 24) * step + c);
+      s += p0;
+      s += p1;
+      s += p2;
+      s += p3;
+    }
+    for (; b < nblk; b += 8) s += __ldg(partial + b * step + c);
+  }
   red[sl][threadIdx.x & 31] = s;
   __syncthreads();
   if (sl == 0 && c < nsum * h) {
@@ -618,12 +910,69 @@ cudaError_t ln_bwd_dx_inst(long long rows, int h, const void* dy, const void* dr
   return cudaGetLastError();
 }
 
+bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 1;
+  return n;
+}
+
+// Blocks of a ring kernel resident per SM at `smem` bytes of dynamic shared memory (0 on
+// failure); raises the kernel's dynamic shared-memory limit first. Cached per (kernel, smem).
+template <typename K>
+int ring_blocks_per_sm(K kern, size_t smem) {
+  struct Entry {
+    const void* fn;
+    size_t smem;
+    int bps;
+  };
+  static std::mutex mu;
+  static Entry cache[32];
+  static int used = 0;
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].smem == smem) return cache[i].bps;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, smem) != cudaSuccess) return 0;
+  if (used < 32) cache[used++] = Entry{fn, smem, n};
+  return n;
+}
+
+template <typename T, int VPL>
+cudaError_t ln_fwd_ring_inst(long long rows, int h, float eps, const void* x, const float* g,
+                             const float* b, void* y, float* mean, float* rstd, int* err,
+                             cudaStream_t s) {
+  auto kern = ln_fwd_ring_kernel<T, VPL, kRingStages>;
+  const size_t smem = (size_t)kRingStages * h * sizeof(T);
+  const int bps = ring_blocks_per_sm(kern, smem);
+  if (bps < 1) return cudaErrorInvalidConfiguration;
+  long long grid = (long long)bps * device_sms();
+  if (grid > rows) grid = rows;
+  kern<<<(unsigned)grid, 256, smem, s>>>(rows, h, eps, reinterpret_cast<const T*>(x), g, b,
+                                        reinterpret_cast<T*>(y), mean, rstd, err);
+  return cudaGetLastError();
+}
+
 // Row-group shapes: a row is spread over W warps with at most VPL 16-byte vectors per thread,
 // so registers stay small and many rows are in flight. bf16: h <= 16384; fp32: h <= 8192.
+// Rows of 256..1024 vectors (bf16 h = 2048..8192) go through the shared-memory ring instead.
 template <typename T>
 cudaError_t ln_fwd_dispatch(long long rows, int h, float eps, const void* x, const float* g,
-                            const float* b, void* y, float* mean, float* rstd, cudaStream_t s) {
+                            const float* b, void* y, float* mean, float* rstd, int* err,
+                            cudaStream_t s) {
   const int nvec = h / Vec<T>::N;
+  if (nvec >= 256 && nvec <= 1024 && aligned16_ptr(x)) {
+    if (nvec <= 256) return ln_fwd_ring_inst<T, 1>(rows, h, eps, x, g, b, y, mean, rstd, err, s);
+    if (nvec <= 512) return ln_fwd_ring_inst<T, 2>(rows, h, eps, x, g, b, y, mean, rstd, err, s);
+    return ln_fwd_ring_inst<T, 4>(rows, h, eps, x, g, b, y, mean, rstd, err, s);
+  }
   if (nvec <= 64) return ln_fwd_inst<T, 1, 2>(rows, h, eps, x, g, b, y, mean, rstd, s);
   if (nvec <= 128) return ln_fwd_inst<T, 1, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
   if (nvec <= 256) return ln_fwd_inst<T, 2, 4>(rows, h, eps, x, g, b, y, mean, rstd, s);
@@ -636,7 +985,7 @@ template <typename T>
 cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* dres,
                             const void* x, const float* g, const float* mean, const float* rstd,
                             void* dx, float* partial, int nblk, float* dgamma, float* dbeta,
-                            float* dres_sum, cudaStream_t s) {
+                            float* dres_sum, int* err, cudaStream_t s) {
   const int nvec = h / Vec<T>::N;
   const int nsum = (dres_sum && dres) ? 3 : 2;
   cudaError_t e;
@@ -649,7 +998,25 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
     const T* px = reinterpret_cast<const T*>(x);
     T* pdx = reinterpret_cast<T*>(dx);
     const unsigned gs = (unsigned)slices;
-    if (nvec <= 256) {
+    const bool ring = nvec >= 256 && aligned16_ptr(x) && aligned16_ptr(dy) &&
+                      (!dres || aligned16_ptr(dres));
+    if (ring) {
+      // x, dy (and dres) rows streamed through the shared-memory ring
+      const size_t smem = (size_t)kRingStages * (dres ? 3 : 2) * h * sizeof(T);
+      auto launch = [&](auto kern) {
+        if (ring_blocks_per_sm(kern, smem) < 1) return cudaErrorInvalidConfiguration;
+        kern<<<gs, 256, smem, s>>>(rows, h, pdy, pdr, px, g, mean, rstd, pdx, partial,
+                                   rows_per, err);
+        return cudaGetLastError();
+      };
+      if (nvec <= 256)
+        e = nsum == 3 ? launch(ln_bwd_ring_kernel<T, 1, 3, kRingStages>)
+                      : launch(ln_bwd_ring_kernel<T, 1, 2, kRingStages>);
+      else
+        e = nsum == 3 ? launch(ln_bwd_ring_kernel<T, 2, 3, kRingStages>)
+                      : launch(ln_bwd_ring_kernel<T, 2, 2, kRingStages>);
+      if (e != cudaSuccess) return e;
+    } else if (nvec <= 256) {
       if (nsum == 3)
         ln_bwd_fused_kernel<T, 1, 3><<<gs, 256, 0, s>>>(rows, h, pdy, pdr, px, g, mean, rstd,
                                                         pdx, partial, rows_per);
@@ -709,10 +1076,11 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
 
 cudaError_t launch_ln_fwd(int dtype, long long rows, int h, float eps, const void* x,
                           const float* gamma, const float* beta, void* y, float* mean,
-                          float* rstd, cudaStream_t s) {
+                          float* rstd, int* err, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  return dtype ? ln_fwd_dispatch<__nv_bfloat16>(rows, h, eps, x, gamma, beta, y, mean, rstd, s)
-               : ln_fwd_dispatch<float>(rows, h, eps, x, gamma, beta, y, mean, rstd, s);
+  return dtype ? ln_fwd_dispatch<__nv_bfloat16>(rows, h, eps, x, gamma, beta, y, mean, rstd,
+                                                err, s)
+               : ln_fwd_dispatch<float>(rows, h, eps, x, gamma, beta, y, mean, rstd, err, s);
 }
 
 int ln_bwd_blocks(long long rows, int num_sms) {
@@ -724,12 +1092,12 @@ int ln_bwd_blocks(long long rows, int num_sms) {
 cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, const void* dres,
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk, float* dgamma,
-                          float* dbeta, float* dres_sum, cudaStream_t s) {
+                          float* dbeta, float* dres_sum, int* err, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   return dtype ? ln_bwd_dispatch<__nv_bfloat16>(rows, h, dy, dres, x, gamma, mean, rstd, dx,
-                                                partial, nblk, dgamma, dbeta, dres_sum, s)
+                                                partial, nblk, dgamma, dbeta, dres_sum, err, s)
                : ln_bwd_dispatch<float>(rows, h, dy, dres, x, gamma, mean, rstd, dx, partial,
-                                        nblk, dgamma, dbeta, dres_sum, s);
+                                        nblk, dgamma, dbeta, dres_sum, err, s);
 }
 
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,

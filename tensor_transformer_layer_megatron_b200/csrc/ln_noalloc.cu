@@ -65,6 +65,6 @@ extern "C" mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int
   // Every partial row is written before it is read, so the array needs no clearing.
   cudaError_t e = mgt::launch_ln_bwd(dtype == MGT_BF16 ? 1 : 0, rows, h, dy, dres, x, gamma,
                                      mean, rstd, dx, scratch, (int)nblk, dgamma, dbeta,
-                                     nullptr, static_cast<cudaStream_t>(stream));
+                                     nullptr, nullptr, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MGT_OK : MGT_ECUDA;
 }

@@ -14,6 +14,7 @@ enum DeviceError : int {
   kErrTimeoutEpilogue = 0x102,  // epilogue waited too long for an accumulator
   kErrTimeoutDrain = 0x103,     // unwinding after a timeout waited too long
   kErrTimeoutAttn = 0x110,
+  kErrTimeoutLn = 0x120,        // a LayerNorm row ring waited too long for a bulk copy
   kErrTimeoutProbe = 0x1F0,     // the bounded-wait probe (mgt_debug_bounded_wait) gave up
 };
 
@@ -108,9 +109,10 @@ cudaError_t launch_gemm_fp8(const GemmArgs& args, int num_sms, cudaStream_t stre
 cudaError_t launch_gemm_simt_f32(const GemmArgs& args, cudaStream_t stream);
 
 // LayerNorm over the last dimension. dtype: 0 fp32, 1 bf16 (x, y); stats and params fp32.
+// err: device status word for bounded-wait timeouts (may be null).
 cudaError_t launch_ln_fwd(int dtype, long long rows, int h, float eps, const void* x,
                           const float* gamma, const float* beta, void* y, float* mean,
-                          float* rstd, cudaStream_t stream);
+                          float* rstd, int* err, cudaStream_t stream);
 // dx = dres + LN'^T(dy); dgamma, dbeta and (if dres_sum and dres are given) dres_sum =
 // sum over rows of dres, through per-slice partials in `partial`, which must hold
 // nblk * (dres_sum ? 3 : 2) * h floats; at most nblk slices are used.
@@ -118,7 +120,8 @@ int ln_bwd_blocks(long long rows, int num_sms);
 cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, const void* dres,
                           const void* x, const float* gamma, const float* mean,
                           const float* rstd, void* dx, float* partial, int nblk,
-                          float* dgamma, float* dbeta, float* dres_sum, cudaStream_t stream);
+                          float* dgamma, float* dbeta, float* dres_sum, int* err,
+                          cudaStream_t stream);
 
 // FP8 quantisation with a per-tensor scale: amax = max |x| over n elements (dtype 0 fp32,
 // 1 bf16), then q = e4m3(x * 448 / amax) with round-to-nearest-even and saturation, and

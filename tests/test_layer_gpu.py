@@ -26,6 +26,12 @@ SMALL = [
     small("h256-d64-p2-tanh", hidden=256, heads=4, ffn=512, seq=33, micro_batch=2, tp_size=2,
           gelu_tanh=1),
     small("h128-d64-p1-s1", hidden=128, heads=2, ffn=256, seq=1, micro_batch=4, tp_size=1),
+    # rows of 256 and 384 16-byte vectors: the LayerNorm kernels' shared-memory row ring (one
+    # and two vectors per thread, the second only for some threads)
+    small("h2048-d128-p2-s72-b2", hidden=2048, heads=16, ffn=2048, seq=72, micro_batch=2,
+          tp_size=2),
+    small("h3072-d128-p4-s40-b3", hidden=3072, heads=24, ffn=3072, seq=40, micro_batch=3,
+          tp_size=4),
 ]
 
 # SwiGLU (fc1 tiles pair a shard's gate and up rows) and no-bias layers. f/p = 128 sends the
@@ -58,6 +64,16 @@ def test_layer_bf16_small(cfg):
 @pytest.mark.parametrize("affine", [False, True])
 def test_layer_f32_tiny(affine):
     cfg = config_by_name("tiny-h64-tp2-f32")
+    errs = full_parity(cfg, nonzero_affine=affine)
+    bad = {k: v for k, v in errs.items() if v > tol(cfg)}
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("affine", [False, True])
+def test_layer_f32_ring_rows(affine):
+    """fp32 layer with h = 1024: LayerNorm rows of 256 vectors take the row-ring kernels."""
+    cfg = LayerConfig("h1024-f32-p2-s24-b2", hidden=1024, heads=16, ffn=1024, seq=24,
+                      micro_batch=2, tp_size=2, dtype="f32", seed=4401)
     errs = full_parity(cfg, nonzero_affine=affine)
     bad = {k: v for k, v in errs.items() if v > tol(cfg)}
     assert not bad, (bad, errs)
