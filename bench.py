@@ -241,7 +241,7 @@ def run_mgt(args):
     run.check()
     torch.cuda.synchronize()
 
-    # ---- timed region. With --graph (default) one step (fwd + bwd, 26 kernel launches through
+    # ---- timed region. With --graph (default) one step (fwd + bwd, 23 kernel launches through
     # the C ABI) is captured once into a CUDA graph and replayed K times; otherwise the C ABI is
     # called eagerly. Per-kernel CUDA events are recorded by the C ABI around every launch of
     # the eager steps (in graph mode: an eager pass of K steps right after the timed replays).
