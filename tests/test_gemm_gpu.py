@@ -13,9 +13,10 @@ def ceil8(v):
     return (v + 7) // 8 * 8
 
 
-# (2048, 12288, 64) selects the 224-wide pair tile for K-major B, the others 128 or 256.
+# For K-major B, (2048, 12288, 64) selects the 224-wide pair tile and (2048, 3000, 72) the
+# 192-wide one with N ragged inside the last tile; the others take 128 or 256.
 SHAPES = [(128, 256, 64), (200, 300, 136), (1, 8, 8), (1000, 520, 1000), (256, 384, 4096),
-          (129, 129, 72), (2048, 12288, 64)]
+          (129, 129, 72), (2048, 12288, 64), (1000, 4096, 200), (2048, 3000, 72)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
