@@ -1,0 +1,51 @@
+"""The backward's second stream (weight gradients and bias column sums, forked from the
+caller's stream and joined back) against the single-stream order that profiling uses: the same
+kernels on the same inputs must give the same dx and parameter gradients. Only the two bias
+column sums accumulate with floating-point atomics (their order varies between runs); every
+other result is bit-identical. Results are read on the caller's stream right after the call,
+so a missing join would show as stale gradients. A second backward overwrites everything."""
+import pytest
+import torch
+
+import tensor_transformer_layer_megatron_b200 as mgt
+from mgt_inputs import LayerConfig, make_inputs, pack_params
+from tensor_transformer_layer_megatron_b200.runner import LayerRun
+
+pytestmark = pytest.mark.gpu
+
+ATOMIC = ("b1", "b_qkv")
+
+
+def _snapshot(run):
+    out = {"dx": run.dx.float().cpu()}
+    out.update({k: v.cpu() for k, v in run.grads.items()})
+    return out
+
+
+@pytest.mark.parametrize("swiglu", [0, 1])
+def test_two_stream_backward_matches_single_stream(swiglu):
+    cfg = LayerConfig("streams-h512-p2-s256-b2", hidden=512, heads=4, ffn=1536, seq=256,
+                      micro_batch=2, tp_size=2, dtype="bf16", seed=4501, swiglu=swiglu)
+    t = make_inputs(cfg, nonzero_affine=True)
+    layer = mgt.Layer.from_config(cfg)
+    run = LayerRun(layer, pack_params(cfg, t), t["x"], t["dy"])
+    run.fwd()
+    layer.profile(True)  # one stream: every launch on the caller's stream
+    run.bwd()
+    run.check()
+    one = _snapshot(run)
+    layer.profile(False)
+    for g in run.grads.values():  # stale values would survive a missing join
+        g.fill_(float("nan"))
+    run.dx.fill_(float("nan"))
+    run.bwd()  # two streams
+    two = _snapshot(run)
+    run.check()
+    for k, ref in one.items():
+        got = two[k]
+        assert torch.isfinite(got).all(), k
+        if k in ATOMIC:
+            scale = ref.abs().max().clamp_min(1e-30)
+            assert ((got - ref).abs().max() / scale).item() <= 1e-6, k
+        else:
+            assert torch.equal(got, ref), k
