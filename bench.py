@@ -335,11 +335,17 @@ def run_mgt(args):
             roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+    # every family against its own roofline: contractions against the sustained bf16 peak
+    # (model FLOPs), memory-bound kernels against the HBM copy bandwidth (algorithmic bytes)
     kernels = {k: {"launches": v["launches"], "ms_per_step": round(v["ms"] / args.steps, 4),
-                   **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)}
+                   **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1),
+                       "frac_of_sustained_bf16": round(v["flops"] / (v["ms"] / 1e3) / 1e12 /
+                                                       peaks["bf16_tflops_sustained"], 4)}
                       if v["flops"] else {}),
-                   **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)}
-                      if v["bytes"] else {})}
+                   **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1),
+                       "frac_of_hbm": round(v["bytes"] / (v["ms"] / 1e3) / 1e9 /
+                                            peaks["hbm_gbs"], 4)}
+                      if v["bytes"] and not v["flops"] else {})}
                for k, v in prof.items()}
     gemm_sites = {k.split("/")[1]: {"ms_per_step": round(v["ms"] / args.steps, 4),
                                     "tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)}
