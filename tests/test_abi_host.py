@@ -108,3 +108,46 @@ def test_region_layout(cfg):
         s = sorted((a, b) for k, a, b in spans if k == buf)
         for (a0, b0), (a1, b1) in zip(s, s[1:]):
             assert b0 <= a1  # regions never overlap
+
+
+# FP8 entry points: argument checks run before any CUDA call, so they are testable on the
+# host. Fake, never-dereferenced addresses stand in for device pointers.
+P16 = 0x10000  # 16-byte aligned
+P_ODD = 0x10001
+
+
+def test_fp8_quantize_rejects():
+    lib = mgt.load_library()
+    assert lib.mgt_fp8_quantize(1, 0, P16, P16, P16, None) == 1       # n < 1
+    assert lib.mgt_fp8_quantize(1, 8, None, P16, P16, None) == 1      # null x
+    assert lib.mgt_fp8_quantize(1, 8, P16, None, P16, None) == 1      # null q
+    assert lib.mgt_fp8_quantize(1, 8, P16, P16, None, None) == 1      # null scales
+    assert lib.mgt_fp8_quantize(7, 8, P16, P16, P16, None) == 2       # unknown dtype
+    assert lib.mgt_fp8_quantize(0, 8, P16, P_ODD, P16, None) == 2     # q not 2-byte aligned
+
+
+@pytest.mark.parametrize("M,N,K,lda,ldb,ldc,cd,code", [
+    (0, 8, 16, 16, 16, 8, 0, 1),      # empty M
+    (8, 0, 16, 16, 16, 8, 0, 1),      # empty N
+    (8, 8, 0, 16, 16, 8, 0, 1),       # empty K
+    (8, 8, 16, 8, 16, 8, 0, 1),       # lda < K
+    (8, 8, 16, 16, 8, 8, 0, 1),       # ldb < K
+    (8, 8, 16, 16, 16, 4, 0, 1),      # ldc < N
+    (8, 8, 16, 16, 16, 8, 5, 2),      # unknown output dtype
+    (8, 8, 24, 24, 32, 8, 0, 2),      # K not a multiple of 16 (TMA K steps of 16 bytes)
+    (8, 8, 16, 24, 16, 8, 0, 2),      # lda not a multiple of 16 bytes
+    (8, 10, 16, 16, 16, 10, 0, 2),    # fp32 rows not 16-byte multiples
+    (8, 12, 16, 16, 16, 12, 1, 2),    # bf16 rows not 16-byte multiples
+])
+def test_gemm_fp8_rejects(M, N, K, lda, ldb, ldc, cd, code):
+    lib = mgt.load_library()
+    assert lib.mgt_gemm_fp8(M, N, K, P16, lda, P16, ldb, P16, P16, P16, cd, ldc, P16,
+                            None) == code
+
+
+def test_gemm_fp8_rejects_null_and_misaligned_pointers():
+    lib = mgt.load_library()
+    assert lib.mgt_gemm_fp8(8, 8, 16, None, 16, P16, 16, P16, P16, P16, 0, 8, P16, None) == 1
+    assert lib.mgt_gemm_fp8(8, 8, 16, P16, 16, P16, 16, P16, P16, P16, 0, 8, None, None) == 1
+    assert lib.mgt_gemm_fp8(8, 8, 16, P_ODD, 16, P16, 16, P16, P16, P16, 0, 8, P16, None) == 2
+    assert lib.mgt_gemm_fp8(8, 8, 16, P16, 16, P16, 16, P16, P16, P_ODD, 0, 8, P16, None) == 2
