@@ -34,16 +34,18 @@ template <int D>
 struct FwdLayout {
   static constexpr int CH = D / 64;              // 64-wide (128-byte) swizzle chunks per row
   static constexpr int TILE = 128 * D * 2;       // one 128-row Q, K or V tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE;             // 2 stages
+  static constexpr int Q_OFF = 0;                // 2 tiles: query blocks q0 and q0 + 1
+  static constexpr int K_OFF = 2 * TILE;         // 2 stages
   static constexpr int V_OFF = K_OFF + 2 * TILE; // 2 stages
   static constexpr int BAR_OFF = V_OFF + 2 * TILE;
   static constexpr int BYTES = BAR_OFF + 256 + 1024;
-  static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
+  // TMEM per query tile: one S buffer (P packed into its first 64 columns) and one O
+  static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
 };
 
-// Forward CTA: warps 0-3 softmax (one TMEM lane quarter each), warp 4 TMA, warp 5 MMA.
-constexpr int kAttnFwdThreads = 192;
+// Forward CTA: warps 0-3 softmax of query tile 0, warps 4-7 of tile 1 (warp w: TMEM lane
+// quarter w % 4), warp 8 TMA, warp 9 MMA.
+constexpr int kAttnFwdThreads = 320;
 // Backward CTAs: warps 0-7 do the elementwise work on TMEM rows (warp w: TMEM lane quarter w%4,
 // column half w/4), warp 8 is the TMA producer, warp 9 owns TMEM and issues MMAs.
 constexpr int kFwdThreads = 320;
@@ -57,26 +59,26 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_full = bars + 1;    // [2] stages
   uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* k_empty = bars + 5;   // [2]: released as soon as S of that block has read K
-  uint64_t* v_empty = bars + 7;   // [2]: released once PV of that block has read V
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* p_full = bars + 11;   // [2]: P of the block written into its S buffer
-  uint64_t* pv_done = bars + 13;
-  uint64_t* drain = bars + 14;    // every MMA done (one-shot: the output waits on it)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* k_empty = bars + 5;   // [2]: released once every S of that block has read K
+  uint64_t* v_empty = bars + 7;   // [2]: released once every PV of that block has read V
+  uint64_t* s_full = bars + 9;    // [2] per tile: S of the tile's current block is in TMEM
+  uint64_t* p_full = bars + 11;   // [2] per tile: P of the tile's current block is in TMEM
+  uint64_t* drain = bars + 13;    // every MMA done (one-shot: the output waits on it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.s, H = a.H, hp = H / a.p;
-  const int nqb = (S + 127) / 128;
-  // Heads vary fastest in the launch order and query blocks run from the longest rows down,
-  // so every head's longest tiles start in the first wave (longest-processing-time order).
-  const int qb = nqb - 1 - blockIdx.y;
+  const int nqb = (S + 127) / 128, npair = (nqb + 1) / 2;
+  // Heads vary fastest in the launch order and pairs of query blocks run from the longest
+  // rows down (longest-processing-time order). Tile u of the pair is query block q0 + u.
+  const int q0 = 2 * (npair - 1 - (int)blockIdx.y);
+  const bool two = q0 + 1 < nqb;   // the pair has a second tile
+  const int last = two ? q0 + 1 : q0;  // last key block any tile of the pair needs
   const int bh = blockIdx.x, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
-  const int nkv = qb + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -88,13 +90,12 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
     }
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -103,15 +104,17 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
-      mbar_arrive_expect_tx(q_full, L::TILE);
+      mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * L::TILE);
+      for (int u = 0; u < (two ? 2 : 1); ++u)
 #pragma unroll
-      for (int c = 0; c < L::CH; ++c)
-        tma_load_3d(&tm, q_full, smem + L::Q_OFF + c * 16384, col_q + c * 64, qb * 128, b);
+        for (int c = 0; c < L::CH; ++c)
+          tma_load_3d(&tm, q_full, smem + L::Q_OFF + u * L::TILE + c * 16384, col_q + c * 64,
+                      (q0 + u) * 128, b);
       int issued_k = 0, issued_v = 0;
-      for (int kb = 0; kb < nkv; ++kb) {
+      for (int kb = 0; kb <= last; ++kb) {
         const int st = kb & 1;
         if (!mbar_wait(&k_empty[st], ((kb >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
           break;
@@ -137,64 +140,78 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       for (int kb = issued_v - 2 < 0 ? 0 : issued_v - 2; kb < issued_v; ++kb)
         mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
+      // Order per key block kb: S0(kb), S1(kb) | PV0(kb), S0(kb+1), PV1(kb), S1(kb+1) | ...
+      // so that one tile's softmax overlaps the other tile's products. A tile's S(kb+1)
+      // overwrites the P that its PV(kb) reads, and is issued after it (tcgen05.mma
+      // operations of one thread execute in issue order); the commit of S(kb+1) therefore
+      // also covers PV(kb), so the softmax may rescale O once it has seen S(kb+1).
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
       bool ok = mbar_wait(q_full, 0, a.err, kErrTimeoutAttn, abort_flag);
-      auto issue_s = [&](int kb) -> bool {
+      auto issue_s = [&](int u, int kb) -> bool {  // S_u = Q_u K_kb^T
         const int st = kb & 1;
         if (!mbar_wait(&k_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
           return false;
         tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF + u * L::TILE);
         const uint32_t k_addr = smem_u32(smem + L::K_OFF + st * L::TILE);
-        const uint32_t d = tmem + (st ? L::TMEM_S1 : L::TMEM_S0);
+        const uint32_t d = tmem + (u ? L::TMEM_S1 : L::TMEM_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
           tc_mma_f16(d, smem_desc_sw128(q_addr + off, 16, 1024),
                      smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[st]);
-        tc_commit(&k_empty[st]);  // K is free once this S has been computed
+        tc_commit(&s_full[u]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int kb = 0; kb < nkv && ok; ++kb) {
-        // S buffer (kb+1)&1 held block kb-1: its softmax finished reading it (p_full of kb-1
-        // was waited for below, one iteration ago) and its PV, which read P from it, was
-        // issued before this S by this thread (MMAs execute in issue order).
-        if (kb + 1 < nkv && !issue_s(kb + 1)) break;
-        if (!mbar_wait(&p_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
-          break;
+      auto issue_pv = [&](int u, int kb) -> bool {  // O_u += P_u V_kb
+        if (!mbar_wait(&p_full[u], kb & 1, a.err, kErrTimeoutAttn, abort_flag)) return false;
         if (!mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
-          break;
+          return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + L::V_OFF + (kb & 1) * L::TILE);
-        const uint32_t p_tmem = tmem + ((kb & 1) ? L::TMEM_S1 : L::TMEM_S0);
+        const uint32_t p_tmem = tmem + (u ? L::TMEM_S1 : L::TMEM_S0);
+        const uint32_t o_tmem = tmem + (u ? L::TMEM_O1 : L::TMEM_O0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA (8 packed P columns)
-          tc_mma_f16_tmem_a(tmem + L::TMEM_O, p_tmem + kk * 8,
+          tc_mma_f16_tmem_a(o_tmem, p_tmem + kk * 8,
                             smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
                             (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(pv_done);
-        tc_commit(&v_empty[kb & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0, 0);
+      if (ok && two) ok = issue_s(1, 0);
+      if (ok) tc_commit(&k_empty[0]);  // every S of block 0 is issued
+      for (int kb = 0; kb <= last && ok; ++kb) {
+        const bool a_on = kb <= q0, a_next = kb + 1 <= q0;  // tile 0 needs blocks 0..q0
+        const bool b_next = two && kb + 1 <= last;          // tile 1 needs blocks 0..q0+1
+        if (a_on && !(ok = issue_pv(0, kb))) break;
+        if (a_next && !(ok = issue_s(0, kb + 1))) break;
+        if (two && !(ok = issue_pv(1, kb))) break;
+        tc_commit(&v_empty[kb & 1]);  // every PV reading V of block kb is issued
+        if (b_next && !(ok = issue_s(1, kb + 1))) break;
+        if (a_next || b_next) tc_commit(&k_empty[(kb + 1) & 1]);
       }
       tc_commit(drain);
       mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
-    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int u = warp >> 2;                 // query tile of this warp group
+    const int qb = q0 + u;
+    const int r = (warp & 3) * 32 + lane;    // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = u ? L::TMEM_S1 : L::TMEM_S0;
+    const uint32_t o_col = u ? L::TMEM_O1 : L::TMEM_O0;
+    const int nkv = (u == 0 || two) ? qb + 1 : 0;  // no blocks for a missing second tile
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int kb = 0; kb < nkv; ++kb) {
-      const int st = kb & 1;
-      const uint32_t s_col = st ? L::TMEM_S1 : L::TMEM_S0;
-      ok = mbar_wait(&s_full[st], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      ok = mbar_wait(&s_full[u], kb & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -240,28 +257,7 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       }
       l_run = l_run * alpha +
               (((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7])));
-      if (kb > 0) {
-        // PV of the previous block must be done before O is rescaled (waited every block,
-        // so the barrier's phases are followed one by one).
-        ok = mbar_wait(pv_done, (kb - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            const uint32_t ta = lane_base + L::TMEM_O + c * 32;
-            tmem_ld_32x32b_x32(ta, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st_32x32b_x32(ta, o);
-          }
-        }
-      }
-      // P (bf16 pairs) into the first 64 columns of this block's S buffer: this thread's own
+      // P (bf16 pairs) into the first 64 columns of this tile's S buffer: this thread's own
       // row, read completely above, so nothing else is overwritten.
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -271,12 +267,25 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
           pw[j] = __uint_as_float(pack_bf16x2(sv[c * 64 + 2 * j], sv[c * 64 + 2 * j + 1]));
         tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);
       }
+      // O holds the sum up to block kb-1 (its PV completed before this S was committed); it
+      // is rescaled before this block's PV, which waits for p_full below.
+      if (kb > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          const uint32_t ta = lane_base + o_col + c * 32;
+          tmem_ld_32x32b_x32(ta, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st_32x32b_x32(ta, o);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[st]);
+      if (lane == 0) mbar_arrive(&p_full[u]);
     }
-    if (ok) {
+    if (ok && nkv > 0) {
       // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
       ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
@@ -288,7 +297,7 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          tmem_ld_32x32b_x32(lane_base + L::TMEM_O + c * 32, o);
+          tmem_ld_32x32b_x32(lane_base + o_col + c * 32, o);
           if (qrow < S) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -934,7 +943,8 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   const uint64_t strides[2] = {three_h, three_h * a.s};
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
-  dim3 grid(a.b * a.H, (a.s + 127) / 128);
+  // one CTA per pair of 128-query blocks of one head
+  dim3 grid(a.b * a.H, ((a.s + 127) / 128 + 1) / 2);
   attn_fwd_tc_kernel<D><<<grid, kAttnFwdThreads, L::BYTES, s>>>(tm, a,
                                                                 kLog2eF / sqrtf((float)D));
   return cudaGetLastError();
