@@ -48,7 +48,7 @@ struct FwdLayout {
 constexpr int kAttnFwdThreads = 320;
 // Backward CTAs: warps 0-7 do the elementwise work on TMEM rows (warp w: TMEM lane quarter w%4,
 // column half w/4), warp 8 is the TMA producer, warp 9 owns TMEM and issues MMAs.
-constexpr int kFwdThreads = 320;
+constexpr int kBwdThreads = 320;
 
 template <int D>
 __global__ void __launch_bounds__(kAttnFwdThreads, 1)
@@ -359,7 +359,7 @@ struct BwdLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                             const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
                             float scale_log2, float scale) {
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                           const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
                           float scale_log2, float scale) {
@@ -917,11 +917,11 @@ cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
   const float scale = 1.f / sqrtf((float)D);
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
   // The dQ kernel goes first: it also forms D = rowsum(dO * O), which the dK/dV kernel reads.
-  attn_bwd_dq_tc_kernel<D><<<grid, kFwdThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
+  attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, L::B_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                   kLog2eF * scale, scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc_kernel<D><<<grid, kFwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kBwdThreads, L::A_BYTES, s>>>(tm_qkv, tm_do, a,
                                                                     kLog2eF * scale, scale);
   return cudaGetLastError();
 }

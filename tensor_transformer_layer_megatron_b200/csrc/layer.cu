@@ -213,14 +213,25 @@ mgt_status ensure_device(mgt_layer* L) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// The backward's second stream (non-blocking) and its events, created on first use.
+// The backward's second stream (non-blocking) and its events, created on first use; on a
+// failure everything created so far is released and the next call tries again.
 cudaError_t ensure_side_stream(mgt_layer* L) {
   if (L->side) return cudaSuccess;
-  cudaError_t e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
-  for (int i = 0; i < 4 && e == cudaSuccess; ++i)
-    e = cudaEventCreateWithFlags(&L->ev_fork[i], cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);
-  return e;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev[5] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+  for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+    e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    for (auto& x : ev)
+      if (x) cudaEventDestroy(x);
+    if (side) cudaStreamDestroy(side);
+    return e;
+  }
+  for (int i = 0; i < 4; ++i) L->ev_fork[i] = ev[i];
+  L->ev_join = ev[4];
+  L->side = side;
+  return cudaSuccess;
 }
 
 // Every parameter (and gradient) pointer must be set and 16-byte aligned, except the four
