@@ -15,3 +15,4 @@ from .layer import (  # noqa: F401
     all_gather_seq, reduce_scatter_seq, layer_fwd_sp, layer_bwd_sp,
 )
 from .fp8 import E4M3_MAX, e4m3_round, quantize_e4m3, gemm_fp8  # noqa: F401
+from .tp_dist import rank_shard, layer_fwd_rank, layer_bwd_rank  # noqa: F401
