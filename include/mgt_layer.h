@@ -266,6 +266,42 @@ mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int32_t h, con
                                      const float* mean, const float* rstd, void* dx,
                                      float* dgamma, float* dbeta, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * One rank of a real tensor-parallel group. The page "Megatron-LM 3D并行原理与万亿参数训练实战指南"
+ * (trdm.cn), section 2.1, sums the row-parallel layers' partial outputs across the ranks with
+ * an AllReduce; the backward's two reductions (the gradients of the replicated inputs of the
+ * column-parallel layers) are its adjoint. A rank holds shard `rank` of the packed parameters:
+ * w_qkv [3][H/p][d][h], b_qkv [3][H/p][d], w_o [h][h/p], w1 [f/p][h] (swiglu: [2][f/p][h]),
+ * b1 [f/p] ([2][f/p]), w2 [h][f/p], and ln1_g, ln1_b, b_o, ln2_g, ln2_b, b2 whole; gradients
+ * have the same shapes (fp32). x, dy are the whole [b, s, h] on every rank; y, dx come out
+ * whole on every rank.
+ *
+ * The caller provides the reduction: `allreduce(buf, count, user, stream)` must replace the
+ * `count` fp32 values at device address `buf` by their sum over all ranks, ordered on
+ * `stream` (work already on `stream` has produced this rank's values; work enqueued after the
+ * callback returns reads the sum), and return MGT_OK. It is called 2 times per forward
+ * (out-proj and fc2 partials) and 2 times per backward (dln2 and dln1 contributions), with
+ * the same `buf` (the workspace region reported by mgt_tp_rank_partial), in that order on
+ * every rank. bf16 layers only; sequence parallelism is not supported here
+ * (MGT_EUNSUPPORTED). Everything runs on `stream`. */
+typedef mgt_status (*mgt_allreduce_fn)(float* buf, int64_t count, void* user, void* stream);
+typedef struct mgt_tp_rank mgt_tp_rank; /* opaque handle, host memory only */
+
+/* Validate `cfg` (as mgt_layer_init) and 0 <= rank < tp_size; create the rank's handle.
+ * Host only. */
+mgt_status mgt_tp_rank_init(const mgt_layer_config* cfg, int32_t rank, mgt_tp_rank** out);
+mgt_status mgt_tp_rank_sizes(const mgt_tp_rank* r, size_t* saved_bytes, size_t* workspace_bytes);
+/* Offset and size in `workspace` of the fp32 [T, h] buffer the reductions run on. */
+mgt_status mgt_tp_rank_partial(const mgt_tp_rank* r, size_t* offset, size_t* bytes);
+mgt_status mgt_tp_rank_fwd(mgt_tp_rank* r, const mgt_layer_params* shard, const void* x, void* y,
+                           void* saved, void* workspace, mgt_allreduce_fn allreduce, void* user,
+                           void* stream);
+mgt_status mgt_tp_rank_bwd(mgt_tp_rank* r, const mgt_layer_params* shard, const void* x,
+                           const void* saved, const void* dy, void* dx,
+                           const mgt_layer_grads* grads, void* workspace,
+                           mgt_allreduce_fn allreduce, void* user, void* stream);
+void mgt_tp_rank_destroy(mgt_tp_rank* r);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,11 @@ class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in PARAM_ORDER]
 
 
+# mgt_allreduce_fn: (float* buf, int64 count, void* user, void* stream) -> mgt_status
+ALLREDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                ctypes.c_void_p)
+
+
 class _KernelStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
                 ("ms", ctypes.c_double), ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -89,6 +94,15 @@ def load_library():
     lib.mgt_fp8_quantize.argtypes = [i32, ctypes.c_int64, vp, vp, vp, vp]
     lib.mgt_gemm_fp8.argtypes = [i32, i32, i32, vp, ctypes.c_int64, vp, ctypes.c_int64, vp, vp,
                                  vp, i32, ctypes.c_int64, vp, vp]
+    lib.mgt_tp_rank_init.argtypes = [ctypes.POINTER(_Config), i32, ctypes.POINTER(vp)]
+    lib.mgt_tp_rank_sizes.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.mgt_tp_rank_partial.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.mgt_tp_rank_fwd.argtypes = [vp, ctypes.POINTER(_Params), vp, vp, vp, vp, ALLREDUCE_FN,
+                                    vp, vp]
+    lib.mgt_tp_rank_bwd.argtypes = [vp, ctypes.POINTER(_Params), vp, vp, vp, vp,
+                                    ctypes.POINTER(_Params), vp, ALLREDUCE_FN, vp, vp]
+    lib.mgt_tp_rank_destroy.argtypes = [vp]
+    lib.mgt_tp_rank_destroy.restype = None
     lib.mgt_debug_bounded_wait.argtypes = [ctypes.c_int64, vp, vp]
     lib.mgt_layer_status_word.argtypes = [vp, vp, ctypes.POINTER(vp)]
     lib.mgt_debug_bounded_wait.restype = ctypes.c_int
@@ -96,7 +110,8 @@ def load_library():
     for name in ("mgt_layer_init", "mgt_layer_sizes", "mgt_layer_region", "mgt_layer_fwd",
                  "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
                  "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc",
-                 "mgt_fp8_quantize", "mgt_gemm_fp8"):
+                 "mgt_fp8_quantize", "mgt_gemm_fp8", "mgt_tp_rank_init", "mgt_tp_rank_sizes",
+                 "mgt_tp_rank_partial", "mgt_tp_rank_fwd", "mgt_tp_rank_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -238,6 +253,80 @@ class Layer:
         return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms,
                                            flops=arr[i].flops, bytes=arr[i].bytes)
                 for i in range(n.value)}
+
+
+class TPRank:
+    """One rank of a real tensor-parallel group (see mgt_tp_rank_* in include/mgt_layer.h):
+    the rank's shard of the packed parameters, whole x / dy / y / dx, and a caller-provided
+    all-reduce.
+
+    allreduce(ptr, count, stream_handle) -> None must replace the `count` fp32 values at device
+    address `ptr` by their sum over all ranks, ordered on the CUDA stream `stream_handle`
+    (an int, 0 for the default stream). It is called 2 times per fwd and 2 per bwd, always on
+    the workspace region `partial_region()` names. bf16 only."""
+
+    def __init__(self, hidden, heads, ffn, seq, micro_batch, tp_size, rank, ln_eps=1e-5,
+                 gelu_tanh=0, swiglu=0, disable_bias_linear=0):
+        self.lib = load_library()
+        self.cfg = _Config(hidden, heads, ffn, seq, micro_batch, tp_size, 1, 1, ln_eps, 1,
+                           gelu_tanh, swiglu, disable_bias_linear, 0)
+        self.dtype = "bf16"
+        self.has_bias = not disable_bias_linear
+        h = ctypes.c_void_p()
+        _check(self.lib.mgt_tp_rank_init(ctypes.byref(self.cfg), rank, ctypes.byref(h)),
+               "mgt_tp_rank_init")
+        self.handle = h
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            self.lib.mgt_tp_rank_destroy(h)
+            self.handle = None
+
+    def sizes(self):
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(self.lib.mgt_tp_rank_sizes(self.handle, ctypes.byref(a), ctypes.byref(b)),
+               "mgt_tp_rank_sizes")
+        return a.value, b.value
+
+    def partial_region(self):
+        o, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(self.lib.mgt_tp_rank_partial(self.handle, ctypes.byref(o), ctypes.byref(n)),
+               "mgt_tp_rank_partial")
+        return o.value, n.value
+
+    def alloc_buffers(self, device="cuda"):
+        import torch
+        s, w = self.sizes()
+        return (torch.empty(max(s, 256), dtype=torch.uint8, device=device),
+                torch.zeros(max(w, 256), dtype=torch.uint8, device=device))
+
+    @staticmethod
+    def _callback(allreduce):
+        def cb(ptr, count, user, stream):
+            try:
+                allreduce(ptr, count, stream or 0)
+                return 0
+            except Exception:  # noqa: BLE001 - reported to the C side as a CUDA-class error
+                import traceback
+                traceback.print_exc()
+                return 3
+        return ALLREDUCE_FN(cb)
+
+    def fwd(self, params, x, y, saved, workspace, allreduce, stream=None):
+        Layer._check_types(self, params, (x, y))
+        cb = self._callback(allreduce)
+        _check(self.lib.mgt_tp_rank_fwd(self.handle, ctypes.byref(Layer._params(params)),
+                                        _ptr(x), _ptr(y), _ptr(saved), _ptr(workspace), cb,
+                                        None, _stream_handle(stream)), "mgt_tp_rank_fwd")
+
+    def bwd(self, params, x, saved, dy, dx, grads, workspace, allreduce, stream=None):
+        Layer._check_types(self, params, (x, dy, dx), grads)
+        cb = self._callback(allreduce)
+        _check(self.lib.mgt_tp_rank_bwd(self.handle, ctypes.byref(Layer._params(params)),
+                                        _ptr(x), _ptr(saved), _ptr(dy), _ptr(dx),
+                                        ctypes.byref(Layer._params(grads)), _ptr(workspace),
+                                        cb, None, _stream_handle(stream)), "mgt_tp_rank_bwd")
 
 
 def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):

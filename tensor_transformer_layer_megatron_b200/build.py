@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmgt.so")
 SOURCES = ["gemm_tc.cu", "attn.cu", "attn_tc.cu", "ln_misc.cu", "layer.cu", "ln_noalloc.cu",
-           "fp8.cu"]
+           "fp8.cu", "layer_tp.cu"]
 HEADERS = ["mgt_device.cuh", "mgt_internal.h"]
 
 

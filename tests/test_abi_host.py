@@ -16,6 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "mgt_layer.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"typedef[^;]*;", "", src)  # type declarations (a function-pointer type too)
     return sorted(set(re.findall(r"\b(mgt_[a-z0-9_]+)\s*\(", src)))
 
 
@@ -151,3 +152,33 @@ def test_gemm_fp8_rejects_null_and_misaligned_pointers():
     assert lib.mgt_gemm_fp8(8, 8, 16, P16, 16, P16, 16, P16, P16, P16, 0, 8, None, None) == 1
     assert lib.mgt_gemm_fp8(8, 8, 16, P_ODD, 16, P16, 16, P16, P16, P16, 0, 8, P16, None) == 2
     assert lib.mgt_gemm_fp8(8, 8, 16, P16, 16, P16, 16, P16, P16, P_ODD, 0, 8, P16, None) == 2
+
+
+def test_tp_rank_init_validates():
+    lib = mgt.load_library()
+    base = dict(hidden=256, heads=4, ffn=512, seq=128, micro_batch=2, tp_size=2)
+
+    def init(rank, **kw):
+        c = dict(base, **kw)
+        cfg = mgt._Config(c["hidden"], c["heads"], c["ffn"], c["seq"], c["micro_batch"],
+                          c["tp_size"], c.get("dtype", 1), 1, 1e-5, 1, 0, 0, 0,
+                          c.get("sp", 0))
+        h = ctypes.c_void_p()
+        st = lib.mgt_tp_rank_init(ctypes.byref(cfg), rank, ctypes.byref(h))
+        if st == 0:
+            lib.mgt_tp_rank_destroy(h)
+        return st
+
+    assert init(0) == 0 and init(1) == 0
+    assert init(2) == 1 and init(-1) == 1                    # rank outside the group
+    assert init(0, dtype=0) == 2                              # bf16 only
+    assert init(0, sp=1) == 2                                 # no sequence parallelism here
+    assert init(0, heads=3) == 1                              # the layer itself is invalid
+    r = mgt.TPRank(256, 4, 512, 128, 2, 2, 1)
+    saved, ws = r.sizes()
+    off, n = r.partial_region()
+    assert n == 256 * 256 * 4 and off % 256 == 0 and off + n <= ws
+    # null pointers and a missing all-reduce are rejected before any CUDA call
+    null = mgt._Params(*([None] * 12))
+    assert lib.mgt_tp_rank_fwd(r.handle, ctypes.byref(null), None, None, None, None,
+                               mgt.ALLREDUCE_FN(0), None, None) == 1
