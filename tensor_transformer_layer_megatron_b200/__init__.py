@@ -329,6 +329,28 @@ class TPRank:
                                         cb, None, _stream_handle(stream)), "mgt_tp_rank_bwd")
 
 
+def process_group_allreduce(workspace, offset, group=None):
+    """The all-reduce a TPRank needs, over a torch.distributed process group (NCCL for device
+    workspaces): the callback views the `count` fp32 values at `offset` of `workspace` (the
+    rank's partial buffer, TPRank.partial_region()) and sums them over the group in place,
+    on the stream the layer passes (torch.distributed enqueues the collective there). Every
+    rank of the group must make the same TPRank calls in the same order."""
+    import torch
+    import torch.distributed as dist
+    base = workspace.data_ptr()
+
+    def allreduce(ptr, count, stream):
+        if ptr != base + offset or count * 4 + offset > workspace.numel():
+            raise ValueError("all-reduce buffer outside the rank's workspace")
+        view = workspace[offset:offset + 4 * count].view(torch.float32)
+        if workspace.is_cuda:
+            with torch.cuda.stream(torch.cuda.ExternalStream(stream, device=workspace.device)):
+                dist.all_reduce(view, group=group)
+        else:
+            dist.all_reduce(view, group=group)
+    return allreduce
+
+
 def gemm_bf16(A, B, C, M, N, K, a_mn, b_mn, lda, ldb, ldc, status, stream=None):
     """C[m, n] = sum_k A(m, k) B(n, k) on the tcgen05 path (see mgt_gemm_bf16)."""
     import torch
