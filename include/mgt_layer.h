@@ -46,14 +46,19 @@
  *   - dtype MGT_BF16: activations, weights and biases are bf16; LN gamma/beta are fp32.
  *     dtype MGT_F32: everything fp32. All gradients of parameters are written in fp32 and
  *     OVERWRITTEN (not accumulated); dx is in the activation dtype.
- *   - All device pointers are owned by the caller. The handle owns host state only (config,
- *     derived sizes, optional profiling events). Calls are asynchronous on `stream`
- *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - All device pointers are owned by the caller. The handle owns host state (config,
+ *     derived sizes) and a few CUDA objects: optional profiling events, and the backward's
+ *     second stream with its fork/join events (created by the first mgt_layer_bwd). Calls are
+ *     asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream).
  *   - The library never allocates device memory. `saved` (written by fwd, read by bwd) and
  *     `workspace` are caller buffers of the sizes mgt_layer_sizes reports, 256-byte aligned.
  *     The first 256 bytes of `workspace` hold the device status word: zero the workspace once
  *     after allocating it; device errors accumulate there until mgt_layer_get_error reads and
  *     clears them.
+ *
+ * The same block split over real tensor-parallel ranks (one shard per rank, the four shard
+ * sums done by a caller-provided all-reduce) is the mgt_tp_rank_* API at the end of this file.
  *
  * Errors: synchronous validation returns MGT_EINVAL / MGT_EUNSUPPORTED without touching the
  * GPU; a failed launch returns MGT_ECUDA; a device-side bounded wait that runs out records
