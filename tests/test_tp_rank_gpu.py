@@ -132,3 +132,28 @@ def test_tp_ranks_match_oracle(cfg):
             errs["d_" + k] = rel_err(b["grads"][k].double().cpu().numpy(), np.asarray(want))
         bad = {k: v for k, v in errs.items() if v > 2e-2}
         assert not bad, (r, bad, errs)
+
+
+def test_tp_rank_reports_a_failed_allreduce():
+    """A collective that fails (here: the callback raises) ends the rank's call with an error
+    status instead of a hang, and leaves the context usable."""
+    cfg = CASES[0]
+    t = make_inputs(cfg)
+    packed = pack_params(cfg, t)
+    dev = torch.device("cuda", 0)
+    rk = mgt.TPRank(cfg.hidden, cfg.heads, cfg.ffn, cfg.seq, cfg.micro_batch, cfg.tp_size, 0)
+    shard = {k: (v[0] if k in SHARDED else v)
+             .to(device=dev, dtype=torch.float32 if k in LN else torch.bfloat16).contiguous()
+             for k, v in packed.items()}
+    x = t["x"].to(device=dev, dtype=torch.bfloat16).contiguous()
+    y = torch.empty_like(x)
+    saved, ws = rk.alloc_buffers(dev)
+
+    def failing(ptr, count, stream):
+        raise RuntimeError("collective failed")
+
+    with pytest.raises(mgt.MgtError) as ei:
+        rk.fwd(shard, x, y, saved, ws, failing)
+    assert ei.value.code == 3
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
