@@ -48,9 +48,10 @@
  *     OVERWRITTEN (not accumulated); dx is in the activation dtype.
  *   - All device pointers are owned by the caller. The handle owns host state (config,
  *     derived sizes) and a few CUDA objects: optional profiling events, and the backward's
- *     second stream with its fork/join events (created by the first mgt_layer_bwd). Calls are
- *     asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
- *     stream).
+ *     second stream with its fork/join events (created by the first mgt_layer_bwd). A handle
+ *     binds to the device current at its first fwd/bwd call; a call from another device
+ *     returns MGT_EUNSUPPORTED. Calls are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = legacy default stream).
  *   - The library never allocates device memory. `saved` (written by fwd, read by bwd) and
  *     `workspace` are caller buffers of the sizes mgt_layer_sizes reports, 256-byte aligned.
  *     The first 256 bytes of `workspace` hold the device status word: zero the workspace once

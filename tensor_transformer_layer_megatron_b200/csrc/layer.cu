@@ -55,6 +55,7 @@ struct mgt_layer {
   Region ws[MGT_WS_COUNT - 64];
   size_t saved_bytes = 0, ws_bytes = 0;
   int num_sms = 0;
+  int device = -1;  // the device the handle is bound to (at its first call)
   // second stream of the backward (weight gradients) and its fork / join events
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork[4] = {};
@@ -195,10 +196,12 @@ mgt_status cuda_status(cudaError_t e) {
     if (_e != cudaSuccess) return MGT_ECUDA;   \
   } while (0)
 
+// The handle binds to the device current at its first call (its SM count, its backward
+// stream); a later call from another device is rejected.
 mgt_status ensure_device(mgt_layer* L) {
-  if (L->num_sms > 0) return MGT_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MGT_ECUDA;
+  if (L->num_sms > 0) return dev == L->device ? MGT_OK : MGT_EUNSUPPORTED;
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return MGT_ECUDA;
@@ -208,6 +211,7 @@ mgt_status ensure_device(mgt_layer* L) {
     if (major != 10) return MGT_EUNSUPPORTED;  // tcgen05 / TMA kernels are built for sm_100a
   }
   L->num_sms = n;
+  L->device = dev;
   return MGT_OK;
 }
 

@@ -102,6 +102,7 @@ struct mgt_tp_rank {
   Reg saved[S_COUNT], ws[W_COUNT];
   size_t saved_bytes = 0, ws_bytes = 0;
   int num_sms = 0;
+  int device = -1;
 };
 
 namespace {
@@ -119,15 +120,17 @@ void place(Reg* r, int n, const size_t* bytes, size_t* total) {
 char* at(void* base, const Reg& r) { return static_cast<char*>(base) + r.off; }
 const char* at(const void* base, const Reg& r) { return static_cast<const char*>(base) + r.off; }
 
+// bound to the device current at the first call, like the layer handle
 mgt_status ensure(mgt_tp_rank* R) {
-  if (R->num_sms > 0) return MGT_OK;
   int dev = 0, n = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MGT_ECUDA;
+  if (R->num_sms > 0) return dev == R->device ? MGT_OK : MGT_EUNSUPPORTED;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return MGT_ECUDA;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   if (major != 10) return MGT_EUNSUPPORTED;
   R->num_sms = n;
+  R->device = dev;
   return MGT_OK;
 }
 
