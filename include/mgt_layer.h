@@ -262,11 +262,15 @@ mgt_status mgt_layer_status_word(mgt_layer* layer, void* workspace, int32_t** wo
  * i.e. the LayerNorm backward of mgt_layer_bwd. dtype: MGT_BF16 (dy, dres, x, dx bf16) or
  * MGT_F32; gamma, mean, rstd, dgamma, dbeta fp32. dres may be NULL. h must be a multiple of 8
  * (bf16) or 4 (f32) and at most 16384 (bf16) / 8192 (f32), else MGT_EUNSUPPORTED.
+ * Alignment: dy, dres, x, dx and gamma 16-byte aligned; mean, rstd, dgamma, dbeta 4-byte
+ * aligned; otherwise MGT_EUNSUPPORTED before anything is launched.
  * Its per-block partial sums live in a fixed 4 MiB array of the library's own device memory,
  * held on every GPU that loads the library until the process exits. The first call on each
- * device looks up that array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture. All calls share the array: calls that overlap on the GPU (other
- * streams, other threads) race on it, so serialise them. Allocates no memory. */
+ * device looks up that array's device address (cudaGetSymbolAddress) and keeps it for the
+ * life of the process: make that first call before any stream capture, and do not reset the
+ * device (cudaDeviceReset) after it. All calls share the array: calls that overlap on the GPU
+ * (other streams, other threads) race on it, so serialise them. The kernels it launches wait
+ * on nothing on the device, so there is no timeout to report. Allocates no memory. */
 mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int32_t h, const void* dy,
                                      const void* dres, const void* x, const float* gamma,
                                      const float* mean, const float* rstd, void* dx,

@@ -998,7 +998,9 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
     const T* px = reinterpret_cast<const T*>(x);
     T* pdx = reinterpret_cast<T*>(dx);
     const unsigned gs = (unsigned)slices;
-    const bool ring = nvec >= 256 && aligned16_ptr(x) && aligned16_ptr(dy) &&
+    // The ring kernel's waits are bounded and report a run-out through `err`; a caller with
+    // no status word gets the wait-free kernels, so a timeout can never go unreported.
+    const bool ring = err && nvec >= 256 && aligned16_ptr(x) && aligned16_ptr(dy) &&
                       (!dres || aligned16_ptr(dres));
     if (ring) {
       // x, dy (and dres) rows streamed through the shared-memory ring

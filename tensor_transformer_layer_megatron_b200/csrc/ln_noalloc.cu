@@ -9,9 +9,14 @@
 // The array is a file-scope __device__ symbol, so every GPU that loads the library holds it
 // until the process exits. Host code must not pass the symbol itself to a kernel (on the host
 // it names a host-side shadow, not device memory); the device address is looked up once per
-// device with cudaGetSymbolAddress and cached.
+// device with cudaGetSymbolAddress and cached for the life of the process, so a device reset
+// (cudaDeviceReset) after the first call on that device is not supported.
+//
+// This entry point has no status word to report a device-side wait that runs out, so it only
+// uses the LayerNorm backward kernels that wait on nothing (never the bulk-copy ring).
 #include <cuda_runtime.h>
 
+#include <cstdint>
 #include <mutex>
 
 #include "../../include/mgt_layer.h"
@@ -55,6 +60,15 @@ extern "C" mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int
   const int vec = dtype == MGT_BF16 ? 8 : 4;
   const int hmax = dtype == MGT_BF16 ? 16384 : 8192;
   if (h % vec || h > hmax) return MGT_EUNSUPPORTED;
+  // The kernels move rows and gamma in 16-byte vectors and the statistics and parameter
+  // gradients as floats; reject misaligned views here, before anything reaches the GPU.
+  auto aligned = [](const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+  };
+  if (!aligned(dy, 16) || !aligned(x, 16) || !aligned(dx, 16) || !aligned(gamma, 16) ||
+      (dres && !aligned(dres, 16)) || !aligned(mean, 4) || !aligned(rstd, 4) ||
+      !aligned(dgamma, 4) || !aligned(dbeta, 4))
+    return MGT_EUNSUPPORTED;
   // One partial row pair (dgamma, dbeta) per block; as many blocks as the array holds.
   long long nblk = kScratchFloats / (2LL * h);
   if (nblk > kMaxBlocks) nblk = kMaxBlocks;
@@ -62,7 +76,8 @@ extern "C" mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int
   float* scratch = nullptr;
   mgt_status st = scratch_for_current_device(&scratch);
   if (st != MGT_OK) return st;
-  // Every partial row is written before it is read, so the array needs no clearing.
+  // Every partial row is written before it is read, so the array needs no clearing. With no
+  // status word (err = nullptr) the dispatch picks kernels without device-side waits.
   cudaError_t e = mgt::launch_ln_bwd(dtype == MGT_BF16 ? 1 : 0, rows, h, dy, dres, x, gamma,
                                      mean, rstd, dx, scratch, (int)nblk, dgamma, dbeta,
                                      nullptr, nullptr, static_cast<cudaStream_t>(stream));

@@ -51,10 +51,16 @@ def run_gpu(cfg, t):
 
 
 def gpu_intermediates(cfg, layer, run):
+    """Every saved / workspace intermediate of the GPU layer, as zero-argument fetchers (each
+    copies one tensor to the host only when called, so the largest layers compare one tensor
+    at a time)."""
     T, h, f, p, H = cfg.tokens, cfg.hidden, cfg.ffn, cfg.tp_size, cfg.heads
     d = h // H
     act = run.act
-    v = lambda buf, n, dt, shp: to_np(layer.view(buf, n, dt, shp))  # noqa: E731
+
+    def v(buf, n, dt, shp):
+        return lambda: to_np(layer.view(buf, n, dt, shp))
+
     out = dict(
         ln1=v(run.saved, "ln1", act, (T, h)),
         qkv=v(run.saved, "qkv", act, (T, p, 3, H // p, d)),
@@ -86,12 +92,14 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
     x, dy = layer_io(cfg, t)
     y_ref, saved = oracle.layer_fwd(cfg, packed, x)
     dx_ref, g_ref, inter = oracle.layer_bwd(cfg, packed, saved, dy)
+    del t, x, dy
     errs = {"y": rel_err(to_np(run.y), y_ref), "dx": rel_err(to_np(run.dx), dx_ref)}
+    del y_ref, dx_ref
     # a layer without linear biases has no bias gradients on either side
     assert set(run.grads) == set(g_ref), (sorted(run.grads), sorted(g_ref))
     for k in GRAD_NAMES:
         if k in g_ref:
-            errs["d_" + k] = rel_err(to_np(run.grads[k]), g_ref[k])
+            errs["d_" + k] = rel_err(to_np(run.grads[k]), g_ref.pop(k))
     if intermediates:
         gi = gpu_intermediates(cfg, layer, run)
         ref = dict(ln1=saved["ln1"], qkv=saved["qkv"], O=saved["O"], lse=saved["lse"],
@@ -99,7 +107,10 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
         if getattr(cfg, "swiglu", 0):
             ref["u"] = saved["u"]
         else:
-            ref["gelu_grad"] = oracle.gelu_grad(saved["u"], cfg.gelu_tanh)
-        for k in gi:
-            errs[k] = rel_err(gi[k], ref[k])
+            ref["gelu_grad"] = lambda: oracle.gelu_grad(saved["u"], cfg.gelu_tanh)
+        del inter
+        for k, fetch in gi.items():
+            r = ref.pop(k)
+            errs[k] = rel_err(fetch(), r() if callable(r) else r)
+            del r
     return errs

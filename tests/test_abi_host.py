@@ -182,3 +182,19 @@ def test_tp_rank_init_validates():
     null = mgt._Params(*([None] * 12))
     assert lib.mgt_tp_rank_fwd(r.handle, ctypes.byref(null), None, None, None, None,
                                mgt.ALLREDUCE_FN(0), None, None) == 1
+
+
+@pytest.mark.parametrize("bad", ["dy", "dres", "x", "gamma", "mean", "rstd", "dx", "dgamma",
+                                 "dbeta"])
+def test_layernorm_bwd_noalloc_rejects_misaligned_pointers(bad):
+    # The pointers are never dereferenced: validation must reject a misaligned view before any
+    # CUDA call (this host has no GPU, so reaching the device lookup would return MGT_ECUDA).
+    lib = mgt.load_library()
+    ptr = {k: 0x10000 + 0x1000 * i for i, k in enumerate(
+        ("dy", "dres", "x", "gamma", "mean", "rstd", "dx", "dgamma", "dbeta"))}
+    ptr[bad] += 2 if bad in ("mean", "rstd", "dgamma", "dbeta") else 4
+    vp = ctypes.c_void_p
+    st = lib.mgt_layernorm_bwd_noalloc(1, 16, 512, vp(ptr["dy"]), vp(ptr["dres"]), vp(ptr["x"]),
+                                       vp(ptr["gamma"]), vp(ptr["mean"]), vp(ptr["rstd"]),
+                                       vp(ptr["dx"]), vp(ptr["dgamma"]), vp(ptr["dbeta"]), None)
+    assert st == 2, (bad, st)
