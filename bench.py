@@ -369,6 +369,8 @@ def run_mgt(args):
     # the LayerNorm backward is one pass plus a reduce up to 512 16-byte vectors per row
     vec = 8 if cfg.dtype == "bf16" else 4
     per_launch["ln_bwd"] = 2 if cfg.hidden // vec <= 512 else 3
+    # head_dim 128: D pre-pass, the single backward kernel and the dQ conversion
+    per_launch["attn_bwd"] = 3 if cfg.dtype == "bf16" and cfg.hidden // cfg.heads == 128 else 2
     launches = sum(v["launches"] * per_launch.get(k, 1) for k, v in prof.items())
 
     cpu = None

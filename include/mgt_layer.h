@@ -148,8 +148,8 @@ typedef enum mgt_region {
   MGT_SAVED_LN2 = 7,        /* ACT [T, h]                                              */
   MGT_SAVED_LN2_MEAN = 8,   /* F32 [T]                                                 */
   MGT_SAVED_LN2_RSTD = 9,   /* F32 [T]                                                 */
-  MGT_SAVED_FC1_DGELU = 10, /* ACT [T][p][f/p]     GeLU'(u), u = fc1 pre-activation;
-                               swiglu: ACT [T][p][2][f/p], u = [gate | up] itself       */
+  MGT_SAVED_FC1_U = 10,     /* ACT [T][p][f/p]     u, the fc1 pre-activation (bias included);
+                               swiglu: ACT [T][p][2][f/p], u = [gate | up]              */
   MGT_SAVED_FC1_A = 11,     /* ACT [T][p][f/p]     GeLU(u) (swiglu: silu(gate) * up)   */
   MGT_SAVED_COUNT = 12,
   MGT_WS_STATUS = 64,       /* int32 device status word (first 256 bytes)              */
@@ -160,15 +160,19 @@ typedef enum mgt_region {
   MGT_WS_DQKV = 69,         /* ACT [T, 3h]  dL/d qkv (packed like qkv)                 */
   MGT_WS_DLN1 = 70,         /* ACT [T, h]   dL/d ln1                                   */
   MGT_WS_ATTN_D = 71,       /* F32 [b][H][s] rowsum(dO * O)                            */
-  MGT_WS_DQ_ACC = 72,       /* unused (0 bytes): dQ is accumulated in tensor memory     */
+  MGT_WS_DQ_ACC = 72,       /* I32 [T, h]   fixed-point dQ accumulator of the attention
+                               backward, then per-head scaling data (bf16 layers with
+                               head_dim 128; 0 bytes otherwise)                         */
   MGT_WS_LN_PARTIAL = 73,   /* F32 [slices][3][h] LayerNorm dgamma/dbeta/residual-grad partial sums */
-  MGT_WS_COUNT = 74
+  MGT_WS_BIAS_PARTIAL = 74, /* F32 [slices][cols] column-sum partials of the b1 / b_qkv gradients
+                               (0 bytes with disable_bias_linear)                        */
+  MGT_WS_COUNT = 75
 } mgt_region;
 mgt_status mgt_layer_region(const mgt_layer* layer, int region, size_t* offset, size_t* bytes);
 
 /* Forward. Reads x [b,s,h]; writes y [b,s,h] and every region of `saved`.
  * Launch order on `stream`: LN1, QKV GEMM(+bias), attention, out-proj GEMM (+shard sum,
- * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores a and GeLU'(u); swiglu: each tile holds a
+ * +b_o, +x), LN2, fc1 GEMM (+b1, GeLU; stores a and u; swiglu: each tile holds a
  * shard's gate and up columns for the same outputs and stores a and [gate | up]), fc2 GEMM
  * (+shard sum, +b2, +h1). */
 mgt_status mgt_layer_fwd(mgt_layer* layer, const mgt_layer_params* params, const void* x,
@@ -290,10 +294,11 @@ mgt_status mgt_layernorm_bwd_noalloc(int32_t dtype, int64_t rows, int32_t h, con
  * `count` fp32 values at device address `buf` by their sum over all ranks, ordered on
  * `stream` (work already on `stream` has produced this rank's values; work enqueued after the
  * callback returns reads the sum), and return MGT_OK. It is called 2 times per forward
- * (out-proj and fc2 partials) and 2 times per backward (dln2 and dln1 contributions), with
- * the same `buf` (the workspace region reported by mgt_tp_rank_partial), in that order on
- * every rank. bf16 layers only; sequence parallelism is not supported here
- * (MGT_EUNSUPPORTED). Everything runs on `stream`. */
+ * (out-proj and fc2 partials) and 2 times per backward (dln2 and dln1 contributions) --
+ * once per row band with mgt_tp_rank_set_bands -- always inside the workspace region reported
+ * by mgt_tp_rank_partial, in the same order on every rank. bf16 layers only; sequence
+ * parallelism is not supported here (MGT_EUNSUPPORTED). Everything runs on `stream`, except
+ * the banded exchanges (below). */
 typedef mgt_status (*mgt_allreduce_fn)(float* buf, int64_t count, void* user, void* stream);
 typedef struct mgt_tp_rank mgt_tp_rank; /* opaque handle, host memory only */
 
@@ -303,6 +308,19 @@ mgt_status mgt_tp_rank_init(const mgt_layer_config* cfg, int32_t rank, mgt_tp_ra
 mgt_status mgt_tp_rank_sizes(const mgt_tp_rank* r, size_t* saved_bytes, size_t* workspace_bytes);
 /* Offset and size in `workspace` of the fp32 [T, h] buffer the reductions run on. */
 mgt_status mgt_tp_rank_partial(const mgt_tp_rank* r, size_t* offset, size_t* bytes);
+/* Row bands of each shard sum (1 <= bands <= 16; default 1; MGT_EINVAL otherwise). With one
+ * band, the callback gets the whole [T, h] partial once per sum, on `stream`, after the
+ * partial GEMM (and, in the backward, after the weight-gradient GEMM enqueued behind it).
+ * With more, the partial GEMM runs over consecutive row bands (an even split of T rounded up
+ * to multiples of 128 rows) and the callback is made once per band, right after that band's
+ * GEMM is enqueued, with `buf` = the band's first row of the partial buffer, `count` = its
+ * rows * h, and `stream` = the rank's communication stream (created by the first such call on
+ * the bound device): work enqueued there runs after the band's partial is written, and
+ * `stream` waits for every band's exchange before the sum is used. An asynchronous collective
+ * (NCCL) therefore exchanges band i while band i+1 is being computed -- the overlap of
+ * communication with the row-parallel GEMM (--tp-comm-overlap on the vampireachao.github.io
+ * page). Every rank must use the same number of bands. */
+mgt_status mgt_tp_rank_set_bands(mgt_tp_rank* r, int32_t bands);
 mgt_status mgt_tp_rank_fwd(mgt_tp_rank* r, const mgt_layer_params* shard, const void* x, void* y,
                            void* saved, void* workspace, mgt_allreduce_fn allreduce, void* user,
                            void* stream);

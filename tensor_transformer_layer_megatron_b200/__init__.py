@@ -21,9 +21,9 @@ PARAM_ORDER = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
 
 REGIONS = {
     "ln1": 0, "ln1_mean": 1, "ln1_rstd": 2, "qkv": 3, "attn_o": 4, "attn_lse": 5, "h1": 6,
-    "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_dgelu": 10, "fc1_a": 11,
+    "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_u": 10, "fc1_a": 11,
     "status": 64, "du": 65, "dln2": 66, "dh1": 67, "dO": 68, "dqkv": 69, "dln1": 70,
-    "attn_D": 71, "dq_acc": 72, "ln_partial": 73,
+    "attn_D": 71, "dq_acc": 72, "ln_partial": 73, "bias_partial": 74,
 }
 
 STATUS = {0: "MGT_OK", 1: "MGT_EINVAL", 2: "MGT_EUNSUPPORTED", 3: "MGT_ECUDA",
@@ -101,6 +101,7 @@ def load_library():
                                     vp, vp]
     lib.mgt_tp_rank_bwd.argtypes = [vp, ctypes.POINTER(_Params), vp, vp, vp, vp,
                                     ctypes.POINTER(_Params), vp, ALLREDUCE_FN, vp, vp]
+    lib.mgt_tp_rank_set_bands.argtypes = [vp, i32]
     lib.mgt_tp_rank_destroy.argtypes = [vp]
     lib.mgt_tp_rank_destroy.restype = None
     lib.mgt_debug_bounded_wait.argtypes = [ctypes.c_int64, vp, vp]
@@ -111,7 +112,8 @@ def load_library():
                  "mgt_layer_bwd", "mgt_layer_get_error", "mgt_layer_profile",
                  "mgt_layer_profile_read", "mgt_gemm_bf16", "mgt_layernorm_bwd_noalloc",
                  "mgt_fp8_quantize", "mgt_gemm_fp8", "mgt_tp_rank_init", "mgt_tp_rank_sizes",
-                 "mgt_tp_rank_partial", "mgt_tp_rank_fwd", "mgt_tp_rank_bwd"):
+                 "mgt_tp_rank_partial", "mgt_tp_rank_fwd", "mgt_tp_rank_bwd",
+                 "mgt_tp_rank_set_bands"):
         getattr(lib, name).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -262,8 +264,9 @@ class TPRank:
 
     allreduce(ptr, count, stream_handle) -> None must replace the `count` fp32 values at device
     address `ptr` by their sum over all ranks, ordered on the CUDA stream `stream_handle`
-    (an int, 0 for the default stream). It is called 2 times per fwd and 2 per bwd, always on
-    the workspace region `partial_region()` names. bf16 only."""
+    (an int, 0 for the default stream). It is called 2 times per fwd and 2 per bwd (times the
+    number of row bands, set_bands), always inside the workspace region `partial_region()`
+    names; banded calls come on the rank's communication stream. bf16 only."""
 
     def __init__(self, hidden, heads, ffn, seq, micro_batch, tp_size, rank, ln_eps=1e-5,
                  gelu_tanh=0, swiglu=0, disable_bias_linear=0):
@@ -288,6 +291,11 @@ class TPRank:
         _check(self.lib.mgt_tp_rank_sizes(self.handle, ctypes.byref(a), ctypes.byref(b)),
                "mgt_tp_rank_sizes")
         return a.value, b.value
+
+    def set_bands(self, bands):
+        """Split every shard sum into `bands` row bands whose exchanges overlap the next band's
+        GEMM (see mgt_tp_rank_set_bands)."""
+        _check(self.lib.mgt_tp_rank_set_bands(self.handle, int(bands)), "mgt_tp_rank_set_bands")
 
     def partial_region(self):
         o, n = ctypes.c_size_t(), ctypes.c_size_t()
@@ -329,20 +337,24 @@ class TPRank:
                                         cb, None, _stream_handle(stream)), "mgt_tp_rank_bwd")
 
 
-def process_group_allreduce(workspace, offset, group=None):
+def process_group_allreduce(workspace, offset, nbytes=None, group=None):
     """The all-reduce a TPRank needs, over a torch.distributed process group (NCCL for device
-    workspaces): the callback views the `count` fp32 values at `offset` of `workspace` (the
-    rank's partial buffer, TPRank.partial_region()) and sums them over the group in place,
-    on the stream the layer passes (torch.distributed enqueues the collective there). Every
-    rank of the group must make the same TPRank calls in the same order."""
+    workspaces): the callback views the `count` fp32 values at the address the layer passes,
+    which must lie inside the rank's partial buffer (`nbytes` bytes at `offset` of
+    `workspace`, TPRank.partial_region(); the rest of the workspace by default) -- the whole
+    buffer, or one row band of it -- and sums them over the group in place, on the stream the
+    layer passes (torch.distributed enqueues the collective there). Every rank of the group
+    must make the same TPRank calls in the same order."""
     import torch
     import torch.distributed as dist
     base = workspace.data_ptr()
+    end = workspace.numel() if nbytes is None else offset + nbytes
 
     def allreduce(ptr, count, stream):
-        if ptr != base + offset or count * 4 + offset > workspace.numel():
-            raise ValueError("all-reduce buffer outside the rank's workspace")
-        view = workspace[offset:offset + 4 * count].view(torch.float32)
+        start = ptr - base
+        if start < offset or (start - offset) % 4 or start + 4 * count > end or count < 1:
+            raise ValueError("all-reduce buffer outside the rank's partial buffer")
+        view = workspace[start:start + 4 * count].view(torch.float32)
         if workspace.is_cuda:
             with torch.cuda.stream(torch.cuda.ExternalStream(stream, device=workspace.device)):
                 dist.all_reduce(view, group=group)

@@ -888,6 +888,537 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ============================================================================ fused backward
+// One key-stationary kernel for head_dim 128 that computes S^T and dP^T once per (key block,
+// query sub-block) and produces all three gradients:
+//   S^T = K Q^T, dP^T = V dO^T           (M = 128 keys, N = 64 queries, fp32 in TMEM)
+//   P^T = exp2(S^T*scale*log2e - lse*log2e), dS^T = P^T * (dP^T - D)   (softmax warps)
+//   dQ^T = K^T dS^T                       (M = d, N = 64 queries) into the dP^T columns
+//   dK += dS^T Q, dV += P^T dO            (TMEM accumulators)
+// P^T goes back into TMEM as packed bf16 (the A operand of dV). dS^T goes to shared memory
+// in the 128-byte swizzled layout, where one buffer serves as the K-major A operand of dK
+// (rows = keys) and as the MN-major B operand of dQ^T (queries contiguous). Four drain warps
+// read each dQ^T tile from TMEM and add it into the accumulator a.dq_fix [T][H][d] with
+// coalesced reductions (a warp covers 32 consecutive d of one query). Five products per
+// (key block, query block) instead of the seven of the two-kernel form.
+//
+// The accumulator is 32-bit fixed point, so the result is bit-reproducible: integer addition
+// is associative, and the key blocks of a query block arrive in no fixed order. Every partial
+// sum of dQ is bounded: |dQ[q,d]| <= max|K| * sum_k |dS[q,k]| and
+// sum_k |dS[q,k]| <= sum_k P[q,k] (|dP[q,k]| + |D[q]|) <= 2 |dO_q| max_k |V_k|
+// (Cauchy-Schwarz for dP = dO.V; |D| = |dO.O| with O a convex combination of the V rows; the
+// probabilities of a row sum to 1). With B = 2 max|K| max|dO_q| max|V_k| over the head, values
+// are scaled by 2^e with B * 2^e < 2^29 and rounded to integers: four times headroom below the
+// int32 limit for rounding, and a resolution of B * 2^-29 per addend.
+//
+// Warps 0-7: softmax (lane quarter w%4 = 32 key rows, query half w/4 of each sub-block);
+// warp 8: TMA producer; warp 9: TMEM owner and MMA issuer; warps 10-13: dQ drain (lane
+// quarter w%4 = 32 of the d rows of dQ^T). Every wait is bounded.
+// Power of two e with B * 2^e < 2^29 for B = 2 max|K| max|dO row| max|V row| over a head's
+// chunk bounds ([nchunk][3]: max |K|, max |V row|^2, max |dO row|^2). Every CTA of a head and
+// nothing else computes it, from the same values, so all agree.
+__device__ __forceinline__ int dq_fixed_exponent(const float* bound, int nchunk) {
+  float km = 0.f, v2 = 0.f, g2 = 0.f;
+  for (int c = 0; c < nchunk; ++c) {
+    km = fmaxf(km, bound[3 * c]);
+    v2 = fmaxf(v2, bound[3 * c + 1]);
+    g2 = fmaxf(g2, bound[3 * c + 2]);
+  }
+  const float B = 2.f * km * sqrtf(v2) * sqrtf(g2);
+  if (!(B > 0.f)) return 100;        // all-zero gradients: any scale is exact
+  if (!(B < INFINITY)) return -100;  // non-finite inputs: the result is undefined anyway
+  int ex;
+  frexpf(B, &ex);                    // B < 2^ex
+  const int e = 29 - ex;
+  return e > 100 ? 100 : (e < -100 ? -100 : e);
+}
+
+template <int D>
+struct FusedBwdLayout {
+  static constexpr int CH = D / 64;
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE, DO_OFF = 4 * TILE;  // Q, dO x2
+  static constexpr int DS_OFF = 6 * TILE;           // dS^T [128 keys][64 queries] bf16
+  static constexpr int STAT_OFF = DS_OFF + 16384;   // float lse2[2][128], dsum[2][128]
+  static constexpr int BAR_OFF = STAT_OFF + 4 * 128 * 4;
+  static constexpr int BYTES = BAR_OFF + 256 + 1024;
+  // TMEM buffer x (sub-block parity) at x*128: S^T in +0..63 (P^T packed into its first
+  // halves), dP^T in +64..127 (then dQ^T); dV and dK accumulators above.
+  static constexpr int T_SUB = 128, T_DV = 256, T_DK = 256 + D;
+};
+constexpr int kFusedBwdThreads = 448;
+
+template <int D>
+__global__ void __launch_bounds__(kFusedBwdThreads, 1)
+    attn_bwd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+                             const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
+                             float scale_log2, float scale) {
+  using L = FusedBwdLayout<D>;
+  static_assert(D == 128, "dQ^T tiles use M = head_dim = 128");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;     // [2]: Q and dO of one query block
+  uint64_t* q_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;     // [2]: S^T, dP^T of a sub-block in buffer x
+  uint64_t* p_full = bars + 7;     // [2]: P^T in TMEM and dS^T in shared memory
+  uint64_t* ds_empty = bars + 9;   // dK and dQ^T of the previous sub-block have read dS^T
+  uint64_t* dq_full = bars + 10;   // [2]: dQ^T of a sub-block is in buffer x
+  uint64_t* dq_empty = bars + 12;  // [2]: the drain warps have read it
+  uint64_t* drain = bars + 14;     // every MMA done (the output reads dV, dK after it)
+  uint64_t* stat_bar = bars + 15;  // [2]: per-query stats of a block staged by the 8 warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lse_s = reinterpret_cast<float*>(smem + L::STAT_OFF);  // [2][128], log2 units
+  float* dsum_s = lse_s + 256;                                   // [2][128]
+  uint8_t* ds_buf = smem + L::DS_OFF;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.s, H = a.H, hp = H / a.p;
+  // Key block; kb = 0 sees the most query blocks. Heads vary fastest in the launch order, so
+  // the longest tiles of every head go first.
+  const int kb = blockIdx.y;
+  const int bh = blockIdx.x, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const int col_q = t * 3 * hp * D + jh * D, col_k = col_q + hp * D, col_v = col_q + 2 * hp * D;
+  const int nq = (S + 127) / 128;
+  const int niter = nq - kb;  // query blocks qi = kb .. nq-1 see keys of this block
+  const int G = 2 * niter;    // 64-query sub-blocks
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&dq_full[i], 1);
+      mbar_init(&dq_empty[i], 4);
+      mbar_init(&stat_bar[i], 256);
+    }
+    mbar_init(ds_empty, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_3d(&tm_qkv, kv_full, smem + L::K_OFF + c * 16384, col_k + c * 64, kb * 128, b);
+        tma_load_3d(&tm_qkv, kv_full, smem + L::V_OFF + c * 16384, col_v + c * 64, kb * 128, b);
+      }
+      int issued = 0;
+      for (int it = 0; it < niter; ++it) {
+        const int st = it & 1, qi = kb + it;
+        if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_3d(&tm_qkv, &q_full[st], smem + L::Q_OFF + st * L::TILE + c * 16384,
+                      col_q + c * 64, qi * 128, b);
+          tma_load_3d(&tm_do, &q_full[st], smem + L::DO_OFF + st * L::TILE + c * 16384,
+                      n * D + c * 64, qi * 128, b);
+        }
+        issued = it + 1;
+      }
+      mbar_wait(kv_full, 0, a.err, kErrTimeoutDrain, nullptr);
+      for (int it = issued - 2 < 0 ? 0 : issued - 2; it < issued; ++it)
+        mbar_wait(&q_full[it & 1], (it >> 1) & 1, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      // Per sub-block g (query block it = g/2, half j = g%2, TMEM buffer x = g%2):
+      //   S^T(g+1), dP^T(g+1) are issued before waiting for the softmax of g, so the tensor
+      //   pipe computes them (and then dQ^T, dK, dV of g) while the softmax warps work.
+      //   dP^T(g+1) overwrites dQ^T(g-1) in the same buffer: it waits until the drain warps
+      //   have read that tile. S^T(g+1) overwrites P^T(g-1), read by dV(g-1) which was issued
+      //   earlier by this thread (tcgen05.mma operations of one thread execute in order).
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, 64, true, true);
+      const uint32_t k_addr = smem_u32(smem + L::K_OFF), v_addr = smem_u32(smem + L::V_OFF);
+      const uint32_t ds_addr = smem_u32(ds_buf);
+      auto issue_sd = [&](int g) -> bool {
+        const int it = g >> 1, j = g & 1, st = it & 1;
+        const uint32_t x = (g & 1) * L::T_SUB;
+        if (j == 0 && !mbar_wait(&q_full[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF + st * L::TILE) + j * 8192;
+        const uint32_t do_addr = smem_u32(smem + L::DO_OFF + st * L::TILE) + j * 8192;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + x, smem_desc_sw128(k_addr + off, 16, 1024),
+                     smem_desc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        if (g >= 2 && !mbar_wait(&dq_empty[g & 1], ((g - 2) >> 1) & 1, a.err, kErrTimeoutAttn,
+                                 abort_flag))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_f16(tmem + x + 64, smem_desc_sw128(v_addr + off, 16, 1024),
+                     smem_desc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[g & 1]);
+        return true;
+      };
+      bool ok = mbar_wait(kv_full, 0, a.err, kErrTimeoutAttn, abort_flag);
+      if (ok && G > 0) ok = issue_sd(0);
+      for (int g = 0; g < G && ok; ++g) {
+        if (g + 1 < G && !(ok = issue_sd(g + 1))) break;
+        if (!(ok = mbar_wait(&p_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag)))
+          break;
+        tc_fence_after();
+        const int it = g >> 1, j = g & 1, st = it & 1;
+        const uint32_t x = (g & 1) * L::T_SUB;
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF + st * L::TILE) + j * 8192;
+        const uint32_t do_addr = smem_u32(smem + L::DO_OFF + st * L::TILE) + j * 8192;
+        // dQ^T(g) = K^T dS^T (128 keys, 16 per MMA): A = K read d-major from its tile, B = dS^T
+        // read query-major; the result replaces dP^T(g), which the softmax has consumed.
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_f16(tmem + x + 64, smem_desc_sw128(k_addr + kk * 2048, 16384, 1024),
+                     smem_desc_sw128(ds_addr + kk * 2048, 16384, 1024), idesc_dq,
+                     kk > 0 ? 1u : 0u);
+        tc_commit(&dq_full[g & 1]);
+        // dK += dS^T Q (64 queries, 16 per MMA): A = dS^T read key-major from shared memory
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_f16(tmem + L::T_DK, smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
+                     smem_desc_sw128(q_addr + kk * 2048, 16384, 1024), idesc_acc,
+                     (g > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(ds_empty);
+        // dV += P^T dO: packed P^T, queries 0-31 in columns 0-15, 32-63 in 32-47
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t pc = kk * 8 + (kk >= 2 ? 16 : 0);
+          tc_mma_f16_tmem_a(tmem + L::T_DV, tmem + x + pc,
+                            smem_desc_sw128(do_addr + kk * 2048, 16384, 1024), idesc_acc,
+                            (g > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (j == 1) tc_commit(&q_empty[st]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, a.err, kErrTimeoutDrain, nullptr);
+    }
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ dQ drain
+    // Thread = row dd of dQ^T (one of the head dimensions); the 64 columns are the queries of
+    // the sub-block. A warp's reduction for one query covers 32 consecutive dd: 128 bytes.
+    const int quarter = warp & 3;
+    const int dd = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int32_t* acc = a.dq_fix + (long long)b * S * H * D + (long long)n * D + dd;
+    const long long ldq = (long long)H * D;
+    // this head's fixed-point scale (the same computation in every CTA of the head)
+    const int e = dq_fixed_exponent(a.dq_bound + (long long)bh * ((S + 127) / 128) * 3,
+                                    (S + 127) / 128);
+    if (kb == 0 && quarter == 0 && lane == 0) a.dq_exp[bh] = e;
+    const float fscale = exp2f((float)e);
+    for (int g = 0; g < G; ++g) {
+      const bool ok = mbar_wait(&dq_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn,
+                                abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t x = (g & 1) * L::T_SUB;
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32_nw(lane_base + x + 64, v0);
+      tmem_ld_32x32b_x32_nw(lane_base + x + 96, v1);
+      tmem_ld_wait();
+      reg_fence(v0);
+      reg_fence(v1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dq_empty[g & 1]);
+      const int q0 = (kb + (g >> 1)) * 128 + (g & 1) * 64;
+      const int nvalid = S - q0 < 64 ? S - q0 : 64;
+      int32_t* row = acc + (long long)q0 * ldq;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nvalid)
+          atomicAdd(row + (long long)i * ldq, __float2int_rn(__uint_as_float(v0[i]) * fscale));
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (32 + i < nvalid)
+          atomicAdd(row + (long long)(32 + i) * ldq,
+                    __float2int_rn(__uint_as_float(v1[i]) * fscale));
+    }
+  } else {
+    // ------------------------------------------------------------ P^T, dS^T and the output
+    // warp w: TMEM lane quarter w%4 (key rows), 32-query half w/4 of each 64-query sub-block
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // key row within the block = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float* lse_g = a.lse + ((long long)b * H + n) * S;
+    const float* dsum_g = a.Dsum + ((long long)b * H + n) * S;
+    // this thread's dS^T row in the swizzled buffer: 16-byte chunk c of the row sits at
+    // chunk c ^ (r % 8)
+    uint8_t* ds_row = ds_buf + r * 128;
+    bool ok = true;
+    const float* stat_g = hf ? dsum_g : lse_g;
+    float* stat_s = hf ? dsum_s : lse_s;
+    auto fetch = [&](int qi) -> float {
+      const int q = qi * 128 + r;  // padded queries get lse = +inf, hence P = 0
+      if (hf == 0) return q < S ? stat_g[q] * kLog2eF : INFINITY;
+      return q < S ? stat_g[q] : 0.f;
+    };
+    float nv = niter > 0 ? fetch(kb) : 0.f;
+    for (int g = 0; g < G; ++g) {
+      const int it = g >> 1, j = g & 1, st = it & 1, qi = kb + it;
+      if (j == 0) {
+        stat_s[st * 128 + r] = nv;
+        if (it + 1 < niter) nv = fetch(qi + 1);
+        mbar_arrive(&stat_bar[st]);
+        ok = mbar_wait(&stat_bar[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+      }
+      ok = mbar_wait(&s_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t x = (g & 1) * L::T_SUB;
+      const int q0 = j * 64 + hf * 32;  // first query (within the block) of this warp's columns
+      const float* ls = lse_s + st * 128 + q0;
+      const float* ds_ = dsum_s + st * 128 + q0;
+      uint32_t sr[32], dr[32];
+      tmem_ld_32x32b_x32_nw(lane_base + x + hf * 32, sr);
+      tmem_ld_32x32b_x32_nw(lane_base + x + 64 + hf * 32, dr);
+      tmem_ld_wait();
+      reg_fence(sr);
+      reg_fence(dr);
+      if (qi == kb) {  // diagonal block: queries before this key see nothing of it
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (q0 + i < r) sr[i] = __float_as_uint(-INFINITY);
+      }
+      uint32_t pw[16], dw[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(ls + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(ds_ + i);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float p4[4], q4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          p4[e] = ex2_approx(fmaf(__uint_as_float(sr[i + e]), scale_log2, -lv[e]));
+          q4[e] = p4[e] * (__uint_as_float(dr[i + e]) - dv[e]);
+        }
+        pw[i >> 1] = pack_bf16x2(p4[0], p4[1]);
+        pw[(i >> 1) + 1] = pack_bf16x2(p4[2], p4[3]);
+        dw[i >> 1] = pack_bf16x2(q4[0], q4[1]);
+        dw[(i >> 1) + 1] = pack_bf16x2(q4[2], q4[3]);
+      }
+      // P^T packed into the first half of the 32 columns this warp itself read, so the other
+      // warp of the quarter (reading its own 32 columns) is never overwritten.
+      tmem_st_32x32b_x16(lane_base + x + hf * 32, pw);
+      // dS^T into shared memory once dK and dQ^T of the previous sub-block have read it
+      if (g > 0) {
+        ok = mbar_wait(ds_empty, (g - 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int chunk = (hf * 4 + c) ^ (r & 7);
+        *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
+            make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[g & 1]);
+    }
+    if (ok && niter > 0) {
+      // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
+      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const int key = kb * 128 + r;
+        const long long ld = 3LL * H * D;
+        __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + ((long long)b * S + key) * ld +
+                            (long long)t * 3 * hp * D + (long long)jh * D + (long long)hp * D;
+        __nv_bfloat16* dv = dk + (long long)hp * D;
+#pragma unroll 1
+        for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {  // this half of d
+          float v[32], kk[32];
+          tmem_ld_32x32b_x32(lane_base + L::T_DV + c * 32, v);
+          tmem_ld_32x32b_x32(lane_base + L::T_DK + c * 32, kk);
+          if (key < S) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 wv, wk;
+              wv.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              wv.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              wv.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              wv.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              wk.x = pack_bf16x2(kk[q * 8 + 0] * scale, kk[q * 8 + 1] * scale);
+              wk.y = pack_bf16x2(kk[q * 8 + 2] * scale, kk[q * 8 + 3] * scale);
+              wk.z = pack_bf16x2(kk[q * 8 + 4] * scale, kk[q * 8 + 5] * scale);
+              wk.w = pack_bf16x2(kk[q * 8 + 6] * scale, kk[q * 8 + 7] * scale);
+              *reinterpret_cast<uint4*>(dv + c * 32 + q * 8) = wv;
+              *reinterpret_cast<uint4*>(dk + c * 32 + q * 8) = wk;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Per head and 128-token chunk c (grid b*H x chunks, 8 warps x 16 tokens): D = rowsum(dO * O)
+// into a.Dsum [b][H][s], the fixed-point dQ accumulator zeroed, and the chunk's max |K|,
+// max |V row|^2 and max |dO row|^2 into a.dq_bound (one lane holds 4 of the 128 dimensions).
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
+  constexpr int D = 128;
+  __shared__ float red[8][3];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x, c = blockIdx.y, nchunk = gridDim.y;
+  const int H = a.H, hp = H / a.p, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
+  const long long ld_qkv = 3LL * H * D, ld_o = (long long)H * D;
+  float kmax = 0.f, v2max = 0.f, g2max = 0.f;
+  for (int i = 0; i < 16; ++i) {
+    const int pos = c * 128 + warp * 16 + i;
+    if (pos >= a.s) break;  // warp-uniform
+    const long long tok = (long long)b * a.s + pos;
+    const long long oo = tok * ld_o + (long long)n * D + lane * 4;
+    const long long ko = tok * ld_qkv + (long long)t * 3 * hp * D + (long long)(hp + jh) * D + lane * 4;
+    const uint2 ov = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + oo);
+    const uint2 gv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.dO) + oo);
+    const uint2 kv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.qkv) + ko);
+    const uint2 vv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.qkv) + ko + (long long)hp * D);
+    const float o[4] = {bf16_lo(ov.x), bf16_hi(ov.x), bf16_lo(ov.y), bf16_hi(ov.y)};
+    const float g[4] = {bf16_lo(gv.x), bf16_hi(gv.x), bf16_lo(gv.y), bf16_hi(gv.y)};
+    const float k[4] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y)};
+    const float v[4] = {bf16_lo(vv.x), bf16_hi(vv.x), bf16_lo(vv.y), bf16_hi(vv.y)};
+    float dsum = 0.f, g2 = 0.f, v2 = 0.f, km = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      dsum = fmaf(o[e], g[e], dsum);
+      g2 = fmaf(g[e], g[e], g2);
+      v2 = fmaf(v[e], v[e], v2);
+      km = fmaxf(km, fabsf(k[e]));
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
+      g2 += __shfl_xor_sync(0xffffffffu, g2, m);
+      v2 += __shfl_xor_sync(0xffffffffu, v2, m);
+      km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, m));
+    }
+    if (lane == 0) a.Dsum[(long long)bh * a.s + pos] = dsum;
+    *reinterpret_cast<int4*>(a.dq_fix + oo) = make_int4(0, 0, 0, 0);
+    kmax = fmaxf(kmax, km);
+    v2max = fmaxf(v2max, v2);
+    g2max = fmaxf(g2max, g2);
+  }
+  if (lane == 0) {
+    red[warp][0] = kmax;
+    red[warp][1] = v2max;
+    red[warp][2] = g2max;
+  }
+  __syncthreads();
+  if (threadIdx.x < 3) {
+    float m = 0.f;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w][threadIdx.x]);
+    a.dq_bound[((long long)bh * nchunk + c) * 3 + threadIdx.x] = m;
+  }
+}
+
+// dQ = dq_fix * 2^-e / sqrt(d) in bf16 into the Q slots of dqkv [T][p][3][H/p][d]: 16 threads
+// per (token, head), 8 elements each.
+__global__ void attn_bwd_dq_convert_kernel(const AttnArgs a, float scale) {
+  const long long rows = (long long)a.b * a.s * a.H;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = idx >> 4;
+  const int part = (int)(idx & 15);
+  if (row >= rows) return;
+  const long long token = row / a.H;
+  const int nh = (int)(row - token * a.H), hp = a.H / a.p, tt = nh / hp, jj = nh - tt * hp;
+  const int bb = (int)(token / a.s);
+  const float f = scale * exp2f((float)-a.dq_exp[(long long)bb * a.H + nh]);
+  const int4* src = reinterpret_cast<const int4*>(a.dq_fix + row * 128 + part * 8);
+  const int4 u = src[0], v = src[1];
+  uint4 w;
+  w.x = pack_bf16x2((float)u.x * f, (float)u.y * f);
+  w.y = pack_bf16x2((float)u.z * f, (float)u.w * f);
+  w.z = pack_bf16x2((float)v.x * f, (float)v.y * f);
+  w.w = pack_bf16x2((float)v.z * f, (float)v.w * f);
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + token * 3LL * a.H * 128 +
+                       (long long)tt * 3 * hp * 128 + (long long)jj * 128 + part * 8;
+  *reinterpret_cast<uint4*>(dst) = w;
+}
+
+cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
+  constexpr int D = 128;
+  using L = FusedBwdLayout<D>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_fused_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap tm_qkv, tm_do;
+  const uint64_t three_h = 3ull * a.H * D, hd = (uint64_t)a.H * D;
+  const uint32_t box[3] = {64, 128, 1};
+  {
+    const uint64_t dims[3] = {three_h, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {three_h, three_h * a.s};
+    if (!make_tensor_map_bf16_3d(&tm_qkv, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {hd, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {hd, hd * a.s};
+    if (!make_tensor_map_bf16_3d(&tm_do, a.dO, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const float scale = 1.f / sqrtf((float)D);
+  const long long threads = (long long)a.b * a.s * a.H * 16;  // 16 per (token, head)
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  attn_bwd_prep_kernel<<<dim3(a.b * a.H, (a.s + 127) / 128), 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.b * a.H, (a.s + 127) / 128);
+  attn_bwd_fused_tc_kernel<D><<<grid, kFusedBwdThreads, L::BYTES, s>>>(tm_qkv, tm_do, a,
+                                                                       kLog2eF * scale, scale);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(a, scale);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t bwd_tc(const AttnArgs& a, cudaStream_t s) {
   using L = BwdLayout<D>;
@@ -953,6 +1484,7 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t s) {
+  if (a.d == 128 && a.dq_fix) return bwd_fused_tc(a, s);
   if (a.d == 64) return bwd_tc<64>(a, s);
   if (a.d == 128) return bwd_tc<128>(a, s);
   return cudaErrorInvalidValue;

@@ -138,7 +138,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
           if (i < count) v[i] += __bfloat162float(r[i]);
       }
     }
-    if (EPI == kEpiDGelu) {  // aux holds GeLU'(u), stored by the forward epilogue
+    if (EPI == kEpiDGelu) {  // aux holds u, stored by the forward epilogue: du = dA GeLU'(u)
       const __nv_bfloat16* g =
           reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col;
       if (count == 32) {
@@ -148,30 +148,30 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            v[q * 8 + 2 * j] *= bf16_lo(ww[j]);
-            v[q * 8 + 2 * j + 1] *= bf16_hi(ww[j]);
+            v[q * 8 + 2 * j] *= gelu_grad_bf16out(bf16_lo(ww[j]), a.gelu_tanh);
+            v[q * 8 + 2 * j + 1] *= gelu_grad_bf16out(bf16_hi(ww[j]), a.gelu_tanh);
           }
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (i < count) v[i] *= __bfloat162float(g[i]);
+          if (i < count) v[i] *= gelu_grad_bf16out(__bfloat162float(g[i]), a.gelu_tanh);
       }
     }
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + off;
-    if (EPI == kEpiGelu) {  // out = GeLU(u), out2 = GeLU'(u) for the backward
+    if (EPI == kEpiGelu) {  // out = GeLU(u), out2 = u for the backward
       __nv_bfloat16* o2 = reinterpret_cast<__nv_bfloat16*>(a.out2) + off;
       if (count == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float ga[8], gd[8];
+          float ga[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) gelu_and_grad_bf16out(v[q * 8 + j], a.gelu_tanh, ga[j], gd[j]);
+          for (int j = 0; j < 8; ++j) ga[j] = gelu_bf16out(v[q * 8 + j], a.gelu_tanh);
           uint4 wd, wa;
-          wd.x = pack_bf16x2(gd[0], gd[1]);
-          wd.y = pack_bf16x2(gd[2], gd[3]);
-          wd.z = pack_bf16x2(gd[4], gd[5]);
-          wd.w = pack_bf16x2(gd[6], gd[7]);
+          wd.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+          wd.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+          wd.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+          wd.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
           *reinterpret_cast<uint4*>(o2 + q * 8) = wd;
           wa.x = pack_bf16x2(ga[0], ga[1]);
           wa.y = pack_bf16x2(ga[2], ga[3]);
@@ -183,10 +183,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i < count) {
-            float ga, gd;
-            gelu_and_grad_bf16out(v[i], a.gelu_tanh, ga, gd);
-            o2[i] = __float2bfloat16_rn(gd);
-            o[i] = __float2bfloat16_rn(ga);
+            o2[i] = __float2bfloat16_rn(v[i]);
+            o[i] = __float2bfloat16_rn(gelu_bf16out(v[i], a.gelu_tanh));
           }
         }
       }
@@ -245,9 +243,9 @@ __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int 
       const uint32_t ww[4] = {r4[q].x, r4[q].y, r4[q].z, r4[q].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (EPI == kEpiDGelu) {  // aux holds GeLU'(u), stored by the forward epilogue
-          v[q * 8 + 2 * j] *= bf16_lo(ww[j]);
-          v[q * 8 + 2 * j + 1] *= bf16_hi(ww[j]);
+        if (EPI == kEpiDGelu) {  // aux holds u, stored by the forward epilogue
+          v[q * 8 + 2 * j] *= gelu_grad_bf16out(bf16_lo(ww[j]), a.gelu_tanh);
+          v[q * 8 + 2 * j + 1] *= gelu_grad_bf16out(bf16_hi(ww[j]), a.gelu_tanh);
         } else {
           v[q * 8 + 2 * j] += bf16_lo(ww[j]);
           v[q * 8 + 2 * j + 1] += bf16_hi(ww[j]);
@@ -282,14 +280,12 @@ __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int 
     }
     return;
   }
-  if constexpr (EPI == kEpiGelu) {
+  if constexpr (EPI == kEpiGelu) {  // w: GeLU(u), w2: u
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float g0, d0, g1, d1;
-      gelu_and_grad_bf16out(v[2 * i], a.gelu_tanh, g0, d0);
-      gelu_and_grad_bf16out(v[2 * i + 1], a.gelu_tanh, g1, d1);
-      w[i] = pack_bf16x2(g0, g1);
-      w2[i] = pack_bf16x2(d0, d1);
+      w[i] = pack_bf16x2(gelu_bf16out(v[2 * i], a.gelu_tanh),
+                         gelu_bf16out(v[2 * i + 1], a.gelu_tanh));
+      w2[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
     }
   } else {
 #pragma unroll

@@ -104,6 +104,21 @@ mgt_status validate(const mgt_layer_config* c) {
   return MGT_OK;
 }
 
+// fixed-point dQ accumulator and scaling data of the single-kernel attention backward (bf16,
+// head_dim 128)
+size_t dq_acc_bytes(const mgt_layer* L) {
+  if (L->cfg.dtype != MGT_BF16 || L->d != 128) return 0;
+  return dq_scratch_layout(L->cfg.micro_batch, L->cfg.seq, L->H).bytes;
+}
+
+// per-slice column sums of du and dqkv (the b1 and b_qkv gradients); one buffer serves both
+size_t bias_partial_bytes(const mgt_layer* L) {
+  if (L->cfg.disable_bias_linear) return 0;
+  const size_t f1 = L->cfg.swiglu ? 2 * (size_t)L->f : (size_t)L->f;
+  const size_t cols = f1 > 3 * (size_t)L->h ? f1 : 3 * (size_t)L->h;
+  return (size_t)kColsumMaxSlices * cols * 4;
+}
+
 void layout(mgt_layer* L) {
   const size_t T = L->T, h = L->h, f = L->f, e = L->esz;
   const size_t f1 = L->cfg.swiglu ? 2 * f : f;  // fc1 outputs: [gate | up] with SwiGLU
@@ -126,8 +141,9 @@ void layout(mgt_layer* L) {
                                    T * 3 * h * e,
                                    T * h * e,
                                    bHs * 4,
-                                   0,
-                                   nblk * 3 * h * 4};
+                                   dq_acc_bytes(L),
+                                   nblk * 3 * h * 4,
+                                   bias_partial_bytes(L)};
   off = 0;
   for (int i = 0; i < MGT_WS_COUNT - 64; ++i) {
     L->ws[i].off = off;
@@ -332,7 +348,7 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   char* ln2 = sp(saved, L->saved[MGT_SAVED_LN2]);
   float* mu2 = reinterpret_cast<float*>(sp(saved, L->saved[MGT_SAVED_LN2_MEAN]));
   float* rs2 = reinterpret_cast<float*>(sp(saved, L->saved[MGT_SAVED_LN2_RSTD]));
-  char* gd = sp(saved, L->saved[MGT_SAVED_FC1_DGELU]);
+  char* u1 = sp(saved, L->saved[MGT_SAVED_FC1_U]);  // fc1 pre-activation u
   char* act = sp(saved, L->saved[MGT_SAVED_FC1_A]);
   const double ln_bytes = (double)T * h * 2 * e + 8.0 * h;
   const bool nb = L->cfg.disable_bias_linear;
@@ -375,19 +391,19 @@ mgt_status mgt_layer_fwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     return launch_ln_fwd(dt, T, h, L->cfg.ln_eps, h1, (const float*)P->ln2_g,
                          (const float*)P->ln2_b, ln2, mu2, rs2, err, s);
   }));
-  // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and GeLU'(u) for the backward).
+  // 6. fc1, column-parallel, + b1, GeLU (stores a = GeLU(u) and u for the backward).
   //    SwiGLU: shard t's gate and up rows go to the two halves of one tile; the epilogue stores
   //    a = silu(gate) * up and [gate | up] for the backward.
   if (L->cfg.swiglu) {
     GemmArgs a = gemm_base(T, f / p, p, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
-    a.epi = kEpiSwiglu; a.out = act; a.ldc = f; a.out2 = gd; a.ldc2 = 2LL * f; a.bias = b1;
+    a.epi = kEpiSwiglu; a.out = act; a.ldc = f; a.out2 = u1; a.ldc2 = 2LL * f; a.bias = b1;
     a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   } else {
     GemmArgs a = gemm_base(T, f, 1, h, 1);
     a.A = ln2; a.lda = h; a.B = P->w1; a.ldb = h;
-    a.epi = kEpiGelu; a.out = act; a.out2 = gd; a.ldc = f; a.bias = b1;
+    a.epi = kEpiGelu; a.out = act; a.out2 = u1; a.ldc = f; a.bias = b1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc1_fwd", a, s));
   }
@@ -432,7 +448,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   const char* ln2 = sp(saved, L->saved[MGT_SAVED_LN2]);
   const float* mu2 = reinterpret_cast<const float*>(sp(saved, L->saved[MGT_SAVED_LN2_MEAN]));
   const float* rs2 = reinterpret_cast<const float*>(sp(saved, L->saved[MGT_SAVED_LN2_RSTD]));
-  const char* gd = sp(saved, L->saved[MGT_SAVED_FC1_DGELU]);
+  const char* u1 = sp(saved, L->saved[MGT_SAVED_FC1_U]);
   const char* act = sp(saved, L->saved[MGT_SAVED_FC1_A]);
   char* du = sp(workspace, L->ws[MGT_WS_DU - 64]);
   char* dln2 = sp(workspace, L->ws[MGT_WS_DLN2 - 64]);
@@ -464,9 +480,10 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
       if (on && cudaEventRecord(L->ev_join, w) == cudaSuccess) cudaStreamWaitEvent(s, L->ev_join, 0);
     }
   } join{L, s, w};
+  float* bias_part = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_BIAS_PARTIAL - 64]));
   auto colsum = [&](const void* src, int cols, void* out) {
     return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, w,
-               [&] { return launch_colsum(dt, T, cols, src, (float*)out, w); });
+               [&] { return launch_colsum(dt, T, cols, src, (float*)out, bias_part, w); });
   };
   const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
   const bool nb = L->cfg.disable_bias_linear, sw = L->cfg.swiglu;
@@ -480,7 +497,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(T, f / p, p, h, 1);  // N grouped by shard
     a.b_mn = 1; a.A = dy; a.lda = h; a.B = P->w2; a.ldb = f / p;
     a.b_ngs = (long long)h * (f / p);
-    a.epi = sw ? kEpiDSwiglu : kEpiDGelu; a.out = du; a.ldc = f1; a.aux = gd; a.ld_aux = f1;
+    a.epi = sw ? kEpiDSwiglu : kEpiDGelu; a.out = du; a.ldc = f1; a.aux = u1; a.ld_aux = f1;
     a.gelu_tanh = L->cfg.gelu_tanh; a.err = err;
     a.a_sp = 1;  // dy is sequence-parallel: its all-gather (adjoint of the reduce-scatter)
     MGT_TRY(gemm(L, "gemm_tc/fc2_dgrad", a, s));
@@ -535,6 +552,13 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   {
     AttnArgs a{L->cfg.micro_batch, L->cfg.seq, L->H, L->d, p, qkv, (void*)O, (float*)lse,
                dO, Dsum, dqkv, err};
+    if (L->ws[MGT_WS_DQ_ACC - 64].bytes) {
+      char* base = sp(workspace, L->ws[MGT_WS_DQ_ACC - 64]);
+      const DqScratch q = dq_scratch_layout(L->cfg.micro_batch, L->cfg.seq, L->H);
+      a.dq_fix = reinterpret_cast<int32_t*>(base + q.fix_off);
+      a.dq_exp = reinterpret_cast<int32_t*>(base + q.exp_off);
+      a.dq_bound = reinterpret_cast<float*>(base + q.bound_off);
+    }
     const double fl = 2.5 * 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;  // model FLOPs incl. one recompute of S
     MGT_TRY(run(L, "attn_bwd", fl, 0, s, [&] { return launch_attn_bwd(dt, a, s); }));
   }

@@ -8,7 +8,10 @@
 //
 // Per reduction: the partial GEMM writes fp32 [T, h] into the workspace, the callback sums
 // it over the ranks in place (ordered on the stream), and a small kernel adds the bias and
-// the residual (forward) or casts to the activation type (backward). Everything else reuses
+// the residual (forward) or casts to the activation type (backward). With row bands
+// (mgt_tp_rank_set_bands) the partial GEMM runs band by band and each band is handed to the
+// callback on a communication stream as soon as its GEMM is enqueued, so the exchange of one
+// band overlaps the GEMM of the next (the page's --tp-comm-overlap). Everything else reuses
 // the single-GPU kernels with one shard: H/p heads, f/p MLP columns.
 #include <cstring>
 #include <new>
@@ -21,6 +24,7 @@ namespace mgt {
 namespace {
 
 constexpr int kMaxLnSlices = 296;  // LayerNorm backward partial rows (2 per SM on 148 SMs)
+constexpr int kMaxBands = 16;      // row bands per shard sum
 
 // out[i] = bf16(part[i] + bias[i % h] + res[i]); bias and res may be null. Eight elements per
 // thread step (h is a multiple of 8, every pointer 16-byte aligned).
@@ -79,7 +83,7 @@ struct Reg {
 enum SavedReg { S_LN1, S_MU1, S_RS1, S_QKV, S_O, S_LSE, S_H1, S_LN2, S_MU2, S_RS2, S_AUX, S_A,
                 S_COUNT };
 enum WsReg { W_STATUS, W_PART, W_DU, W_DLN2, W_DH1, W_DO, W_DQKV, W_DLN1, W_D, W_LNP,
-             W_COUNT };
+             W_DQACC, W_BIASP, W_COUNT };
 
 GemmArgs base(int M, int N, int K) {
   GemmArgs a;
@@ -103,6 +107,13 @@ struct mgt_tp_rank {
   size_t saved_bytes = 0, ws_bytes = 0;
   int num_sms = 0;
   int device = -1;
+  // Row bands of each shard sum (1: one exchange after the whole partial GEMM, on the
+  // caller's stream). With more, the exchanges run on `comm`, each ordered after its band's
+  // GEMM by ev_ready[i]; ev_done joins the last one back into the caller's stream.
+  int bands = 1;
+  cudaStream_t comm = nullptr;
+  cudaEvent_t ev_ready[kMaxBands] = {};
+  cudaEvent_t ev_done = nullptr;
 };
 
 namespace {
@@ -157,9 +168,85 @@ mgt_status check_ptrs(const mgt_tp_rank* R, const void* const* q) {
     if (_s != MGT_OK) return _s;                  \
   } while (0)
 
+// The communication stream and its events, created on the first banded call on the bound
+// device; on a failure everything created so far is released and the next call tries again.
+cudaError_t ensure_comm(mgt_tp_rank* R) {
+  if (R->comm) return cudaSuccess;
+  cudaStream_t comm = nullptr;
+  cudaEvent_t ev[kMaxBands + 1] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&comm, cudaStreamNonBlocking);
+  for (int i = 0; i <= kMaxBands && e == cudaSuccess; ++i)
+    e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    for (auto& x : ev)
+      if (x) cudaEventDestroy(x);
+    if (comm) cudaStreamDestroy(comm);
+    return e;
+  }
+  for (int i = 0; i < kMaxBands; ++i) R->ev_ready[i] = ev[i];
+  R->ev_done = ev[kMaxBands];
+  R->comm = comm;
+  return cudaSuccess;
+}
+
+// Rows per band: an even split of T rounded up to whole 128-row tiles.
+int band_rows(const mgt_tp_rank* R) {
+  const int per = (R->T + R->bands - 1) / R->bands;
+  return (per + 127) / 128 * 128;
+}
+
+// First half of a shard sum. `a` is the partial GEMM over all T rows (K-major A at `A` with
+// `lda` elements per row, fp32 output `part` [T, h]). One band: the GEMM only (the exchange
+// follows in reduce_end, on the caller's stream). Several bands: each band's GEMM, then that
+// band's exchange on the communication stream, ordered after the GEMM by an event, so band
+// i's exchange overlaps band i+1's GEMM.
+mgt_status reduce_begin(mgt_tp_rank* R, GemmArgs a, const void* A, long long lda, float* part,
+                        mgt_allreduce_fn allreduce, void* user, cudaStream_t s) {
+  if (R->bands == 1) {
+    a.A = A;
+    a.out = part;
+    TP_TRY(launch_gemm_tc(a, R->num_sms, s));
+    return MGT_OK;
+  }
+  TP_TRY(ensure_comm(R));
+  const int per = band_rows(R);
+  for (int i = 0, r0 = 0; r0 < R->T; ++i, r0 += per) {
+    const int rows = R->T - r0 < per ? R->T - r0 : per;
+    GemmArgs b = a;
+    b.M = rows;
+    b.A = static_cast<const __nv_bfloat16*>(A) + (long long)r0 * lda;
+    b.out = part + (long long)r0 * R->h;
+    TP_TRY(launch_gemm_tc(b, R->num_sms, s));
+    TP_TRY(cudaEventRecord(R->ev_ready[i], s));
+    TP_TRY(cudaStreamWaitEvent(R->comm, R->ev_ready[i], 0));
+    TP_TRY_ST(allreduce(part + (long long)r0 * R->h, (int64_t)rows * R->h, user, R->comm));
+  }
+  return MGT_OK;
+}
+
+// Second half: one band -- the exchange of the whole partial on the caller's stream; several
+// -- the caller's stream waits for the last band's exchange (the communication stream runs
+// them in order).
+mgt_status reduce_end(mgt_tp_rank* R, float* part, mgt_allreduce_fn allreduce, void* user,
+                      cudaStream_t s) {
+  if (R->bands == 1) {
+    TP_TRY_ST(allreduce(part, (int64_t)R->T * R->h, user, s));
+    return MGT_OK;
+  }
+  TP_TRY(cudaEventRecord(R->ev_done, R->comm));
+  TP_TRY(cudaStreamWaitEvent(s, R->ev_done, 0));
+  return MGT_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+mgt_status mgt_tp_rank_set_bands(mgt_tp_rank* R, int32_t bands) {
+  if (!R || bands < 1 || bands > kMaxBands) return MGT_EINVAL;
+  R->bands = bands;
+  return MGT_OK;
+}
 
 mgt_status mgt_tp_rank_init(const mgt_layer_config* cfg, int32_t rank, mgt_tp_rank** out) {
   if (!out) return MGT_EINVAL;
@@ -193,7 +280,16 @@ mgt_status mgt_tp_rank_init(const mgt_layer_config* cfg, int32_t rank, mgt_tp_ra
                               T * R->fl * e};
   const size_t wb[W_COUNT] = {256, T * h * 4, T * R->f1l * e, T * h * e, T * h * e,
                               T * R->hl * e, T * 3 * R->hl * e, T * h * e, lse,
-                              (size_t)R->nblk * 3 * h * 4};
+                              (size_t)R->nblk * 3 * h * 4,
+                              // fixed-point dQ accumulator and its scaling data
+                              R->d == 128 ? dq_scratch_layout(cfg->micro_batch, cfg->seq,
+                                                              R->Hl).bytes
+                                          : 0,
+                              // column-sum partials of the b1 / b_qkv gradients
+                              cfg->disable_bias_linear
+                                  ? 0
+                                  : (size_t)kColsumMaxSlices *
+                                        (R->f1l > 3 * R->hl ? R->f1l : 3 * R->hl) * 4};
   place(R->saved, S_COUNT, sb, &R->saved_bytes);
   place(R->ws, W_COUNT, wb, &R->ws_bytes);
   *out = R;
@@ -214,7 +310,17 @@ mgt_status mgt_tp_rank_partial(const mgt_tp_rank* R, size_t* offset, size_t* byt
   return MGT_OK;
 }
 
-void mgt_tp_rank_destroy(mgt_tp_rank* R) { delete R; }
+void mgt_tp_rank_destroy(mgt_tp_rank* R) {
+  if (!R) return;
+  if (R->comm) {
+    cudaStreamSynchronize(R->comm);
+    for (auto& e : R->ev_ready)
+      if (e) cudaEventDestroy(e);
+    if (R->ev_done) cudaEventDestroy(R->ev_done);
+    cudaStreamDestroy(R->comm);
+  }
+  delete R;
+}
 
 mgt_status mgt_tp_rank_fwd(mgt_tp_rank* R, const mgt_layer_params* P, const void* x, void* y,
                            void* saved, void* workspace, mgt_allreduce_fn allreduce, void* user,
@@ -261,11 +367,11 @@ mgt_status mgt_tp_rank_fwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
   // out-proj partial -> all-reduce -> h1 = x + b_o + sum
   {
     GemmArgs a = base(T, h, hl);
-    a.A = O; a.lda = hl; a.B = P->w_o; a.ldb = hl;
-    a.epi = kEpiStoreF32; a.out = part; a.ldc = h; a.err = err;
-    TP_TRY(launch_gemm_tc(a, R->num_sms, s));
+    a.lda = hl; a.B = P->w_o; a.ldb = hl;
+    a.epi = kEpiStoreF32; a.ldc = h; a.err = err;
+    TP_TRY_ST(reduce_begin(R, a, O, hl, part, allreduce, user, s));
   }
-  TP_TRY_ST(allreduce(part, (int64_t)T * h, user, stream));
+  TP_TRY_ST(reduce_end(R, part, allreduce, user, s));
   TP_TRY(sum_epilogue((long long)T * h, h, part, nb ? nullptr : P->b_o, x, h1, R->num_sms, s));
   // LN2, fc1 of this rank's columns (+ activation)
   TP_TRY(launch_ln_fwd(1, T, h, R->cfg.ln_eps, h1, (const float*)P->ln2_g,
@@ -286,11 +392,11 @@ mgt_status mgt_tp_rank_fwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
   // fc2 partial -> all-reduce -> y = h1 + b2 + sum
   {
     GemmArgs a = base(T, h, fl);
-    a.A = act; a.lda = fl; a.B = P->w2; a.ldb = fl;
-    a.epi = kEpiStoreF32; a.out = part; a.ldc = h; a.err = err;
-    TP_TRY(launch_gemm_tc(a, R->num_sms, s));
+    a.lda = fl; a.B = P->w2; a.ldb = fl;
+    a.epi = kEpiStoreF32; a.ldc = h; a.err = err;
+    TP_TRY_ST(reduce_begin(R, a, act, fl, part, allreduce, user, s));
   }
-  TP_TRY_ST(allreduce(part, (int64_t)T * h, user, stream));
+  TP_TRY_ST(reduce_end(R, part, allreduce, user, s));
   TP_TRY(sum_epilogue((long long)T * h, h, part, nb ? nullptr : P->b2, h1, y, R->num_sms, s));
   return MGT_OK;
 }
@@ -336,6 +442,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
   char* dln1 = at(workspace, R->ws[W_DLN1]);
   float* Dsum = reinterpret_cast<float*>(at(workspace, R->ws[W_D]));
   float* lnp = reinterpret_cast<float*>(at(workspace, R->ws[W_LNP]));
+  float* biasp = reinterpret_cast<float*>(at(workspace, R->ws[W_BIASP]));
   // fc2: du = (dy W2_t) * act'(u) (the activation backward in the dgrad epilogue); dW2_t
   {
     GemmArgs a = base(T, fl, h);
@@ -351,12 +458,12 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     TP_TRY(launch_gemm_tc(a, R->num_sms, s));
   }
   // fc1: db1_t, dln2 partial -> all-reduce -> bf16, dW1_t
-  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, biasp, s));
   {
     GemmArgs a = base(T, h, f1l);
-    a.b_mn = 1; a.A = du; a.lda = f1l; a.B = P->w1; a.ldb = h;
-    a.epi = kEpiStoreF32; a.out = part; a.ldc = h; a.err = err;
-    TP_TRY(launch_gemm_tc(a, R->num_sms, s));
+    a.b_mn = 1; a.lda = f1l; a.B = P->w1; a.ldb = h;
+    a.epi = kEpiStoreF32; a.ldc = h; a.err = err;
+    TP_TRY_ST(reduce_begin(R, a, du, f1l, part, allreduce, user, s));
   }
   {
     GemmArgs a = base(f1l, h, T);
@@ -364,7 +471,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err;
     TP_TRY(launch_gemm_tc(a, R->num_sms, s));
   }
-  TP_TRY_ST(allreduce(part, (int64_t)T * h, user, stream));
+  TP_TRY_ST(reduce_end(R, part, allreduce, user, s));
   TP_TRY(sum_epilogue((long long)T * h, h, part, nullptr, nullptr, dln2, R->num_sms, s));
   // LN2 backward (replicated): dh1 = dy + LN2'(dln2); the dres sum is db2
   TP_TRY(launch_ln_bwd(1, T, h, dln2, dy, h1, (const float*)P->ln2_g, mu2, rs2, dh1, lnp,
@@ -387,15 +494,22 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
   {
     AttnArgs a{R->cfg.micro_batch, R->cfg.seq, R->Hl, R->d, 1, qkv, (void*)O, (float*)lse,
                dO, Dsum, dqkv, err};
+    if (R->ws[W_DQACC].bytes) {
+      char* base = at(workspace, R->ws[W_DQACC]);
+      const DqScratch q = dq_scratch_layout(R->cfg.micro_batch, R->cfg.seq, R->Hl);
+      a.dq_fix = reinterpret_cast<int32_t*>(base + q.fix_off);
+      a.dq_exp = reinterpret_cast<int32_t*>(base + q.exp_off);
+      a.dq_bound = reinterpret_cast<float*>(base + q.bound_off);
+    }
     TP_TRY(launch_attn_bwd(1, a, s));
   }
   // QKV: db_qkv_t, dln1 partial -> all-reduce -> bf16, dW_qkv,t
-  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, biasp, s));
   {
     GemmArgs a = base(T, h, 3 * hl);
-    a.b_mn = 1; a.A = dqkv; a.lda = 3 * hl; a.B = P->w_qkv; a.ldb = h;
-    a.epi = kEpiStoreF32; a.out = part; a.ldc = h; a.err = err;
-    TP_TRY(launch_gemm_tc(a, R->num_sms, s));
+    a.b_mn = 1; a.lda = 3 * hl; a.B = P->w_qkv; a.ldb = h;
+    a.epi = kEpiStoreF32; a.ldc = h; a.err = err;
+    TP_TRY_ST(reduce_begin(R, a, dqkv, 3 * hl, part, allreduce, user, s));
   }
   {
     GemmArgs a = base(3 * hl, h, T);
@@ -403,7 +517,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err;
     TP_TRY(launch_gemm_tc(a, R->num_sms, s));
   }
-  TP_TRY_ST(allreduce(part, (int64_t)T * h, user, stream));
+  TP_TRY_ST(reduce_end(R, part, allreduce, user, s));
   TP_TRY(sum_epilogue((long long)T * h, h, part, nullptr, nullptr, dln1, R->num_sms, s));
   // LN1 backward (replicated): dx = dh1 + LN1'(dln1); the dres sum is db_o
   TP_TRY(launch_ln_bwd(1, T, h, dln1, dh1, x, (const float*)P->ln1_g, mu1, rs1, dx, lnp,

@@ -758,12 +758,15 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
 }
 
 // ---------------------------------------------------------------------------- column sums
-// out[c] = sum_r x[r, c]. Block = 32 x 8 threads covering 32*VEC columns; blockIdx.y splits
-// the rows; partial sums are combined with fp32 atomics into a zeroed `out`.
+// out[c] = sum_r x[r, c] in two deterministic passes. Pass 1: block = 32 x 8 threads covering
+// 32*VEC columns, blockIdx.y a slice of rows; each block writes its column sums to
+// partial[slice][c]. Pass 2 (colsum_reduce_kernel) adds the slices in a fixed order, so the
+// result does not depend on scheduling.
 template <typename T>
 __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
                                                      const T* __restrict__ x,
-                                                     float* __restrict__ out, long long rows_per) {
+                                                     float* __restrict__ partial,
+                                                     long long rows_per) {
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
   const int c0 = (blockIdx.x * 32 + threadIdx.x) * V;
@@ -800,9 +803,28 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
       float s = 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) s += red[k][cc];
-      atomicAdd(out + col, s);
+      partial[(long long)blockIdx.y * cols + col] = s;
     }
   }
+}
+
+// out[c] = sum over slices of partial[slice][c], slices in increasing order; four
+// independent chains per thread keep loads in flight.
+__global__ void __launch_bounds__(256) colsum_reduce_kernel(int cols, int slices,
+                                                            const float* __restrict__ partial,
+                                                            float* __restrict__ out) {
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  if (c >= cols) return;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int k = 0;
+  for (; k + 3 < slices; k += 4) {
+    a0 += partial[(long long)k * cols + c];
+    a1 += partial[(long long)(k + 1) * cols + c];
+    a2 += partial[(long long)(k + 2) * cols + c];
+    a3 += partial[(long long)(k + 3) * cols + c];
+  }
+  for (; k < slices; ++k) a0 += partial[(long long)k * cols + c];
+  out[c] = (a0 + a1) + (a2 + a3);
 }
 
 // ---------------------------------------------------------------------------- fp32 GEMM
@@ -865,16 +887,15 @@ __global__ void gemm_simt_f32_kernel(const GemmArgs a) {
       out[off] = acc;
       break;
     }
-    case kEpiGelu: {
+    case kEpiGelu: {  // out = GeLU(u), out2 = u
       if (bias) acc += bias[col];
-      float g, dg;
-      gelu_and_grad_f(acc, a.gelu_tanh, g, dg);
-      reinterpret_cast<float*>(a.out2)[off] = dg;
-      out[off] = g;
+      reinterpret_cast<float*>(a.out2)[off] = acc;
+      out[off] = gelu_f(acc, a.gelu_tanh);
       break;
     }
-    case kEpiDGelu: {
-      out[off] = acc * reinterpret_cast<const float*>(a.aux)[(long long)m * a.ld_aux + col];
+    case kEpiDGelu: {  // du = dA GeLU'(u), aux = u
+      out[off] = acc * gelu_grad_f(reinterpret_cast<const float*>(a.aux)[(long long)m * a.ld_aux + col],
+                                   a.gelu_tanh);
       break;
     }
     case kEpiDSwiglu: {  // acc = dA(m, ng*Ng + n); aux and out laid out [M][NG][2][Ng]
@@ -1102,23 +1123,34 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
                                         nblk, dgamma, dbeta, dres_sum, err, s);
 }
 
-cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
-                          cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * cols, s);
-  if (e != cudaSuccess || rows <= 0) return e;
+int colsum_slices(long long rows, int cols, int dtype) {
   const int V = dtype ? 8 : 4;
   const int cb = (cols + 32 * V - 1) / (32 * V);
   long long splits = (4 * 148 + cb - 1) / cb;  // aim for ~4 blocks per SM
+  if (splits > kColsumMaxSlices) splits = kColsumMaxSlices;
   if (splits > (rows + 7) / 8) splits = (rows + 7) / 8;
   if (splits < 1) splits = 1;
   const long long rows_per = (rows + splits - 1) / splits;
-  dim3 grid(cb, (unsigned)splits), block(32, 8);
+  return (int)((rows + rows_per - 1) / rows_per);
+}
+
+cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
+                          float* partial, cudaStream_t s) {
+  if (rows <= 0) return cudaMemsetAsync(out, 0, sizeof(float) * cols, s);
+  const int V = dtype ? 8 : 4;
+  const int cb = (cols + 32 * V - 1) / (32 * V);
+  const int slices = colsum_slices(rows, cols, dtype);
+  const long long rows_per = (rows + slices - 1) / slices;
+  dim3 grid(cb, (unsigned)slices), block(32, 8);
   if (dtype)
     colsum_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        rows, cols, reinterpret_cast<const __nv_bfloat16*>(x), out, rows_per);
+        rows, cols, reinterpret_cast<const __nv_bfloat16*>(x), partial, rows_per);
   else
     colsum_kernel<float><<<grid, block, 0, s>>>(rows, cols, reinterpret_cast<const float*>(x),
-                                                 out, rows_per);
+                                                 partial, rows_per);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  colsum_reduce_kernel<<<(cols + 255) / 256, 256, 0, s>>>(cols, slices, partial, out);
   return cudaGetLastError();
 }
 

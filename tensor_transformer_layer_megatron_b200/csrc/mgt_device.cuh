@@ -460,6 +460,16 @@ __device__ __forceinline__ void gelu_and_grad_bf16out(float u, int tanh_form, fl
   g = u * cdf;
   dg = fmaf(u * 0.3989422804014327f, e, cdf);
 }
+__device__ __forceinline__ float gelu_bf16out(float u, int tanh_form) {
+  float g, dg;
+  gelu_and_grad_bf16out(u, tanh_form, g, dg);
+  return g;
+}
+__device__ __forceinline__ float gelu_grad_bf16out(float u, int tanh_form) {
+  float g, dg;
+  gelu_and_grad_bf16out(u, tanh_form, g, dg);
+  return dg;
+}
 // SiLU z*sigmoid(z) and its derivative sigmoid(z)*(1 + z*(1 - sigmoid(z))): accurate form
 // (expf, IEEE division) for fp32 results, and a form from ex2.approx and rcp.approx for bf16
 // results (relative error near 2^-21, far below bf16 rounding).

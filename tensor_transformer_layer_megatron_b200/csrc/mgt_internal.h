@@ -22,8 +22,8 @@ enum DeviceError : int {
 enum Epilogue : int {
   kEpiStoreF32 = 0,  // out (fp32) = acc                     (weight gradients)
   kEpiBf16 = 1,      // out (act) = acc [+ bias] [+ residual] (QKV, out-proj, fc2, dgrads)
-  kEpiGelu = 2,      // u = acc + bias; out = GeLU(u), out2 = GeLU'(u) (fc1)
-  kEpiDGelu = 3,     // out = acc * aux, aux = GeLU'(u)        (fc2 dgrad -> du)
+  kEpiGelu = 2,      // u = acc + bias; out = GeLU(u), out2 = u (fc1)
+  kEpiDGelu = 3,     // out = acc * GeLU'(aux), aux = u        (fc2 dgrad -> du)
   // SwiGLU fc1 (GLU tiles): group ng holds Ng outputs; B rows ng*2Ng + n (gate) and
   // ng*2Ng + Ng + n (up) feed output (m, ng*Ng + n). out[m*ldc + ng*Ng + n] = silu(g) * u;
   // out2[m*ldc2 + ng*2Ng + n] = g, out2[... + Ng] = u (g, u include the bias, indexed like
@@ -52,11 +52,11 @@ struct GemmArgs {
   // Epilogue.
   int epi;
   void* out; long long ldc; int out_ng; long long out_gs;
-  void* out2;                           // kEpiGelu: GeLU'(u) (same addressing as out)
+  void* out2;                           // kEpiGelu: u (same addressing as out)
   long long ldc2;                       // kEpiSwiglu: row stride of out2
   const void* bias;                     // indexed by col; nullable
   const void* res; long long ldr;       // residual, res[m*ldr + col]; nullable
-  const void* aux; long long ld_aux;    // kEpiDGelu: GeLU'(u)[m*ld_aux + col]
+  const void* aux; long long ld_aux;    // kEpiDGelu: u[m*ld_aux + col]
   int gelu_tanh;
   int* err;                             // device status word
   // Sequence-parallel layout: token m (= batch * seq + position) of an operand or output held
@@ -133,9 +133,13 @@ cudaError_t launch_fp8_quantize(int dtype, long long n, const void* x, uint8_t* 
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
 
-// Column sums of a [rows, cols] activation matrix into fp32 (bias gradients).
+// Column sums of a [rows, cols] activation matrix into fp32 (bias gradients), deterministic:
+// per-slice partial sums in `partial` (colsum_slices(...) * cols floats, at most
+// kColsumMaxSlices * cols), then a fixed-order reduction of the slices.
+constexpr int kColsumMaxSlices = 32;
+int colsum_slices(long long rows, int cols, int dtype);
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
-                          cudaStream_t stream);
+                          float* partial, cudaStream_t stream);
 
 // Causal attention over packed qkv [T][p][3][H/p][d]; O [T][p][H/p][d]; lse [b][H][s].
 struct AttnArgs {
@@ -143,11 +147,36 @@ struct AttnArgs {
   const void* qkv; void* o; float* lse;
   const void* dO; float* Dsum; void* dqkv;
   int* err;
+  // Single-kernel backward (head_dim 128; null dq_fix selects the two-kernel backward):
+  //   dq_fix   int32 [T][H][d]: dQ accumulated in fixed point (integer adds are associative,
+  //            so the sum does not depend on the order in which key blocks arrive)
+  //   dq_bound float [b*H][ceil(s/128)][3]: per 128-token chunk, max |K|, max |V row|^2,
+  //            max |dO row|^2, from which every partial sum of dQ is bounded
+  //   dq_exp   int32 [b*H]: the power of two that scales each head's dQ to fixed point
+  int32_t* dq_fix;
+  float* dq_bound;
+  int32_t* dq_exp;
 };
+// Bytes of the single-kernel backward's dQ scratch (dq_fix, dq_exp, dq_bound) and where each
+// part starts, for b sequences of s tokens, H heads of 128.
+struct DqScratch {
+  size_t fix_off, exp_off, bound_off, bytes;
+};
+inline DqScratch dq_scratch_layout(long long b, long long s, long long H) {
+  DqScratch r;
+  const long long nchunk = (s + 127) / 128;
+  r.fix_off = 0;
+  r.exp_off = (size_t)b * s * H * 128 * 4;
+  r.bound_off = r.exp_off + (((size_t)b * H * 4 + 255) / 256) * 256;
+  r.bytes = r.bound_off + (size_t)b * H * nchunk * 3 * 4;
+  return r;
+}
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t stream);  // bf16, d in {64, 128}
-// bf16 backward: dQ kernel (which also writes a.Dsum = rowsum(dO * O)) then dK/dV kernel,
-// both tcgen05.
+// bf16 backward on tcgen05. With a.dq_fix (head_dim 128): D = rowsum(dO * O), the bounds of
+// dQ and a zeroed fixed-point dQ accumulator, then one key-stationary kernel computing dK, dV
+// and adding dQ, then the dQ conversion to bf16. Otherwise: dQ kernel (which also writes
+// a.Dsum) then dK/dV kernel.
 cudaError_t launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_bwd(int dtype, const AttnArgs& a, cudaStream_t stream);
 

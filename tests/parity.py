@@ -75,12 +75,10 @@ def gpu_intermediates(cfg, layer, run):
         dqkv=v(run.ws, "dqkv", act, (T, p, 3, H // p, d)),
         dln1=v(run.ws, "dln1", act, (T, h)),
     )
-    if getattr(cfg, "swiglu", 0):  # the fc1 pre-activations [gate | up] and their gradient
-        out["u"] = v(run.saved, "fc1_dgelu", act, (T, p, 2, f // p))
-        out["du"] = v(run.ws, "du", act, (T, p, 2, f // p))
-    else:
-        out["gelu_grad"] = v(run.saved, "fc1_dgelu", act, (T, p, f // p))
-        out["du"] = v(run.ws, "du", act, (T, p, f // p))
+    # the fc1 pre-activations u (SwiGLU: [gate | up]) and their gradient
+    u_shape = (T, p, 2, f // p) if getattr(cfg, "swiglu", 0) else (T, p, f // p)
+    out["u"] = v(run.saved, "fc1_u", act, u_shape)
+    out["du"] = v(run.ws, "du", act, u_shape)
     return out
 
 
@@ -103,11 +101,7 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
     if intermediates:
         gi = gpu_intermediates(cfg, layer, run)
         ref = dict(ln1=saved["ln1"], qkv=saved["qkv"], O=saved["O"], lse=saved["lse"],
-                   h1=saved["h1"], ln2=saved["ln2"], a=saved["a"], **inter)
-        if getattr(cfg, "swiglu", 0):
-            ref["u"] = saved["u"]
-        else:
-            ref["gelu_grad"] = lambda: oracle.gelu_grad(saved["u"], cfg.gelu_tanh)
+                   h1=saved["h1"], ln2=saved["ln2"], a=saved["a"], u=saved["u"], **inter)
         del inter
         for k, fetch in gi.items():
             r = ref.pop(k)

@@ -95,7 +95,7 @@ def test_region_layout(cfg):
     T, h, f, e = cfg.tokens, cfg.hidden, cfg.ffn, 2 if cfg.dtype == "bf16" else 4
     f1 = cfg.fc1_rows  # SwiGLU keeps [gate | up] and its gradient: 2f columns
     expect = {"ln1": T * h * e, "qkv": 3 * T * h * e, "attn_o": T * h * e,
-              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_dgelu": T * f1 * e,
+              "attn_lse": cfg.micro_batch * cfg.heads * cfg.seq * 4, "fc1_u": T * f1 * e,
               "fc1_a": T * f * e, "du": T * f1 * e, "dqkv": 3 * T * h * e}
     spans = []
     for name, rid in mgt.REGIONS.items():

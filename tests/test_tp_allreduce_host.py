@@ -1,8 +1,9 @@
 """The process-group all-reduce that tensor-parallel ranks get from the binding
 (process_group_allreduce), on two gloo ranks with CPU workspaces: the callback must locate
-the partial buffer inside the rank's workspace from the pointer the layer passes, sum it over
-the ranks in place, leave the rest of the workspace alone, and reject a pointer outside the
-workspace."""
+the partial buffer inside the rank's workspace from the pointer the layer passes -- the whole
+buffer, or one row band of it when the shard sums are banded (mgt_tp_rank_set_bands) -- sum it
+over the ranks in place, leave the rest of the workspace alone, and reject a pointer outside
+the partial buffer."""
 import datetime
 import os
 import socket
@@ -34,16 +35,25 @@ def _rank(rank, world, port, out):
         ws[:off] = 7
         part = ws[off:off + 4 * count].view(torch.float32)
         part.copy_(torch.arange(count, dtype=torch.float32) * (rank + 1))
-        ar = mgt.process_group_allreduce(ws, off)
+        ar = mgt.process_group_allreduce(ws, off, 4 * count)
         ar(ws.data_ptr() + off, count, 0)
-        want = torch.arange(count, dtype=torch.float32) * sum(r + 1 for r in range(world))
+        total = sum(r + 1 for r in range(world))
+        want = torch.arange(count, dtype=torch.float32) * total
         ok = torch.equal(part, want) and bool((ws[:off] == 7).all()) and \
             bool((ws[off + 4 * count:] == 0).all())
-        try:
-            ar(ws.data_ptr(), count, 0)
-            rejected = False
-        except ValueError:
-            rejected = True
+        # banded: three row bands in order, each summed on its own
+        part.copy_(torch.arange(count, dtype=torch.float32) * (rank + 1))
+        for b0, b1 in ((0, 400), (400, 800), (800, 1000)):
+            ar(ws.data_ptr() + off + 4 * b0, b1 - b0, 0)
+        ok = ok and torch.equal(part, want) and bool((ws[off + 4 * count:] == 0).all())
+        rejected = True
+        for ptr, n in ((ws.data_ptr(), count), (ws.data_ptr() + off + 4, count),
+                       (ws.data_ptr() + off + 2, 10), (ws.data_ptr() + off + 4 * 990, 20)):
+            try:
+                ar(ptr, n, 0)
+                rejected = False
+            except ValueError:
+                pass
         out.put((rank, ok, rejected))
     finally:
         dist.destroy_process_group()

@@ -27,7 +27,13 @@ SHARDED = ("w_qkv", "b_qkv", "w_o", "w1", "b1", "w2")
 LN = ("ln1_g", "ln1_b", "ln2_g", "ln2_b")
 
 
-def _run_ranks(cfg, t):
+def _band_sizes(T, bands):
+    """Rows of each band: an even split rounded up to whole 128-row tiles."""
+    per = ((T + bands - 1) // bands + 127) // 128 * 128
+    return [min(per, T - r0) for r0 in range(0, T, per)]
+
+
+def _run_ranks(cfg, t, bands=1):
     p = cfg.tp_size
     packed = pack_params(cfg, t)
     dev = torch.device("cuda", 0)
@@ -36,6 +42,8 @@ def _run_ranks(cfg, t):
         rk = mgt.TPRank(cfg.hidden, cfg.heads, cfg.ffn, cfg.seq, cfg.micro_batch, p, r,
                         cfg.ln_eps, cfg.gelu_tanh, swiglu=cfg.swiglu,
                         disable_bias_linear=cfg.disable_bias_linear)
+        if bands > 1:
+            rk.set_bands(bands)
         shard = {k: (v[r] if k in SHARDED else v)
                  .to(device=dev, dtype=torch.float32 if k in LN else torch.bfloat16)
                  .contiguous() for k, v in packed.items()}
@@ -57,14 +65,21 @@ def _run_ranks(cfg, t):
     shared = {}
     calls = [0] * p
 
+    sizes = _band_sizes(cfg.tokens, bands)
+    row_bytes = 4 * cfg.hidden
+
     def make_allreduce(r):
         def allreduce(ptr, count, stream):
+            # the reductions arrive band by band, in row order, inside the partial buffer; one
+            # band comes on the caller's stream, several on the rank's communication stream
             ws = bufs[r]["ws"]
-            assert ptr == ws.data_ptr() + off and count * 4 == nbytes
-            assert stream == streams[r].cuda_stream
+            band = calls[r] % len(sizes)
+            start = off + row_bytes * sum(sizes[:band])
+            assert ptr == ws.data_ptr() + start and count * 4 == row_bytes * sizes[band]
+            assert (stream == streams[r].cuda_stream) == (bands == 1)
             calls[r] += 1
-            view = ws[off:off + nbytes].view(torch.float32)
-            streams[r].synchronize()
+            view = ws[start:start + 4 * count].view(torch.float32)
+            torch.cuda.ExternalStream(stream, device=dev).synchronize()
             views[r] = view
             barrier.wait()
             if r == 0:
@@ -75,7 +90,7 @@ def _run_ranks(cfg, t):
                 shared["total"] = total
             barrier.wait()
             view.copy_(shared["total"])
-            streams[r].synchronize()
+            torch.cuda.synchronize(dev)
             barrier.wait()  # every rank holds the sum before the next reduction reuses it
         return allreduce
 
@@ -101,7 +116,7 @@ def _run_ranks(cfg, t):
         th.join(timeout=300)
     torch.cuda.synchronize()
     assert not errors, errors
-    assert calls == [4] * p, calls
+    assert calls == [4 * len(sizes)] * p, calls
     for b in bufs:  # device status word: no bounded wait gave up
         assert int(b["ws"][:4].view(torch.int32).item()) == 0
     return packed, bufs
@@ -118,10 +133,11 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("bands", [1, 2])
 @pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
-def test_tp_ranks_match_oracle(cfg):
+def test_tp_ranks_match_oracle(cfg, bands):
     t = make_inputs(cfg, nonzero_affine=True)
-    packed, bufs = _run_ranks(cfg, t)
+    packed, bufs = _run_ranks(cfg, t, bands)
     y_ref, saved = oracle.layer_fwd(cfg, packed, t["x"])
     dx_ref, g_ref, _ = oracle.layer_bwd(cfg, packed, saved, t["dy"])
     for r, b in enumerate(bufs):
