@@ -105,6 +105,8 @@ def load_library():
     lib.mgt_tp_rank_destroy.argtypes = [vp]
     lib.mgt_tp_rank_destroy.restype = None
     lib.mgt_debug_bounded_wait.argtypes = [ctypes.c_int64, vp, vp]
+    lib.mgt_debug_exp2.argtypes = [i32, ctypes.c_int64, vp, vp, vp]
+    lib.mgt_debug_exp2.restype = ctypes.c_int
     lib.mgt_layer_status_word.argtypes = [vp, vp, ctypes.POINTER(vp)]
     lib.mgt_debug_bounded_wait.restype = ctypes.c_int
     lib.mgt_layer_status_word.restype = ctypes.c_int
@@ -416,6 +418,17 @@ def layernorm_bwd_noalloc(dtype, rows, h, dy, dres, x, gamma, mean, rstd, dx, dg
                                          _ptr(dres), _ptr(x), _ptr(gamma), _ptr(mean),
                                          _ptr(rstd), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
                                          _stream_handle(stream)), "mgt_layernorm_bwd_noalloc")
+
+
+def debug_exp2(x, y, path, stream=None):
+    """y = 2^x through the attention kernels' exponential (see mgt_debug_exp2): path 0 the
+    hardware approximation, 1 the FMA-pipe polynomial. x, y fp32 device tensors."""
+    import torch
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or y.numel() < x.numel():
+        raise TypeError("debug_exp2 takes fp32 x and y")
+    lib = load_library()
+    _check(lib.mgt_debug_exp2(int(path), x.numel(), _ptr(x), _ptr(y), _stream_handle(stream)),
+           "mgt_debug_exp2")
 
 
 def debug_bounded_wait(limit_ns, status_ptr, stream=None):

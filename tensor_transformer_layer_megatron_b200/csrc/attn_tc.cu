@@ -217,56 +217,85 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[128];
-      {
-        uint32_t raw[4][32];
+      // Two passes over the row in TMEM, 64 then 32 scores in registers at a time: the row
+      // maximum first, then P = 2^(S*scale*log2e - m) chunk by chunk, packed to bf16 and
+      // written back over the scores already consumed (P of chunk c -> columns 16c..16c+15),
+      // so that the exponentials' temporaries fit beside the scores.
+      const bool diag = kb == qb;  // keys after this query are masked
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, raw[c]);
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, ra);
+        tmem_ld_32x32b_x32_nw(lane_base + s_col + (c + 1) * 32, rb);
         tmem_ld_wait();
+        reg_fence(ra);
+        reg_fence(rb);
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          reg_fence(raw[c]);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[c][i]);
+          for (int i = 0; i < 32; ++i) {
+            if (c * 32 + i > r) ra[i] = __float_as_uint(-INFINITY);
+            if ((c + 1) * 32 + i > r) rb[i] = __float_as_uint(-INFINITY);
+          }
         }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            m4[k] = fmax3(m4[k], __uint_as_float(ra[i + k]), __uint_as_float(rb[i + k]));
       }
-      if (kb == qb) {  // diagonal block: keys after this query are masked
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > r) sv[i] = -INFINITY;
-      }
-      // row max (raw scores; the scale is positive): eight independent chains, then a tree
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = sv[k];
-#pragma unroll
-      for (int i = 8; i < 128; i += 8)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], sv[i + k]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;
+      const float mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
       const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
-      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // exponentials on pairs of scores; off the diagonal (no masked -inf) three pairs in
+      // eight take the polynomial 2^x on the FMA pipe, the rest the special-function unit
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
+      uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const float p = ex2_approx(fmaf(sv[i], scale_log2, -m_run));
-        sv[i] = p;
-        r8[i & 7] += p;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t raw[32];
+        tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, raw);
+        tmem_ld_wait();
+        reg_fence(raw);
+        uint32_t pw[16];
+        if (diag) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float pa, pb;
+            f2_unpack(f2_fma(f2_pack(c * 32 + i > r ? -INFINITY : __uint_as_float(raw[i]),
+                                     c * 32 + i + 1 > r ? -INFINITY : __uint_as_float(raw[i + 1])),
+                             c2, nm2),
+                      pa, pb);
+            pa = ex2_approx(pa);
+            pb = ex2_approx(pb);
+            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(pa, pb));
+            pw[i >> 1] = pack_bf16x2(pa, pb);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float pa, pb;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1])), c2,
+                             nm2),
+                      pa, pb);
+            const int jp = (i >> 1) & 7;
+            if (jp == 1 || jp == 4 || jp == 6) {
+              exp2_poly_pair(pa, pb);
+            } else {
+              pa = ex2_approx(pa);
+              pb = ex2_approx(pb);
+            }
+            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(pa, pb));
+            pw[i >> 1] = pack_bf16x2(pa, pb);
+          }
+        }
+        tmem_st_32x32b_x16(lane_base + s_col + c * 16, pw);
       }
-      l_run = l_run * alpha +
-              (((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7])));
-      // P (bf16 pairs) into the first 64 columns of this tile's S buffer: this thread's own
-      // row, read completely above, so nothing else is overwritten.
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float pw[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          pw[j] = __uint_as_float(pack_bf16x2(sv[c * 64 + 2 * j], sv[c * 64 + 2 * j + 1]));
-        tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);
-      }
+      float rs[4];
+      f2_unpack(acc2[0], rs[0], rs[1]);
+      f2_unpack(acc2[1], rs[2], rs[3]);
+      l_run = l_run * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       // O holds the sum up to block kb-1 (its PV completed before this S was committed); it
       // is rescaled before this block's PV, which waits for p_full below.
       if (kb > 0 && __any_sync(0xffffffffu, need)) {
@@ -939,8 +968,9 @@ struct FusedBwdLayout {
   static constexpr int TILE = 128 * D * 2;
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE, DO_OFF = 4 * TILE;  // Q, dO x2
   static constexpr int DS_OFF = 6 * TILE;           // dS^T [128 keys][64 queries] bf16
-  static constexpr int STAT_OFF = DS_OFF + 16384;   // float lse2[2][128], dsum[2][128]
-  static constexpr int BAR_OFF = STAT_OFF + 4 * 128 * 4;
+  static constexpr int STG_OFF = DS_OFF + 16384;    // dQ staging: 4 warps x [16 q][32 d] int32
+  static constexpr int STAT_OFF = STG_OFF + 8192;   // [2 stages][-lse*log2e | -D][128 queries]
+  static constexpr int BAR_OFF = STAT_OFF + 2048;
   static constexpr int BYTES = BAR_OFF + 256 + 1024;
   // TMEM buffer x (sub-block parity) at x*128: S^T in +0..63 (P^T packed into its first
   // halves), dP^T in +64..127 (then dQ^T); dV and dK accumulators above.
@@ -951,7 +981,8 @@ constexpr int kFusedBwdThreads = 448;
 template <int D>
 __global__ void __launch_bounds__(kFusedBwdThreads, 1)
     attn_bwd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
-                             const __grid_constant__ CUtensorMap tm_do, const AttnArgs a,
+                             const __grid_constant__ CUtensorMap tm_do,
+                             const __grid_constant__ CUtensorMap tm_dq, const AttnArgs a,
                              float scale_log2, float scale) {
   using L = FusedBwdLayout<D>;
   static_assert(D == 128, "dQ^T tiles use M = head_dim = 128");
@@ -967,12 +998,10 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
   uint64_t* dq_full = bars + 10;   // [2]: dQ^T of a sub-block is in buffer x
   uint64_t* dq_empty = bars + 12;  // [2]: the drain warps have read it
   uint64_t* drain = bars + 14;     // every MMA done (the output reads dV, dK after it)
-  uint64_t* stat_bar = bars + 15;  // [2]: per-query stats of a block staged by the 8 warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* lse_s = reinterpret_cast<float*>(smem + L::STAT_OFF);  // [2][128], log2 units
-  float* dsum_s = lse_s + 256;                                   // [2][128]
   uint8_t* ds_buf = smem + L::DS_OFF;
+  float* stat_s = reinterpret_cast<float*>(smem + L::STAT_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.s, H = a.H, hp = H / a.p;
@@ -994,7 +1023,6 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
       mbar_init(&p_full[i], 8);
       mbar_init(&dq_full[i], 1);
       mbar_init(&dq_empty[i], 4);
-      mbar_init(&stat_bar[i], 256);
     }
     mbar_init(ds_empty, 1);
     mbar_init(drain, 1);
@@ -1002,6 +1030,7 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -1026,7 +1055,7 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
         const int st = it & 1, qi = kb + it;
         if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, a.err, kErrTimeoutAttn, abort_flag))
           break;
-        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE);
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + 1024);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c) {
           tma_load_3d(&tm_qkv, &q_full[st], smem + L::Q_OFF + st * L::TILE + c * 16384,
@@ -1034,6 +1063,10 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
           tma_load_3d(&tm_do, &q_full[st], smem + L::DO_OFF + st * L::TILE + c * 16384,
                       n * D + c * 64, qi * 128, b);
         }
+        // the block's -lse*log2(e) and -D rows (padded past the sequence by the pre-pass)
+        const float* srow = a.dq_stat + (long long)bh * 2 * (nq * 128) + qi * 128;
+        bulk_load_1d(stat_s + st * 256, srow, 512, &q_full[st]);
+        bulk_load_1d(stat_s + st * 256 + 128, srow + nq * 128, 512, &q_full[st]);
         issued = it + 1;
       }
       mbar_wait(kv_full, 0, a.err, kErrTimeoutDrain, nullptr);
@@ -1123,77 +1156,67 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
   } else if (warp >= 10) {
     // ------------------------------------------------------------ dQ drain
     // Thread = row dd of dQ^T (one of the head dimensions); the 64 columns are the queries of
-    // the sub-block. A warp's reduction for one query covers 32 consecutive dd: 128 bytes.
+    // the sub-block. Each warp converts its 32 rows to fixed point, stages them 16 queries at
+    // a time as a [query][d] box in shared memory and hands the box to one bulk tensor
+    // reduce-add (integer add in L2), so the additions cost the warp no per-element
+    // instructions.
     const int quarter = warp & 3;
-    const int dd = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    int32_t* acc = a.dq_fix + (long long)b * S * H * D + (long long)n * D + dd;
-    const long long ldq = (long long)H * D;
+    int32_t* stg = reinterpret_cast<int32_t*>(smem + L::STG_OFF) + (warp - 10) * 512;
     // this head's fixed-point scale (the same computation in every CTA of the head)
     const int e = dq_fixed_exponent(a.dq_bound + (long long)bh * ((S + 127) / 128) * 3,
                                     (S + 127) / 128);
     if (kb == 0 && quarter == 0 && lane == 0) a.dq_exp[bh] = e;
     const float fscale = exp2f((float)e);
+    bool issued = false;
     for (int g = 0; g < G; ++g) {
       const bool ok = mbar_wait(&dq_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn,
                                 abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t x = (g & 1) * L::T_SUB;
-      uint32_t v0[32], v1[32];
-      tmem_ld_32x32b_x32_nw(lane_base + x + 64, v0);
-      tmem_ld_32x32b_x32_nw(lane_base + x + 96, v1);
+      uint32_t v[2][32];
+      tmem_ld_32x32b_x32_nw(lane_base + x + 64, v[0]);
+      tmem_ld_32x32b_x32_nw(lane_base + x + 96, v[1]);
       tmem_ld_wait();
-      reg_fence(v0);
-      reg_fence(v1);
+      reg_fence(v[0]);
+      reg_fence(v[1]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dq_empty[g & 1]);
       const int q0 = (kb + (g >> 1)) * 128 + (g & 1) * 64;
-      const int nvalid = S - q0 < 64 ? S - q0 : 64;
-      int32_t* row = acc + (long long)q0 * ldq;
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i < nvalid)
-          atomicAdd(row + (long long)i * ldq, __float2int_rn(__uint_as_float(v0[i]) * fscale));
+      for (int hh = 0; hh < 4; ++hh) {  // four boxes of 16 queries
+        if (q0 + hh * 16 >= S) break;  // rows past the sequence are clipped; none left here
+        if (lane == 0 && issued) bulk_wait_read0();  // the previous box has been read
+        __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (32 + i < nvalid)
-          atomicAdd(row + (long long)(32 + i) * ldq,
-                    __float2int_rn(__uint_as_float(v1[i]) * fscale));
+        for (int i = 0; i < 16; ++i)
+          stg[i * 32 + lane] = __float2int_rn(__uint_as_float(v[hh >> 1][(hh & 1) * 16 + i]) * fscale);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stg, n * D + quarter * 32, q0 + hh * 16, b);
+          bulk_commit();
+        }
+        issued = true;
+      }
     }
+    if (lane == 0 && issued) bulk_wait0();  // every reduction has landed in global memory
   } else {
     // ------------------------------------------------------------ P^T, dS^T and the output
     // warp w: TMEM lane quarter w%4 (key rows), 32-query half w/4 of each 64-query sub-block
     const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // key row within the block = TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const float* lse_g = a.lse + ((long long)b * H + n) * S;
-    const float* dsum_g = a.Dsum + ((long long)b * H + n) * S;
+    // per-query -lse*log2(e) and -D of the current query block (padded past the sequence
+    // with -inf and 0, so P = 0 there), brought into shared memory with Q and dO
     // this thread's dS^T row in the swizzled buffer: 16-byte chunk c of the row sits at
     // chunk c ^ (r % 8)
     uint8_t* ds_row = ds_buf + r * 128;
     bool ok = true;
-    const float* stat_g = hf ? dsum_g : lse_g;
-    float* stat_s = hf ? dsum_s : lse_s;
-    auto fetch = [&](int qi) -> float {
-      const int q = qi * 128 + r;  // padded queries get lse = +inf, hence P = 0
-      if (hf == 0) return q < S ? stat_g[q] * kLog2eF : INFINITY;
-      return q < S ? stat_g[q] : 0.f;
-    };
-    float nv = niter > 0 ? fetch(kb) : 0.f;
     for (int g = 0; g < G; ++g) {
       const int it = g >> 1, j = g & 1, st = it & 1, qi = kb + it;
-      if (j == 0) {
-        stat_s[st * 128 + r] = nv;
-        if (it + 1 < niter) nv = fetch(qi + 1);
-        mbar_arrive(&stat_bar[st]);
-        ok = mbar_wait(&stat_bar[st], (it >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-      }
       ok = mbar_wait(&s_full[g & 1], (g >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
@@ -1202,8 +1225,8 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
       tc_fence_after();
       const uint32_t x = (g & 1) * L::T_SUB;
       const int q0 = j * 64 + hf * 32;  // first query (within the block) of this warp's columns
-      const float* ls = lse_s + st * 128 + q0;
-      const float* ds_ = dsum_s + st * 128 + q0;
+      const float* ls = stat_s + st * 256 + q0;
+      const float* ds_ = stat_s + st * 256 + 128 + q0;
       uint32_t sr[32], dr[32];
       tmem_ld_32x32b_x32_nw(lane_base + x + hf * 32, sr);
       tmem_ld_32x32b_x32_nw(lane_base + x + 64 + hf * 32, dr);
@@ -1215,22 +1238,37 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
         for (int i = 0; i < 32; ++i)
           if (q0 + i < r) sr[i] = __float_as_uint(-INFINITY);
       }
+      // P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D) on pairs of queries;
+      // off the diagonal (no masked -inf) three pairs in eight take the polynomial 2^x on the
+      // FMA pipe, the rest the SFU
       uint32_t pw[16], dw[16];
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+      const bool diag = qi == kb;
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(ls + i);
-        const float4 d4 = *reinterpret_cast<const float4*>(ds_ + i);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float p4[4], q4[4];
+        const float4 l4 = *reinterpret_cast<const float4*>(ls + i);   // -lse * log2e
+        const float4 d4 = *reinterpret_cast<const float4*>(ds_ + i);  // -D
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          p4[e] = ex2_approx(fmaf(__uint_as_float(sr[i + e]), scale_log2, -lv[e]));
-          q4[e] = p4[e] * (__uint_as_float(dr[i + e]) - dv[e]);
+        for (int e = 0; e < 4; e += 2) {
+          float pa, pb;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i + e]), __uint_as_float(sr[i + e + 1])),
+                           c2, e ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y)),
+                    pa, pb);
+          const int jp = ((i + e) >> 1) & 7;
+          if (!diag && (jp == 1 || jp == 4 || jp == 6)) {
+            exp2_poly_pair(pa, pb);
+          } else {
+            pa = ex2_approx(pa);
+            pb = ex2_approx(pb);
+          }
+          const uint64_t dpd = f2_add(
+              f2_pack(__uint_as_float(dr[i + e]), __uint_as_float(dr[i + e + 1])),
+              e ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y));
+          float qa, qb;
+          f2_unpack(f2_mul(f2_pack(pa, pb), dpd), qa, qb);
+          pw[(i + e) >> 1] = pack_bf16x2(pa, pb);
+          dw[(i + e) >> 1] = pack_bf16x2(qa, qb);
         }
-        pw[i >> 1] = pack_bf16x2(p4[0], p4[1]);
-        pw[(i >> 1) + 1] = pack_bf16x2(p4[2], p4[3]);
-        dw[i >> 1] = pack_bf16x2(q4[0], q4[1]);
-        dw[(i >> 1) + 1] = pack_bf16x2(q4[2], q4[3]);
       }
       // P^T packed into the first half of the 32 columns this warp itself read, so the other
       // warp of the quarter (reading its own 32 columns) is never overwritten.
@@ -1310,9 +1348,17 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
   const int H = a.H, hp = H / a.p, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const long long ld_qkv = 3LL * H * D, ld_o = (long long)H * D;
   float kmax = 0.f, v2max = 0.f, g2max = 0.f;
+  const long long nqp = (long long)nchunk * 128;
+  float* stat = a.dq_stat + (long long)bh * 2 * nqp;
   for (int i = 0; i < 16; ++i) {
     const int pos = c * 128 + warp * 16 + i;
-    if (pos >= a.s) break;  // warp-uniform
+    if (pos >= a.s) {  // warp-uniform: padding of the softmax statistics (P = 0 there)
+      if (lane == 0) {
+        stat[pos] = -INFINITY;
+        stat[nqp + pos] = 0.f;
+      }
+      continue;
+    }
     const long long tok = (long long)b * a.s + pos;
     const long long oo = tok * ld_o + (long long)n * D + lane * 4;
     const long long ko = tok * ld_qkv + (long long)t * 3 * hp * D + (long long)(hp + jh) * D + lane * 4;
@@ -1339,7 +1385,11 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
       v2 += __shfl_xor_sync(0xffffffffu, v2, m);
       km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, m));
     }
-    if (lane == 0) a.Dsum[(long long)bh * a.s + pos] = dsum;
+    if (lane == 0) {
+      a.Dsum[(long long)bh * a.s + pos] = dsum;
+      stat[pos] = -a.lse[(long long)bh * a.s + pos] * kLog2eF;
+      stat[nqp + pos] = -dsum;
+    }
     *reinterpret_cast<int4*>(a.dq_fix + oo) = make_int4(0, 0, 0, 0);
     kmax = fmaxf(kmax, km);
     v2max = fmaxf(v2max, v2);
@@ -1411,9 +1461,17 @@ cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
   attn_bwd_prep_kernel<<<dim3(a.b * a.H, (a.s + 127) / 128), 256, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  CUtensorMap tm_dq;  // the fixed-point dQ accumulator as [b][s][H*d] int32, 32 x 16 boxes
+  {
+    const uint64_t dims[3] = {hd, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {hd, hd * a.s};
+    const uint32_t qbox[3] = {32, 16, 1};
+    if (!make_tensor_map_i32_3d(&tm_dq, a.dq_fix, dims, strides, qbox))
+      return cudaErrorInvalidValue;
+  }
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
-  attn_bwd_fused_tc_kernel<D><<<grid, kFusedBwdThreads, L::BYTES, s>>>(tm_qkv, tm_do, a,
-                                                                       kLog2eF * scale, scale);
+  attn_bwd_fused_tc_kernel<D><<<grid, kFusedBwdThreads, L::BYTES, s>>>(
+      tm_qkv, tm_do, tm_dq, a, kLog2eF * scale, scale);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(a, scale);
   return cudaGetLastError();

@@ -959,6 +959,20 @@ bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t di
   return r == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_i32_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
+                            const uint64_t strides[2], const uint32_t box[3]) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t gs[2] = {strides[0] * 4, strides[1] * 4};
+  cuuint32_t bd[3] = {box[0], box[1], box[2]};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, const_cast<void*>(base), gd, gs, bd, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],

@@ -558,6 +558,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
       a.dq_fix = reinterpret_cast<int32_t*>(base + q.fix_off);
       a.dq_exp = reinterpret_cast<int32_t*>(base + q.exp_off);
       a.dq_bound = reinterpret_cast<float*>(base + q.bound_off);
+      a.dq_stat = reinterpret_cast<float*>(base + q.stat_off);
     }
     const double fl = 2.5 * 2.0 * L->cfg.micro_batch * (double)L->cfg.seq * L->cfg.seq * h;  // model FLOPs incl. one recompute of S
     MGT_TRY(run(L, "attn_bwd", fl, 0, s, [&] { return launch_attn_bwd(dt, a, s); }));
@@ -663,6 +664,12 @@ mgt_status mgt_debug_bounded_wait(int64_t limit_ns, int32_t* status, void* strea
   return cuda_status(launch_bounded_wait_probe(reinterpret_cast<int*>(status),
                                                (unsigned long long)limit_ns,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+mgt_status mgt_debug_exp2(int32_t path, int64_t n, const float* x, float* y, void* stream) {
+  if (n < 0 || (n && (!x || !y)) || (path != 0 && path != 1)) return MGT_EINVAL;
+  if (n == 0) return MGT_OK;
+  return cuda_status(launch_exp2_probe(path, n, x, y, static_cast<cudaStream_t>(stream)));
 }
 
 mgt_status mgt_layer_status_word(mgt_layer* L, void* workspace, int32_t** word) {

@@ -500,6 +500,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
       a.dq_fix = reinterpret_cast<int32_t*>(base + q.fix_off);
       a.dq_exp = reinterpret_cast<int32_t*>(base + q.exp_off);
       a.dq_bound = reinterpret_cast<float*>(base + q.bound_off);
+      a.dq_stat = reinterpret_cast<float*>(base + q.stat_off);
     }
     TP_TRY(launch_attn_bwd(1, a, s));
   }

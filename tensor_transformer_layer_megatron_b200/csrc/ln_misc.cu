@@ -1167,6 +1167,26 @@ __global__ void bounded_wait_probe_kernel(int* status, unsigned long long limit_
   if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, status, kErrTimeoutProbe, nullptr, limit_ns);
 }
 
+__global__ void exp2_probe_kernel(int path, long long n, const float* x, float* y) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  if (path == 1) {
+    exp2_poly_pair(a, b);
+  } else {
+    a = ex2_approx(a);
+    b = ex2_approx(b);
+  }
+  y[i] = a;
+  if (i + 1 < n) y[i + 1] = b;
+}
+
+cudaError_t launch_exp2_probe(int path, long long n, const float* x, float* y, cudaStream_t s) {
+  const long long pairs = (n + 1) / 2;
+  exp2_probe_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(path, n, x, y);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns, cudaStream_t s) {
   bounded_wait_probe_kernel<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();

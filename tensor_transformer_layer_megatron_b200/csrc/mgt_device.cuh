@@ -127,6 +127,16 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// 3-D tiled bulk tensor reduction (element-wise add of the box into global memory, in the
+// tensor map's element type) from this CTA's shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -279,6 +289,63 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ----------------------------------------------------------------------------- paired fp32
+// Blackwell issues two fp32 additions, multiplications or fused multiply-adds as one
+// instruction on a pair of values held in a 64-bit register pair (PTX .f32x2 forms).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max(a, b, c) in one instruction (three-input form of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of finite x <= 127 on the FMA and integer pipes, leaving the special-function
+// unit to other values: x = j + f with j = rint(x) (adding 1.5 * 2^23 leaves rint(x) in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients
+// were fitted for relative error by iteratively reweighted least squares on [-1/2, 1/2] (max
+// relative error 7.5e-5, below the bf16 rounding of the probabilities); 2^j is applied by
+// adding j to the exponent field (the shifted-out high bits of the rounding constant vanish
+// in the 32-bit sum). Inputs below -125 are clamped there (2^-125 instead of a smaller
+// number), so callers keep exact zeros (masked scores, -inf) on the hardware path.
+__device__ __forceinline__ void exp2_poly_pair(float& a, float& b) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f, f2_pack(0.05517155f, 0.05517155f), f2_pack(0.24261114f, 0.24261114f));
+  p = f2_fma(p, f, f2_pack(0.69326103f, 0.69326103f));
+  p = f2_fma(p, f, f2_pack(0.99992806f, 0.99992806f));
+  float tl, th, pl, ph;
+  f2_unpack(t, tl, th);
+  f2_unpack(p, pl, ph);
+  a = __int_as_float(__float_as_int(pl) + (__float_as_int(tl) << 23));
+  b = __int_as_float(__float_as_int(ph) + (__float_as_int(th) << 23));
 }
 
 // Shared-memory matrix descriptor for tcgen05 (128-byte swizzle, sm_100 version field = 1).

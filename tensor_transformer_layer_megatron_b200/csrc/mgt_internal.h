@@ -73,6 +73,7 @@ struct GemmArgs {
   const float* b_scale;
 };
 
+
 // Row of token m in the sequence-parallel layout [p][b][s/p]: shard t = pos / (s/p) owns
 // positions t*s/p .. of every sequence.
 __host__ __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
@@ -98,6 +99,9 @@ struct SeqCursor {
 // 3-D bf16 tensor map (128-byte swizzle, zero fill out of bounds); strides in elements.
 bool make_tensor_map_bf16_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
                              const uint64_t strides[2], const uint32_t box[3]);
+// 3-D int32 tensor map without swizzle (row-major boxes); strides in elements.
+bool make_tensor_map_i32_3d(CUtensorMap* m, const void* base, const uint64_t dims[3],
+                            const uint64_t strides[2], const uint32_t box[3]);
 
 // tcgen05 / TMA GEMM for bf16 operands (fp32 accumulate in tensor memory).
 // Builds the tensor maps from the pointers in `args` (A, B, strides) and launches a persistent
@@ -130,6 +134,10 @@ cudaError_t launch_fp8_quantize(int dtype, long long n, const void* x, uint8_t* 
                                 float* scale_out, cudaStream_t stream);
 
 // Device-side failure-path probe (see mgt_debug_bounded_wait).
+// y[i] = 2^x[i] through the attention kernels' exponential: path 0 the special-function unit
+// (ex2.approx), path 1 the polynomial on the FMA pipe (exp2_poly_pair), pairs (i, i+1).
+cudaError_t launch_exp2_probe(int path, long long n, const float* x, float* y,
+                              cudaStream_t stream);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
 
@@ -153,14 +161,17 @@ struct AttnArgs {
   //   dq_bound float [b*H][ceil(s/128)][3]: per 128-token chunk, max |K|, max |V row|^2,
   //            max |dO row|^2, from which every partial sum of dQ is bounded
   //   dq_exp   int32 [b*H]: the power of two that scales each head's dQ to fixed point
+  //   dq_stat  float [b*H][2][ceil(s/128)*128]: -lse*log2(e) and -D per query, padded past s
+  //            with -inf and 0 (the softmax reads them as they are, no bounds checks)
   int32_t* dq_fix;
   float* dq_bound;
   int32_t* dq_exp;
+  float* dq_stat;
 };
 // Bytes of the single-kernel backward's dQ scratch (dq_fix, dq_exp, dq_bound) and where each
 // part starts, for b sequences of s tokens, H heads of 128.
 struct DqScratch {
-  size_t fix_off, exp_off, bound_off, bytes;
+  size_t fix_off, exp_off, bound_off, stat_off, bytes;
 };
 inline DqScratch dq_scratch_layout(long long b, long long s, long long H) {
   DqScratch r;
@@ -168,7 +179,8 @@ inline DqScratch dq_scratch_layout(long long b, long long s, long long H) {
   r.fix_off = 0;
   r.exp_off = (size_t)b * s * H * 128 * 4;
   r.bound_off = r.exp_off + (((size_t)b * H * 4 + 255) / 256) * 256;
-  r.bytes = r.bound_off + (size_t)b * H * nchunk * 3 * 4;
+  r.stat_off = r.bound_off + (((size_t)b * H * nchunk * 3 * 4 + 255) / 256) * 256;
+  r.bytes = r.stat_off + (size_t)b * H * 2 * nchunk * 128 * 4;
   return r;
 }
 cudaError_t launch_attn_fwd(int dtype, const AttnArgs& a, cudaStream_t stream);

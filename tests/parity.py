@@ -108,3 +108,112 @@ def full_parity(cfg, nonzero_affine=True, intermediates=True):
             errs[k] = rel_err(fetch(), r() if callable(r) else r)
             del r
     return errs
+
+
+def stage_parity(cfg, nonzero_affine=True):
+    """Every intermediate of the GPU layer against the oracle's primitives applied to the GPU's
+    own inputs of that stage (the bf16 values the kernel actually consumed), so each kernel's
+    own error is measured apart from the bf16 rounding of the activations upstream of it.
+    Stages: LN1, QKV GEMM, attention (O, lse), out-proj (h1), LN2, fc1 (u, a), fc2 (y), fc2
+    dgrad with the activation backward (du), fc1 dgrad (dln2), LN2 backward (dh1), out-proj
+    dgrad (dO), attention backward (dqkv), QKV dgrad (dln1), LN1 backward (dx). Plain layer
+    only (no sequence parallelism). Returns the dict of relative errors."""
+    assert not getattr(cfg, "sequence_parallel", 0)
+    t = make_inputs(cfg, nonzero_affine=nonzero_affine)
+    packed, layer, run = run_gpu(cfg, t)
+    h, H, f, p = cfg.hidden, cfg.heads, cfg.ffn, cfg.tp_size
+    b, s, T, d, hp = cfg.micro_batch, cfg.seq, cfg.tokens, cfg.hidden // cfg.heads, \
+        cfg.heads // cfg.tp_size
+    sw, nb = bool(getattr(cfg, "swiglu", 0)), bool(getattr(cfg, "disable_bias_linear", 0))
+    Pm = {k: np.asarray(v.double().numpy() if hasattr(v, "double") else v, np.float64)
+          for k, v in packed.items()}
+    bias = (lambda k: 0.0) if nb else (lambda k: Pm[k])  # noqa: E731
+    gi = gpu_intermediates(cfg, layer, run)
+    x = to_np(run.x).reshape(T, h)
+    dy = to_np(run.dy).reshape(T, h)
+    errs = {}
+    # forward
+    errs["ln1"] = rel_err(gi["ln1"](), oracle.layer_norm(x, Pm["ln1_g"], Pm["ln1_b"],
+                                                         cfg.ln_eps)[0])
+    ln1 = gi["ln1"]()
+    qkv = np.empty((T, p, 3, hp, d))
+    for tt in range(p):
+        qkv[:, tt] = (ln1 @ Pm["w_qkv"][tt].reshape(3 * hp * d, h).T +
+                      (0.0 if nb else Pm["b_qkv"][tt].reshape(-1))).reshape(T, 3, hp, d)
+    errs["qkv"] = rel_err(gi["qkv"](), qkv)
+    del ln1, qkv
+    qkv = gi["qkv"]()
+    O, lse = oracle.attention_fwd(qkv, b, s, H, p)
+    errs["O"] = rel_err(gi["O"](), O)
+    errs["lse"] = rel_err(gi["lse"](), lse)
+    del O, lse
+    Og = gi["O"]()
+    acc = np.zeros((T, h))
+    for tt in range(p):
+        acc += Og[:, tt].reshape(T, h // p) @ Pm["w_o"][tt].T
+    errs["h1"] = rel_err(gi["h1"](), x + bias("b_o") + acc)
+    del Og, acc
+    h1 = gi["h1"]()
+    errs["ln2"] = rel_err(gi["ln2"](), oracle.layer_norm(h1, Pm["ln2_g"], Pm["ln2_b"],
+                                                         cfg.ln_eps)[0])
+    ln2 = gi["ln2"]()
+    if sw:
+        u = np.empty((T, p, 2, f // p))
+        for tt in range(p):
+            for c in range(2):
+                u[:, tt, c] = ln2 @ Pm["w1"][tt, c].T + (0.0 if nb else Pm["b1"][tt, c])
+        a = oracle.swiglu(u[:, :, 0], u[:, :, 1])
+    else:
+        u = np.empty((T, p, f // p))
+        for tt in range(p):
+            u[:, tt] = ln2 @ Pm["w1"][tt].T + (0.0 if nb else Pm["b1"][tt])
+        a = oracle.gelu(u, cfg.gelu_tanh)
+    errs["u"] = rel_err(gi["u"](), u)
+    errs["a"] = rel_err(gi["a"](), a)
+    del ln2, u, a
+    ag = gi["a"]()
+    acc = np.zeros((T, h))
+    for tt in range(p):
+        acc += ag[:, tt] @ Pm["w2"][tt].T
+    errs["y"] = rel_err(to_np(run.y).reshape(T, h), h1 + bias("b2") + acc)
+    del ag, acc
+    # backward
+    ug = gi["u"]()
+    da = np.empty((T, p, f // p))
+    for tt in range(p):
+        da[:, tt] = dy @ Pm["w2"][tt]
+    if sw:
+        du = np.stack(oracle.swiglu_grad(ug[:, :, 0], ug[:, :, 1], da), axis=2)
+    else:
+        du = da * oracle.gelu_grad(ug, cfg.gelu_tanh)
+    errs["du"] = rel_err(gi["du"](), du)
+    del ug, da, du
+    dug = gi["du"]()
+    rows = (2 if sw else 1) * (f // p)
+    dln2 = np.zeros((T, h))
+    for tt in range(p):
+        dln2 += dug[:, tt].reshape(T, rows) @ Pm["w1"][tt].reshape(rows, h)
+    errs["dln2"] = rel_err(gi["dln2"](), dln2)
+    del dug, dln2
+    _, _, rstd2, xhat2 = oracle.layer_norm(h1, Pm["ln2_g"], Pm["ln2_b"], cfg.ln_eps)
+    dl, _, _ = oracle.layer_norm_grad(gi["dln2"](), xhat2, rstd2, Pm["ln2_g"])
+    errs["dh1"] = rel_err(gi["dh1"](), dy + dl)
+    del h1, xhat2, rstd2, dl
+    dh1 = gi["dh1"]()
+    dO = np.empty((T, p, hp, d))
+    for tt in range(p):
+        dO[:, tt] = (dh1 @ Pm["w_o"][tt]).reshape(T, hp, d)
+    errs["dO"] = rel_err(gi["dO"](), dO)
+    del dO
+    errs["dqkv"] = rel_err(gi["dqkv"](), oracle.attention_bwd(qkv, gi["dO"](), b, s, H, p))
+    del qkv
+    dqg = gi["dqkv"]()
+    dln1 = np.zeros((T, h))
+    for tt in range(p):
+        dln1 += dqg[:, tt].reshape(T, 3 * hp * d) @ Pm["w_qkv"][tt].reshape(3 * hp * d, h)
+    errs["dln1"] = rel_err(gi["dln1"](), dln1)
+    del dqg, dln1
+    _, _, rstd1, xhat1 = oracle.layer_norm(x, Pm["ln1_g"], Pm["ln1_b"], cfg.ln_eps)
+    dl, _, _ = oracle.layer_norm_grad(gi["dln1"](), xhat1, rstd1, Pm["ln1_g"])
+    errs["dx"] = rel_err(to_np(run.dx).reshape(T, h), dh1 + dl)
+    return errs

@@ -198,3 +198,12 @@ def test_layernorm_bwd_noalloc_rejects_misaligned_pointers(bad):
                                        vp(ptr["gamma"]), vp(ptr["mean"]), vp(ptr["rstd"]),
                                        vp(ptr["dx"]), vp(ptr["dgamma"]), vp(ptr["dbeta"]), None)
     assert st == 2, (bad, st)
+
+
+def test_debug_exp2_rejects_bad_arguments():
+    lib = mgt.load_library()
+    vp = ctypes.c_void_p
+    assert lib.mgt_debug_exp2(2, 4, vp(P16), vp(P16), None) == 1   # unknown path
+    assert lib.mgt_debug_exp2(1, -1, vp(P16), vp(P16), None) == 1  # negative count
+    assert lib.mgt_debug_exp2(1, 4, None, vp(P16), None) == 1      # null input
+    assert lib.mgt_debug_exp2(0, 0, None, None, None) == 0         # nothing to do
