@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // warp 8: TMA producer; warp 9: TMEM owner and MMA issuer; warps 10-13: dQ drain (lane
 // quarter w%4 = 32 of the d rows of dQ^T). Every wait is bounded.
 // Power of two e with B * 2^e < 2^29 for B = 2 max|K| max|dO row| max|V row| over a head's
-// chunk bounds ([nchunk][3]: max |K|, max |V row|^2, max |dO row|^2). Every CTA of a head and
+// 32-token chunk bounds ([nchunk][3]: max |K|, max |V row|^2, max |dO row|^2). Every CTA of a head and
 // nothing else computes it, from the same values, so all agree.
 __device__ __forceinline__ int dq_fixed_exponent(const float* bound, int nchunk) {
   float km = 0.f, v2 = 0.f, g2 = 0.f;
@@ -1164,8 +1164,7 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int32_t* stg = reinterpret_cast<int32_t*>(smem + L::STG_OFF) + (warp - 10) * 512;
     // this head's fixed-point scale (the same computation in every CTA of the head)
-    const int e = dq_fixed_exponent(a.dq_bound + (long long)bh * ((S + 127) / 128) * 3,
-                                    (S + 127) / 128);
+    const int e = dq_fixed_exponent(a.dq_bound + (long long)bh * nq * 4 * 3, nq * 4);
     if (kb == 0 && quarter == 0 && lane == 0) a.dq_exp[bh] = e;
     const float fscale = exp2f((float)e);
     bool issued = false;
@@ -1337,9 +1336,11 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
   }
 }
 
-// Per head and 128-token chunk c (grid b*H x chunks, 8 warps x 16 tokens): D = rowsum(dO * O)
-// into a.Dsum [b][H][s], the fixed-point dQ accumulator zeroed, and the chunk's max |K|,
-// max |V row|^2 and max |dO row|^2 into a.dq_bound (one lane holds 4 of the 128 dimensions).
+// Per head and 32-token chunk c (grid b*H x ceil(s/128)*4, 8 warps x 4 tokens): D = rowsum(dO * O)
+// into a.Dsum [b][H][s], the fixed-point dQ accumulator zeroed, the per-query statistics rows
+// (-lse*log2e, -D, padded to whole 128-query blocks with -inf and 0) and the chunk's max |K|,
+// max |V row|^2 and max |dO row|^2 into a.dq_bound. A lane holds 4 of the 128 dimensions; each
+// warp issues the loads of its 4 tokens before using any, so that enough bytes are in flight.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
   constexpr int D = 128;
   __shared__ float red[8][3];
@@ -1347,11 +1348,30 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
   const int bh = blockIdx.x, c = blockIdx.y, nchunk = gridDim.y;
   const int H = a.H, hp = H / a.p, b = bh / H, n = bh % H, t = n / hp, jh = n % hp;
   const long long ld_qkv = 3LL * H * D, ld_o = (long long)H * D;
-  float kmax = 0.f, v2max = 0.f, g2max = 0.f;
-  const long long nqp = (long long)nchunk * 128;
+  const long long nqp = (long long)nchunk * 32;
   float* stat = a.dq_stat + (long long)bh * 2 * nqp;
-  for (int i = 0; i < 16; ++i) {
-    const int pos = c * 128 + warp * 16 + i;
+  const __nv_bfloat16* o_ = reinterpret_cast<const __nv_bfloat16*>(a.o);
+  const __nv_bfloat16* g_ = reinterpret_cast<const __nv_bfloat16*>(a.dO);
+  const __nv_bfloat16* qkv_ = reinterpret_cast<const __nv_bfloat16*>(a.qkv);
+  uint2 ov[4], gv[4], kv[4], vv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int pos = c * 32 + warp * 4 + i;
+    if (pos < a.s) {
+      const long long tok = (long long)b * a.s + pos;
+      const long long oo = tok * ld_o + (long long)n * D + lane * 4;
+      const long long ko = tok * ld_qkv + (long long)t * 3 * hp * D + (long long)(hp + jh) * D +
+                           lane * 4;
+      ov[i] = *reinterpret_cast<const uint2*>(o_ + oo);
+      gv[i] = *reinterpret_cast<const uint2*>(g_ + oo);
+      kv[i] = *reinterpret_cast<const uint2*>(qkv_ + ko);
+      vv[i] = *reinterpret_cast<const uint2*>(qkv_ + ko + (long long)hp * D);
+    }
+  }
+  float kmax = 0.f, v2max = 0.f, g2max = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int pos = c * 32 + warp * 4 + i;
     if (pos >= a.s) {  // warp-uniform: padding of the softmax statistics (P = 0 there)
       if (lane == 0) {
         stat[pos] = -INFINITY;
@@ -1360,16 +1380,10 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
       continue;
     }
     const long long tok = (long long)b * a.s + pos;
-    const long long oo = tok * ld_o + (long long)n * D + lane * 4;
-    const long long ko = tok * ld_qkv + (long long)t * 3 * hp * D + (long long)(hp + jh) * D + lane * 4;
-    const uint2 ov = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + oo);
-    const uint2 gv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.dO) + oo);
-    const uint2 kv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.qkv) + ko);
-    const uint2 vv = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(a.qkv) + ko + (long long)hp * D);
-    const float o[4] = {bf16_lo(ov.x), bf16_hi(ov.x), bf16_lo(ov.y), bf16_hi(ov.y)};
-    const float g[4] = {bf16_lo(gv.x), bf16_hi(gv.x), bf16_lo(gv.y), bf16_hi(gv.y)};
-    const float k[4] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y)};
-    const float v[4] = {bf16_lo(vv.x), bf16_hi(vv.x), bf16_lo(vv.y), bf16_hi(vv.y)};
+    const float o[4] = {bf16_lo(ov[i].x), bf16_hi(ov[i].x), bf16_lo(ov[i].y), bf16_hi(ov[i].y)};
+    const float g[4] = {bf16_lo(gv[i].x), bf16_hi(gv[i].x), bf16_lo(gv[i].y), bf16_hi(gv[i].y)};
+    const float k[4] = {bf16_lo(kv[i].x), bf16_hi(kv[i].x), bf16_lo(kv[i].y), bf16_hi(kv[i].y)};
+    const float v[4] = {bf16_lo(vv[i].x), bf16_hi(vv[i].x), bf16_lo(vv[i].y), bf16_hi(vv[i].y)};
     float dsum = 0.f, g2 = 0.f, v2 = 0.f, km = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -1390,7 +1404,8 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
       stat[pos] = -a.lse[(long long)bh * a.s + pos] * kLog2eF;
       stat[nqp + pos] = -dsum;
     }
-    *reinterpret_cast<int4*>(a.dq_fix + oo) = make_int4(0, 0, 0, 0);
+    *reinterpret_cast<int4*>(a.dq_fix + tok * ld_o + (long long)n * D + lane * 4) =
+        make_int4(0, 0, 0, 0);
     kmax = fmaxf(kmax, km);
     v2max = fmaxf(v2max, v2);
     g2max = fmaxf(g2max, g2);
@@ -1458,7 +1473,7 @@ cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
   const float scale = 1.f / sqrtf((float)D);
   const long long threads = (long long)a.b * a.s * a.H * 16;  // 16 per (token, head)
   const unsigned blocks = (unsigned)((threads + 255) / 256);
-  attn_bwd_prep_kernel<<<dim3(a.b * a.H, (a.s + 127) / 128), 256, 0, s>>>(a);
+  attn_bwd_prep_kernel<<<dim3(a.b * a.H, (a.s + 127) / 128 * 4), 256, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tm_dq;  // the fixed-point dQ accumulator as [b][s][H*d] int32, 32 x 16 boxes

@@ -732,17 +732,15 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
   const int sl = threadIdx.x >> 5;
   float s = 0.f;
   if (c < nsum * h) {
-    // four loads in flight per thread; the additions keep the order b = sl, sl + 8, ...
+    // eight loads in flight per thread; the additions keep the order b = sl, sl + 8, ...
     const long long step = (long long)nsum * h;
     int b = sl;
-    for (; b + 24 < nblk; b += 32) {
-      const float p0 = __ldg(partial + b * step + c), p1 = __ldg(partial + (b + 8) * step + c);
-      const float p2 = __ldg(partial + (b + 16) * step + c);
-      const float p3 = __ldg(partial + (b + 24) * step + c);
-      s += p0;
-      s += p1;
-      s += p2;
-      s += p3;
+    for (; b + 56 < nblk; b += 64) {
+      float p[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) p[u] = __ldg(partial + (b + 8 * u) * step + c);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += p[u];
     }
     for (; b < nblk; b += 8) s += __ldg(partial + b * step + c);
   }
@@ -808,23 +806,22 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
   }
 }
 
-// out[c] = sum over slices of partial[slice][c], slices in increasing order; four
-// independent chains per thread keep loads in flight.
-__global__ void __launch_bounds__(256) colsum_reduce_kernel(int cols, int slices,
-                                                            const float* __restrict__ partial,
-                                                            float* __restrict__ out) {
-  const int c = blockIdx.x * 256 + threadIdx.x;
+// out[c] = sum over slices of partial[slice][c] in a fixed order: every slice's value is loaded
+// before any is added (at most kColsumMaxSlices in flight per thread), then added in slice
+// order. Small blocks spread the columns over every SM.
+__global__ void __launch_bounds__(64) colsum_reduce_kernel(int cols, int slices,
+                                                           const float* __restrict__ partial,
+                                                           float* __restrict__ out) {
+  const int c = blockIdx.x * 64 + threadIdx.x;
   if (c >= cols) return;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int k = 0;
-  for (; k + 3 < slices; k += 4) {
-    a0 += partial[(long long)k * cols + c];
-    a1 += partial[(long long)(k + 1) * cols + c];
-    a2 += partial[(long long)(k + 2) * cols + c];
-    a3 += partial[(long long)(k + 3) * cols + c];
-  }
-  for (; k < slices; ++k) a0 += partial[(long long)k * cols + c];
-  out[c] = (a0 + a1) + (a2 + a3);
+  float p[kColsumMaxSlices];
+#pragma unroll
+  for (int k = 0; k < kColsumMaxSlices; ++k)
+    p[k] = k < slices ? __ldg(partial + (long long)k * cols + c) : 0.f;
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < kColsumMaxSlices; ++k) acc += p[k];
+  out[c] = acc;
 }
 
 // ---------------------------------------------------------------------------- fp32 GEMM
@@ -1150,7 +1147,7 @@ cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, fl
                                                  partial, rows_per);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  colsum_reduce_kernel<<<(cols + 255) / 256, 256, 0, s>>>(cols, slices, partial, out);
+  colsum_reduce_kernel<<<(cols + 63) / 64, 64, 0, s>>>(cols, slices, partial, out);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,8 @@ struct GemmArgs {
   int f8;
   const float* a_scale;
   const float* b_scale;
+  // Tile order (set by the launcher): 1 = N fastest within a group, 0 = M fastest.
+  int n_fast;
 };
 
 
@@ -158,7 +160,7 @@ struct AttnArgs {
   // Single-kernel backward (head_dim 128; null dq_fix selects the two-kernel backward):
   //   dq_fix   int32 [T][H][d]: dQ accumulated in fixed point (integer adds are associative,
   //            so the sum does not depend on the order in which key blocks arrive)
-  //   dq_bound float [b*H][ceil(s/128)][3]: per 128-token chunk, max |K|, max |V row|^2,
+  //   dq_bound float [b*H][4*ceil(s/128)][3]: per 32-token chunk, max |K|, max |V row|^2,
   //            max |dO row|^2, from which every partial sum of dQ is bounded
   //   dq_exp   int32 [b*H]: the power of two that scales each head's dQ to fixed point
   //   dq_stat  float [b*H][2][ceil(s/128)*128]: -lse*log2(e) and -D per query, padded past s
@@ -179,7 +181,7 @@ inline DqScratch dq_scratch_layout(long long b, long long s, long long H) {
   r.fix_off = 0;
   r.exp_off = (size_t)b * s * H * 128 * 4;
   r.bound_off = r.exp_off + (((size_t)b * H * 4 + 255) / 256) * 256;
-  r.stat_off = r.bound_off + (((size_t)b * H * nchunk * 3 * 4 + 255) / 256) * 256;
+  r.stat_off = r.bound_off + (((size_t)b * H * nchunk * 4 * 3 * 4 + 255) / 256) * 256;
   r.bytes = r.stat_off + (size_t)b * H * 2 * nchunk * 128 * 4;
   return r;
 }
