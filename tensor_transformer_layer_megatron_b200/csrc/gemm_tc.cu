@@ -47,13 +47,22 @@ struct TileCoord {
   int ng, mb, nb;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n) {
+// Tile order within a group. The CTAs of one wave run consecutive tiles, and the operand that
+// the fast index sweeps is read again by every wave, so the fast index is the one whose
+// operand is smaller (it then stays in L2): M fastest (the wave shares B tiles and sweeps A)
+// unless A is the larger operand (M > N, the wide weight gradients), then N fastest.
+__device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n, int n_fast) {
   TileCoord t;
   const int per_group = num_m * num_n;
   t.ng = tile / per_group;
   const int r = tile - t.ng * per_group;
-  t.nb = r / num_m;  // m fastest: consecutive CTAs share the same weight (B) tile
-  t.mb = r - t.nb * num_m;
+  if (n_fast) {
+    t.mb = r / num_n;
+    t.nb = r - t.mb * num_n;
+  } else {
+    t.nb = r / num_m;
+    t.mb = r - t.nb * num_m;
+  }
   return t;
 }
 
@@ -411,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     SeqCursor cur{0, 0};
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, num_m, num_n);
+      const TileCoord tc = tile_coord(tile, num_m, num_n, args.n_fast);
       // token coordinates go through the sequence-parallel row map where set: M of a
       // K-major A once per tile, the K of an MN-major operand through the cursor
       const int ma = (!A_MN && args.a_sp) ? seq_row(args, tc.mb * BM) : tc.mb * BM;
@@ -521,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, num_m, num_n);
+      const TileCoord tc = tile_coord(tile, num_m, num_n, args.n_fast);
       const int row = tc.mb * BM + ew * 32 + lane;
       if (k_iters > 0) {
         const bool ok = mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue,
@@ -678,7 +687,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     SeqCursor cur{0, 0};
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-      const TileCoord tc = tile_coord(tile, num_m2, num_n);
+      const TileCoord tc = tile_coord(tile, num_m2, num_n, args.n_fast);
       const int m0 = tc.mb * 256 + rank * 128;
       const int n0 = tc.nb * BN + rank * (BN / 2);
       // token coordinates go through the sequence-parallel row map where set: M of a
@@ -798,7 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
-      const TileCoord tc = tile_coord(tile, num_m2, num_n);
+      const TileCoord tc = tile_coord(tile, num_m2, num_n, args.n_fast);
       const int row = tc.mb * 256 + rank * 128 + ew * 32 + lane;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue,
                                 abort_flag);
@@ -1254,9 +1263,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) 
     }
     if (!make_map(&tb, a.B, dims, str, box)) return cudaErrorInvalidValue;
   }
-  if (pair) return launch_pair(ta, tb, a, num_sms, pair_bn, stream);
-  if (BN == 128) return launch_bn<128>(ta, tb, a, num_sms, stream);
-  return launch_bn<256>(ta, tb, a, num_sms, stream);
+  GemmArgs ka = a;
+  ka.n_fast = (long long)a.M > (long long)a.Ng * a.NG ? 1 : 0;
+  if (pair) return launch_pair(ta, tb, ka, num_sms, pair_bn, stream);
+  if (BN == 128) return launch_bn<128>(ta, tb, ka, num_sms, stream);
+  return launch_bn<256>(ta, tb, ka, num_sms, stream);
 }
 
 }  // namespace mgt
