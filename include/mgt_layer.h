@@ -254,10 +254,11 @@ mgt_status mgt_gemm_fp8(int32_t M, int32_t N, int32_t K, const uint8_t* A, int64
  * mgt_layer_get_error report MGT_ETIMEOUT. */
 mgt_status mgt_debug_bounded_wait(int64_t limit_ns, int32_t* status, void* stream);
 
-/* Numerics probe (tests; no counterpart in the pages): y[i] = 2^x[i] for n floats through the
- * exponential the attention kernels use for softmax probabilities: path 0 = the hardware
- * approximation (ex2.approx), path 1 = the polynomial evaluated on the FMA pipe (relative
- * error below 7.5e-5 for -125 <= x <= 127; inputs below -125 give 2^-125). x, y device
+/* Numerics probe (tests; no counterpart in the pages): y[i] = 2^x[i] for n floats: path 0 =
+ * the hardware approximation (ex2.approx) that the attention kernels use for the softmax
+ * probabilities, path 1 = an alternative polynomial evaluated on the FMA pipe (relative
+ * error below 7.5e-5 for -125 <= x <= 127; inputs below -125 give 2^-125), which the kernels
+ * do not use because it made none of their loops faster on B200. x, y device
  * pointers; asynchronous on `stream`; MGT_EINVAL for n < 0, null pointers or another path. */
 mgt_status mgt_debug_exp2(int32_t path, int64_t n, const float* x, float* y, void* stream);
 

@@ -52,7 +52,8 @@ constexpr int kBwdThreads = 320;
 
 template <int D>
 __global__ void __launch_bounds__(kAttnFwdThreads, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a,
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm,
+                       const __grid_constant__ CUtensorMap tm_o, const AttnArgs a,
                        float scale_log2) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -217,85 +219,68 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         break;
       }
       tc_fence_after();
-      // Two passes over the row in TMEM, 64 then 32 scores in registers at a time: the row
-      // maximum first, then P = 2^(S*scale*log2e - m) chunk by chunk, packed to bf16 and
-      // written back over the scores already consumed (P of chunk c -> columns 16c..16c+15),
-      // so that the exponentials' temporaries fit beside the scores.
+      // The whole row of scores in registers (one TMEM read), the row maximum, then
+      // P = 2^(S*scale*log2e - m) on pairs of scores, packed to bf16 and written over the
+      // first 64 columns of the row's own scores.
       const bool diag = kb == qb;  // keys after this query are masked
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float sv[128];
+      {
+        uint32_t raw[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; c += 2) {
-        uint32_t ra[32], rb[32];
-        tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, ra);
-        tmem_ld_32x32b_x32_nw(lane_base + s_col + (c + 1) * 32, rb);
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, raw[c]);
         tmem_ld_wait();
-        reg_fence(ra);
-        reg_fence(rb);
-        if (diag) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (c * 32 + i > r) ra[i] = __float_as_uint(-INFINITY);
-            if ((c + 1) * 32 + i > r) rb[i] = __float_as_uint(-INFINITY);
-          }
+        for (int c = 0; c < 4; ++c) {
+          reg_fence(raw[c]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[c][i]);
         }
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            m4[k] = fmax3(m4[k], __uint_as_float(ra[i + k]), __uint_as_float(rb[i + k]));
       }
-      const float mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * scale_log2;
+      if (diag) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i > r) sv[i] = -INFINITY;
+      }
+      // row max of the raw scores (the scale is positive): eight chains, then a tree
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmax3(sv[k], sv[8 + k], sv[16 + k]);
+#pragma unroll
+      for (int i = 24; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], sv[i + k], sv[i + 8 + k]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                             fmaxf(m8[6], m8[7])) * scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
       const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
-      // exponentials on pairs of scores; off the diagonal (no masked -inf) three pairs in
-      // eight take the polynomial 2^x on the FMA pipe, the rest the special-function unit
+      // exponent arguments on pairs of scores (paired fp32 FMA), 2^x on the special-function
+      // unit, row sums in four paired accumulators
       const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
-      uint64_t acc2[2] = {0ull, 0ull};
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32];
-        tmem_ld_32x32b_x32_nw(lane_base + s_col + c * 32, raw);
-        tmem_ld_wait();
-        reg_fence(raw);
-        uint32_t pw[16];
-        if (diag) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pa, pb;
-            f2_unpack(f2_fma(f2_pack(c * 32 + i > r ? -INFINITY : __uint_as_float(raw[i]),
-                                     c * 32 + i + 1 > r ? -INFINITY : __uint_as_float(raw[i + 1])),
-                             c2, nm2),
-                      pa, pb);
-            pa = ex2_approx(pa);
-            pb = ex2_approx(pb);
-            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(pa, pb));
-            pw[i >> 1] = pack_bf16x2(pa, pb);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pa, pb;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1])), c2,
-                             nm2),
-                      pa, pb);
-            const int jp = (i >> 1) & 7;
-            if (jp == 1 || jp == 4 || jp == 6) {
-              exp2_poly_pair(pa, pb);
-            } else {
-              pa = ex2_approx(pa);
-              pb = ex2_approx(pb);
-            }
-            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(pa, pb));
-            pw[i >> 1] = pack_bf16x2(pa, pb);
-          }
-        }
-        tmem_st_32x32b_x16(lane_base + s_col + c * 16, pw);
+      for (int i = 0; i < 128; i += 2) {
+        float pa, pb;
+        f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), c2, nm2), pa, pb);
+        pa = ex2_approx(pa);
+        pb = ex2_approx(pb);
+        sv[i] = pa;
+        sv[i + 1] = pb;
+        acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(pa, pb));
       }
-      float rs[4];
-      f2_unpack(acc2[0], rs[0], rs[1]);
-      f2_unpack(acc2[1], rs[2], rs[3]);
-      l_run = l_run * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float pw[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          pw[j] = __uint_as_float(pack_bf16x2(sv[c * 64 + 2 * j], sv[c * 64 + 2 * j + 1]));
+        tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);
+      }
+      float rs[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f2_unpack(acc2[k], rs[2 * k], rs[2 * k + 1]);
+      l_run = l_run * alpha +
+              (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
       // O holds the sum up to block kb-1 (its PV completed before this S was committed); it
       // is rescaled before this block's PV, which waits for p_full below.
       if (kb > 0 && __any_sync(0xffffffffu, need)) {
@@ -314,32 +299,46 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[u]);
     }
-    if (ok && nkv > 0) {
+    if (nkv > 0) {
       // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
-      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
+      if (ok) ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      // O / l in bf16 into this tile's Q buffer (every MMA has completed, so Q is no longer
+      // read), laid out as the 128-byte-swizzled boxes the tensor map describes: 16-byte piece
+      // j of row r's 64-column chunk at r * 128 + (j ^ (r % 8)) * 16. A bulk tensor store per
+      // chunk then writes whole rows; rows past the sequence end are clipped by the map.
+      uint8_t* stage = smem + L::Q_OFF + u * L::TILE;
+      const int qrow = qb * 128 + r;
+      if (ok) {
         tc_fence_after();
-        const int qrow = qb * 128 + r;
         const float inv = 1.f / l_run;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) +
-                              ((long long)b * S + qrow) * H * D + (long long)n * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tmem_ld_32x32b_x32(lane_base + o_col + c * 32, o);
-          if (qrow < S) {
+          uint8_t* rowp = stage + (c >> 1) * 16384 + r * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 w;
-              w.x = pack_bf16x2(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
-              w.y = pack_bf16x2(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
-              w.z = pack_bf16x2(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
-              w.w = pack_bf16x2(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
-              *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = w;
-            }
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(o[q * 8 + 0] * inv, o[q * 8 + 1] * inv);
+            w.y = pack_bf16x2(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
+            w.z = pack_bf16x2(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
+            w.w = pack_bf16x2(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
+            const int j = (c & 1) * 4 + q;
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (r & 7)) << 4)) = w;
           }
         }
+        fence_proxy_async_smem();
         if (qrow < S) a.lse[((long long)b * H + n) * S + qrow] = (m_run + log2f(l_run)) * kLn2F;
+      }
+      // the tile's four warps always meet here (also after an error), then one thread stores
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + u) : "memory");
+      if ((warp & 3) == 0 && lane == 0 && ok && !*abort_flag) {
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c)
+          tma_store_3d(&tm_o, stage + c * 16384, n * D + c * 64, qb * 128, b);
+        bulk_commit();
+        bulk_wait0();
       }
     }
   }
@@ -1237,12 +1236,10 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
         for (int i = 0; i < 32; ++i)
           if (q0 + i < r) sr[i] = __float_as_uint(-INFINITY);
       }
-      // P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D) on pairs of queries;
-      // off the diagonal (no masked -inf) three pairs in eight take the polynomial 2^x on the
-      // FMA pipe, the rest the SFU
+      // P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D) on pairs of queries
+      // (paired fp32 ops; 2^x on the special-function unit)
       uint32_t pw[16], dw[16];
       const uint64_t c2 = f2_pack(scale_log2, scale_log2);
-      const bool diag = qi == kb;
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(ls + i);   // -lse * log2e
@@ -1253,13 +1250,8 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i + e]), __uint_as_float(sr[i + e + 1])),
                            c2, e ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y)),
                     pa, pb);
-          const int jp = ((i + e) >> 1) & 7;
-          if (!diag && (jp == 1 || jp == 4 || jp == 6)) {
-            exp2_poly_pair(pa, pb);
-          } else {
-            pa = ex2_approx(pa);
-            pb = ex2_approx(pb);
-          }
+          pa = ex2_approx(pa);
+          pb = ex2_approx(pb);
           const uint64_t dpd = f2_add(
               f2_pack(__uint_as_float(dr[i + e]), __uint_as_float(dr[i + e + 1])),
               e ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y));
@@ -1547,9 +1539,15 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   const uint64_t strides[2] = {three_h, three_h * a.s};
   const uint32_t box[3] = {64, 128, 1};
   if (!make_tensor_map_bf16_3d(&tm, a.qkv, dims, strides, box)) return cudaErrorInvalidValue;
+  // o viewed as [b][s][H*D], written in the same 64-column, 128-row boxes
+  CUtensorMap tm_o;
+  const uint64_t hd = (uint64_t)a.H * D;
+  const uint64_t dims_o[3] = {hd, (uint64_t)a.s, (uint64_t)a.b};
+  const uint64_t strides_o[2] = {hd, hd * a.s};
+  if (!make_tensor_map_bf16_3d(&tm_o, a.o, dims_o, strides_o, box)) return cudaErrorInvalidValue;
   // one CTA per pair of 128-query blocks of one head
   dim3 grid(a.b * a.H, ((a.s + 127) / 128 + 1) / 2);
-  attn_fwd_tc_kernel<D><<<grid, kAttnFwdThreads, L::BYTES, s>>>(tm, a,
+  attn_fwd_tc_kernel<D><<<grid, kAttnFwdThreads, L::BYTES, s>>>(tm, tm_o, a,
                                                                 kLog2eF / sqrtf((float)D));
   return cudaGetLastError();
 }
