@@ -164,9 +164,7 @@ typedef enum mgt_region {
                                backward, then per-head scaling data (bf16 layers with
                                head_dim 128; 0 bytes otherwise)                         */
   MGT_WS_LN_PARTIAL = 73,   /* F32 [slices][3][h] LayerNorm dgamma/dbeta/residual-grad partial sums */
-  MGT_WS_BIAS_PARTIAL = 74, /* F32 [slices][cols] column-sum partials of the b1 / b_qkv gradients
-                               (0 bytes with disable_bias_linear)                        */
-  MGT_WS_COUNT = 75
+  MGT_WS_COUNT = 74
 } mgt_region;
 mgt_status mgt_layer_region(const mgt_layer* layer, int region, size_t* offset, size_t* bytes);
 

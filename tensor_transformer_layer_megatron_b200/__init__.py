@@ -23,7 +23,7 @@ REGIONS = {
     "ln1": 0, "ln1_mean": 1, "ln1_rstd": 2, "qkv": 3, "attn_o": 4, "attn_lse": 5, "h1": 6,
     "ln2": 7, "ln2_mean": 8, "ln2_rstd": 9, "fc1_u": 10, "fc1_a": 11,
     "status": 64, "du": 65, "dln2": 66, "dh1": 67, "dO": 68, "dqkv": 69, "dln1": 70,
-    "attn_D": 71, "dq_acc": 72, "ln_partial": 73, "bias_partial": 74,
+    "attn_D": 71, "dq_acc": 72, "ln_partial": 73,
 }
 
 STATUS = {0: "MGT_OK", 1: "MGT_EINVAL", 2: "MGT_EUNSUPPORTED", 3: "MGT_ECUDA",

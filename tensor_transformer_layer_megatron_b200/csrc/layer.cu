@@ -111,14 +111,6 @@ size_t dq_acc_bytes(const mgt_layer* L) {
   return dq_scratch_layout(L->cfg.micro_batch, L->cfg.seq, L->H).bytes;
 }
 
-// per-slice column sums of du and dqkv (the b1 and b_qkv gradients); one buffer serves both
-size_t bias_partial_bytes(const mgt_layer* L) {
-  if (L->cfg.disable_bias_linear) return 0;
-  const size_t f1 = L->cfg.swiglu ? 2 * (size_t)L->f : (size_t)L->f;
-  const size_t cols = f1 > 3 * (size_t)L->h ? f1 : 3 * (size_t)L->h;
-  return (size_t)kColsumMaxSlices * cols * 4;
-}
-
 void layout(mgt_layer* L) {
   const size_t T = L->T, h = L->h, f = L->f, e = L->esz;
   const size_t f1 = L->cfg.swiglu ? 2 * f : f;  // fc1 outputs: [gate | up] with SwiGLU
@@ -142,8 +134,7 @@ void layout(mgt_layer* L) {
                                    T * h * e,
                                    bHs * 4,
                                    dq_acc_bytes(L),
-                                   nblk * 3 * h * 4,
-                                   bias_partial_bytes(L)};
+                                   nblk * 3 * h * 4};
   off = 0;
   for (int i = 0; i < MGT_WS_COUNT - 64; ++i) {
     L->ws[i].off = off;
@@ -480,10 +471,9 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
       if (on && cudaEventRecord(L->ev_join, w) == cudaSuccess) cudaStreamWaitEvent(s, L->ev_join, 0);
     }
   } join{L, s, w};
-  float* bias_part = reinterpret_cast<float*>(sp(workspace, L->ws[MGT_WS_BIAS_PARTIAL - 64]));
   auto colsum = [&](const void* src, int cols, void* out) {
     return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, w,
-               [&] { return launch_colsum(dt, T, cols, src, (float*)out, bias_part, w); });
+               [&] { return launch_colsum(dt, T, cols, src, (float*)out, w); });
   };
   const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
   const bool nb = L->cfg.disable_bias_linear, sw = L->cfg.swiglu;

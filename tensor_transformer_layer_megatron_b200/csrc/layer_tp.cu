@@ -83,7 +83,7 @@ struct Reg {
 enum SavedReg { S_LN1, S_MU1, S_RS1, S_QKV, S_O, S_LSE, S_H1, S_LN2, S_MU2, S_RS2, S_AUX, S_A,
                 S_COUNT };
 enum WsReg { W_STATUS, W_PART, W_DU, W_DLN2, W_DH1, W_DO, W_DQKV, W_DLN1, W_D, W_LNP,
-             W_DQACC, W_BIASP, W_COUNT };
+             W_DQACC, W_COUNT };
 
 GemmArgs base(int M, int N, int K) {
   GemmArgs a;
@@ -284,12 +284,7 @@ mgt_status mgt_tp_rank_init(const mgt_layer_config* cfg, int32_t rank, mgt_tp_ra
                               // fixed-point dQ accumulator and its scaling data
                               R->d == 128 ? dq_scratch_layout(cfg->micro_batch, cfg->seq,
                                                               R->Hl).bytes
-                                          : 0,
-                              // column-sum partials of the b1 / b_qkv gradients
-                              cfg->disable_bias_linear
-                                  ? 0
-                                  : (size_t)kColsumMaxSlices *
-                                        (R->f1l > 3 * R->hl ? R->f1l : 3 * R->hl) * 4};
+                                          : 0};
   place(R->saved, S_COUNT, sb, &R->saved_bytes);
   place(R->ws, W_COUNT, wb, &R->ws_bytes);
   *out = R;
@@ -442,7 +437,6 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
   char* dln1 = at(workspace, R->ws[W_DLN1]);
   float* Dsum = reinterpret_cast<float*>(at(workspace, R->ws[W_D]));
   float* lnp = reinterpret_cast<float*>(at(workspace, R->ws[W_LNP]));
-  float* biasp = reinterpret_cast<float*>(at(workspace, R->ws[W_BIASP]));
   // fc2: du = (dy W2_t) * act'(u) (the activation backward in the dgrad epilogue); dW2_t
   {
     GemmArgs a = base(T, fl, h);
@@ -458,7 +452,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     TP_TRY(launch_gemm_tc(a, R->num_sms, s));
   }
   // fc1: db1_t, dln2 partial -> all-reduce -> bf16, dW1_t
-  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, biasp, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, s));
   {
     GemmArgs a = base(T, h, f1l);
     a.b_mn = 1; a.lda = f1l; a.B = P->w1; a.ldb = h;
@@ -505,7 +499,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     TP_TRY(launch_attn_bwd(1, a, s));
   }
   // QKV: db_qkv_t, dln1 partial -> all-reduce -> bf16, dW_qkv,t
-  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, biasp, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, s));
   {
     GemmArgs a = base(T, h, 3 * hl);
     a.b_mn = 1; a.lda = 3 * hl; a.B = P->w_qkv; a.ldb = h;

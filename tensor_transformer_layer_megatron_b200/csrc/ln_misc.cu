@@ -756,17 +756,27 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
 }
 
 // ---------------------------------------------------------------------------- column sums
-// out[c] = sum_r x[r, c] in two deterministic passes. Pass 1: block = 32 x 8 threads covering
-// 32*VEC columns, blockIdx.y a slice of rows; each block writes its column sums to
-// partial[slice][c]. Pass 2 (colsum_reduce_kernel) adds the slices in a fixed order, so the
-// result does not depend on scheduling.
+// out[c] = sum_r x[r, c] in one launch. A cluster of kColsumSlices CTAs along y covers one
+// stripe of 32*VEC columns; CTA y of the cluster takes the y-th slice of the rows. Thread (x, t)
+// takes rows t, t + 8, ... of the slice, kColsumBatch 16-byte loads in flight at a time (rows
+// past the slice read as zeros); the eight row groups of the CTA are added in order into a
+// per-column slice sum in shared memory, and after a cluster barrier CTA 0 adds the slices'
+// sums, read from the other CTAs' shared memory, in rank order. Every addition has a fixed
+// order, so the result does not depend on scheduling.
+constexpr int kColsumSlices = 8;
+constexpr int kColsumBatch = 8;
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 template <typename T>
-__global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
-                                                     const T* __restrict__ x,
-                                                     float* __restrict__ partial,
-                                                     long long rows_per) {
+__global__ void __cluster_dims__(1, kColsumSlices, 1) __launch_bounds__(256, 4)
+    colsum_kernel(long long rows, int cols, const T* __restrict__ x, float* __restrict__ out,
+                  long long rows_per) {
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
+  __shared__ float slice_sum[32 * V];
   const int c0 = (blockIdx.x * 32 + threadIdx.x) * V;
   const long long r0 = blockIdx.y * rows_per;
   const long long r1 = min(rows, r0 + rows_per);
@@ -774,21 +784,19 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
 #pragma unroll
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
   if (c0 < cols) {
-    long long r = r0 + threadIdx.y;
-    for (; r + 56 < r1; r += 64) {  // eight independent rows in flight per thread
-      float v[8][V];
+    for (long long r = r0 + threadIdx.y; r < r1; r += 8 * kColsumBatch) {
+      uint4 w[kColsumBatch];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) Vec<T>::load(x + (r + 8 * u) * cols + c0, v[u]);
+      for (int u = 0; u < kColsumBatch; ++u)
+        w[u] = r + 8 * u < r1 ? __ldg(reinterpret_cast<const uint4*>(x + (r + 8 * u) * cols + c0))
+                              : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int j = 0; j < V; ++j)
-        acc[j] += ((v[0][j] + v[1][j]) + (v[2][j] + v[3][j])) +
-                  ((v[4][j] + v[5][j]) + (v[6][j] + v[7][j]));
-    }
-    for (; r < r1; r += 8) {
-      float v[V];
-      Vec<T>::load(x + r * cols + c0, v);
+      for (int u = 0; u < kColsumBatch; ++u) {
+        float v[V];
+        Vec<T>::unpack(w[u], v);
 #pragma unroll
-      for (int j = 0; j < V; ++j) acc[j] += v[j];
+        for (int j = 0; j < V; ++j) acc[j] += v[j];
+      }
     }
   }
 #pragma unroll
@@ -796,32 +804,26 @@ __global__ void __launch_bounds__(256) colsum_kernel(long long rows, int cols,
   __syncthreads();
   const int t = threadIdx.y * 32 + threadIdx.x;
   for (int cc = t; cc < 32 * V; cc += 256) {
-    const int col = blockIdx.x * 32 * V + cc;
-    if (col < cols) {
-      float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) s += red[k][cc];
-      partial[(long long)blockIdx.y * cols + col] = s;
+    for (int k = 0; k < 8; ++k) sum += red[k][cc];
+    slice_sum[cc] = sum;
+  }
+  cluster_sync_all();  // every slice sum of the cluster is written
+  if (cluster_ctarank() == 0) {
+    for (int cc = t; cc < 32 * V; cc += 256) {
+      const int col = blockIdx.x * 32 * V + cc;
+      const uint32_t local = smem_u32(&slice_sum[cc]);
+      float p[kColsumSlices];
+#pragma unroll
+      for (int q = 0; q < kColsumSlices; ++q) p[q] = ld_shared_cluster_f32(mapa_shared(local, q));
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kColsumSlices; ++q) sum += p[q];
+      if (col < cols) out[col] = sum;
     }
   }
-}
-
-// out[c] = sum over slices of partial[slice][c] in a fixed order: every slice's value is loaded
-// before any is added (at most kColsumMaxSlices in flight per thread), then added in slice
-// order. Small blocks spread the columns over every SM.
-__global__ void __launch_bounds__(64) colsum_reduce_kernel(int cols, int slices,
-                                                           const float* __restrict__ partial,
-                                                           float* __restrict__ out) {
-  const int c = blockIdx.x * 64 + threadIdx.x;
-  if (c >= cols) return;
-  float p[kColsumMaxSlices];
-#pragma unroll
-  for (int k = 0; k < kColsumMaxSlices; ++k)
-    p[k] = k < slices ? __ldg(partial + (long long)k * cols + c) : 0.f;
-  float acc = 0.f;
-#pragma unroll
-  for (int k = 0; k < kColsumMaxSlices; ++k) acc += p[k];
-  out[c] = acc;
+  cluster_sync_all();  // no CTA leaves while CTA 0 may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------- fp32 GEMM
@@ -999,6 +1001,14 @@ cudaError_t ln_fwd_dispatch(long long rows, int h, float eps, const void* x, con
   return ln_fwd_inst<T, 8, 8>(rows, h, eps, x, g, b, y, mean, rstd, s);
 }
 
+// dgamma, dbeta (and dres_sum) from the per-block partial rows, in a fixed order.
+cudaError_t launch_param_reduce(int h, long long slices, int nsum, const float* partial,
+                                float* dgamma, float* dbeta, float* dres_sum, cudaStream_t s) {
+  ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
+                                                             dgamma, dbeta, dres_sum);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* dres,
                             const void* x, const float* g, const float* mean, const float* rstd,
@@ -1052,9 +1062,7 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
                                                         pdx, partial, rows_per);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
-                                                               dgamma, dbeta, dres_sum);
-    return cudaGetLastError();
+    return launch_param_reduce(h, slices, nsum, partial, dgamma, dbeta, dres_sum, s);
   }
   // Wider rows: a dx kernel, then a parameter-partial kernel over slices of rows.
   if (nvec <= 64)
@@ -1087,9 +1095,7 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
         rows, h, reinterpret_cast<const T*>(dy), reinterpret_cast<const T*>(x), nullptr, mean,
         rstd, partial, rows_per);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
-                                                             dgamma, dbeta, dres_sum);
-  return cudaGetLastError();
+  return launch_param_reduce(h, slices, nsum, partial, dgamma, dbeta, dres_sum, s);
 }
 
 }  // namespace
@@ -1120,34 +1126,19 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
                                         nblk, dgamma, dbeta, dres_sum, err, s);
 }
 
-int colsum_slices(long long rows, int cols, int dtype) {
-  const int V = dtype ? 8 : 4;
-  const int cb = (cols + 32 * V - 1) / (32 * V);
-  long long splits = (4 * 148 + cb - 1) / cb;  // aim for ~4 blocks per SM
-  if (splits > kColsumMaxSlices) splits = kColsumMaxSlices;
-  if (splits > (rows + 7) / 8) splits = (rows + 7) / 8;
-  if (splits < 1) splits = 1;
-  const long long rows_per = (rows + splits - 1) / splits;
-  return (int)((rows + rows_per - 1) / rows_per);
-}
-
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
-                          float* partial, cudaStream_t s) {
+                          cudaStream_t s) {
   if (rows <= 0) return cudaMemsetAsync(out, 0, sizeof(float) * cols, s);
   const int V = dtype ? 8 : 4;
   const int cb = (cols + 32 * V - 1) / (32 * V);
-  const int slices = colsum_slices(rows, cols, dtype);
-  const long long rows_per = (rows + slices - 1) / slices;
-  dim3 grid(cb, (unsigned)slices), block(32, 8);
+  const long long rows_per = (rows + kColsumSlices - 1) / kColsumSlices;
+  dim3 grid(cb, kColsumSlices), block(32, 8);
   if (dtype)
     colsum_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        rows, cols, reinterpret_cast<const __nv_bfloat16*>(x), partial, rows_per);
+        rows, cols, reinterpret_cast<const __nv_bfloat16*>(x), out, rows_per);
   else
     colsum_kernel<float><<<grid, block, 0, s>>>(rows, cols, reinterpret_cast<const float*>(x),
-                                                 partial, rows_per);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  colsum_reduce_kernel<<<(cols + 63) / 64, 64, 0, s>>>(cols, slices, partial, out);
+                                                 out, rows_per);
   return cudaGetLastError();
 }
 

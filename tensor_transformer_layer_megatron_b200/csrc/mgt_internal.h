@@ -143,13 +143,10 @@ cudaError_t launch_exp2_probe(int path, long long n, const float* x, float* y,
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
 
-// Column sums of a [rows, cols] activation matrix into fp32 (bias gradients), deterministic:
-// per-slice partial sums in `partial` (colsum_slices(...) * cols floats, at most
-// kColsumMaxSlices * cols), then a fixed-order reduction of the slices.
-constexpr int kColsumMaxSlices = 32;
-int colsum_slices(long long rows, int cols, int dtype);
+// Column sums of a [rows, cols] activation matrix into fp32 (bias gradients), deterministic
+// (fixed-order additions; one launch, no scratch memory).
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
-                          float* partial, cudaStream_t stream);
+                          cudaStream_t stream);
 
 // Causal attention over packed qkv [T][p][3][H/p][d]; O [T][p][H/p][d]; lse [b][H][s].
 struct AttnArgs {
