@@ -217,13 +217,33 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, int row, int c
   }
 }
 
+// The per-element source of a bf16 epilogue chunk (32 columns from col of row `row`): the
+// residual (kEpiBf16 with a residual) or u (kEpiDGelu); zeros for a row past M. Loaded ahead
+// of the accumulator so that its latency overlaps the TMEM read (and the previous chunk).
+template <int EPI>
+__device__ __forceinline__ bool epi_has_src(const GemmArgs& a) {
+  return (EPI == kEpiBf16 && a.res) || EPI == kEpiDGelu;
+}
+template <int EPI>
+__device__ __forceinline__ void epi_load_src(const GemmArgs& a, int row, int col, bool row_ok,
+                                             uint4 (&r4)[4]) {
+  const __nv_bfloat16* src =
+      EPI == kEpiDGelu
+          ? reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col
+          : reinterpret_cast<const __nv_bfloat16*>(a.res) + (long long)row * a.ldr + col;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    r4[q] = row_ok ? *reinterpret_cast<const uint4*>(src + q * 8) : make_uint4(0, 0, 0, 0);
+}
+
 // Values of one whole 32-column chunk of a bf16 epilogue, packed as bf16 pairs for a staged
-// (TMA) store: w holds out, w2 out2 (kEpiGelu only). Rows at or past M (row_ok false) read no
-// residual or aux; the store clips them.
+// (TMA) store: w holds out, w2 out2 (kEpiGelu only); r4 is the chunk's source as loaded by
+// epi_load_src (read when epi_has_src). Rows at or past M (row_ok false) read no residual or
+// aux; the store clips them.
 template <int EPI>
 __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int col, bool row_ok,
-                                                float (&v)[32], uint32_t (&w)[16],
-                                                uint32_t (&w2)[16]) {
+                                                float (&v)[32], const uint4 (&r4)[4],
+                                                uint32_t (&w)[16], uint32_t (&w2)[16]) {
   const __nv_bfloat16* bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
   if ((EPI == kEpiBf16 || EPI == kEpiGelu) && bias) {
     const uint4* bp = reinterpret_cast<const uint4*>(bias + col);
@@ -238,15 +258,7 @@ __device__ __forceinline__ void epi_values_bf16(const GemmArgs& a, int row, int 
       }
     }
   }
-  if ((EPI == kEpiBf16 && a.res) || EPI == kEpiDGelu) {
-    const __nv_bfloat16* src =
-        EPI == kEpiDGelu
-            ? reinterpret_cast<const __nv_bfloat16*>(a.aux) + (long long)row * a.ld_aux + col
-            : reinterpret_cast<const __nv_bfloat16*>(a.res) + (long long)row * a.ldr + col;
-    uint4 r4[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      r4[q] = row_ok ? *reinterpret_cast<const uint4*>(src + q * 8) : make_uint4(0, 0, 0, 0);
+  if (epi_has_src<EPI>(a)) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t ww[4] = {r4[q].x, r4[q].y, r4[q].z, r4[q].w};
@@ -809,6 +821,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
       const TileCoord tc = tile_coord(tile, num_m2, num_n, args.n_fast);
       const int row = tc.mb * 256 + rank * 128 + ew * 32 + lane;
+      // bf16 epilogues with a residual or u: each staged chunk's source is loaded one chunk
+      // ahead, the first one before the accumulator is ready
+      constexpr bool kSrcEpi = !kGlu && (EPI == kEpiBf16 || EPI == kEpiDGelu);
+      const int src_row0 = tc.mb * 256 + rank * 128 + ew * 32;
+      const int src_orow = args.out_sp ? seq_row(args, row) : row;
+      auto src_chunk = [&](int c) {  // chunk c is stored staged and reads a source
+        const int n0 = tc.nb * BN + c * 32;
+        return epi_has_src<EPI>(args) && staged && n0 + 32 <= args.Ng && src_row0 < args.M;
+      };
+      uint4 src_next[4] = {};
+      if constexpr (kSrcEpi)
+        if (c_begin < c_end && src_chunk(c_begin))
+          epi_load_src<EPI>(args, src_orow, tc.ng * args.Ng + tc.nb * BN + c_begin * 32,
+                            row < args.M, src_next);
       const bool ok = mbar_wait(&tfull[acc], acc_phase, args.err, kErrTimeoutEpilogue,
                                 abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -855,6 +881,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll 1
       for (int c = c_begin; c < c_end; ++c) {
+        uint4 src_cur[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) src_cur[q] = src_next[q];
+        if constexpr (kSrcEpi)
+          if (c + 1 < c_end && src_chunk(c + 1))
+            epi_load_src<EPI>(args, src_orow, tc.ng * args.Ng + tc.nb * BN + (c + 1) * 32,
+                              row < args.M, src_next);
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * 256 + c * 32,
                            v);
@@ -884,7 +917,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                   make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           } else {
             uint32_t w[16], w2[16];
-            epi_values_bf16<EPI>(args, orow, col, row < args.M, v, w, w2);
+            epi_values_bf16<EPI>(args, orow, col, row < args.M, v, src_cur, w, w2);
             constexpr bool two = EPI == kEpiGelu || EPI == kEpiDSwiglu;
             if (lane == 0) bulk_wait_read0();
             __syncwarp();
