@@ -1346,6 +1346,9 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
   const __nv_bfloat16* g_ = reinterpret_cast<const __nv_bfloat16*>(a.dO);
   const __nv_bfloat16* qkv_ = reinterpret_cast<const __nv_bfloat16*>(a.qkv);
   uint2 ov[4], gv[4], kv[4], vv[4];
+  // lane i < 4 fetches token i's lse with the rows, so no load waits inside the loop below
+  const int lpos = c * 32 + warp * 4 + lane;
+  const float lse_l = (lane < 4 && lpos < a.s) ? a.lse[(long long)bh * a.s + lpos] : 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int pos = c * 32 + warp * 4 + i;
@@ -1364,6 +1367,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int pos = c * 32 + warp * 4 + i;
+    const float lse_i = __shfl_sync(0xffffffffu, lse_l, i);
     if (pos >= a.s) {  // warp-uniform: padding of the softmax statistics (P = 0 there)
       if (lane == 0) {
         stat[pos] = -INFINITY;
@@ -1393,7 +1397,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
     }
     if (lane == 0) {
       a.Dsum[(long long)bh * a.s + pos] = dsum;
-      stat[pos] = -a.lse[(long long)bh * a.s + pos] * kLog2eF;
+      stat[pos] = -lse_i * kLog2eF;
       stat[nqp + pos] = -dsum;
     }
     *reinterpret_cast<int4*>(a.dq_fix + tok * ld_o + (long long)n * D + lane * 4) =
