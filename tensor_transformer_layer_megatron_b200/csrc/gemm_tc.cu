@@ -881,6 +881,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll 1
       for (int c = c_begin; c < c_end; ++c) {
+        if constexpr (EPI == kEpiStoreF32) {
+          // fp32 chunk written straight from registers: two 16-lane loads in the 16x256b
+          // layout, so each group of four threads stores 32 consecutive bytes of one row
+          // (whole sectors) and nothing passes through shared memory, whose port the
+          // operand traffic of the next tile's mainloop needs.
+          const int n0 = tc.nb * BN + c * 32;
+          const int row0 = tc.mb * 256 + rank * 128 + ew * 32;
+          if (staged && n0 + 32 <= args.Ng && row0 < args.M) {
+            const int col = tc.ng * args.Ng + n0;
+            float* o = reinterpret_cast<float*>(args.out) +
+                       (long long)(col / args.out_ng) * args.out_gs + (col % args.out_ng) +
+                       2 * (lane & 3);
+            uint32_t r16[2][16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              tmem_ld_16x256b_x4_nw(tmem_base + (static_cast<uint32_t>(ew * 32 + hh * 16) << 16) +
+                                        acc * 256 + c * 32,
+                                    r16[hh]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              reg_fence(r16[hh]);
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {  // rows t/4 and t/4 + 8 of this 16-lane half
+                const int rr = row0 + hh * 16 + e * 8 + (lane >> 2);
+                if (rr < args.M) {
+                  float* orow = o + (long long)(args.out_sp ? seq_row(args, rr) : rr) * args.ldc;
+#pragma unroll
+                  for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<float2*>(orow + 8 * k) =
+                        make_float2(__uint_as_float(r16[hh][4 * k + 2 * e]) * dq,
+                                    __uint_as_float(r16[hh][4 * k + 2 * e + 1]) * dq);
+                }
+              }
+            }
+            continue;
+          }
+        }
         uint4 src_cur[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) src_cur[q] = src_next[q];

@@ -275,6 +275,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32_nw(uint32_t taddr, uint32_t (
         "=r"(r[31])
       : "r"(taddr));
 }
+// 16 lanes x 32 consecutive 32-bit columns, four repetitions of the 16x256b shape: thread t
+// receives lane (base + t/4) in r[4k], r[4k+1] and lane (base + 8 + t/4) in r[4k+2], r[4k+3],
+// both at columns 8k + 2(t%4) and 8k + 2(t%4) + 1 (k = 0..3), so four consecutive threads
+// hold 32 consecutive bytes of a row. No wait: call tmem_ld_wait() and reg_fence() after it.
+__device__ __forceinline__ void tmem_ld_16x256b_x4_nw(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
