@@ -603,13 +603,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // `tfull` in both CTAs; both CTAs' epilogue warps arrive on the leader's `tempty` (count 8).
 // A cluster barrier after initialisation and another before exit bracket all cross-CTA
 // traffic; every wait in between is bounded.
-// Six 32 KB stages; the SwiGLU forward keeps five to make room for its three staged outputs.
-constexpr int pair_stages(int epi) { return epi == kEpiSwiglu ? 5 : 6; }
-constexpr int stage_out_bytes(int epi) { return epi == kEpiSwiglu ? 6144 : 4096; }
+// Six 32 KB stages; the SwiGLU forward keeps five to make room for its three staged outputs,
+// and the fp32 store, which stages nothing, takes seven.
+constexpr int pair_stages(int epi) {
+  return epi == kEpiSwiglu ? 5 : (epi == kEpiStoreF32 ? 7 : 6);
+}
+constexpr int stage_out_bytes(int epi) {
+  return epi == kEpiSwiglu ? 6144 : (epi == kEpiStoreF32 ? 0 : 4096);
+}
 constexpr int kPairAB = BM * BK * 2;            // 16 KB: this CTA's A rows or B half
 constexpr int kPairStageBytes = 2 * kPairAB;    // 32 KB per CTA per stage
-// Output staging per epilogue warp: one 32 x 32 fp32 chunk (128-byte rows), or up to three
-// 32 x 32 bf16 chunks (64-byte rows, 2 KB apart: out, then out2 / the second GLU half).
+// Output staging per epilogue warp: up to three 32 x 32 bf16 chunks (64-byte rows, 2 KB apart:
+// out, then out2 / the second GLU half); none for fp32 outputs, which are stored from registers.
 // stages | barriers (padded to 1 KB) | output staging | 1 KB alignment slack
 constexpr int pair_smem(int epi) {
   return pair_stages(epi) * kPairStageBytes + 1024 + kEpiWarps * stage_out_bytes(epi) + 1024;
@@ -624,12 +629,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmC2, const GemmArgs args, int num_m2,
                     int num_n, int BN, int staged) {
-  // tmC (tmC2: out2 of kEpiGelu): output viewed as {out_ng, M, groups}; each epilogue warp
-  // stages a 32 x 32 chunk in a swizzled shared buffer (128-byte rows for fp32, 64-byte rows
-  // for bf16) and stores it with one TMA bulk tensor store (full lines, coalesced; rows past M
-  // are clipped). A chunk that straddles N is written element by element instead, and so is
-  // every chunk when `staged` is 0 (the host found a column offset that is not a multiple of
-  // 16 bytes, which a TMA store cannot start at).
+  // tmC (tmC2: out2 of kEpiGelu): output viewed as {out_ng, M, groups}; for bf16 outputs each
+  // epilogue warp stages a 32 x 32 chunk in a swizzled shared buffer (64-byte rows) and stores
+  // it with one TMA bulk tensor store (full lines, coalesced; rows past M are clipped); fp32
+  // chunks are stored from registers in whole 32-byte sectors. A chunk that straddles N is
+  // written element by element instead, and so is every chunk when `staged` is 0 (the host
+  // found a column offset that is not a multiple of 16 bytes, which a TMA store cannot start
+  // at and the 8-byte fp32 stores assume).
   // BN: the pair's N tile, a multiple of 32 up to 256 (256 when B is MN-major); each CTA
   // loads BN/2 rows of B. Accumulator buffers stay 256 columns apart in TMEM.
   constexpr int STAGES = pair_stages(EPI);
@@ -945,15 +951,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (n0 < args.Ng && (n0 + 32 > args.Ng || !staged)) {
           if (row < args.M) epilogue_chunk<EPI>(args, orow, col, min(32, args.Ng - n0), v);
         } else if (n0 < args.Ng && row0 < args.M) {  // warp-uniform
-          uint8_t* buf = stage_out + (warp - 2) * kStageOut;
-          if constexpr (EPI == kEpiStoreF32) {
-            if (lane == 0) bulk_wait_read0();  // the previous chunk's store has read the buffer
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          } else {
+          // (bf16 outputs only: whole fp32 chunks were stored from registers above)
+          if constexpr (EPI != kEpiStoreF32) {
+            uint8_t* buf = stage_out + (warp - 2) * kStageOut;
             uint32_t w[16], w2[16];
             epi_values_bf16<EPI>(args, orow, col, row < args.M, v, src_cur, w, w2);
             constexpr bool two = EPI == kEpiGelu || EPI == kEpiDSwiglu;
@@ -970,19 +970,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(buf + 2048 + lane * 64 + ((j ^ sw) << 4)) =
                     make_uint4(w2[4 * j], w2[4 * j + 1], w2[4 * j + 2], w2[4 * j + 3]);
             }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (EPI == kEpiDSwiglu) {  // tmC views dz as {Ng, M, 2*NG}
-              tma_store_3d(&tmC, buf, n0, orow0, 2 * tc.ng);
-              tma_store_3d(&tmC, buf + 2048, n0, orow0, 2 * tc.ng + 1);
-            } else {
-              tma_store_3d(&tmC, buf, col % args.out_ng, orow0, col / args.out_ng);
-              if (EPI == kEpiGelu)
-                tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, orow0, col / args.out_ng);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (EPI == kEpiDSwiglu) {  // tmC views dz as {Ng, M, 2*NG}
+                tma_store_3d(&tmC, buf, n0, orow0, 2 * tc.ng);
+                tma_store_3d(&tmC, buf + 2048, n0, orow0, 2 * tc.ng + 1);
+              } else {
+                tma_store_3d(&tmC, buf, col % args.out_ng, orow0, col / args.out_ng);
+                if (EPI == kEpiGelu)
+                  tma_store_3d(&tmC2, buf + 2048, col % args.out_ng, orow0, col / args.out_ng);
+              }
+              bulk_commit();
             }
-            bulk_commit();
           }
         }
       }
