@@ -1,26 +1,29 @@
-// Causal attention forward on the fifth-generation tensor cores (tcgen05 + TMEM + TMA).
+// Causal attention on the fifth-generation tensor cores (tcgen05 + TMEM + TMA): the forward,
+// and the backward with the probabilities recomputed from the saved log-sum-exp (below).
 //
-// One CTA owns one 128-query tile of one head. The heads are local to their tensor-parallel
-// shard (the column split of W_q/W_k/W_v on the trdm.cn page, section 2.1, keeps whole heads
-// on a shard), so the softmax never needs another shard's data. Softmax arithmetic is fp32
-// (section 3.2, attention_softmax_in_fp32); scale 1/sqrt(d); key j visible to query i iff
-// j <= i.
+// The heads are local to their tensor-parallel shard (the column split of W_q/W_k/W_v on the
+// trdm.cn page, section 2.1, keeps whole heads on a shard), so the softmax never needs another
+// shard's data. Softmax arithmetic is fp32 (section 3.2, attention_softmax_in_fp32); scale
+// 1/sqrt(d); key j visible to query i iff j <= i.
 //
-// Per key block of 128 (double-buffered K/V tiles from TMA):
-//   S = Q K^T            tcgen05.mma M=128 N=128, fp32 in TMEM (two S buffers, so the next
-//                        block's S is computed while the softmax works on this one)
+// Forward: one CTA per pair of consecutive 128-query tiles of one head, longest pairs first.
+// Per tile and key block of 128 (double-buffered K/V tiles from TMA):
+//   S = Q K^T            tcgen05.mma M=128 N=128, fp32 into the tile's S buffer in TMEM
 //   softmax warps        one thread per query row reads all 128 of its scores with tcgen05.ld,
 //                        so the row max and sum need no exchange between threads;
 //                        P = exp2(S*scale*log2e - m) is packed to bf16 and written back into the
 //                        first 64 columns of the same S buffer
 //   O += P V             tcgen05.mma M=128 N=d with A = P read from TMEM and V read N-major
 //                        straight from its TMA tile
-// The running max is updated lazily: O and the row sum are rescaled only when a row's max grows
-// by more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16).
-// Finally O / l is written in bf16 and lse = (m + log2 l) * ln 2.
+// One tile's softmax runs while the tensor pipe works on the other tile's products. The
+// running max is updated lazily: O and the row sum are rescaled only when a row's max grows by
+// more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16). Finally O / l is
+// staged in bf16 in the tile's Q buffer and written by bulk tensor stores, and
+// lse = (m + log2 l) * ln 2.
 //
-// Warps 0-3: softmax + output (warp w owns TMEM lanes 32w..32w+31, i.e. query rows);
-// warp 4: TMA producer; warp 5: TMEM owner and MMA issuer. Every wait is bounded.
+// Forward warps: 0-3 softmax and output of query tile 0, 4-7 of tile 1 (warp w owns TMEM lanes
+// 32 (w % 4) .., i.e. query rows); warp 8 TMA producer; warp 9 TMEM owner and MMA issuer.
+// Every wait is bounded.
 #include "mgt_device.cuh"
 
 namespace mgt {
