@@ -355,7 +355,10 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
 }
 
 // ============================================================================ backward
-// Two kernels, both on tcgen05 with the probabilities recomputed from the saved log-sum-exp:
+// Head dimension 128 (bf16) runs the single key-stationary kernel further below
+// (attn_bwd_fused_tc_kernel: S and dP once per tile pair, dQ accumulated in 32-bit fixed point
+// through bulk tensor reduce-adds) between a pre-pass and a conversion. Head dimension 64 uses
+// two kernels, both on tcgen05 with the probabilities recomputed from the saved log-sum-exp:
 //   dK/dV kernel, one CTA per 128-key block (key-stationary), looping over query blocks in
 //     64-query sub-blocks with double-buffered TMEM: S^T = K Q^T and dP^T = V dO^T; one
 //     thread per key row forms P^T = exp2(S^T*scale*log2e - lse*log2e) and
