@@ -68,9 +68,10 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   uint64_t* k_empty = bars + 5;   // [2]: released once every S of that block has read K
   uint64_t* v_empty = bars + 7;   // [2]: released once every PV of that block has read V
   uint64_t* s_full = bars + 9;    // [2] per tile: S of the tile's current block is in TMEM
-  uint64_t* p_full = bars + 11;   // [2] per tile: P of the tile's current block is in TMEM
-  uint64_t* drain = bars + 13;    // every MMA done (one-shot: the output waits on it)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  // [2 tiles][2 halves]: P of keys 0-63 / 64-127 of the tile's current block is in TMEM
+  uint64_t* p_half = bars + 11;
+  uint64_t* drain = bars + 15;    // every MMA done (one-shot: the output waits on it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,7 +93,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_half[2 * i], 4);
+      mbar_init(&p_half[2 * i + 1], 4);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -173,19 +175,23 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
         tc_commit(&s_full[u]);
         return true;
       };
-      auto issue_pv = [&](int u, int kb) -> bool {  // O_u += P_u V_kb
-        if (!mbar_wait(&p_full[u], kb & 1, a.err, kErrTimeoutAttn, abort_flag)) return false;
+      auto issue_pv = [&](int u, int kb) -> bool {  // O_u += P_u V_kb, keys 0-63 first
         if (!mbar_wait(&v_full[kb & 1], (kb >> 1) & 1, a.err, kErrTimeoutAttn, abort_flag))
           return false;
-        tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + L::V_OFF + (kb & 1) * L::TILE);
         const uint32_t p_tmem = tmem + (u ? L::TMEM_S1 : L::TMEM_S0);
         const uint32_t o_tmem = tmem + (u ? L::TMEM_O1 : L::TMEM_O0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA (8 packed P columns)
-          tc_mma_f16_tmem_a(o_tmem, p_tmem + kk * 8,
-                            smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                            (kb > 0 || kk > 0) ? 1u : 0u);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!mbar_wait(&p_half[2 * u + hf], kb & 1, a.err, kErrTimeoutAttn, abort_flag))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = hf * 4; kk < hf * 4 + 4; ++kk)  // 16 keys (8 packed P columns) each
+            tc_mma_f16_tmem_a(o_tmem, p_tmem + kk * 8,
+                              smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                              (kb > 0 || kk > 0) ? 1u : 0u);
+        }
         return true;
       };
       if (ok) ok = issue_s(0, 0);
@@ -258,49 +264,45 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
       const float alpha = need ? ex2_approx(m_run - mx) : 1.f;
       if (need) m_run = mx;
       // exponent arguments on pairs of scores (paired fp32 FMA), 2^x on the special-function
-      // unit, row sums in four paired accumulators
+      // unit, row sums in four paired accumulators; P of keys 0-63 is handed to the MMA before
+      // keys 64-127 are computed, so the first half of this block's PV overlaps the second
       const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
       uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        float pa, pb;
-        f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), c2, nm2), pa, pb);
-        pa = ex2_approx(pa);
-        pb = ex2_approx(pb);
-        sv[i] = pa;
-        sv[i + 1] = pb;
-        acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(pa, pb));
-      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float pw[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          pw[j] = __uint_as_float(pack_bf16x2(sv[c * 64 + 2 * j], sv[c * 64 + 2 * j + 1]));
-        tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);
+        for (int i = 0; i < 64; i += 2) {
+          float pa, pb;
+          f2_unpack(f2_fma(f2_pack(sv[c * 64 + i], sv[c * 64 + i + 1]), c2, nm2), pa, pb);
+          pa = ex2_approx(pa);
+          pb = ex2_approx(pb);
+          acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(pa, pb));
+          pw[i >> 1] = __uint_as_float(pack_bf16x2(pa, pb));
+        }
+        tmem_st_32x32b_x32(lane_base + s_col + c * 32, pw);  // includes the store wait
+        // O holds the sum up to block kb-1 (its PV completed before this S was committed); it
+        // is rescaled before this block's first PV, which waits for the first half of P
+        if (c == 0 && kb > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int oc = 0; oc < D / 32; ++oc) {
+            float o[32];
+            const uint32_t ta = lane_base + o_col + oc * 32;
+            tmem_ld_32x32b_x32(ta, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st_32x32b_x32(ta, o);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_half[2 * u + c]);
       }
       float rs[8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) f2_unpack(acc2[k], rs[2 * k], rs[2 * k + 1]);
       l_run = l_run * alpha +
               (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
-      // O holds the sum up to block kb-1 (its PV completed before this S was committed); it
-      // is rescaled before this block's PV, which waits for p_full below.
-      if (kb > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          const uint32_t ta = lane_base + o_col + c * 32;
-          tmem_ld_32x32b_x32(ta, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st_32x32b_x32(ta, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[u]);
     }
     if (nkv > 0) {
       // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
