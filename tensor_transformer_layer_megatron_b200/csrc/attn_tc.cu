@@ -15,7 +15,8 @@
 //                        first 64 columns of the same S buffer
 //   O += P V             tcgen05.mma M=128 N=d with A = P read from TMEM and V read N-major
 //                        straight from its TMA tile
-// One tile's softmax runs while the tensor pipe works on the other tile's products. The
+// One tile's softmax runs while the tensor pipe works on the other tile's products, and P
+// reaches the MMA in two halves of 64 keys so that PV starts before the softmax ends. The
 // running max is updated lazily: O and the row sum are rescaled only when a row's max grows by
 // more than 2^8 (P stays <= 256 otherwise, exact in fp32 and safe in bf16). Finally O / l is
 // staged in bf16 in the tile's Q buffer and written by bulk tensor stores, and
