@@ -990,7 +990,8 @@ template <int D>
 __global__ void __launch_bounds__(kFusedBwdThreads, 1)
     attn_bwd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                              const __grid_constant__ CUtensorMap tm_do,
-                             const __grid_constant__ CUtensorMap tm_dq, const AttnArgs a,
+                             const __grid_constant__ CUtensorMap tm_dq,
+                             const __grid_constant__ CUtensorMap tm_dqkv, const AttnArgs a,
                              float scale_log2, float scale) {
   using L = FusedBwdLayout<D>;
   static_assert(D == 128, "dQ^T tiles use M = head_dim = 128");
@@ -1039,6 +1040,7 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
+    tma_prefetch_desc(&tm_dqkv);
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -1293,38 +1295,59 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[g & 1]);
     }
-    if (ok && niter > 0) {
+    if (niter > 0) {
       // drain is committed once, after the last MMA (a one-shot barrier: no phase aliasing)
-      ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
+      if (ok) ok = mbar_wait(drain, 0, a.err, kErrTimeoutAttn, abort_flag);
+      // the eight warps meet at both barriers below on every path, and decide together
+      uint32_t all_ok;
+      asm volatile(
+          "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.and.pred po, 1, 256, pi; "
+          "selp.u32 %0, 1, 0, po; }"
+          : "=r"(all_ok)
+          : "r"((uint32_t)__all_sync(0xffffffffu, ok))
+          : "memory");
+      // dK (scaled) and dV in bf16 into the K and V tile buffers (every MMA has completed, so
+      // they are no longer read), as the 128-byte-swizzled boxes of the dqkv tensor map:
+      // 16-byte piece j of row r's 64-column chunk at r * 128 + (j ^ (r % 8)) * 16; rows past
+      // the sequence are clipped by the map.
+      uint8_t* stage_k = smem + L::K_OFF;
+      uint8_t* stage_v = smem + L::V_OFF;
+      if (all_ok) {
         tc_fence_after();
-        const int key = kb * 128 + r;
-        const long long ld = 3LL * H * D;
-        __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(a.dqkv) + ((long long)b * S + key) * ld +
-                            (long long)t * 3 * hp * D + (long long)jh * D + (long long)hp * D;
-        __nv_bfloat16* dv = dk + (long long)hp * D;
 #pragma unroll 1
         for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {  // this half of d
           float v[32], kk[32];
           tmem_ld_32x32b_x32(lane_base + L::T_DV + c * 32, v);
           tmem_ld_32x32b_x32(lane_base + L::T_DK + c * 32, kk);
-          if (key < S) {
+          const int off = (c >> 1) * 16384 + r * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 wv, wk;
-              wv.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-              wv.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-              wv.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-              wv.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              wk.x = pack_bf16x2(kk[q * 8 + 0] * scale, kk[q * 8 + 1] * scale);
-              wk.y = pack_bf16x2(kk[q * 8 + 2] * scale, kk[q * 8 + 3] * scale);
-              wk.z = pack_bf16x2(kk[q * 8 + 4] * scale, kk[q * 8 + 5] * scale);
-              wk.w = pack_bf16x2(kk[q * 8 + 6] * scale, kk[q * 8 + 7] * scale);
-              *reinterpret_cast<uint4*>(dv + c * 32 + q * 8) = wv;
-              *reinterpret_cast<uint4*>(dk + c * 32 + q * 8) = wk;
-            }
+          for (int q = 0; q < 4; ++q) {
+            uint4 wv, wk;
+            wv.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+            wv.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+            wv.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+            wv.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            wk.x = pack_bf16x2(kk[q * 8 + 0] * scale, kk[q * 8 + 1] * scale);
+            wk.y = pack_bf16x2(kk[q * 8 + 2] * scale, kk[q * 8 + 3] * scale);
+            wk.z = pack_bf16x2(kk[q * 8 + 4] * scale, kk[q * 8 + 5] * scale);
+            wk.w = pack_bf16x2(kk[q * 8 + 6] * scale, kk[q * 8 + 7] * scale);
+            const int jj = ((c & 1) * 4 + q) ^ (r & 7);
+            *reinterpret_cast<uint4*>(stage_v + off + jj * 16) = wv;
+            *reinterpret_cast<uint4*>(stage_k + off + jj * 16) = wk;
           }
         }
+        fence_proxy_async_smem();
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // every row of both tiles is staged
+      if (warp == 0 && lane == 0 && all_ok && !*abort_flag) {
+        const int col_dk = t * 3 * hp * D + hp * D + jh * D, col_dv = col_dk + hp * D;
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_store_3d(&tm_dqkv, stage_k + c * 16384, col_dk + c * 64, kb * 128, b);
+          tma_store_3d(&tm_dqkv, stage_v + c * 16384, col_dv + c * 64, kb * 128, b);
+        }
+        bulk_commit();
+        bulk_wait0();
       }
     }
   }
@@ -1489,9 +1512,16 @@ cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
     if (!make_tensor_map_i32_3d(&tm_dq, a.dq_fix, dims, strides, qbox))
       return cudaErrorInvalidValue;
   }
+  CUtensorMap tm_dqkv;  // dK and dV written into dqkv, viewed as qkv is
+  {
+    const uint64_t dims[3] = {three_h, (uint64_t)a.s, (uint64_t)a.b};
+    const uint64_t strides[2] = {three_h, three_h * a.s};
+    if (!make_tensor_map_bf16_3d(&tm_dqkv, a.dqkv, dims, strides, box))
+      return cudaErrorInvalidValue;
+  }
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
   attn_bwd_fused_tc_kernel<D><<<grid, kFusedBwdThreads, L::BYTES, s>>>(
-      tm_qkv, tm_do, tm_dq, a, kLog2eF * scale, scale);
+      tm_qkv, tm_do, tm_dq, tm_dqkv, a, kLog2eF * scale, scale);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(a, scale);
   return cudaGetLastError();
