@@ -111,6 +111,8 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();  // qkv is the previous kernel's result
+  grid_dependents_launch();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -1050,6 +1052,8 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();  // the pre-pass's statistics and zeroed accumulator
+  grid_dependents_launch();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -1366,6 +1370,8 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
 // max |V row|^2 and max |dO row|^2 into a.dq_bound. A lane holds 4 of the 128 dimensions; each
 // warp issues the loads of its 4 tokens before using any, so that enough bytes are in flight.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   constexpr int D = 128;
   __shared__ float red[8][3];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1454,6 +1460,8 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
 // dQ = dq_fix * 2^-e / sqrt(d) in bf16 into the Q slots of dqkv [T][p][3][H/p][d]: 16 threads
 // per (token, head), 8 elements each.
 __global__ void attn_bwd_dq_convert_kernel(const AttnArgs a, float scale) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const long long rows = (long long)a.b * a.s * a.H;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = idx >> 4;
@@ -1501,8 +1509,8 @@ cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
   const float scale = 1.f / sqrtf((float)D);
   const long long threads = (long long)a.b * a.s * a.H * 16;  // 16 per (token, head)
   const unsigned blocks = (unsigned)((threads + 255) / 256);
-  attn_bwd_prep_kernel<<<dim3(a.b * a.H, (a.s + 127) / 128 * 4), 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(true, attn_bwd_prep_kernel,
+                                dim3(a.b * a.H, (a.s + 127) / 128 * 4), dim3(256), 0, s, a);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_dq;  // the fixed-point dQ accumulator as [b][s][H*d] int32, 32 x 16 boxes
   {
@@ -1520,11 +1528,11 @@ cudaError_t bwd_fused_tc(const AttnArgs& a, cudaStream_t s) {
       return cudaErrorInvalidValue;
   }
   dim3 grid(a.b * a.H, (a.s + 127) / 128);
-  attn_bwd_fused_tc_kernel<D><<<grid, kFusedBwdThreads, L::BYTES, s>>>(
-      tm_qkv, tm_do, tm_dq, tm_dqkv, a, kLog2eF * scale, scale);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(a, scale);
-  return cudaGetLastError();
+  e = launch_kernel(true, attn_bwd_fused_tc_kernel<D>, grid, dim3(kFusedBwdThreads), L::BYTES,
+                    s, tm_qkv, tm_do, tm_dq, tm_dqkv, a, kLog2eF * scale, scale);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(true, attn_bwd_dq_convert_kernel, dim3(blocks), dim3(256), 0, s, a,
+                       scale);
 }
 
 template <int D>
@@ -1590,9 +1598,8 @@ cudaError_t fwd_tc(const AttnArgs& a, cudaStream_t s) {
   if (!make_tensor_map_bf16_3d(&tm_o, a.o, dims_o, strides_o, box)) return cudaErrorInvalidValue;
   // one CTA per pair of 128-query blocks of one head
   dim3 grid(a.b * a.H, ((a.s + 127) / 128 + 1) / 2);
-  attn_fwd_tc_kernel<D><<<grid, kAttnFwdThreads, L::BYTES, s>>>(tm, tm_o, a,
-                                                                kLog2eF / sqrtf((float)D));
-  return cudaGetLastError();
+  return launch_kernel(true, attn_fwd_tc_kernel<D>, grid, dim3(kAttnFwdThreads), L::BYTES, s,
+                       tm, tm_o, a, kLog2eF / sqrtf((float)D));
 }
 
 }  // namespace

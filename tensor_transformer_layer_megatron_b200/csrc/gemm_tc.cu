@@ -697,6 +697,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrive or load
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();  // the operands are the previous kernel's results
+  grid_dependents_launch();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -1175,9 +1177,8 @@ cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tb, const
   const int num_n = (a.Ng + tile_cols - 1) / tile_cols;
   const int tiles = a.NG * num_m2 * num_n;
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  kern<<<2 * pairs, kThreads, smem_bytes, stream>>>(ta, tb, tc, tc2, a, num_m2, num_n, bn,
-                                                     staged);
-  return cudaGetLastError();
+  return launch_kernel(!a.plain_launch, kern, dim3(2 * pairs), dim3(kThreads), smem_bytes,
+                       stream, ta, tb, tc, tc2, a, num_m2, num_n, bn, staged);
 }
 
 template <bool A_MN, bool B_MN>

@@ -473,7 +473,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
   } join{L, s, w};
   auto colsum = [&](const void* src, int cols, void* out) {
     return run(L, "colsum", 0, (double)T * cols * e + 4.0 * cols, w,
-               [&] { return launch_colsum(dt, T, cols, src, (float*)out, w); });
+               [&] { return launch_colsum(dt, T, cols, src, (float*)out, !two, w); });
   };
   const double lnb_bytes = (double)T * h * 6 * e + 3.0 * nblk * h * 4 * 2;
   const bool nb = L->cfg.disable_bias_linear, sw = L->cfg.swiglu;
@@ -496,6 +496,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(h, f, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dy; a.lda = h; a.B = act; a.ldb = f;
     a.epi = kEpiStoreF32; a.out = G->w2; a.ldc = f / p; a.out_ng = f / p;
+    a.plain_launch = two;  // the side stream's predecessor is not an input
     a.out_gs = (long long)h * (f / p); a.err = err; a.a_sp = 1;
     MGT_TRY(gemm(L, "gemm_tc/fc2_wgrad", a, w));
   }
@@ -513,6 +514,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(f1, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = du; a.lda = f1; a.B = ln2; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w1; a.ldc = h; a.err = err; a.b_sp = 1;
+    a.plain_launch = two;  // the side stream's predecessor is not an input
     MGT_TRY(gemm(L, "gemm_tc/fc1_wgrad", a, w));
   }
   // B4. LN2 backward + residual gradient dy -> dh1
@@ -535,6 +537,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dh1; a.lda = h; a.B = O; a.ldb = h; a.a_sp = 1;
     a.epi = kEpiStoreF32; a.out = G->w_o; a.ldc = h / p; a.out_ng = h / p;
+    a.plain_launch = two;  // the side stream's predecessor is not an input
     a.out_gs = (long long)h * (h / p); a.err = err;
     MGT_TRY(gemm(L, "gemm_tc/outproj_wgrad", a, w));
   }
@@ -566,6 +569,7 @@ mgt_status mgt_layer_bwd(mgt_layer* L, const mgt_layer_params* P, const void* x,
     GemmArgs a = gemm_base(3 * h, h, 1, T, 1);
     a.a_mn = 1; a.b_mn = 1; a.A = dqkv; a.lda = 3 * h; a.B = ln1; a.ldb = h;
     a.epi = kEpiStoreF32; a.out = G->w_qkv; a.ldc = h; a.err = err; a.b_sp = 1;
+    a.plain_launch = two;  // the side stream's predecessor is not an input
     MGT_TRY(gemm(L, "gemm_tc/qkv_wgrad", a, w));
   }
   // B8. LN1 backward + residual gradient dh1 -> dx

@@ -452,7 +452,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     TP_TRY(launch_gemm_tc(a, R->num_sms, s));
   }
   // fc1: db1_t, dln2 partial -> all-reduce -> bf16, dW1_t
-  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, f1l, du, (float*)G->b1, true, s));
   {
     GemmArgs a = base(T, h, f1l);
     a.b_mn = 1; a.lda = f1l; a.B = P->w1; a.ldb = h;
@@ -499,7 +499,7 @@ mgt_status mgt_tp_rank_bwd(mgt_tp_rank* R, const mgt_layer_params* P, const void
     TP_TRY(launch_attn_bwd(1, a, s));
   }
   // QKV: db_qkv_t, dln1 partial -> all-reduce -> bf16, dW_qkv,t
-  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, s));
+  if (!nb) TP_TRY(launch_colsum(1, T, 3 * hl, dqkv, (float*)G->b_qkv, true, s));
   {
     GemmArgs a = base(T, h, 3 * hl);
     a.b_mn = 1; a.lda = 3 * hl; a.B = P->w_qkv; a.ldb = h;

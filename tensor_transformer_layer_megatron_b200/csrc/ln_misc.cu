@@ -385,6 +385,8 @@ __global__ void __launch_bounds__(256) ln_fwd_ring_kernel(long long rows, int h,
                                                           T* __restrict__ y,
                                                           float* __restrict__ mean,
                                                           float* __restrict__ rstd, int* err) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[S];
@@ -503,6 +505,8 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int
                                                           T* __restrict__ dx,
                                                           float* __restrict__ partial,
                                                           long long rows_per, int* err) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[S];
@@ -727,6 +731,8 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
                                                               float* __restrict__ dgamma,
                                                               float* __restrict__ dbeta,
                                                               float* __restrict__ dres_sum) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   __shared__ float red[8][33];
   const int c = blockIdx.x * 32 + (threadIdx.x & 31);
   const int sl = threadIdx.x >> 5;
@@ -774,6 +780,8 @@ template <typename T>
 __global__ void __cluster_dims__(1, kColsumSlices, 1) __launch_bounds__(256, 4)
     colsum_kernel(long long rows, int cols, const T* __restrict__ x, float* __restrict__ out,
                   long long rows_per) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
   __shared__ float slice_sum[32 * V];
@@ -975,9 +983,9 @@ cudaError_t ln_fwd_ring_inst(long long rows, int h, float eps, const void* x, co
   if (bps < 1) return cudaErrorInvalidConfiguration;
   long long grid = (long long)bps * device_sms();
   if (grid > rows) grid = rows;
-  kern<<<(unsigned)grid, 256, smem, s>>>(rows, h, eps, reinterpret_cast<const T*>(x), g, b,
-                                        reinterpret_cast<T*>(y), mean, rstd, err);
-  return cudaGetLastError();
+  return launch_kernel(true, kern, dim3((unsigned)grid), dim3(256), smem, s, rows, h, eps,
+                       reinterpret_cast<const T*>(x), g, b, reinterpret_cast<T*>(y), mean, rstd,
+                       err);
 }
 
 // Row-group shapes: a row is spread over W warps with at most VPL 16-byte vectors per thread,
@@ -1004,9 +1012,8 @@ cudaError_t ln_fwd_dispatch(long long rows, int h, float eps, const void* x, con
 // dgamma, dbeta (and dres_sum) from the per-block partial rows, in a fixed order.
 cudaError_t launch_param_reduce(int h, long long slices, int nsum, const float* partial,
                                 float* dgamma, float* dbeta, float* dres_sum, cudaStream_t s) {
-  ln_param_reduce_kernel<<<(nsum * h + 31) / 32, 256, 0, s>>>(h, (int)slices, nsum, partial,
-                                                             dgamma, dbeta, dres_sum);
-  return cudaGetLastError();
+  return launch_kernel(true, ln_param_reduce_kernel, dim3((nsum * h + 31) / 32), dim3(256), 0,
+                       s, h, (int)slices, nsum, partial, dgamma, dbeta, dres_sum);
 }
 
 template <typename T>
@@ -1035,9 +1042,8 @@ cudaError_t ln_bwd_dispatch(long long rows, int h, const void* dy, const void* d
       const size_t smem = (size_t)kRingStages * (dres ? 3 : 2) * h * sizeof(T);
       auto launch = [&](auto kern) {
         if (ring_blocks_per_sm(kern, smem) < 1) return cudaErrorInvalidConfiguration;
-        kern<<<gs, 256, smem, s>>>(rows, h, pdy, pdr, px, g, mean, rstd, pdx, partial,
-                                   rows_per, err);
-        return cudaGetLastError();
+        return launch_kernel(true, kern, dim3(gs), dim3(256), smem, s, rows, h, pdy, pdr, px,
+                             g, mean, rstd, pdx, partial, rows_per, err);
       };
       if (nvec <= 256)
         e = nsum == 3 ? launch(ln_bwd_ring_kernel<T, 1, 3, kRingStages>)
@@ -1127,6 +1133,7 @@ cudaError_t launch_ln_bwd(int dtype, long long rows, int h, const void* dy, cons
 }
 
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
+                          bool programmatic,
                           cudaStream_t s) {
   if (rows <= 0) return cudaMemsetAsync(out, 0, sizeof(float) * cols, s);
   const int V = dtype ? 8 : 4;
@@ -1134,12 +1141,10 @@ cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, fl
   const long long rows_per = (rows + kColsumSlices - 1) / kColsumSlices;
   dim3 grid(cb, kColsumSlices), block(32, 8);
   if (dtype)
-    colsum_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        rows, cols, reinterpret_cast<const __nv_bfloat16*>(x), out, rows_per);
-  else
-    colsum_kernel<float><<<grid, block, 0, s>>>(rows, cols, reinterpret_cast<const float*>(x),
-                                                 out, rows_per);
-  return cudaGetLastError();
+    return launch_kernel(programmatic, colsum_kernel<__nv_bfloat16>, grid, block, 0, s, rows,
+                         cols, reinterpret_cast<const __nv_bfloat16*>(x), out, rows_per);
+  return launch_kernel(programmatic, colsum_kernel<float>, grid, block, 0, s, rows, cols,
+                       reinterpret_cast<const float*>(x), out, rows_per);
 }
 
 // One thread waits on an mbarrier that nothing ever arrives on, through the same bounded

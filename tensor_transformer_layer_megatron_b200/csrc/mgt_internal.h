@@ -4,7 +4,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mgt {
+
+// Kernel launch, with programmatic stream serialization when `programmatic`: the kernel's CTAs
+// may then be scheduled while the previous kernel of `s` is finishing (its tail wave, its
+// memory flush), run their set-up, and wait inside the kernel (grid_dependency_wait) for that
+// kernel's results. Only kernels that call grid_dependency_wait before touching global memory
+// may be launched this way. A launch whose stream predecessor produces none of its inputs (a
+// weight gradient on the backward's second stream) stays plain, so that its CTAs do not hold
+// SMs idle while they wait.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(bool programmatic, void (*kern)(KArgs...), dim3 grid,
+                                 dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = programmatic ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Device status codes written into the caller's status word (first failure wins).
 enum DeviceError : int {
@@ -73,6 +98,8 @@ struct GemmArgs {
   const float* b_scale;
   // Tile order (set by the launcher): 1 = N fastest within a group, 0 = M fastest.
   int n_fast;
+  // 1: plain launch; 0: programmatic stream serialization (see launch_kernel)
+  int plain_launch;
 };
 
 
@@ -146,6 +173,7 @@ cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
 // Column sums of a [rows, cols] activation matrix into fp32 (bias gradients), deterministic
 // (fixed-order additions; one launch, no scratch memory).
 cudaError_t launch_colsum(int dtype, long long rows, int cols, const void* x, float* out,
+                          bool programmatic,
                           cudaStream_t stream);
 
 // Causal attention over packed qkv [T][p][3][H/p][d]; O [T][p][H/p][d]; lse [b][H][s].
