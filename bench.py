@@ -160,9 +160,12 @@ def e2e_steps(run, host, steps, stream, graph=True):
     """K steps through the C ABI with host buffers; returns the device-timed ms. Every step
     copies its own x, dy from pinned host memory and its y, dx back. The device buffers are
     double-buffered and the copies run on two copy streams, so step i+1's inputs arrive and
-    step i-1's results leave while step i computes (a training loop with prefetch). With
-    `graph`, the C-ABI calls of a step (which allocate nothing and never synchronise) are
-    captured once per buffer set into a CUDA graph and replayed; the copies stay outside."""
+    step i-1's results leave while step i computes (a training loop with prefetch). Within a
+    step the forward waits only for x and the backward for dy, and y leaves while the backward
+    runs, so only the first x and the last dx are not hidden behind compute. With `graph`, the
+    C-ABI forward and backward calls of a step (which allocate nothing and never synchronise)
+    are captured once per buffer set into two CUDA graphs and replayed; the copies stay
+    outside."""
     import torch
     x_h, dy_h, y_h, dx_h = host
     first = (run.x, run.dy, run.y, run.dx)
@@ -171,16 +174,17 @@ def e2e_steps(run, host, steps, stream, graph=True):
     if graph:
         for b in range(2):
             run.x, run.dy, run.y, run.dx = bufs[b]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                run.step()
-            graphs[b] = g
+            gf, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gf):
+                run.fwd()
+            with torch.cuda.graph(gb):
+                run.bwd()
+            graphs[b] = (gf, gb)
         run.x, run.dy, run.y, run.dx = first
         torch.cuda.synchronize()
     s_in, s_out = torch.cuda.Stream(run.x.device), torch.cuda.Stream(run.x.device)
-    in_ready = [torch.cuda.Event(), torch.cuda.Event()]
-    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
-    out_done = [torch.cuda.Event(), torch.cuda.Event()]
+    ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]  # noqa: E731
+    x_ready, dy_ready, fwd_done, comp_done, y_out, dx_out = ev(), ev(), ev(), ev(), ev(), ev()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     s_in.wait_event(t0)
@@ -191,23 +195,34 @@ def e2e_steps(run, host, steps, stream, graph=True):
             if i >= 2:
                 s_in.wait_event(comp_done[b])  # step i-2 has finished reading x[b], dy[b]
             x.copy_(x_h, non_blocking=True)
+            x_ready[b].record(s_in)
             dy.copy_(dy_h, non_blocking=True)
-            in_ready[b].record(s_in)
-        stream.wait_event(in_ready[b])
+            dy_ready[b].record(s_in)
+        stream.wait_event(x_ready[b])
         if i >= 2:
-            stream.wait_event(out_done[b])  # step i-2's y[b], dx[b] have been copied out
+            stream.wait_event(y_out[b])  # step i-2's y[b] has been copied out
         if graphs[b] is not None:
-            graphs[b].replay()
+            graphs[b][0].replay()
         else:
             run.x, run.dy, run.y, run.dx = x, dy, y, dx
-            run.step(stream)
+            run.fwd(stream)
+        fwd_done[b].record(stream)
+        stream.wait_event(dy_ready[b])
+        if i >= 2:
+            stream.wait_event(dx_out[b])  # step i-2's dx[b] has been copied out
+        if graphs[b] is not None:
+            graphs[b][1].replay()
+        else:
+            run.bwd(stream)
         comp_done[b].record(stream)
         with torch.cuda.stream(s_out):
-            s_out.wait_event(comp_done[b])
+            s_out.wait_event(fwd_done[b])
             y_h.copy_(y, non_blocking=True)
+            y_out[b].record(s_out)
+            s_out.wait_event(comp_done[b])
             dx_h.copy_(dx, non_blocking=True)
-            out_done[b].record(s_out)
-    stream.wait_event(out_done[(steps - 1) & 1])
+            dx_out[b].record(s_out)
+    stream.wait_event(dx_out[(steps - 1) & 1])
     t1.record(stream)
     torch.cuda.synchronize()
     run.x, run.dy, run.y, run.dx = first
