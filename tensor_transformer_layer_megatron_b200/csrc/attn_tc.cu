@@ -112,7 +112,6 @@ __global__ void __launch_bounds__(kAttnFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   grid_dependency_wait();  // qkv is the previous kernel's result
-  grid_dependents_launch();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -1053,7 +1052,6 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   grid_dependency_wait();  // the pre-pass's statistics and zeroed accumulator
-  grid_dependents_launch();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -1371,7 +1369,6 @@ __global__ void __launch_bounds__(kFusedBwdThreads, 1)
 // warp issues the loads of its 4 tokens before using any, so that enough bytes are in flight.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
   grid_dependency_wait();
-  grid_dependents_launch();
   constexpr int D = 128;
   __shared__ float red[8][3];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1461,7 +1458,6 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
 // per (token, head), 8 elements each.
 __global__ void attn_bwd_dq_convert_kernel(const AttnArgs a, float scale) {
   grid_dependency_wait();
-  grid_dependents_launch();
   const long long rows = (long long)a.b * a.s * a.H;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = idx >> 4;

@@ -25,7 +25,11 @@ using namespace mgt;
 
 namespace {
 
-constexpr int kMaxLnBlocks = 296;  // LayerNorm backward partial rows (2 per SM on 148 SMs)
+// LayerNorm backward blocks, each writing one partial row of dgamma/dbeta (and the residual
+// gradient's column sum): one per SM on 148 SMs. A block's bulk-copy row ring keeps enough
+// bytes in flight on its own, and half the partial rows of two per SM take 7 us per step off
+// the two fixed-order parameter reduces.
+constexpr int kMaxLnBlocks = 148;
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 

@@ -386,7 +386,6 @@ __global__ void __launch_bounds__(256) ln_fwd_ring_kernel(long long rows, int h,
                                                           float* __restrict__ mean,
                                                           float* __restrict__ rstd, int* err) {
   grid_dependency_wait();
-  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[S];
@@ -506,7 +505,6 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int
                                                           float* __restrict__ partial,
                                                           long long rows_per, int* err) {
   grid_dependency_wait();
-  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[S];
@@ -732,7 +730,6 @@ __global__ void __launch_bounds__(256) ln_param_reduce_kernel(int h, int nblk, i
                                                               float* __restrict__ dbeta,
                                                               float* __restrict__ dres_sum) {
   grid_dependency_wait();
-  grid_dependents_launch();
   __shared__ float red[8][33];
   const int c = blockIdx.x * 32 + (threadIdx.x & 31);
   const int sl = threadIdx.x >> 5;
@@ -781,7 +778,6 @@ __global__ void __cluster_dims__(1, kColsumSlices, 1) __launch_bounds__(256, 4)
     colsum_kernel(long long rows, int cols, const T* __restrict__ x, float* __restrict__ out,
                   long long rows_per) {
   grid_dependency_wait();
-  grid_dependents_launch();
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
   __shared__ float slice_sum[32 * V];

@@ -171,17 +171,15 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // Programmatic dependent launch. A kernel launched with programmatic stream serialization
-// (launch_dependent) may start while the previous kernel of its stream is still running;
-// every thread calls grid_dependency_wait() after its shared-memory and TMEM set-up and before
-// its first global-memory access, which returns once that kernel has completed and its
-// writes are visible. grid_dependents_launch() lets the next such kernel be scheduled onto
-// SMs that this grid leaves free, once every CTA of this grid has called it or exited.
-// Without a programmatic predecessor the wait returns at once.
+// (launch_kernel) may be scheduled once every CTA of the previous kernel of its stream has
+// exited, before that grid has completed and flushed its writes; every thread calls
+// grid_dependency_wait() after its shared-memory and TMEM set-up and before its first
+// global-memory access, which returns once that kernel has completed and its writes are
+// visible. No kernel triggers its dependents earlier than its own exit: CTAs that were
+// resident early would hold SMs idle that the backward's second stream fills. Without a
+// programmatic predecessor the wait returns at once.
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dependents_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, fp32 accumulate).

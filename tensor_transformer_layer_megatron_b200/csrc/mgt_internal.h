@@ -9,12 +9,12 @@
 namespace mgt {
 
 // Kernel launch, with programmatic stream serialization when `programmatic`: the kernel's CTAs
-// may then be scheduled while the previous kernel of `s` is finishing (its tail wave, its
-// memory flush), run their set-up, and wait inside the kernel (grid_dependency_wait) for that
-// kernel's results. Only kernels that call grid_dependency_wait before touching global memory
-// may be launched this way. A launch whose stream predecessor produces none of its inputs (a
-// weight gradient on the backward's second stream) stays plain, so that its CTAs do not hold
-// SMs idle while they wait.
+// may then be scheduled as soon as the previous kernel of `s` has no CTA left, while that
+// grid completes and flushes its writes, run their set-up, and wait inside the kernel
+// (grid_dependency_wait) for that kernel's results. Only kernels that call
+// grid_dependency_wait before touching global memory may be launched this way. A launch whose
+// stream predecessor produces none of its inputs (a weight gradient on the backward's second
+// stream) stays plain.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(bool programmatic, void (*kern)(KArgs...), dim3 grid,
                                  dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
