@@ -936,9 +936,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // P^T goes back into TMEM as packed bf16 (the A operand of dV). dS^T goes to shared memory
 // in the 128-byte swizzled layout, where one buffer serves as the K-major A operand of dK
 // (rows = keys) and as the MN-major B operand of dQ^T (queries contiguous). Four drain warps
-// read each dQ^T tile from TMEM and add it into the accumulator a.dq_fix [T][H][d] with
-// coalesced reductions (a warp covers 32 consecutive d of one query). Five products per
-// (key block, query block) instead of the seven of the two-kernel form.
+// read each dQ^T tile from TMEM, convert it to fixed point and stage it 16 queries at a time
+// as [query][d] boxes that bulk tensor reduce-adds add into the accumulator a.dq_fix [T][H][d].
+// Five products per (key block, query block) instead of the seven of the two-kernel form.
+// After the last sub-block dK and dV leave through bulk tensor stores staged in the K and V
+// tile buffers. The kernel is bound by shared-memory bandwidth: the N = 64 products read a
+// 4 KB A tile and a 2 KB B tile per 32 cycles of math.
 //
 // The accumulator is 32-bit fixed point, so the result is bit-reproducible: integer addition
 // is associative, and the key blocks of a query block arrive in no fixed order. Every partial
