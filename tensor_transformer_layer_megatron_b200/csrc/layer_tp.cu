@@ -23,7 +23,7 @@
 namespace mgt {
 namespace {
 
-constexpr int kMaxLnSlices = 296;  // LayerNorm backward partial rows (2 per SM on 148 SMs)
+constexpr int kMaxLnSlices = 148;  // LayerNorm backward partial rows (one block per SM)
 constexpr int kMaxBands = 16;      // row bands per shard sum
 
 // out[i] = bf16(part[i] + bias[i % h] + res[i]); bias and res may be null. Eight elements per

@@ -492,9 +492,13 @@ __global__ void __launch_bounds__(256) ln_fwd_ring_kernel(long long rows, int h,
 
 // LayerNorm backward over a contiguous slice of rows per block (rows_per each): dx per row and
 // the parameter partials of the slice, as ln_bwd_fused_kernel, with x, dy and dres streamed
-// through the ring (one stage = the three rows) instead of prefetched into registers.
+// through the ring (one stage = the three rows) instead of prefetched into registers. Rows are
+// taken two at a time: the two rows' sums are reduced together, behind one block barrier, so
+// the shuffle chains and the barrier of one row overlap the other's (a row alone left the SM
+// mostly waiting on that chain). Each row's sums and each column's partial sums are formed in
+// the same order as one row at a time, so the results do not depend on the pairing.
 template <typename T, int VPL, int NSUM, int S>
-__global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int h,
+__global__ void __launch_bounds__(256, 1) ln_bwd_ring_kernel(long long rows, int h,
                                                           const T* __restrict__ dy,
                                                           const T* __restrict__ dres,
                                                           const T* __restrict__ x,
@@ -505,10 +509,11 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int
                                                           float* __restrict__ partial,
                                                           long long rows_per, int* err) {
   grid_dependency_wait();
+  static_assert(S % 2 == 0, "rows are taken in pairs of stages");
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[S];
-  __shared__ float2 red[2][8];
+  __shared__ float4 red[2][8];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int nvec = h / V;
   const uint32_t row_bytes = (uint32_t)h * sizeof(T);
@@ -539,29 +544,32 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int
 #pragma unroll
     for (int j = 0; j < V; ++j) ag[k][j] = ab[k][j] = ar[k][j] = 0.f;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  float cmu = nloc ? mean[r0] : 0.f, crs = nloc ? rstd[r0] : 0.f;
+  float cmu[2], crs[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    cmu[q] = q < nloc ? mean[r0 + q] : 0.f;
+    crs[q] = q < nloc ? rstd[r0 + q] : 0.f;
+  }
   int par = 0;
-  for (long long i = 0; i < nloc; ++i, par ^= 1) {
+  for (long long i = 0; i < nloc; i += 2, par ^= 1) {
     const long long r = r0 + i;
-    const int st = (int)(i % S);
-    const float nmu = i + 1 < nloc ? mean[r + 1] : 0.f;
-    const float nrs = i + 1 < nloc ? rstd[r + 1] : 0.f;
-    const bool ok = mbar_wait(&full[st], (uint32_t)((i / S) & 1), err, kErrTimeoutLn, nullptr);
-    const uint4* sx = reinterpret_cast<const uint4*>(ring + (size_t)st * stage_bytes);
-    const uint4* sd = sx + row_bytes / 16;
-    const uint4* sr = sd + row_bytes / 16;
-    uint4 cx[VPL], cd[VPL], cr[VPL];
-    float s1 = 0.f, s2 = 0.f;
+    const bool two = i + 1 < nloc;  // the slice's last row may come alone
+    float nmu[2], nrs[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      nmu[q] = i + 2 + q < nloc ? mean[r + 2 + q] : 0.f;
+      nrs[q] = i + 2 + q < nloc ? rstd[r + 2 + q] : 0.f;
+    }
+    bool ok = mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), err, kErrTimeoutLn, nullptr);
+    if (two && ok)
+      ok = mbar_wait(&full[(i + 1) % S], (uint32_t)(((i + 1) / S) & 1), err, kErrTimeoutLn,
+                     nullptr);
+    uint4 cx[2][VPL], cd[2][VPL], cr[2][VPL];
+    float s1[2] = {0.f, 0.f}, s2[2] = {0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
       const int vi = t + k * 256;
-      const bool in = ok && vi < nvec;
-      cx[k] = in ? sx[vi] : zero;
-      cd[k] = in ? sd[vi] : zero;
-      cr[k] = (in && dres) ? sr[vi] : zero;
-      float xv[V], dv[V], gv[V];
-      Vec<T>::unpack(cx[k], xv);
-      Vec<T>::unpack(cd[k], dv);
+      float gv[V];
       if (vi < nvec) {
         load_param<V>(gamma, vi * V, gv);
       } else {
@@ -569,55 +577,84 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_ring_kernel(long long rows, int
         for (int j = 0; j < V; ++j) gv[j] = 0.f;
       }
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
-        s1 += g;
-        s2 += g * xh;
-        ag[k][j] += dv[j] * xh;
-        ab[k][j] += dv[j];
+      for (int q = 0; q < 2; ++q) {
+        const uint4* sx =
+            reinterpret_cast<const uint4*>(ring + (size_t)((i + q) % S) * stage_bytes);
+        const uint4* sd = sx + row_bytes / 16;
+        const uint4* sr = sd + row_bytes / 16;
+        const bool in = ok && vi < nvec && (q == 0 || two);
+        cx[q][k] = in ? sx[vi] : zero;
+        cd[q][k] = in ? sd[vi] : zero;
+        cr[q][k] = (in && dres) ? sr[vi] : zero;
+        float xv[V], dv[V];
+        Vec<T>::unpack(cx[q][k], xv);
+        Vec<T>::unpack(cd[q][k], dv);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const float xh = (xv[j] - cmu[q]) * crs[q], g = dv[j] * gv[j];
+          s1[q] += g;
+          s2[q] += g * xh;
+          ag[k][j] += dv[j] * xh;  // a missing second row has dy = 0: it adds nothing
+          ab[k][j] += dv[j];
+        }
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      s1[0] += __shfl_xor_sync(0xffffffffu, s1[0], o);
+      s2[0] += __shfl_xor_sync(0xffffffffu, s2[0], o);
+      s1[1] += __shfl_xor_sync(0xffffffffu, s1[1], o);
+      s2[1] += __shfl_xor_sync(0xffffffffu, s2[1], o);
     }
-    // Two buffers by row parity: a buffer is rewritten two rows later, after every thread has
-    // passed the next row's barrier and so has finished reading it.
-    if (lane == 0) red[par][warp] = make_float2(s1, s2);
+    // Two buffers by pair parity: a buffer is rewritten two pairs later, after every thread
+    // has passed the next pair's barrier and so has finished reading it.
+    if (lane == 0) red[par][warp] = make_float4(s1[0], s2[0], s1[1], s2[1]);
     if (__syncthreads_or(!ok)) {
       if (t == 0) ring_drain<S>(full, i, nloc, err);
       return;
     }
-    if (t == 0 && i + S < nloc) issue(i + S);  // the stage has been read into registers
-    float S1 = 0.f, S2 = 0.f;
+    if (t == 0) {  // both stages have been read into registers: refill them
+      if (i + S < nloc) issue(i + S);
+      if (i + 1 + S < nloc) issue(i + 1 + S);
+    }
+    float S1[2] = {0.f, 0.f}, S2[2] = {0.f, 0.f};
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-      const float2 v = red[par][w];
-      S1 += v.x;
-      S2 += v.y;
+      const float4 v = red[par][w];
+      S1[0] += v.x;
+      S2[0] += v.y;
+      S1[1] += v.z;
+      S2[1] += v.w;
     }
-    const float m1 = S1 * inv_h, m2 = S2 * inv_h;
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
       const int vi = t + k * 256;
       if (vi < nvec) {
-        float xv[V], dv[V], rv[V], gv[V], o[V];
-        Vec<T>::unpack(cx[k], xv);
-        Vec<T>::unpack(cd[k], dv);
-        Vec<T>::unpack(cr[k], rv);
+        float gv[V];
         load_param<V>(gamma, vi * V, gv);
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-          const float xh = (xv[j] - cmu) * crs, g = dv[j] * gv[j];
-          o[j] = crs * (g - m1 - xh * m2) + rv[j];
-          if constexpr (NSUM == 3) ar[k][j] += rv[j];
+        for (int q = 0; q < 2; ++q) {
+          if (q == 1 && !two) break;
+          const float m1 = S1[q] * inv_h, m2 = S2[q] * inv_h;
+          float xv[V], dv[V], rv[V], o[V];
+          Vec<T>::unpack(cx[q][k], xv);
+          Vec<T>::unpack(cd[q][k], dv);
+          Vec<T>::unpack(cr[q][k], rv);
+#pragma unroll
+          for (int j = 0; j < V; ++j) {
+            const float xh = (xv[j] - cmu[q]) * crs[q], g = dv[j] * gv[j];
+            o[j] = crs[q] * (g - m1 - xh * m2) + rv[j];
+            if constexpr (NSUM == 3) ar[k][j] += rv[j];
+          }
+          Vec<T>::store(dx + (r + q) * h + vi * V, o);
         }
-        Vec<T>::store(dx + r * h + vi * V, o);
       }
     }
-    cmu = nmu;
-    crs = nrs;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      cmu[q] = nmu[q];
+      crs[q] = nrs[q];
+    }
   }
   float* pg = partial + (long long)blockIdx.x * NSUM * h;
 #pragma unroll
